@@ -1,0 +1,265 @@
+"""fp64 CPU oracle for mixed-head (retrieval / streaming) KV-cache attention.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this module.  It shares no code
+with the CUDA library (``head_wise_kv_b200``) and imports nothing from it; the
+library never imports this.
+
+Plain, slow and meant to be checked by eye against the pages:
+
+* "DuoAttention: Dual Retrieval & Streaming Heads Guide" (the DuoAttention
+  guide below), sections 1 (KV-cache-size equation), 2 ("Retrieval Heads vs.
+  Streaming Heads", "Cache Partitioning Mechanics" and its memory equation)
+  and its Python simulation of the dual-head cache;
+* "Attention Variants and KV-Cache Compression", sections "MHA and GQA"
+  (size formula) and "When Is Reuse Exact?" (chunked-prefill mask rule,
+  original positions kept after eviction);
+* "Attention Variants and Memory Efficiency", sections "Multi-Query and
+  Grouped-Query Attention" (``repeat_kv``) and "Sliding-Window and Mixed
+  Attention" (window rule and ``SlidingKVCache`` ring).
+
+Every bf16 input is widened exactly to float64; all arithmetic is float64.
+
+Readings taken where the pages leave a step open (each listed in the design
+notes of the repository):
+  * the recent window includes the current token: keys t-W+1 .. t;
+  * when fewer than S+W tokens exist, a streaming head sees every token
+    (sinks and window overlap; union, no duplicates);
+  * the ring slot of token p is p for p < S, else S + ((p - S) mod W): the
+    sliding-window ring's "slot = appended-count mod W" rule applied to the
+    tokens that come after the sinks;
+  * query head h reads KV head h // (Hq / n_kv) (``repeat_interleave``);
+  * a decode query sits at t = T - 1, the token just appended; prefill row i
+    of a chunk that follows P cached tokens sits at t = P + i.
+
+Parity pins for every function live in ``tests/test_oracle_pins.py``.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+__all__ = [
+    "kv_cache_bytes", "duo_effective_context", "duo_cache_bytes", "duo_slots",
+    "StreamingCache", "ring_positions", "keep_set", "key_mask", "kv_head_of",
+    "attend", "decode_attention", "prefill_attention", "brute_force_attention",
+]
+
+
+# ---------------------------------------------------------------- sizes
+def kv_cache_bytes(layers: int, n_kv: int, d: int, tokens: int, elem_bytes: int = 2) -> int:
+    """Dense KV-cache bytes: keys and values (x2), ``elem_bytes`` per element,
+    for every layer, KV head, head-dim element and token.
+    DuoAttention guide, section 1, KV-cache-size equation; the same product
+    as the size formula of "Attention Variants and KV-Cache Compression",
+    section "MHA and GQA"."""
+    return 2 * elem_bytes * layers * n_kv * d * tokens
+
+
+def duo_effective_context(tokens: int, sink: int, window: int, retrieval_frac: float) -> float:
+    """Tokens held per KV head on average: R*T + (1-R)*(S+W).
+    DuoAttention guide, section 2, memory equation and its 128k worked line."""
+    return retrieval_frac * tokens + (1.0 - retrieval_frac) * (sink + window)
+
+
+def duo_cache_bytes(layers: int, n_kv: int, d: int, tokens: int, sink: int, window: int,
+                    n_retrieval, elem_bytes: int = 2) -> int:
+    """Bytes of the DuoAttention cache for one sequence with ``tokens`` rows
+    reserved per retrieval head: retrieval heads keep all T tokens, streaming
+    heads keep S + W (DuoAttention guide, section 2, memory equation,
+    with R = retrieval heads / n_kv).  ``n_retrieval`` is one count for all
+    layers or a per-layer list; the result is exact integer arithmetic."""
+    per_layer = list(n_retrieval) if hasattr(n_retrieval, "__len__") else [n_retrieval] * layers
+    assert len(per_layer) == layers
+    total = 0
+    for n_r in per_layer:
+        n_s = n_kv - int(n_r)
+        total += 2 * elem_bytes * d * (int(n_r) * tokens + n_s * (sink + window))
+    return total
+
+
+def duo_slots(tokens: int, sink: int, window: int, n_retrieval: int, n_streaming: int) -> int:
+    """Occupied cache rows after ``tokens`` appends: every token in each
+    retrieval head, at most S + W in each streaming head (the DuoAttention
+    guide's simulation counts slots this way in its memory statistics)."""
+    return n_retrieval * tokens + n_streaming * min(tokens, sink + window)
+
+
+# ---------------------------------------------------------------- ring
+class StreamingCache:
+    """Literal per-token model of one streaming head's cache.
+
+    Tokens go to the sink region until it holds S tokens (DuoAttention guide,
+    simulation, ``append_token``); every later token goes to the recent
+    window, a W-slot ring that overwrites its oldest entry, its slot being the
+    number of window appends so far modulo W ("Attention Variants and Memory
+    Efficiency", ``SlidingKVCache.append``).  Slots 0..S-1 are the sinks, slots
+    S..S+W-1 the ring.  ``pos[slot]`` keeps each token's original position
+    (-1 = empty): "Attention Variants and KV-Cache Compression", section
+    "When Is Reuse Exact?" -- positions are not renumbered after eviction."""
+
+    def __init__(self, sink: int, window: int):
+        assert sink >= 0 and window >= 1
+        self.sink, self.window = sink, window
+        self.pos = np.full(sink + window, -1, dtype=np.int64)
+        self.items = [None] * (sink + window)
+        self.n_sink = 0
+        self.n_window = 0
+
+    def append(self, position: int, item=None) -> int:
+        if self.n_sink < self.sink:
+            slot = self.n_sink
+            self.n_sink += 1
+        else:
+            slot = self.sink + (self.n_window % self.window)
+            self.n_window += 1
+        self.pos[slot] = position
+        self.items[slot] = item
+        return slot
+
+    def ordered(self):
+        """Held (position, item) pairs, sinks first, then the window oldest to
+        newest (the ring's ordered view)."""
+        sinks = [(int(self.pos[s]), self.items[s]) for s in range(self.n_sink)]
+        count = min(self.n_window, self.window)
+        win = [(int(self.pos[self.sink + (k % self.window)]), self.items[self.sink + (k % self.window)])
+               for k in range(self.n_window - count, self.n_window)]
+        return sinks + win
+
+
+def ring_positions(tokens: int, sink: int, window: int) -> np.ndarray:
+    """pos table [S+W] after appending positions 0 .. tokens-1 one by one."""
+    c = StreamingCache(sink, window)
+    for p in range(tokens):
+        c.append(p)
+    return c.pos.copy()
+
+
+# ---------------------------------------------------------------- key sets
+def keep_set(t: int, sink: int, window: int) -> np.ndarray:
+    """Key positions a streaming head attends from query position t: the
+    attention sinks 0..S-1 and the recent window max(0, t-W+1) .. t
+    (DuoAttention guide, section 2, streaming heads; window rule of
+    "Attention Variants and Memory Efficiency", section "Sliding-Window and
+    Mixed Attention")."""
+    j = np.arange(t + 1)
+    return j[(j < sink) | (j >= t - window + 1)]
+
+
+def key_mask(rows_t: np.ndarray, n_keys: int, retrieval: bool, sink: int, window: int) -> np.ndarray:
+    """bool [len(rows_t)][n_keys]: may the query at absolute position
+    rows_t[i] read the key at absolute position j?  Retrieval heads: every
+    j <= t (full causal).  Streaming heads: j <= t and j in keep_set(t)."""
+    t = np.asarray(rows_t)[:, None]
+    j = np.arange(n_keys)[None, :]
+    m = j <= t
+    if not retrieval:
+        m &= (j < sink) | (j >= t - window + 1)
+    return m
+
+
+def kv_head_of(h: int, hq: int, n_kv: int) -> int:
+    """KV head read by query head h: K/V repeated along the head axis with
+    ``repeat_interleave(hq // n_kv)`` ("Attention Variants and Memory
+    Efficiency", section "Multi-Query and Grouped-Query Attention")."""
+    assert hq % n_kv == 0
+    return h // (hq // n_kv)
+
+
+# ---------------------------------------------------------------- attention
+def attend(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float):
+    """Softmax attention of one query over the given keys (float64).
+    Returns (o [d], lse) with lse = log sum_j exp(s_j)."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    s = scale * (k @ q)
+    m = s.max()
+    e = np.exp(s - m)
+    z = e.sum()
+    return (e @ v) / z, m + math.log(z)
+
+
+def decode_attention(q, k_hist, v_hist, lens_after, mask, sink, window, scale):
+    """One decode step of one layer.
+
+    q: [B][Hq][d] (the newest token's query per sequence);
+    k_hist(b, g) / v_hist(b, g): callables returning the full history
+    [lens_after[b]][d] of KV head g of sequence b (tokens 0 .. T_b-1);
+    mask: [n_kv], 1 = retrieval head.  Query position t = T_b - 1.
+    Returns out [B][Hq][d] and lse [B][Hq] (float64)."""
+    q = np.asarray(q, dtype=np.float64)
+    B, hq, d = q.shape
+    n_kv = len(mask)
+    out = np.zeros((B, hq, d))
+    lse = np.zeros((B, hq))
+    for b in range(B):
+        t = int(lens_after[b]) - 1
+        for g in range(n_kv):
+            keys = np.arange(t + 1) if mask[g] else keep_set(t, sink, window)
+            K = np.asarray(k_hist(b, g), dtype=np.float64)[keys]
+            V = np.asarray(v_hist(b, g), dtype=np.float64)[keys]
+            for h in range(hq):
+                if kv_head_of(h, hq, n_kv) != g:
+                    continue
+                out[b, h], lse[b, h] = attend(q[b, h], K, V, scale)
+    return out, lse
+
+
+def prefill_attention(q, k_hist, v_hist, prefix, mask, sink, window, scale,
+                      rows=None, row_block: int = 256):
+    """Attention of a prefill chunk of C queries that follows ``prefix[b]``
+    cached tokens ("Attention Variants and KV-Cache Compression", section
+    "When Is Reuse Exact?": row i sits at absolute position P + i and may read
+    keys through P + i, not an upper-left C x (P + C) triangle).
+
+    q: [B][Hq][C][d]; k_hist(b, g) / v_hist(b, g): history [P_b + C][d]
+    (cached prefix followed by the chunk's own keys); rows: optional list of
+    chunk rows to evaluate (others are left as NaN).
+    Returns out [B][Hq][C][d] (float64)."""
+    q = np.asarray(q, dtype=np.float64)
+    B, hq, C, d = q.shape
+    n_kv = len(mask)
+    rows = np.arange(C) if rows is None else np.asarray(sorted(rows))
+    out = np.full((B, hq, C, d), np.nan)
+    for b in range(B):
+        P = int(prefix[b])
+        for g in range(n_kv):
+            K = np.asarray(k_hist(b, g), dtype=np.float64)
+            V = np.asarray(v_hist(b, g), dtype=np.float64)
+            assert K.shape[0] >= P + C
+            for h in range(hq):
+                if kv_head_of(h, hq, n_kv) != g:
+                    continue
+                for r0 in range(0, len(rows), row_block):
+                    rr = rows[r0:r0 + row_block]
+                    t = P + rr
+                    n_keys = int(t.max()) + 1
+                    allowed = key_mask(t, n_keys, bool(mask[g]), sink, window)
+                    s = scale * (q[b, h, rr] @ K[:n_keys].T)
+                    s = np.where(allowed, s, -np.inf)
+                    m = s.max(axis=1, keepdims=True)
+                    e = np.exp(s - m)
+                    out[b, h, rr] = (e @ V[:n_keys]) / e.sum(axis=1, keepdims=True)
+    return out
+
+
+def brute_force_attention(q, k, v, keys, scale):
+    """Pure-Python loops (tiny inputs only): softmax over the listed key
+    positions of scale * <q, k_j>, weights applied to v_j."""
+    d = len(q)
+    scores = []
+    for j in keys:
+        acc = 0.0
+        for x in range(d):
+            acc += float(q[x]) * float(k[j][x])
+        scores.append(scale * acc)
+    m = max(scores)
+    w = [math.exp(s - m) for s in scores]
+    z = sum(w)
+    o = [0.0] * d
+    for wj, j in zip(w, keys):
+        for x in range(d):
+            o[x] += wj * float(v[j][x])
+    return [ox / z for ox in o], m + math.log(z)

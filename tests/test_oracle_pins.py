@@ -1,0 +1,393 @@
+"""Pins for the fp64 oracle, against values the pages print, closed forms,
+library routines and brute force -- never against the oracle itself.
+
+The last section plants plausible mistakes in the oracle (monkeypatched, on
+the CPU) and checks that some pin fails for each.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import duo_oracle as O
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def fixture(name):
+    rows = []
+    with open(os.path.join(GOLD, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                rows.append(line)
+    return rows
+
+
+def fixture_kv(name):
+    out = {}
+    for r in fixture(name):
+        k, v = r.split(None, 1)
+        out[k] = v
+    return out
+
+
+# ------------------------------------------------------------------ sizes
+def test_dense_sizes_match_printed_values():
+    n = 0
+    for row in fixture("kv_sizes.txt"):
+        lhs, rhs = row.split("=")
+        kind, L, n_kv, d, T = lhs.split()
+        assert kind == "dense"
+        assert O.kv_cache_bytes(int(L), int(n_kv), int(d), int(T)) == int(rhs)
+        n += 1
+    assert n == 3
+
+
+def test_four_gqa_sequences_equal_one_mha_sequence():
+    # "Attention Variants and KV-Cache Compression", MHA and GQA: four equal-length
+    # GQA sequences use 2 GiB, as one MHA sequence does.
+    assert 4 * O.kv_cache_bytes(32, 8, 128, 4096) == O.kv_cache_bytes(32, 32, 128, 4096) == 2 ** 31
+
+
+def test_effective_context_printed_value():
+    f = fixture_kv("duo_effective_context.txt")
+    got = O.duo_effective_context(int(f["tokens"]), int(f["sink"]), int(f["window"]),
+                                  float(f["retrieval_frac"]))
+    assert got == pytest.approx(int(f["effective_context"]), abs=1e-9)
+
+
+def test_duo_bytes_of_the_guides_example():
+    # 80 layers, 8 KV heads, d=128, T=128,000, S=32, W=128 and R = 0.25 (2 of 8 heads):
+    # the printed effective context (32,120 tokens per head) times the printed dense
+    # bytes per token (41,943,040,000 / 128,000).
+    f = fixture_kv("duo_effective_context.txt")
+    dense_per_token = 41943040000 // 128000
+    got = O.duo_cache_bytes(80, 8, 128, 128000, 32, 128, 2)
+    assert got == int(f["effective_context"]) * dense_per_token == 10525081600
+
+
+def test_duo_bytes_limits():
+    # all heads retrieval: the dense formula; no retrieval heads: T replaced by S+W
+    assert O.duo_cache_bytes(3, 4, 64, 1000, 16, 64, 4) == O.kv_cache_bytes(3, 4, 64, 1000)
+    assert O.duo_cache_bytes(3, 4, 64, 1000, 16, 64, 0) == O.kv_cache_bytes(3, 4, 64, 80)
+    assert O.duo_cache_bytes(2, 8, 128, 5000, 64, 256, [2, 5]) == \
+        O.kv_cache_bytes(1, 7, 128, 5000) + O.kv_cache_bytes(1, 9, 128, 320)
+
+
+# ------------------------------------------------------------------ ring
+def test_sliding_window_printed_example():
+    f = fixture_kv("sliding_window_ring.txt")
+    c = O.StreamingCache(0, int(f["window"]))
+    for p in range(int(f["appends"])):
+        c.append(p, int(f["value_factor"]) * p)
+    want = [tuple(int(x) for x in e.split(":")) for e in f["ordered"].split()]
+    assert [(p, it) for p, it in c.ordered()] == want
+    # slot layout: slot = appended count mod 3 -> positions 3, 4, 2 in slots 0, 1, 2
+    assert list(c.pos) == [3, 4, 2]
+
+
+def _list_simulation(T, S, W):
+    """The guide's simulation: a sink list filled first, then a window list
+    that drops its oldest entry once it holds more than W."""
+    sinks, window = [], []
+    for p in range(T):
+        if len(sinks) < S:
+            sinks.append(p)
+        else:
+            window.append(p)
+            if len(window) > W:
+                window.pop(0)
+    return sinks, window
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_ring_matches_list_simulation(seed):
+    rng = np.random.default_rng(seed)
+    for _ in range(40):
+        S, W = int(rng.integers(0, 9)), int(rng.integers(1, 12))
+        T = int(rng.integers(0, 60))
+        c = O.StreamingCache(S, W)
+        for p in range(T):
+            c.append(p)
+        sinks, window = _list_simulation(T, S, W)
+        assert [p for p, _ in c.ordered()] == sinks + window
+        held = sorted(int(p) for p in c.pos if p >= 0)
+        assert held == sorted(sinks + window)
+        if T:
+            # the keep set of the newest token is exactly what the cache holds
+            assert held == list(O.keep_set(T - 1, S, W))
+
+
+def test_needle_simulation_statements():
+    f = fixture_kv("duo_simulation_needle.txt")
+    L, H, S, W, T = (int(f[k]) for k in ("layers", "heads", "sink", "window", "tokens"))
+    needle = int(f["needle"])
+    # head assignment of the page's simulation: max(1, int(L*H*R)) retrieval heads,
+    # taken from layers >= 1 at even head indices
+    count = max(1, int(L * H * float(f["retrieval_frac"])))
+    roles, taken = {}, 0
+    for l in range(L):
+        for h in range(H):
+            r = taken < count and l >= 1 and h % 2 == 0
+            roles[(l, h)] = r
+            taken += r
+    n_r = sum(roles.values())
+    held = set(int(p) for p in O.ring_positions(T, S, W) if p >= 0)
+    # every retrieval head keeps all T tokens (the needle included); streaming heads not
+    assert f["needle_in_retrieval"] == "all" and needle < T
+    assert f["needle_in_streaming"] == "none" and needle not in held
+    assert O.duo_slots(T, S, W, n_r, L * H - n_r) == int(f["derived_duo_slots"])
+    assert L * H * T == int(f["derived_dense_slots"])
+
+
+def test_worked_positions_tiny_config():
+    # S=16, W=64 after 513 and 528 appends (repository-derived worked values;
+    # cross-checked against the list simulation above)
+    pos = O.ring_positions(513, 16, 64)
+    assert list(pos[:16]) == list(range(16))
+    assert (pos[16], pos[64], pos[65], pos[79]) == (464, 512, 449, 463)
+    pos = O.ring_positions(528, 16, 64)
+    assert [pos[16 + k] for k in range(16)] == [464 + k for k in range(16)]
+    pos = O.ring_positions(50, 16, 64)
+    assert list(pos[:50]) == list(range(50)) and all(p == -1 for p in pos[50:])
+    pos = O.ring_positions(32769, 64, 256)
+    assert (pos[64], pos[256], pos[257]) == (32576, 32768, 32513)
+
+
+# ------------------------------------------------------------------ attention
+def _rand(rng, *shape):
+    x = torch.from_numpy(rng.standard_normal(shape).astype(np.float32)).to(torch.bfloat16)
+    return x.double().numpy()
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_brute_force_matches_vectorised(seed):
+    rng = np.random.default_rng(100 + seed)
+    d, T = 8, 23
+    q, k, v = _rand(rng, d), _rand(rng, T, d), _rand(rng, T, d)
+    keys = sorted(rng.choice(T, size=9, replace=False).tolist())
+    scale = float(rng.uniform(0.1, 1.0))
+    o_ref, lse_ref = O.brute_force_attention(q, k, v, keys, scale)
+    o, lse = O.attend(q, k[keys], v[keys], scale)
+    np.testing.assert_allclose(o, o_ref, rtol=1e-13, atol=1e-13)
+    assert lse == pytest.approx(lse_ref, rel=1e-13)
+
+
+def test_weights_sum_to_one_and_closed_forms():
+    rng = np.random.default_rng(7)
+    d = 16
+    q, k, v = _rand(rng, d), _rand(rng, 40, d), _rand(rng, 40, d)
+    _, lse = O.attend(q, k, v, 0.25)
+    assert np.exp(0.25 * (k @ q) - lse).sum() == pytest.approx(1.0, abs=1e-12)
+    # one key: the output is that key's value
+    o, _ = O.attend(q, k[:1], v[:1], 0.25)
+    np.testing.assert_allclose(o, v[0], rtol=0, atol=1e-15)
+    # identical keys: the plain mean of the values
+    o, _ = O.attend(q, np.repeat(k[:1], 7, 0), v[:7], 0.25)
+    np.testing.assert_allclose(o, v[:7].mean(0), rtol=1e-13, atol=1e-14)
+    # two keys: logistic weights
+    o, _ = O.attend(q, k[:2], v[:2], 0.5)
+    s0, s1 = 0.5 * q @ k[0], 0.5 * q @ k[1]
+    w0 = 1.0 / (1.0 + math.exp(s1 - s0))
+    np.testing.assert_allclose(o, w0 * v[0] + (1 - w0) * v[1], rtol=1e-13, atol=1e-14)
+
+
+def _hist(rng, B, n_kv, T, d):
+    return _rand(rng, B, n_kv, T, d), _rand(rng, B, n_kv, T, d)
+
+
+def _sdpa(q, k, v, mask, scale):
+    """torch fp64 scaled_dot_product_attention, one query row set."""
+    q = torch.from_numpy(q)[None, None]
+    k = torch.from_numpy(k)[None, None]
+    v = torch.from_numpy(v)[None, None]
+    m = torch.from_numpy(mask)[None, None]
+    return torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=m, scale=scale)[0, 0].numpy()
+
+
+@pytest.mark.parametrize("S,W,T", [(4, 8, 30), (0, 5, 17), (3, 1, 9), (16, 64, 513), (2, 40, 20)])
+def test_decode_matches_sdpa_with_ring_contents(S, W, T):
+    """Streaming heads: attention over exactly what a literal ring simulation
+    holds after T appends, computed by torch's SDPA.  Retrieval heads: SDPA
+    with every key."""
+    rng = np.random.default_rng(S * 1000 + W * 10 + T)
+    B, hq, n_kv, d = 2, 4, 2, 16
+    K, V = _hist(rng, B, n_kv, T, d)
+    q = _rand(rng, B, hq, d)
+    mask = np.array([1, 0], dtype=np.uint8)
+    lens = np.array([T, T])
+    out, lse = O.decode_attention(q, lambda b, g: K[b, g], lambda b, g: V[b, g], lens, mask, S, W, 0.3)
+    held = np.zeros(T, dtype=bool)
+    held[[p for p in O.ring_positions(T, S, W) if p >= 0]] = True
+    for b in range(B):
+        for h in range(hq):
+            g = h // (hq // n_kv)
+            m = np.ones(T, dtype=bool) if mask[g] else held
+            want = _sdpa(q[b, h][None], K[b, g], V[b, g], m[None], 0.3)[0]
+            np.testing.assert_allclose(out[b, h], want, rtol=1e-12, atol=1e-12)
+
+
+def test_streaming_equals_full_when_window_covers_context():
+    rng = np.random.default_rng(3)
+    B, hq, n_kv, d, T = 1, 4, 4, 8, 50
+    K, V = _hist(rng, B, n_kv, T, d)
+    q = _rand(rng, B, hq, d)
+    kh, vh = (lambda b, g: K[b, g]), (lambda b, g: V[b, g])
+    full, _ = O.decode_attention(q, kh, vh, [T], np.ones(4, np.uint8), 10, 40, 0.35)
+    for S, W in [(10, 40), (0, 50), (50, 1), (20, 200)]:
+        strm, _ = O.decode_attention(q, kh, vh, [T], np.zeros(4, np.uint8), S, W, 0.35)
+        np.testing.assert_allclose(strm, full, rtol=1e-14, atol=1e-14)
+    # one token short of covering: differs
+    strm, _ = O.decode_attention(q, kh, vh, [T], np.zeros(4, np.uint8), 10, 39, 0.35)
+    assert np.abs(strm - full).max() > 1e-6
+
+
+def test_gqa_equals_mha_with_repeated_kv():
+    """GQA with n_kv heads == MHA on K/V repeated with repeat_interleave
+    ("Attention Variants and Memory Efficiency", repeat_kv)."""
+    rng = np.random.default_rng(11)
+    B, hq, n_kv, d, T = 2, 8, 2, 16, 40
+    K, V = _hist(rng, B, n_kv, T, d)
+    q = _rand(rng, B, hq, d)
+    mask = np.array([0, 1], np.uint8)
+    Kr = torch.from_numpy(K).repeat_interleave(hq // n_kv, dim=1).numpy()
+    Vr = torch.from_numpy(V).repeat_interleave(hq // n_kv, dim=1).numpy()
+    mask_r = np.repeat(mask, hq // n_kv)
+    lens = np.array([T, T - 7])
+    a, la = O.decode_attention(q, lambda b, g: K[b, g, :lens[b]], lambda b, g: V[b, g, :lens[b]],
+                               lens, mask, 3, 6, 0.25)
+    m, lm = O.decode_attention(q, lambda b, g: Kr[b, g, :lens[b]], lambda b, g: Vr[b, g, :lens[b]],
+                               lens, mask_r, 3, 6, 0.25)
+    np.testing.assert_allclose(a, m, rtol=1e-14, atol=1e-14)
+    np.testing.assert_allclose(la, lm, rtol=1e-14)
+
+
+# ------------------------------------------------------------------ prefill
+def _prefill_case(seed, T=96, d=16, hq=4, n_kv=2):
+    rng = np.random.default_rng(seed)
+    K, V = _hist(rng, 1, n_kv, T, d)
+    Q = _rand(rng, 1, hq, T, d)
+    return K, V, Q
+
+
+def test_prefill_retrieval_rows_equal_causal_sdpa():
+    """Chunk rows after a cached prefix P equal rows P.. of one-shot causal
+    attention over the whole sequence (torch SDPA, is_causal) -- the
+    offset-causal rule of "When Is Reuse Exact?"."""
+    K, V, Q = _prefill_case(1)
+    T, P, C = 96, 40, 56
+    mask = np.array([1, 1], np.uint8)
+    out = O.prefill_attention(Q[:, :, P:P + C], lambda b, g: K[b, g], lambda b, g: V[b, g],
+                              [P], mask, 4, 8, 0.25)
+    for h in range(4):
+        g = h // 2
+        full = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(Q[0, h])[None], torch.from_numpy(K[0, g])[None],
+            torch.from_numpy(V[0, g])[None], is_causal=True, scale=0.25)[0].numpy()
+        np.testing.assert_allclose(out[0, h], full[P:P + C], rtol=1e-12, atol=1e-12)
+    # the naive upper-left C x (P+C) triangle hides cached keys and gives other rows
+    naive = np.tril(np.ones((C, P + C), dtype=bool))
+    got_naive = _sdpa(Q[0, 0, P:P + C], K[0, 0], V[0, 0], naive, 0.25)
+    assert np.abs(got_naive - out[0, 0]).max() > 1e-3
+
+
+def test_prefill_streaming_rows_equal_ring_contents():
+    """Each streaming row reads exactly what a ring holds right after its own
+    token was appended (literal simulation, then torch SDPA)."""
+    K, V, Q = _prefill_case(2)
+    T, P, C, S, W = 96, 30, 66, 5, 12
+    mask = np.array([0, 0], np.uint8)
+    out = O.prefill_attention(Q[:, :, P:P + C], lambda b, g: K[b, g], lambda b, g: V[b, g],
+                              [P], mask, S, W, 0.3)
+    ring = O.StreamingCache(S, W)
+    rows = []
+    for p in range(T):
+        ring.append(p)
+        if p >= P:
+            m = np.zeros(T, dtype=bool)
+            m[[x for x in ring.pos if x >= 0]] = True
+            rows.append(m)
+    rows = np.stack(rows)
+    for h in range(4):
+        want = _sdpa(Q[0, h, P:P + C], K[0, h // 2], V[0, h // 2], rows, 0.3)
+        np.testing.assert_allclose(out[0, h], want, rtol=1e-12, atol=1e-12)
+
+
+def test_chunked_equals_one_shot_and_last_row_equals_decode():
+    K, V, Q = _prefill_case(3)
+    T = 96
+    mask = np.array([1, 0], np.uint8)
+    kh, vh = (lambda b, g: K[b, g]), (lambda b, g: V[b, g])
+    one = O.prefill_attention(Q, kh, vh, [0], mask, 4, 10, 0.25)
+    parts = []
+    for P, C in [(0, 32), (32, 40), (72, 24)]:
+        parts.append(O.prefill_attention(Q[:, :, P:P + C], kh, vh, [P], mask, 4, 10, 0.25))
+    np.testing.assert_allclose(np.concatenate(parts, axis=2), one, rtol=1e-13, atol=1e-13)
+    dec, _ = O.decode_attention(Q[:, :, T - 1], kh, vh, [T], mask, 4, 10, 0.25)
+    np.testing.assert_allclose(one[:, :, T - 1], dec, rtol=1e-13, atol=1e-13)
+    # sampled rows equal the full evaluation
+    some = O.prefill_attention(Q, kh, vh, [0], mask, 4, 10, 0.25, rows=[0, 5, 95])
+    np.testing.assert_allclose(some[:, :, [0, 5, 95]], one[:, :, [0, 5, 95]], rtol=0, atol=0)
+
+
+# ------------------------------------------------------------------ planted mistakes
+def _fails(fn, *a, **kw):
+    try:
+        fn(*a, **kw)
+    except AssertionError:
+        return True
+    return False
+
+
+def test_planted_window_off_by_one_is_caught(monkeypatch):
+    def bad_keep(t, sink, window):
+        j = np.arange(t + 1)
+        return j[(j < sink) | (j >= t - window)]
+    monkeypatch.setattr(O, "keep_set", bad_keep)
+    assert _fails(test_ring_matches_list_simulation, 0)
+    assert _fails(test_decode_matches_sdpa_with_ring_contents, 4, 8, 30)
+
+
+def test_planted_ring_slot_error_is_caught(monkeypatch):
+    orig = O.StreamingCache.append
+
+    def bad_append(self, position, item=None):
+        if self.n_sink < self.sink:
+            return orig(self, position, item)
+        slot = self.sink + (position % self.window)   # forgets to count from the sinks
+        self.n_window += 1
+        self.pos[slot] = position
+        self.items[slot] = item
+        return slot
+    monkeypatch.setattr(O.StreamingCache, "append", bad_append)
+    assert _fails(test_worked_positions_tiny_config)
+    monkeypatch.setattr(O.StreamingCache, "append", orig)
+
+
+def test_planted_gqa_mapping_error_is_caught(monkeypatch):
+    monkeypatch.setattr(O, "kv_head_of", lambda h, hq, n_kv: h % n_kv)
+    assert _fails(test_gqa_equals_mha_with_repeated_kv)
+
+
+def test_planted_causal_offset_error_is_caught(monkeypatch):
+    orig = O.key_mask
+
+    def upper_left(rows_t, n_keys, retrieval, sink, window):
+        t = np.asarray(rows_t)
+        return orig(t - t.min(), n_keys, retrieval, sink, window)
+    monkeypatch.setattr(O, "key_mask", upper_left)
+    assert _fails(test_prefill_retrieval_rows_equal_causal_sdpa)
+
+
+def test_planted_missing_scale_is_caught(monkeypatch):
+    orig = O.attend
+    monkeypatch.setattr(O, "attend", lambda q, k, v, scale: orig(q, k, v, 1.0))
+    assert _fails(test_decode_matches_sdpa_with_ring_contents, 4, 8, 30)
+
+
+def test_planted_size_factor_error_is_caught(monkeypatch):
+    monkeypatch.setattr(O, "kv_cache_bytes", lambda L, n, d, T, elem_bytes=2: elem_bytes * L * n * d * T)
+    assert _fails(test_dense_sizes_match_printed_values)
