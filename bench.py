@@ -1,0 +1,441 @@
+"""Benchmark: mixed-head decode attention, one layer-step = KV append of the
+new token + decode attention for every sequence and query head, on the
+GQA 128K workload (Llama-3-8B attention shape: 32 query / 8 KV heads,
+d=128, batch 8 with ragged lengths U[16K, 128K], 4 of 8 KV heads retrieval,
+sink 64 + window 256, 32 distinct decode steps cycled).
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+Prints one JSON line (rank 0).  Multi-GPU: one process per GPU (torchrun),
+each rank decodes its own 8 sequences of a global batch of 8N (weak scaling,
+no collective on the data path); timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import duo_workloads as W  # noqa: E402
+
+METRIC = "mixed-head decode attn: µs/layer-step, achieved HBM GB/s (% of B200 peak)"
+WORKLOAD = "gqa128k"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ---------------------------------------------------------------- helpers
+def kv_bytes(lens_after, mask, d, S, Wn, cap):
+    """Algorithmic KV bytes of one layer-step: full K and V rows of every
+    retrieval head, the min(T, S+W) filled ring slots of every streaming head."""
+    n_r = int(mask.sum())
+    n_s = len(mask) - n_r
+    tot = 0
+    for T in lens_after:
+        tot += n_r * 4 * d * min(int(T), cap) + n_s * 4 * d * min(int(T), S + Wn)
+    return tot
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits", "-lms", "50",
+                 "-i", str(self.index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.15)
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            out, _ = self.proc.communicate(timeout=10)
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx or None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def max_over_ranks(x: float, world: int, dev) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def rank_workload(rank: int, world: int):
+    """Rank r decodes sequences 8r .. 8r+7 of a global batch of 8 * world."""
+    base = W.WORKLOADS[WORKLOAD]
+    g = W.scaled(base, batch=base.batch * world)
+    lens = W.context_lengths(g)[rank * base.batch:(rank + 1) * base.batch]
+    return base, g, lens
+
+
+# ---------------------------------------------------------------- our arm
+def fill_rank(cache, gw, lens0, first_b, dev, slab=16384):
+    """Bulk-append the seeded history of this rank's sequences."""
+    B = len(lens0)
+    top = int(lens0.max())
+    for p0 in range(0, top, slab):
+        n = min(slab, top - p0)
+        k = torch.zeros(B, gw.n_kv, n, gw.d, dtype=torch.bfloat16)
+        v = torch.zeros_like(k)
+        cnt = np.clip(lens0 - p0, 0, n).astype(np.int32)
+        for b in range(B):
+            c = int(cnt[b])
+            for g in range(gw.n_kv):
+                if c:
+                    k[b, g, :c] = W.tokens(gw, 0, first_b + b, g, W.TENSOR_K, p0, p0 + c)
+                    v[b, g, :c] = W.tokens(gw, 0, first_b + b, g, W.TENSOR_V, p0, p0 + c)
+        cache.append(0, k.to(dev), v.to(dev), torch.from_numpy(np.minimum(lens0, p0).astype(np.int32)).to(dev),
+                     torch.from_numpy(cnt).to(dev))
+
+
+def step_inputs(gw, lens0, first_b, steps):
+    """Per decode step s: q [B][Hq][d], k/v [B][n_kv][1][d] (CPU bf16)."""
+    B = len(lens0)
+    q = torch.empty(steps, B, gw.hq, gw.d, dtype=torch.bfloat16)
+    k = torch.empty(steps, B, gw.n_kv, 1, gw.d, dtype=torch.bfloat16)
+    v = torch.empty_like(k)
+    for b in range(B):
+        p = int(lens0[b])
+        for h in range(gw.hq):
+            q[:, b, h] = W.tokens(gw, 0, first_b + b, h, W.TENSOR_Q, p, p + steps)
+        for g in range(gw.n_kv):
+            k[:, b, g, 0] = W.tokens(gw, 0, first_b + b, g, W.TENSOR_K, p, p + steps)
+            v[:, b, g, 0] = W.tokens(gw, 0, first_b + b, g, W.TENSOR_V, p, p + steps)
+    return ([q[s].contiguous() for s in range(steps)], [k[s].contiguous() for s in range(steps)],
+            [v[s].contiguous() for s in range(steps)])
+
+
+def run_ours(args, rank, world, local):
+    from head_wise_kv_b200 import DuoKVCache
+    from head_wise_kv_b200 import _lib as L
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    base, gw, lens0 = rank_workload(rank, world)
+    first_b = rank * base.batch
+    mask = W.retrieval_mask(gw, 0)
+    steps = base.steps
+    cap = int(lens0.max()) + steps
+    B = base.batch
+    cache = DuoKVCache(1, B, base.hq, base.n_kv, base.d, base.sink, base.window, cap, mask[None], device=dev)
+    fill_rank(cache, gw, lens0, first_b, dev)
+    qs, ks, vs = step_inputs(gw, lens0, first_b, steps)
+    dq = [q.to(dev) for q in qs]
+    dk = [k.to(dev) for k in ks]
+    dv = [v.to(dev) for v in vs]
+    lb = [torch.from_numpy((lens0 + s).astype(np.int32)).to(dev) for s in range(steps)]
+    la = [torch.from_numpy((lens0 + s + 1).astype(np.int32)).to(dev) for s in range(steps)]
+    out = torch.empty(B, base.hq, base.d, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    scale = base.scale
+
+    def one(i):
+        s = i % steps
+        cache.append(0, dk[s], dv[s], lb[s])
+        cache.decode(0, dq[s], la[s], scale, out=out)
+
+    for i in range(args.warmup):
+        one(i)
+    torch.cuda.synchronize()
+    assert cache.status() == 0, "device status set during warm-up"
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(K):
+            s = i % steps
+            ev[i][0].record(stream)
+            cache.append(0, dk[s], dv[s], lb[s])
+            ev[i][1].record(stream)
+            cache.decode(0, dq[s], la[s], scale, out=out)
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    total_ms = ev[0][0].elapsed_time(ev[-1][2])
+    dec_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+    app_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
+    assert cache.status() == 0, "device status set during the timed region"
+    total_ms = max_over_ranks(total_ms, world, dev)
+    us_per_step = total_ms * 1e3 / K
+
+    # algorithmic bytes of the decode launch, averaged over the steps timed
+    bytes_steps = [kv_bytes(lens0 + (i % steps) + 1, mask, base.d, base.sink, base.window, cap) for i in range(K)]
+    avg_bytes = sum(bytes_steps) / K
+    dec_avg_ms = sum(dec_ms) / K
+    hbm_peak, peak_kind = peaks()
+    achieved = avg_bytes / (dec_avg_ms * 1e-3) / 1e9
+    step_gbs = avg_bytes / (us_per_step * 1e-6) / 1e9
+
+    # ---------------- e2e: host buffers in, host result out, copies timed
+    pin_q = [q.pin_memory() for q in qs]
+    pin_k = [k.pin_memory() for k in ks]
+    pin_v = [v.pin_memory() for v in vs]
+    pin_lb = [x.cpu().pin_memory() for x in lb]
+    pin_la = [x.cpu().pin_memory() for x in la]
+    host_out = torch.empty(B, base.hq, base.d, dtype=torch.float32).pin_memory()
+    dq_e = torch.empty_like(dq[0])
+    dk_e = torch.empty_like(dk[0])
+    dv_e = torch.empty_like(dv[0])
+    dlb = torch.empty_like(lb[0])
+    dla = torch.empty_like(la[0])
+
+    def e2e_step(i):
+        s = i % steps
+        dq_e.copy_(pin_q[s], non_blocking=True)
+        dk_e.copy_(pin_k[s], non_blocking=True)
+        dv_e.copy_(pin_v[s], non_blocking=True)
+        dlb.copy_(pin_lb[s], non_blocking=True)
+        dla.copy_(pin_la[s], non_blocking=True)
+        cache.append(0, dk_e, dv_e, dlb)
+        cache.decode(0, dq_e, dla, scale, out=out)
+        host_out.copy_(out, non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(K):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    h2d = (dq_e.numel() + dk_e.numel() + dv_e.numel()) * 2 + (dlb.numel() + dla.numel()) * 4
+    d2h = host_out.numel() * 4
+
+    res = {
+        "metric": METRIC,
+        "value": round(us_per_step, 3),
+        "unit": "us/layer-step",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / K, 6),
+        "higher_is_better": False,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": "gqa128k: GQA 32q/8kv d=128, B=8/GPU ragged T~U[16384,131072], 4/8 KV heads "
+                        "retrieval, S=64 W=256, append+decode per layer-step, 32 distinct steps cycled",
+            "global_batch": B * world,
+            "seq_len": [int(x) for x in lens0],
+            "kv_bytes_per_layer_step": int(avg_bytes),
+            "l2": "not flushed: the KV read per step (~1.2 GB) is larger than L2 (126 MB)",
+            "parallelism": f"replicas/dp{world} (independent sequences per GPU)",
+        },
+        "hbm_gbs_step": round(step_gbs * world, 1),
+        "append_us": round(1e3 * sum(app_ms) / K, 3),
+        "decode_us": round(1e3 * dec_avg_ms, 3),
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "decode (split-K attention + LSE merge launch pair)",
+            "achieved": round(achieved, 1),
+            "peak": hbm_peak,
+            "peak_kind": peak_kind,
+            "unit": "GB/s",
+            "frac": round(achieved / hbm_peak, 4),
+            "traffic": None,
+        },
+        "e2e": {"value": round(e2e_ms * 1e3 / K, 3), "unit": "us/layer-step",
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": 3 * K,
+        "clocks": clk.summary(),
+    }
+    cache.close()
+    return res, (gw, lens0, mask, first_b)
+
+
+# ---------------------------------------------------------------- oracle timing
+def oracle_step_sample(gw, lens0, mask, first_b, seqs):
+    """Time the fp64 oracle on one full layer-step of the given sequences
+    (every query head); returns (seconds, KV bytes covered)."""
+    from oracle import duo_oracle as O
+    secs, nbytes = 0.0, 0
+    base = W.WORKLOADS[WORKLOAD]
+    for b in seqs:
+        T = int(lens0[b]) + 1
+        hist_k = {g: W.tokens(gw, 0, first_b + b, g, W.TENSOR_K, 0, T).float().numpy() for g in range(gw.n_kv)}
+        hist_v = {g: W.tokens(gw, 0, first_b + b, g, W.TENSOR_V, 0, T).float().numpy() for g in range(gw.n_kv)}
+        q = torch.stack([W.tokens(gw, 0, first_b + b, h, W.TENSOR_Q, T - 1, T)[0] for h in range(gw.hq)])
+        t0 = time.perf_counter()
+        O.decode_attention(q[None].double().numpy(), lambda _b, g: hist_k[g], lambda _b, g: hist_v[g], [T], mask,
+                           gw.sink, gw.window, gw.scale)
+        secs += time.perf_counter() - t0
+        nbytes += kv_bytes([T], mask, base.d, base.sink, base.window, 1 << 40)
+    return secs, nbytes
+
+
+def cpu_baseline(ctx):
+    gw, lens0, mask, first_b = ctx
+    cores = len(os.sched_getaffinity(0))
+    secs, nbytes = oracle_step_sample(gw, lens0, mask, first_b, range(len(lens0)))
+    total = kv_bytes(lens0 + 1, mask, gw.d, gw.sink, gw.window, 1 << 40)
+    return {"value": round(secs * 1e6 * total / nbytes, 1), "unit": "us/layer-step", "cores": cores,
+            "kind": "oracle",
+            "sample": f"numpy fp64 oracle on one full layer-step (all {len(lens0)} sequences, all 32 query "
+                      f"heads, first decode step), {secs:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm: each step times the oracle's decode of
+    the 4 query heads of one retrieval KV head over a 4,096-token prefix of
+    one sequence's cache (cycling sequences and heads) plus one streaming KV
+    head, scaled to a full layer-step by KV bytes."""
+    if rank != 0:
+        return None
+    from oracle import duo_oracle as O
+    base, gw, lens0 = rank_workload(0, 1)
+    mask = W.retrieval_mask(gw, 0)
+    r_heads = [g for g in range(gw.n_kv) if mask[g]]
+    s_heads = [g for g in range(gw.n_kv) if not mask[g]]
+    Tw = 4096
+    samples = []
+    for i in range(min(8, base.batch)):
+        b, g, gs = i % base.batch, r_heads[i % len(r_heads)], s_heads[i % len(s_heads)]
+        T = int(lens0[b]) + 1
+        K = W.tokens(gw, 0, b, g, W.TENSOR_K, 0, Tw).float().numpy()
+        V = W.tokens(gw, 0, b, g, W.TENSOR_V, 0, Tw).float().numpy()
+        keep = O.keep_set(T - 1, gw.sink, gw.window)
+        Ks = W.tokens(gw, 0, b, gs, W.TENSOR_K, 0, T).float().numpy()[keep]
+        Vs = W.tokens(gw, 0, b, gs, W.TENSOR_V, 0, T).float().numpy()[keep]
+        q = torch.stack([W.tokens(gw, 0, b, h, W.TENSOR_Q, T - 1, T)[0] for h in range(gw.hq)]).double().numpy()
+        samples.append((K, V, Ks, Vs, q, g, gs))
+    G = gw.hq // gw.n_kv
+    sample_bytes = 4 * gw.d * (Tw + len(samples[0][2]))
+    total = kv_bytes(lens0 + 1, mask, gw.d, gw.sink, gw.window, 1 << 40)
+
+    def one(i):
+        K, V, Ks, Vs, q, g, gs = samples[i % len(samples)]
+        for h in range(g * G, (g + 1) * G):
+            O.attend(q[h], K, V, gw.scale)
+        for h in range(gs * G, (gs + 1) * G):
+            O.attend(q[h], Ks, Vs, gw.scale)
+
+    for i in range(args.warmup):
+        one(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        one(i)
+    secs = (time.perf_counter() - t0) / args.steps
+    val = secs * 1e6 * total / sample_bytes
+    cores = len(os.sched_getaffinity(0))
+    sample = (f"per step: fp64 oracle decode of one retrieval KV head (4 query heads) over a {Tw}-token "
+              f"prefix plus one streaming KV head, scaled to the full layer-step by KV bytes")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(val, 1), "unit": "us/layer-step",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(val / 1e3, 4),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": "gqa128k (oracle on a bounded sample per step)", "global_batch": base.batch,
+                   "parallelism": "rank 0 only"},
+        "cpu_baseline": {"value": round(val, 1), "unit": "us/layer-step", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(val, 1), "unit": "us/layer-step", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2048)
+    ap.add_argument("--warmup", type=int, default=64)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(args.warmup, 3)
+    rank, world, local = dist_init()
+    try:
+        if args.impl == "reference":
+            res = run_reference(args, rank, world)
+        else:
+            res, ctx = run_ours(args, rank, world, local)
+            if rank == 0 and world == 1 and not args.no_cpu_baseline:
+                res["cpu_baseline"] = cpu_baseline(ctx)
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,142 @@
+"""Torch-facing wrapper of the C ABI: owns the cache buffer and workspace as
+torch tensors and passes their device pointers and the current stream to
+libduo_kv.  Shape / dtype / device checks and pointer marshalling only --
+every step of the path runs in the library's CUDA kernels."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import _lib as L
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _need(t: torch.Tensor, name: str, dtype, shape, device):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.device != device:
+        raise ValueError(f"{name}: on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+class DuoKVCache:
+    """Mixed-head KV cache for ``num_layers`` layers and ``batch`` sequences.
+
+    retrieval_mask: [num_layers][num_kv_heads] (1 = retrieval KV head).
+    """
+
+    def __init__(self, num_layers, batch, num_q_heads, num_kv_heads, head_dim, sink, window, capacity,
+                 retrieval_mask, device="cuda"):
+        self.device = torch.device(device)
+        if self.device.type != "cuda":
+            raise ValueError("DuoKVCache lives on a CUDA device")
+        if self.device.index is None:
+            self.device = torch.device("cuda", torch.cuda.current_device())
+        mask = np.asarray(retrieval_mask, dtype=np.uint8).reshape(num_layers, num_kv_heads)
+        self.mask = mask.copy()
+        self.L, self.B, self.hq, self.n_kv, self.d = num_layers, batch, num_q_heads, num_kv_heads, head_dim
+        self.S, self.W, self.cap = sink, window, capacity
+        self._desc, self._mask_buf = L.make_desc(num_layers, batch, num_q_heads, num_kv_heads, head_dim,
+                                                 sink, window, capacity, mask.tobytes())
+        self.total_bytes, self.cache_bytes = L.duo_kv_required_bytes(self._desc)
+        with torch.cuda.device(self.device):
+            self.buf = torch.empty(self.total_bytes, dtype=torch.uint8, device=self.device)
+            self.handle = L.duo_kv_alloc(self._desc, self.buf.data_ptr(), self.total_bytes, _stream(self.device))
+        self._ws = None
+        self._alloc_workspace()
+
+    # ------------------------------------------------------------ housekeeping
+    def _alloc_workspace(self):
+        n = L.duo_decode_workspace_bytes(self.handle)
+        self._ws = torch.empty(max(n, 256), dtype=torch.uint8, device=self.device)
+
+    def set_decode_ctas(self, ctas: int):
+        L.duo_kv_set_decode_ctas(self.handle, ctas)
+        self._alloc_workspace()
+
+    def close(self):
+        if getattr(self, "handle", None):
+            L.duo_kv_free(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def status(self, clear: bool = True) -> int:
+        return L.duo_kv_read_status(self.handle, clear, _stream(self.device))
+
+    def layer_views(self, layer: int) -> dict:
+        """Torch views of one layer's cache regions (see duo_kv_layer_view)."""
+        v = L.duo_kv_layer_view_get(self.handle, layer)
+        base = self.buf.data_ptr()
+        B, d, SW, cap = self.B, self.d, self.S + self.W, self.cap
+
+        def region(ptr, nbytes):
+            off = ptr - base
+            return self.buf[off:off + nbytes]
+        nr, ns = v.n_retrieval, v.n_streaming
+        kr = region(v.k_retrieval, B * nr * cap * d * 2).view(torch.bfloat16).view(B, nr, cap, d)
+        vr = region(v.v_retrieval, B * nr * cap * d * 2).view(torch.bfloat16).view(B, nr, cap, d)
+        ks = region(v.k_streaming, B * ns * SW * d * 2).view(torch.bfloat16).view(B, ns, SW, d)
+        vs = region(v.v_streaming, B * ns * SW * d * 2).view(torch.bfloat16).view(B, ns, SW, d)
+        pos = region(v.positions, B * SW * 4).view(torch.int32).view(B, SW)
+        rank = [v.head_rank[g] for g in range(self.n_kv)]
+        is_r = [bool(v.is_retrieval[g]) for g in range(self.n_kv)]
+        return dict(k_retrieval=kr, v_retrieval=vr, k_streaming=ks, v_streaming=vs, positions=pos,
+                    head_rank=rank, is_retrieval=is_r)
+
+    # ------------------------------------------------------------ the path
+    def append(self, layer: int, k_new, v_new, len_before, n_new=None):
+        """k_new, v_new: bf16 [B][n_kv][n][d]; len_before: int32 [B] (device);
+        n_new: optional int32 [B] per-sequence counts (<= n)."""
+        n = k_new.shape[2]
+        shp = (self.B, self.n_kv, n, self.d)
+        kp = _need(k_new, "k_new", torch.bfloat16, shp, self.device)
+        vp = _need(v_new, "v_new", torch.bfloat16, shp, self.device)
+        lp = _need(len_before, "len_before", torch.int32, (self.B,), self.device)
+        np_ = _need(n_new, "n_new", torch.int32, (self.B,), self.device) if n_new is not None else None
+        L.duo_kv_append(self.handle, layer, kp, vp, lp, np_, n, _stream(self.device))
+
+    def decode(self, layer: int, q, lengths, scale: float, out=None, lse=None, want_lse=False):
+        """q: bf16 [B][Hq][d]; lengths: int32 [B] after this step's append.
+        Returns fp32 out [B][Hq][d] (and lse [B][Hq] if asked)."""
+        qp = _need(q, "q", torch.bfloat16, (self.B, self.hq, self.d), self.device)
+        lp = _need(lengths, "lengths", torch.int32, (self.B,), self.device)
+        if out is None:
+            out = torch.empty(self.B, self.hq, self.d, dtype=torch.float32, device=self.device)
+        op = _need(out, "out", torch.float32, (self.B, self.hq, self.d), self.device)
+        if want_lse and lse is None:
+            lse = torch.empty(self.B, self.hq, dtype=torch.float32, device=self.device)
+        sp = _need(lse, "lse", torch.float32, (self.B, self.hq), self.device) if lse is not None else None
+        L.duo_decode_attn(self.handle, layer, qp, lp, float(scale), op, sp, self._ws.data_ptr(),
+                          self._ws.numel(), _stream(self.device))
+        return (out, lse) if lse is not None else out
+
+    def prefill(self, layer: int, q, k_chunk, v_chunk, prefix_len, scale: float, out=None):
+        """q: bf16 [B][Hq][C][d]; k_chunk, v_chunk: bf16 [B][n_kv][C][d];
+        prefix_len: int32 [B].  Returns fp32 out [B][Hq][C][d]."""
+        C = q.shape[2]
+        qp = _need(q, "q", torch.bfloat16, (self.B, self.hq, C, self.d), self.device)
+        kp = _need(k_chunk, "k_chunk", torch.bfloat16, (self.B, self.n_kv, C, self.d), self.device)
+        vp = _need(v_chunk, "v_chunk", torch.bfloat16, (self.B, self.n_kv, C, self.d), self.device)
+        pp = _need(prefix_len, "prefix_len", torch.int32, (self.B,), self.device)
+        if out is None:
+            out = torch.empty(self.B, self.hq, C, self.d, dtype=torch.float32, device=self.device)
+        op = _need(out, "out", torch.float32, (self.B, self.hq, C, self.d), self.device)
+        n = L.duo_prefill_workspace_bytes(self.handle, C)
+        ws = torch.empty(max(n, 256), dtype=torch.uint8, device=self.device)
+        L.duo_prefill_attn(self.handle, layer, qp, kp, vp, pp, C, float(scale), op, ws.data_ptr(), ws.numel(),
+                           _stream(self.device))
+        return out

@@ -1,0 +1,278 @@
+// Host side of libduo_kv: argument checks, cache layout in the caller's
+// buffer, and kernel launches.  No device allocation, no synchronisation
+// (except duo_kv_read_status).
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <new>
+
+#include "duo_internal.cuh"
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;   // 1 s per pipeline wait
+
+size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int check_desc(const duo_kv_desc* d) {
+    if (!d || !d->retrieval_mask) return DUO_ERR_INVALID_ARG;
+    if (d->num_layers < 1 || d->batch < 1 || d->num_q_heads < 1 || d->num_kv_heads < 1)
+        return DUO_ERR_INVALID_ARG;
+    if (d->num_q_heads % d->num_kv_heads != 0) return DUO_ERR_INVALID_ARG;
+    if (d->sink < 0 || d->window < 1 || d->capacity < 1) return DUO_ERR_INVALID_ARG;
+    if (d->capacity > 0x7fffffffLL) return DUO_ERR_INVALID_ARG;       // positions are int32
+    if (int64_t(d->sink) + d->window > (1 << 20)) return DUO_ERR_INVALID_ARG;
+    if (d->head_dim != 64 && d->head_dim != 128) return DUO_ERR_UNSUPPORTED;
+    const int g = d->num_q_heads / d->num_kv_heads;
+    if (g != 1 && g != 2 && g != 4 && g != 8) return DUO_ERR_UNSUPPORTED;
+    if (d->num_kv_heads > duo::kMaxKvHeads) return DUO_ERR_UNSUPPORTED;
+    if (d->batch > 65536) return DUO_ERR_UNSUPPORTED;
+    return DUO_OK;
+}
+
+// Layout: [status 256 B] then per layer [Kr][Vr][Ks][Vs][pos], each 256-aligned.
+size_t plan_layout(const duo_kv_desc* d, std::vector<duo::LayerLayout>* layers, size_t* cache_bytes) {
+    size_t off = kAlign;   // status word
+    size_t cache = 0;
+    const size_t D = size_t(d->head_dim), B = size_t(d->batch), SW = size_t(d->sink) + d->window;
+    for (int l = 0; l < d->num_layers; ++l) {
+        duo::LayerLayout L;
+        memset(L.rank, 0, sizeof L.rank);
+        memset(L.r_before, 0, sizeof L.r_before);
+        memset(L.is_r, 0, sizeof L.is_r);
+        for (int g = 0; g < d->num_kv_heads; ++g) {
+            const bool r = d->retrieval_mask[size_t(l) * d->num_kv_heads + g] != 0;
+            L.r_before[g] = L.n_r;
+            L.is_r[g] = r;
+            L.rank[g] = r ? L.n_r++ : L.n_s++;
+        }
+        L.r_before[d->num_kv_heads] = L.n_r;
+        const size_t kr = B * L.n_r * size_t(d->capacity) * D * 2;
+        const size_t ks = B * L.n_s * SW * D * 2;
+        L.off_kr = off; off = align_up(off + kr);
+        L.off_vr = off; off = align_up(off + kr);
+        L.off_ks = off; off = align_up(off + ks);
+        L.off_vs = off; off = align_up(off + ks);
+        L.off_pos = off; off = align_up(off + B * SW * 4);
+        cache += 2 * kr + 2 * ks;
+        if (layers) layers->push_back(L);
+    }
+    if (cache_bytes) *cache_bytes = cache;
+    return off;
+}
+
+int cuda_err(cudaError_t e) { return e == cudaSuccess ? DUO_OK : DUO_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int duo_kv_required_bytes(const duo_kv_desc* desc, size_t* total_bytes, size_t* cache_bytes) {
+    const int rc = check_desc(desc);
+    if (rc) return rc;
+    if (!total_bytes) return DUO_ERR_INVALID_ARG;
+    *total_bytes = plan_layout(desc, nullptr, cache_bytes);
+    return DUO_OK;
+}
+
+int duo_kv_alloc(const duo_kv_desc* desc, void* dev_buf, size_t buf_bytes, duo_stream_t stream,
+                 duo_kv** out) {
+    int rc = check_desc(desc);
+    if (rc) return rc;
+    if (!out || !dev_buf) return DUO_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (reinterpret_cast<uintptr_t>(dev_buf) % kAlign) return DUO_ERR_ALIGNMENT;
+    duo_kv* h = new (std::nothrow) duo_kv();
+    if (!h) return DUO_ERR_INVALID_ARG;
+    h->desc = *desc;
+    h->desc.retrieval_mask = nullptr;
+    const size_t need = plan_layout(desc, &h->layers, nullptr);
+    if (buf_bytes < need) {
+        delete h;
+        return DUO_ERR_BUFFER_TOO_SMALL;
+    }
+    h->base = static_cast<char*>(dev_buf);
+    h->bytes = need;
+    h->status = reinterpret_cast<int32_t*>(h->base);
+    if (cudaGetDevice(&h->device) != cudaSuccess ||
+        cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess) {
+        delete h;
+        return DUO_ERR_CUDA;
+    }
+    cudaError_t e = cudaMemsetAsync(h->status, 0, kAlign, stream);
+    const size_t SW = size_t(desc->sink) + desc->window;
+    for (size_t l = 0; l < h->layers.size() && e == cudaSuccess; ++l)
+        e = cudaMemsetAsync(h->base + h->layers[l].off_pos, 0xff, size_t(desc->batch) * SW * 4, stream);
+    if (e != cudaSuccess) {
+        delete h;
+        return DUO_ERR_CUDA;
+    }
+    *out = h;
+    return DUO_OK;
+}
+
+int duo_kv_free(duo_kv* kv) {
+    delete kv;
+    return DUO_OK;
+}
+
+int duo_kv_layer_view_get(const duo_kv* kv, int32_t layer, duo_kv_layer_view* out) {
+    if (!kv || !out || layer < 0 || layer >= kv->desc.num_layers) return DUO_ERR_INVALID_ARG;
+    const duo::LayerLayout& L = kv->layers[layer];
+    memset(out, 0, sizeof *out);
+    out->k_retrieval = reinterpret_cast<uint16_t*>(kv->base + L.off_kr);
+    out->v_retrieval = reinterpret_cast<uint16_t*>(kv->base + L.off_vr);
+    out->k_streaming = reinterpret_cast<uint16_t*>(kv->base + L.off_ks);
+    out->v_streaming = reinterpret_cast<uint16_t*>(kv->base + L.off_vs);
+    out->positions = reinterpret_cast<int32_t*>(kv->base + L.off_pos);
+    out->n_retrieval = L.n_r;
+    out->n_streaming = L.n_s;
+    for (int g = 0; g < kv->desc.num_kv_heads; ++g) {
+        out->head_rank[g] = L.rank[g];
+        out->is_retrieval[g] = L.is_r[g];
+    }
+    return DUO_OK;
+}
+
+int duo_kv_append(duo_kv* kv, int32_t layer, const uint16_t* k_new, const uint16_t* v_new,
+                  const int32_t* len_before, const int32_t* n_new, int32_t n_new_max,
+                  duo_stream_t stream) {
+    if (!kv || layer < 0 || layer >= kv->desc.num_layers || n_new_max < 0) return DUO_ERR_INVALID_ARG;
+    if (n_new_max == 0) return DUO_OK;
+    if (!k_new || !v_new || !len_before) return DUO_ERR_INVALID_ARG;
+    if (!aligned16(k_new) || !aligned16(v_new) || (reinterpret_cast<uintptr_t>(len_before) & 3) ||
+        (reinterpret_cast<uintptr_t>(n_new) & 3))
+        return DUO_ERR_ALIGNMENT;
+    const duo::LayerLayout& L = kv->layers[layer];
+    duo::AppendParams p;
+    p.k_new = k_new;
+    p.v_new = v_new;
+    p.len_before = len_before;
+    p.n_new = n_new;
+    p.kr = reinterpret_cast<uint16_t*>(kv->base + L.off_kr);
+    p.vr = reinterpret_cast<uint16_t*>(kv->base + L.off_vr);
+    p.ks = reinterpret_cast<uint16_t*>(kv->base + L.off_ks);
+    p.vs = reinterpret_cast<uint16_t*>(kv->base + L.off_vs);
+    p.pos = reinterpret_cast<int32_t*>(kv->base + L.off_pos);
+    p.status = kv->status;
+    p.cap = kv->desc.capacity;
+    p.B = kv->desc.batch;
+    p.n_kv = kv->desc.num_kv_heads;
+    p.n_r = L.n_r;
+    p.n_s = L.n_s;
+    p.S = kv->desc.sink;
+    p.W = kv->desc.window;
+    p.d = kv->desc.head_dim;
+    p.n_new_max = n_new_max;
+    memcpy(p.rank, L.rank, sizeof p.rank);
+    memcpy(p.is_r, L.is_r, sizeof p.is_r);
+    return cuda_err(duo::launch_append(p, stream));
+}
+
+static int decode_slots(const duo_kv* kv) {
+    const int ctas = kv->decode_ctas > 0 ? kv->decode_ctas
+                                         : duo::decode_ctas_default(kv->num_sms, kv->desc.head_dim,
+                                                                    kv->desc.num_q_heads / kv->desc.num_kv_heads);
+    return kv->desc.batch * kv->desc.num_kv_heads + ctas;
+}
+
+int duo_decode_workspace_bytes(const duo_kv* kv, size_t* bytes) {
+    if (!kv || !bytes) return DUO_ERR_INVALID_ARG;
+    *bytes = duo::decode_workspace_bytes(decode_slots(kv), kv->desc.head_dim,
+                                         kv->desc.num_q_heads / kv->desc.num_kv_heads);
+    return DUO_OK;
+}
+
+int duo_decode_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const int32_t* len, float scale,
+                    float* out, float* lse, void* workspace, size_t workspace_bytes,
+                    duo_stream_t stream) {
+    if (!kv || layer < 0 || layer >= kv->desc.num_layers || !q || !len || !out) return DUO_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || scale != scale) return DUO_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(out) || (reinterpret_cast<uintptr_t>(len) & 3) ||
+        (reinterpret_cast<uintptr_t>(lse) & 3))
+        return DUO_ERR_ALIGNMENT;
+    const int G = kv->desc.num_q_heads / kv->desc.num_kv_heads;
+    const int D = kv->desc.head_dim;
+    const int slots = decode_slots(kv);
+    const size_t need = duo::decode_workspace_bytes(slots, D, G);
+    if (!workspace || workspace_bytes < need) return DUO_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return DUO_ERR_ALIGNMENT;
+    const duo::LayerLayout& L = kv->layers[layer];
+    duo::DecodeParams p;
+    p.kr = reinterpret_cast<const uint16_t*>(kv->base + L.off_kr);
+    p.vr = reinterpret_cast<const uint16_t*>(kv->base + L.off_vr);
+    p.ks = reinterpret_cast<const uint16_t*>(kv->base + L.off_ks);
+    p.vs = reinterpret_cast<const uint16_t*>(kv->base + L.off_vs);
+    p.q = q;
+    p.len = len;
+    p.out = out;
+    p.lse = lse;
+    p.ws_o = static_cast<float*>(workspace);
+    p.ws_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                       ((size_t(slots) * G * D * 4 + 255) & ~size_t(255)));
+    p.status = kv->status;
+    p.cap = kv->desc.capacity;
+    p.B = kv->desc.batch;
+    p.n_kv = kv->desc.num_kv_heads;
+    p.hq = kv->desc.num_q_heads;
+    p.n_r = L.n_r;
+    p.n_s = L.n_s;
+    p.S = kv->desc.sink;
+    p.W = kv->desc.window;
+    p.num_ctas = slots - p.B * p.n_kv;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.timeout_ns = kWaitLimitNs;
+    memcpy(p.rank, L.rank, sizeof p.rank);
+    memcpy(p.r_before, L.r_before, sizeof p.r_before);
+    memcpy(p.is_r, L.is_r, sizeof p.is_r);
+    return cuda_err(duo::launch_decode(p, D, G, stream));
+}
+
+int duo_prefill_workspace_bytes(const duo_kv* kv, int32_t chunk, size_t* bytes) {
+    if (!kv || !bytes || chunk < 1) return DUO_ERR_INVALID_ARG;
+    *bytes = 0;
+    return DUO_OK;
+}
+
+int duo_prefill_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const uint16_t* k_chunk,
+                     const uint16_t* v_chunk, const int32_t* prefix_len, int32_t chunk, float scale,
+                     float* out, void* workspace, size_t workspace_bytes, duo_stream_t stream) {
+    if (!kv || layer < 0 || layer >= kv->desc.num_layers || !q || !k_chunk || !v_chunk || !prefix_len ||
+        !out || chunk < 1)
+        return DUO_ERR_INVALID_ARG;
+    (void)scale; (void)workspace; (void)workspace_bytes; (void)stream;
+    return DUO_ERR_UNSUPPORTED;
+}
+
+int duo_kv_read_status(duo_kv* kv, int32_t* status, int32_t clear, duo_stream_t stream) {
+    if (!kv || !status) return DUO_ERR_INVALID_ARG;
+    cudaError_t e = cudaMemcpyAsync(status, kv->status, sizeof(int32_t), cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e == cudaSuccess && clear) e = cudaMemsetAsync(kv->status, 0, sizeof(int32_t), stream);
+    return cuda_err(e);
+}
+
+int duo_kv_set_decode_ctas(duo_kv* kv, int32_t ctas) {
+    if (!kv || ctas < 0 || ctas > (1 << 20)) return DUO_ERR_INVALID_ARG;
+    kv->decode_ctas = ctas;
+    return DUO_OK;
+}
+
+const char* duo_strerror(int code) {
+    switch (code) {
+        case DUO_OK: return "ok";
+        case DUO_ERR_INVALID_ARG: return "invalid argument";
+        case DUO_ERR_UNSUPPORTED: return "unsupported shape (head_dim must be 64 or 128, group 1/2/4/8, <= 64 KV heads)";
+        case DUO_ERR_BUFFER_TOO_SMALL: return "device buffer smaller than duo_kv_required_bytes";
+        case DUO_ERR_WORKSPACE: return "workspace missing or smaller than required";
+        case DUO_ERR_CUDA: return "CUDA runtime error";
+        case DUO_ERR_ALIGNMENT: return "misaligned device pointer";
+    }
+    return "unknown error";
+}
+
+}  // extern "C"

@@ -1,0 +1,104 @@
+// KV append + window eviction for one layer.
+//
+// Retrieval heads store every token at its own row ("Tokens are stored
+// sequentially from step 1 to T", DuoAttention guide, section 2).  Streaming
+// heads keep the first S tokens in the sink slots and the most recent W in a
+// W-slot ring that overwrites its oldest entry (the guide's simulation,
+// append_token; the ring rule of "Attention Variants and Memory Efficiency",
+// "Sliding-Window and Mixed Attention").  A bulk append writes only the
+// tokens that survive the whole append (p < S or p >= T_new - W), so the
+// result equals appending one token at a time and no two threads write the
+// same slot.  The position table keeps each slot's original position ("When
+// Is Reuse Exact?": positions are not renumbered after eviction).
+//
+// One row (d bf16 = 128 or 256 bytes) is moved by d/8 threads with 16-byte
+// loads and stores; a trailing set of work items resets the position table
+// of sequences that start over (len_before == 0).
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "duo_internal.cuh"
+
+namespace duo {
+
+namespace {
+
+constexpr int kThreads = 256;
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) append_kernel(const __grid_constant__ AppendParams p) {
+    constexpr int TPR = D / 8;   // threads per row, 16 bytes each
+    const int64_t rows_total = int64_t(p.B) * p.n_kv * p.n_new_max;
+    const int64_t item = (int64_t(blockIdx.x) * kThreads + threadIdx.x) / TPR;
+    const int part = threadIdx.x % TPR;
+    const int SW = p.S + p.W;
+
+    if (item >= rows_total) {
+        // position-table reset for sequences that start from empty
+        const int64_t r = (item - rows_total) * TPR + part;
+        if (r >= int64_t(p.B) * SW) return;
+        const int b = int(r / SW), slot = int(r % SW);
+        if (p.len_before[b] != 0) return;
+        const int nb = p.n_new ? p.n_new[b] : p.n_new_max;
+        // slots 0 .. min(nb, S+W)-1 are filled by this append; the rest start empty
+        if (slot >= nb) p.pos[size_t(b) * SW + slot] = -1;
+        return;
+    }
+
+    const int i = int(item % p.n_new_max);
+    const int g = int((item / p.n_new_max) % p.n_kv);
+    const int b = int(item / (int64_t(p.n_new_max) * p.n_kv));
+    const int nb = p.n_new ? p.n_new[b] : p.n_new_max;
+    const int lb = p.len_before[b];
+    if (lb < 0 || nb < 0 || nb > p.n_new_max) {
+        if (part == 0 && i == 0 && g == 0) set_status(p.status, DUO_STATUS_BAD_LENGTH);
+        return;
+    }
+    if (i >= nb) return;
+    const int64_t pos = int64_t(lb) + i;
+    const int64_t t_new = int64_t(lb) + nb;
+    const bool survives = pos < p.S || pos >= t_new - p.W;   // still held once all nb are in
+    const int slot = pos < p.S ? int(pos) : p.S + int((pos - p.S) % p.W);
+    // one writer per (sequence, slot) of the position table: KV head 0, first thread of the row
+    if (g == 0 && part == 0 && survives) p.pos[size_t(b) * SW + slot] = int32_t(pos);
+
+    const size_t src = ((size_t(b) * p.n_kv + g) * p.n_new_max + i) * D + part * 8;
+    if (p.is_r[g]) {
+        if (pos >= p.cap) {
+            if (part == 0) set_status(p.status, DUO_STATUS_OVER_CAPACITY);
+            return;
+        }
+        const uint4 kv = *reinterpret_cast<const uint4*>(p.k_new + src);
+        const uint4 vv = *reinterpret_cast<const uint4*>(p.v_new + src);
+        const size_t dst = ((size_t(b) * p.n_r + p.rank[g]) * size_t(p.cap) + pos) * D + part * 8;
+        *reinterpret_cast<uint4*>(p.kr + dst) = kv;
+        *reinterpret_cast<uint4*>(p.vr + dst) = vv;
+    } else if (survives) {
+        const uint4 kv = *reinterpret_cast<const uint4*>(p.k_new + src);
+        const uint4 vv = *reinterpret_cast<const uint4*>(p.v_new + src);
+        const size_t dst = ((size_t(b) * p.n_s + p.rank[g]) * SW + slot) * D + part * 8;
+        *reinterpret_cast<uint4*>(p.ks + dst) = kv;
+        *reinterpret_cast<uint4*>(p.vs + dst) = vv;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_append(const AppendParams& p, cudaStream_t s) {
+    const int tpr = p.d / 8;
+    const int64_t rows = int64_t(p.B) * p.n_kv * p.n_new_max;
+    const int64_t reset_items = (int64_t(p.B) * (p.S + p.W) + tpr - 1) / tpr;
+    const int64_t threads = (rows + reset_items) * tpr;
+    const int64_t blocks = (threads + kThreads - 1) / kThreads;
+    if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
+    if (p.d == 128) {
+        append_kernel<128><<<unsigned(blocks), kThreads, 0, s>>>(p);
+    } else if (p.d == 64) {
+        append_kernel<64><<<unsigned(blocks), kThreads, 0, s>>>(p);
+    } else {
+        return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace duo

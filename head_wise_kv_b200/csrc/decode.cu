@@ -1,0 +1,550 @@
+// Mixed-head decode attention (one new query token per sequence).
+//
+// Retrieval KV heads attend over their full cache, streaming KV heads over
+// their sink + window ring (DuoAttention guide, section 2; decode reads
+// "Coalesced Autoregressive Reads" under "Zero-Gather Hardware Efficiency").
+// Each (sequence b, KV head g) pair is a *segment* of keys: min(len, cap) rows
+// of the retrieval cache, or min(len, S + W) filled slots of the ring (slot
+// order does not matter to a softmax, and once the token is appended the
+// ring holds exactly the sink + window key set of the query).
+//
+// Work split (split-K, load balanced): all segments are laid end to end in
+// units of 16 tokens; a persistent grid of C CTAs takes C equal contiguous
+// ranges of that axis.  A CTA walks its range piece by piece (a piece = the
+// part of one segment inside the range); pieces that cover a whole segment
+// are normalised and written straight to `out`, the others leave an
+// unnormalised partial (o, max, sum) in the workspace, slot = segment + CTA
+// (unique: moving along the axis crosses either a segment or a CTA boundary).
+// A second small kernel merges the partials by log-sum-exp.
+//
+// Inside a CTA: one producer warp streams K and V tiles of 56 rows into a
+// 4-stage shared-memory ring with TMA bulk copies (cp.async.bulk, completion
+// on mbarriers, L2 evict-first); 7 consumer warps compute.  GQA packing: a
+// KV tile is read once from shared memory and feeds all G query heads of the
+// group (the K/V of "Multi-Query and Grouped-Query Attention" reused without
+// copies).  A consumer lane group of LPT lanes owns one token per step; each
+// lane holds D/LPT dims of q (fp32) for all G heads and of the running output.
+// Dot products reduce with xor-shuffles inside the lane group; the softmax
+// is online, in the log2 domain, fp32 throughout.
+#include <cuda_runtime.h>
+#include <math_constants.h>
+#include <stdint.h>
+
+#include "duo_internal.cuh"
+
+namespace duo {
+
+namespace {
+
+// 7 consumer warps + 1 producer warp = 2 warps per SM sub-partition, so each
+// thread may hold up to 255 registers (q and the running output of all G
+// heads stay in registers).  A tile holds exactly two (four for LPT = 16)
+// warp steps of 7 warps x TPW tokens.
+constexpr int kTile = 56;        // rows per pipeline stage
+constexpr int kStages = 4;
+constexpr int kConsumerWarps = 7;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kBlk = 16;         // partition granularity in tokens
+constexpr float kNegBig = -1.0e30f;   // finite "minus infinity" for running maxima
+
+template <int D, int G>
+struct Cfg {
+    static constexpr int LPT = (D == 128 && G == 8) ? 16 : 8;   // lanes per token
+    static constexpr int TPW = 32 / LPT;                         // tokens per warp step
+    static constexpr int NCL = D / 8 / LPT;                      // 16-byte chunks per lane
+    static constexpr int STEPS = kTile / (TPW * kConsumerWarps);
+    static constexpr int ROW_BYTES = D * 2;
+    static constexpr int STAGE_BYTES = kTile * ROW_BYTES;        // one of K or V
+    static constexpr int RED_STRIDE = D + 4;                     // floats; keeps float4 alignment
+    static constexpr int RED_FLOATS = kConsumerWarps * G * RED_STRIDE;
+    static constexpr size_t SMEM = size_t(2) * kStages * STAGE_BYTES + RED_FLOATS * 4 + 1024;
+    static_assert(STEPS * TPW * kConsumerWarps == kTile, "tile must be whole warp steps");
+    static_assert(STAGE_BYTES % 1024 == 0, "stage buffers stay 1024-byte aligned");
+};
+
+__device__ __forceinline__ int blocks_of(int64_t rows) { return int((rows + kBlk - 1) / kBlk); }
+
+__device__ __forceinline__ int64_t rows_r(int len, int64_t cap) {
+    int64_t r = len < 0 ? 0 : len;
+    return r < cap ? r : cap;
+}
+__device__ __forceinline__ int64_t rows_s(int len, int S, int W) {
+    int64_t r = len < 0 ? 0 : len;
+    return r < S + W ? r : S + W;
+}
+
+// Fill bpre[0..B] (shared) with the running count of 16-token blocks per
+// sequence; warp 0 does a chunked shuffle scan.  Caller syncs afterwards.
+__device__ void build_prefix(const DecodeParams& p, int32_t* bpre) {
+    if (threadIdx.x >= 32) return;
+    const int lane = threadIdx.x;
+    int run = 0;
+    if (lane == 0) bpre[0] = 0;
+    for (int base = 0; base < p.B; base += 32) {
+        const int b = base + lane;
+        int c = 0;
+        if (b < p.B) {
+            const int L = p.len[b];
+            c = p.n_r * blocks_of(rows_r(L, p.cap)) + p.n_s * blocks_of(rows_s(L, p.S, p.W));
+        }
+        int x = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (b < p.B) bpre[b + 1] = run + x;
+        run += __shfl_sync(0xffffffffu, x, 31);
+    }
+}
+
+// First block index owned by CTA c when `total` blocks are split over n CTAs.
+__device__ __forceinline__ int64_t cta_start(int64_t c, int64_t total, int64_t n) { return c * total / n; }
+// CTA that owns block gb.
+__device__ __forceinline__ int cta_owner(int64_t gb, int64_t total, int64_t n) {
+    int64_t c = ((gb + 1) * n - 1) / total;
+    return int(c < n - 1 ? c : n - 1);
+}
+
+struct Piece {
+    int b, g, seg;          // sequence, KV head, segment index b * n_kv + g
+    int64_t seg_gb;         // first global block of the segment
+    int seg_nb;             // blocks in the segment
+    int64_t tok0, tok1;     // token rows of this piece inside the segment
+    int64_t end_gb;         // global block after the piece
+    bool whole;             // the piece is the whole segment
+};
+
+// Locate the piece that starts at global block gb (gb < range end).
+__device__ __forceinline__ Piece locate(const DecodeParams& p, const int32_t* bpre, int64_t gb,
+                                        int64_t range_end) {
+    Piece pc;
+    // b = last index with bpre[b] <= gb  (binary search over B + 1 entries)
+    int lo = 0, hi = p.B;   // invariant: bpre[lo] <= gb < bpre[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (bpre[mid] <= gb) lo = mid; else hi = mid;
+    }
+    pc.b = lo;
+    const int L = p.len[lo];
+    const int64_t rr = rows_r(L, p.cap), rs = rows_s(L, p.S, p.W);
+    const int nbr = blocks_of(rr), nbs = blocks_of(rs);
+    const int64_t local = gb - bpre[lo];
+    int g = 0;
+    int64_t start = 0;
+    for (; g < p.n_kv; ++g) {
+        start = int64_t(p.r_before[g]) * nbr + int64_t(g - p.r_before[g]) * nbs;
+        const int nb = p.is_r[g] ? nbr : nbs;
+        if (local < start + nb) break;
+    }
+    pc.g = g;
+    pc.seg = lo * p.n_kv + g;
+    pc.seg_nb = p.is_r[g] ? nbr : nbs;
+    pc.seg_gb = bpre[lo] + start;
+    const int64_t seg_end = pc.seg_gb + pc.seg_nb;
+    pc.end_gb = seg_end < range_end ? seg_end : range_end;
+    const int64_t rows = p.is_r[g] ? rr : rs;
+    pc.tok0 = (gb - pc.seg_gb) * kBlk;
+    const int64_t t1 = (pc.end_gb - pc.seg_gb) * kBlk;
+    pc.tok1 = t1 < rows ? t1 : rows;
+    pc.whole = (gb == pc.seg_gb) && (pc.end_gb == seg_end);
+    return pc;
+}
+
+template <int D>
+__device__ __forceinline__ void seg_ptrs(const DecodeParams& p, int b, int g, const uint16_t*& k,
+                                         const uint16_t*& v) {
+    const int r = p.rank[g];
+    if (p.is_r[g]) {
+        const size_t off = (size_t(b) * p.n_r + r) * size_t(p.cap) * D;
+        k = p.kr + off;
+        v = p.vr + off;
+    } else {
+        const size_t off = (size_t(b) * p.n_s + r) * size_t(p.S + p.W) * D;
+        k = p.ks + off;
+        v = p.vs + off;
+    }
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
+    using C = Cfg<D, G>;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    // 1024-byte aligned carve-up
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    unsigned char* sK = smem;
+    unsigned char* sV = sK + kStages * C::STAGE_BYTES;
+    float* red = reinterpret_cast<float*>(sV + kStages * C::STAGE_BYTES);
+    __shared__ __align__(8) uint64_t full_bar[kStages];
+    __shared__ __align__(8) uint64_t empty_bar[kStages];
+    __shared__ int abort_flag;
+
+    // bpre lives after the reduction buffer; sized B + 1 by the launcher
+    int32_t* bpre = reinterpret_cast<int32_t*>(red + C::RED_FLOATS);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(smem_addr(&full_bar[s]), 1);
+            mbar_init(smem_addr(&empty_bar[s]), kConsumerWarps);
+        }
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    build_prefix(p, bpre);
+    __syncthreads();
+
+    const int64_t total = bpre[p.B];
+    if (total == 0) return;
+    const int64_t n = p.num_ctas;
+    const int64_t gb_begin = cta_start(blockIdx.x, total, n);
+    const int64_t gb_end = cta_start(blockIdx.x + 1, total, n);
+    if (gb_begin >= gb_end) return;
+
+    if (warp == kConsumerWarps) {
+        // ------------------------------------------------------------ producer
+        if (lane != 0) return;
+        const uint64_t policy = l2_evict_first_policy();
+        uint32_t it = 0;
+        bool ok = true;
+        for (int64_t gb = gb_begin; gb < gb_end && ok;) {
+            const Piece pc = locate(p, bpre, gb, gb_end);
+            const uint16_t *kp, *vp;
+            seg_ptrs<D>(p, pc.b, pc.g, kp, vp);
+            for (int64_t t = pc.tok0; t < pc.tok1; t += kTile, ++it) {
+                const int rows = int(pc.tok1 - t < kTile ? pc.tok1 - t : kTile);
+                const int st = it % kStages;
+                const uint32_t ph = (it / kStages) & 1;
+                if (!mbar_wait(smem_addr(&empty_bar[st]), ph ^ 1, p.timeout_ns) ||
+                    *((volatile int*)&abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t bytes = uint32_t(rows) * C::ROW_BYTES;
+                mbar_arrive_expect_tx(smem_addr(&full_bar[st]), 2 * bytes);
+                bulk_g2s(smem_addr(sK + st * C::STAGE_BYTES), kp + t * D, bytes,
+                         smem_addr(&full_bar[st]), policy);
+                bulk_g2s(smem_addr(sV + st * C::STAGE_BYTES), vp + t * D, bytes,
+                         smem_addr(&full_bar[st]), policy);
+            }
+            gb = pc.end_gb;
+        }
+        if (!ok) {
+            set_status(p.status, DUO_STATUS_WAIT_TIMEOUT);
+            atomicExch(&abort_flag, 1);
+        }
+        // Do not leave while copies issued by this CTA may still land in its
+        // shared memory: wait (bounded) for every stage's last issued phase.
+        for (uint32_t k = 0; k < kStages && k < it; ++k) {
+            const uint32_t last = it - 1 - k;
+            mbar_wait(smem_addr(&full_bar[last % kStages]), (last / kStages) & 1, p.timeout_ns);
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------------- consumers
+    const int grp = lane / C::LPT;          // token slot within the warp step
+    const int li = lane % C::LPT;           // lane within the token group
+    uint32_t it = 0;
+    bool aborted = false;
+    const uint32_t sK0 = smem_addr(sK), sV0 = smem_addr(sV);
+
+    for (int64_t gb = gb_begin; gb < gb_end;) {
+        const Piece pc = locate(p, bpre, gb, gb_end);
+        gb = pc.end_gb;
+
+        // q of the G query heads of this KV head, this lane's dims, fp32
+        float2 q2[G][C::NCL * 4];
+        {
+            const uint16_t* qb = p.q + (size_t(pc.b) * p.hq + size_t(pc.g) * G) * D;
+#pragma unroll
+            for (int h = 0; h < G; ++h)
+#pragma unroll
+                for (int k = 0; k < C::NCL; ++k) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(qb + h * D + (li + k * C::LPT) * 8);
+                    q2[h][k * 4 + 0] = bf2_to_f2(v.x);
+                    q2[h][k * 4 + 1] = bf2_to_f2(v.y);
+                    q2[h][k * 4 + 2] = bf2_to_f2(v.z);
+                    q2[h][k * 4 + 3] = bf2_to_f2(v.w);
+                }
+        }
+        float2 o2[G][C::NCL * 4];
+        float m[G], l[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            m[h] = kNegBig;
+            l[h] = 0.f;
+#pragma unroll
+            for (int j = 0; j < C::NCL * 4; ++j) o2[h][j] = make_float2(0.f, 0.f);
+        }
+
+        for (int64_t t = pc.tok0; t < pc.tok1 && !aborted; t += kTile, ++it) {
+            const int rows = int(pc.tok1 - t < kTile ? pc.tok1 - t : kTile);
+            const int st = it % kStages;
+            const uint32_t ph = (it / kStages) & 1;
+            if (*((volatile int*)&abort_flag)) {
+                aborted = true;
+                break;
+            }
+            if (!mbar_wait(smem_addr(&full_bar[st]), ph, p.timeout_ns)) {
+                // Stop consuming; keep taking part in the named barriers below so
+                // that no warp of this CTA waits on one forever.
+                set_status(p.status, DUO_STATUS_WAIT_TIMEOUT);
+                atomicExch(&abort_flag, 1);
+                aborted = true;
+                break;
+            }
+            const uint32_t kbase = sK0 + st * C::STAGE_BYTES;
+            const uint32_t vbase = sV0 + st * C::STAGE_BYTES;
+
+            float sc[C::STEPS][G];
+#pragma unroll
+            for (int s = 0; s < C::STEPS; ++s) {
+                const int row = (s * kConsumerWarps + warp) * C::TPW + grp;
+                float2 acc[G];
+#pragma unroll
+                for (int h = 0; h < G; ++h) acc[h] = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int k = 0; k < C::NCL; ++k) {
+                    const uint4 kv = lds128(kbase + row * C::ROW_BYTES + (li + k * C::LPT) * 16);
+                    const float2 k0 = bf2_to_f2(kv.x), k1 = bf2_to_f2(kv.y);
+                    const float2 k2 = bf2_to_f2(kv.z), k3 = bf2_to_f2(kv.w);
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        acc[h] = ffma2(q2[h][k * 4 + 0], k0, acc[h]);
+                        acc[h] = ffma2(q2[h][k * 4 + 1], k1, acc[h]);
+                        acc[h] = ffma2(q2[h][k * 4 + 2], k2, acc[h]);
+                        acc[h] = ffma2(q2[h][k * 4 + 3], k3, acc[h]);
+                    }
+                }
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    float x = acc[h].x + acc[h].y;
+#pragma unroll
+                    for (int o = 1; o < C::LPT; o <<= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+                    sc[s][h] = row < rows ? x * p.scale_log2 : -CUDART_INF_F;
+                }
+            }
+            // online softmax: one rescale per tile
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                float mt = sc[0][h];
+#pragma unroll
+                for (int s = 1; s < C::STEPS; ++s) mt = fmaxf(mt, sc[s][h]);
+                if (mt > m[h]) {
+                    const float a = fast_exp2(m[h] - mt);
+                    m[h] = mt;
+                    l[h] *= a;
+                    const float2 a2 = make_float2(a, a);
+#pragma unroll
+                    for (int j = 0; j < C::NCL * 4; ++j) o2[h][j] = fmul2(o2[h][j], a2);
+                }
+#pragma unroll
+                for (int s = 0; s < C::STEPS; ++s) {
+                    sc[s][h] = fast_exp2(sc[s][h] - m[h]);
+                    l[h] += sc[s][h];
+                }
+            }
+#pragma unroll
+            for (int s = 0; s < C::STEPS; ++s) {
+                const int row = (s * kConsumerWarps + warp) * C::TPW + grp;
+                if (row < rows) {
+#pragma unroll
+                    for (int k = 0; k < C::NCL; ++k) {
+                        const uint4 vv = lds128(vbase + row * C::ROW_BYTES + (li + k * C::LPT) * 16);
+                        const float2 v0 = bf2_to_f2(vv.x), v1 = bf2_to_f2(vv.y);
+                        const float2 v2 = bf2_to_f2(vv.z), v3 = bf2_to_f2(vv.w);
+#pragma unroll
+                        for (int h = 0; h < G; ++h) {
+                            const float2 pp = make_float2(sc[s][h], sc[s][h]);
+                            o2[h][k * 4 + 0] = ffma2(pp, v0, o2[h][k * 4 + 0]);
+                            o2[h][k * 4 + 1] = ffma2(pp, v1, o2[h][k * 4 + 1]);
+                            o2[h][k * 4 + 2] = ffma2(pp, v2, o2[h][k * 4 + 2]);
+                            o2[h][k * 4 + 3] = ffma2(pp, v3, o2[h][k * 4 + 3]);
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&empty_bar[st]));
+        }
+
+        // -------- merge the token groups of this warp (same lanes li, other grp)
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            float M = m[h];
+#pragma unroll
+            for (int o = C::LPT; o < 32; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+            const float f = fast_exp2(m[h] - M);
+            float L = l[h] * f;
+#pragma unroll
+            for (int o = C::LPT; o < 32; o <<= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+            m[h] = M;
+            l[h] = L;
+#pragma unroll
+            for (int j = 0; j < C::NCL * 4; ++j) {
+                float2 x = make_float2(o2[h][j].x * f, o2[h][j].y * f);
+#pragma unroll
+                for (int o = C::LPT; o < 32; o <<= 1) {
+                    x.x += __shfl_xor_sync(0xffffffffu, x.x, o);
+                    x.y += __shfl_xor_sync(0xffffffffu, x.y, o);
+                }
+                o2[h][j] = x;
+            }
+        }
+        // lanes of token group 0 publish the warp's partial: red[warp][h][o(D), m, l]
+        if (grp == 0) {
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                float* dst = red + (warp * G + h) * C::RED_STRIDE;
+#pragma unroll
+                for (int k = 0; k < C::NCL; ++k) {
+                    float4* d4 = reinterpret_cast<float4*>(dst + (li + k * C::LPT) * 8);
+                    d4[0] = make_float4(o2[h][k * 4 + 0].x, o2[h][k * 4 + 0].y, o2[h][k * 4 + 1].x,
+                                        o2[h][k * 4 + 1].y);
+                    d4[1] = make_float4(o2[h][k * 4 + 2].x, o2[h][k * 4 + 2].y, o2[h][k * 4 + 3].x,
+                                        o2[h][k * 4 + 3].y);
+                }
+                if (li == 0) {
+                    dst[D] = m[h];
+                    dst[D + 1] = l[h];
+                }
+            }
+        }
+        named_bar_sync(1, kConsumerWarps * 32);
+        // -------- merge the warps and write
+        for (int e = threadIdx.x; e < G * D; e += kConsumerWarps * 32) {
+            const int h = e / D, x = e % D;
+            float M = kNegBig;
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, red[(w * G + h) * C::RED_STRIDE + D]);
+            float L = 0.f, acc = 0.f;
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w) {
+                const float* src = red + (w * G + h) * C::RED_STRIDE;
+                const float f = fast_exp2(src[D] - M);
+                L += src[D + 1] * f;
+                acc += src[x] * f;
+            }
+            const int qh = pc.g * G + h;
+            if (pc.whole) {
+                p.out[(size_t(pc.b) * p.hq + qh) * D + x] = L > 0.f ? acc / L : 0.f;
+                if (x == 0 && p.lse != nullptr)
+                    p.lse[size_t(pc.b) * p.hq + qh] =
+                        L > 0.f ? (M + __log2f(L)) * 0.69314718055994530942f : -CUDART_INF_F;
+            } else {
+                const size_t slot = size_t(pc.seg) + blockIdx.x;
+                p.ws_o[(slot * G + h) * D + x] = acc;
+                if (x == 0) {
+                    p.ws_ml[(slot * G + h) * 2 + 0] = M;
+                    p.ws_ml[(slot * G + h) * 2 + 1] = L;
+                }
+            }
+        }
+        named_bar_sync(1, kConsumerWarps * 32);
+    }
+}
+
+// Merge the partials of segments that more than one CTA touched, and handle
+// empty / over-capacity sequences.  One CTA per segment, one warp per query
+// head of the group.
+template <int D, int G>
+__global__ void __launch_bounds__(32 * G) merge_kernel(const __grid_constant__ DecodeParams p) {
+    extern __shared__ int32_t bpre[];
+    build_prefix(p, bpre);
+    __syncthreads();
+    const int seg = blockIdx.x;
+    const int b = seg / p.n_kv, g = seg % p.n_kv;
+    const int h = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int qh = g * G + h;
+    const int L = p.len[b];
+    if (threadIdx.x == 0 && g == 0) {
+        if (L < 0) set_status(p.status, DUO_STATUS_BAD_LENGTH);
+        if (int64_t(L) > p.cap && p.n_r > 0) set_status(p.status, DUO_STATUS_OVER_CAPACITY);
+        if (L < 1) set_status(p.status, DUO_STATUS_EMPTY_SEQUENCE);
+    }
+    float* out = p.out + (size_t(b) * p.hq + qh) * D;
+    if (L < 1) {
+        for (int x = lane; x < D; x += 32) out[x] = 0.f;
+        if (lane == 0 && p.lse != nullptr) p.lse[size_t(b) * p.hq + qh] = -CUDART_INF_F;
+        return;
+    }
+    const int64_t total = bpre[p.B];
+    const int nbr = blocks_of(rows_r(L, p.cap)), nbs = blocks_of(rows_s(L, p.S, p.W));
+    const int64_t seg_gb = bpre[b] + int64_t(p.r_before[g]) * nbr + int64_t(g - p.r_before[g]) * nbs;
+    const int seg_nb = p.is_r[g] ? nbr : nbs;
+    const int c0 = cta_owner(seg_gb, total, p.num_ctas);
+    const int c1 = cta_owner(seg_gb + seg_nb - 1, total, p.num_ctas);
+    if (c0 == c1) return;
+    float M = kNegBig;
+    for (int c = c0; c <= c1; ++c) M = fmaxf(M, p.ws_ml[((size_t(seg) + c) * G + h) * 2]);
+    float Lsum = 0.f;
+    float acc[D / 32];
+#pragma unroll
+    for (int j = 0; j < D / 32; ++j) acc[j] = 0.f;
+    for (int c = c0; c <= c1; ++c) {
+        const size_t slot = size_t(seg) + c;
+        const float f = fast_exp2(p.ws_ml[(slot * G + h) * 2] - M);
+        Lsum += p.ws_ml[(slot * G + h) * 2 + 1] * f;
+        const float* src = p.ws_o + (slot * G + h) * D;
+#pragma unroll
+        for (int j = 0; j < D / 32; ++j) acc[j] += src[lane + 32 * j] * f;
+    }
+#pragma unroll
+    for (int j = 0; j < D / 32; ++j) out[lane + 32 * j] = Lsum > 0.f ? acc[j] / Lsum : 0.f;
+    if (lane == 0 && p.lse != nullptr)
+        p.lse[size_t(b) * p.hq + qh] =
+            Lsum > 0.f ? (M + __log2f(Lsum)) * 0.69314718055994530942f : -CUDART_INF_F;
+}
+
+template <int D, int G>
+cudaError_t launch_t(const DecodeParams& p, cudaStream_t s) {
+    using C = Cfg<D, G>;
+    const size_t smem = C::SMEM + size_t(p.B + 1) * 4;
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(smem));
+    if (e != cudaSuccess) return e;
+    decode_kernel<D, G><<<p.num_ctas, kThreads, smem, s>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    merge_kernel<D, G><<<p.B * p.n_kv, 32 * G, size_t(p.B + 1) * 4, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+int decode_ctas_default(int num_sms, int d, int group) {
+    (void)d;
+    (void)group;
+    return num_sms;   // one persistent CTA per SM
+}
+
+size_t decode_workspace_bytes(int slots, int d, int group) {
+    const size_t o = size_t(slots) * group * d * 4;
+    const size_t ml = size_t(slots) * group * 2 * 4;
+    return ((o + 255) & ~size_t(255)) + ml;
+}
+
+cudaError_t launch_decode(const DecodeParams& p, int d, int group, cudaStream_t s) {
+    if (d == 128) {
+        switch (group) {
+            case 1: return launch_t<128, 1>(p, s);
+            case 2: return launch_t<128, 2>(p, s);
+            case 4: return launch_t<128, 4>(p, s);
+            case 8: return launch_t<128, 8>(p, s);
+        }
+    } else if (d == 64) {
+        switch (group) {
+            case 1: return launch_t<64, 1>(p, s);
+            case 2: return launch_t<64, 2>(p, s);
+            case 4: return launch_t<64, 4>(p, s);
+            case 8: return launch_t<64, 8>(p, s);
+        }
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace duo

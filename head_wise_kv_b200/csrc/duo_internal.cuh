@@ -1,0 +1,204 @@
+// Internal definitions shared by the libduo_kv kernels and host code.
+// Not part of the C ABI (include/duo_kv.h is).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <vector>
+
+#include "duo_kv.h"
+
+namespace duo {
+
+constexpr int kMaxKvHeads = 64;
+
+// One layer's slice of the caller's device buffer (byte offsets from the base).
+struct LayerLayout {
+    int n_r = 0, n_s = 0;
+    size_t off_kr = 0, off_vr = 0, off_ks = 0, off_vs = 0, off_pos = 0;
+    int32_t rank[kMaxKvHeads];      // index among the layer's retrieval or streaming heads
+    int32_t r_before[kMaxKvHeads + 1];  // retrieval heads among KV heads 0..g-1
+    uint8_t is_r[kMaxKvHeads];
+};
+
+}  // namespace duo
+
+struct duo_kv {
+    duo_kv_desc desc;                       // retrieval_mask pointer cleared (not kept)
+    std::vector<duo::LayerLayout> layers;
+    char* base = nullptr;                   // caller's device buffer
+    size_t bytes = 0;
+    int32_t* status = nullptr;              // device status word
+    int device = 0;
+    int num_sms = 0;
+    int decode_ctas = 0;                    // 0 = default persistent wave
+};
+
+namespace duo {
+
+// ----------------------------------------------------------------- launch params
+struct DecodeParams {
+    const uint16_t* kr;
+    const uint16_t* vr;
+    const uint16_t* ks;
+    const uint16_t* vs;
+    const uint16_t* q;
+    const int32_t* len;
+    float* out;
+    float* lse;
+    float* ws_o;      // [slots][G][D]  partial outputs (unnormalised)
+    float* ws_ml;     // [slots][G][2]  partial (max, sum) in the log2 domain
+    int32_t* status;
+    int64_t cap;
+    int B, n_kv, hq, n_r, n_s, S, W;
+    int num_ctas;
+    float scale_log2;
+    unsigned long long timeout_ns;
+    int32_t rank[kMaxKvHeads];
+    int32_t r_before[kMaxKvHeads + 1];
+    uint8_t is_r[kMaxKvHeads];
+};
+
+struct AppendParams {
+    const uint16_t* k_new;
+    const uint16_t* v_new;
+    const int32_t* len_before;
+    const int32_t* n_new;   // may be null
+    uint16_t* kr;
+    uint16_t* vr;
+    uint16_t* ks;
+    uint16_t* vs;
+    int32_t* pos;
+    int32_t* status;
+    int64_t cap;
+    int B, n_kv, n_r, n_s, S, W, d, n_new_max;
+    int32_t rank[kMaxKvHeads];
+    uint8_t is_r[kMaxKvHeads];
+};
+
+// Host-side launchers (defined in the kernel translation units).
+cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
+int decode_ctas_default(int num_sms, int d, int group);
+size_t decode_workspace_bytes(int slots, int d, int group);
+cudaError_t launch_decode(const DecodeParams& p, int d, int group, cudaStream_t s);
+
+// ----------------------------------------------------------------- device helpers
+#ifdef __CUDACC__
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for the given phase parity of an mbarrier, giving up after limit_ns
+// nanoseconds of wall time.  Returns false on timeout.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned long long limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = global_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_ns() - t0 > limit_ns) return false;
+    }
+    return true;
+}
+
+// Bulk (TMA engine) copy of `bytes` contiguous bytes global -> shared,
+// completing on mbarrier `bar`.  16-byte aligned addresses, bytes % 16 == 0.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar,
+                                         uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+        "[%0], [%1], %2, [%3], %4;" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr));
+    return v;
+}
+
+// bf16 pair (low half = element 0) -> two fp32 (exact widening).
+__device__ __forceinline__ float2 bf2_to_f2(uint32_t x) {
+    float2 r;
+    r.x = __uint_as_float(x << 16);
+    r.y = __uint_as_float(x & 0xffff0000u);
+    return r;
+}
+
+// Packed fp32x2 fused multiply-add (sm_100): d = a * b + c, per lane of the pair.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    unsigned long long av = *reinterpret_cast<unsigned long long*>(&a);
+    unsigned long long bv = *reinterpret_cast<unsigned long long*>(&b);
+    unsigned long long cv = *reinterpret_cast<unsigned long long*>(&c);
+    unsigned long long dv;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(dv) : "l"(av), "l"(bv), "l"(cv));
+    return *reinterpret_cast<float2*>(&dv);
+}
+
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+    unsigned long long av = *reinterpret_cast<unsigned long long*>(&a);
+    unsigned long long bv = *reinterpret_cast<unsigned long long*>(&b);
+    unsigned long long dv;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(dv) : "l"(av), "l"(bv));
+    return *reinterpret_cast<float2*>(&dv);
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ void set_status(int32_t* status, int32_t bits) {
+    atomicOr(reinterpret_cast<int*>(status), bits);
+}
+#endif
+
+}  // namespace duo

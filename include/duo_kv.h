@@ -1,0 +1,224 @@
+/*
+ * duo_kv.h -- mixed-head (retrieval / streaming) KV cache and attention
+ * for NVIDIA B200 (sm_100a).  C ABI of libduo_kv.so.
+ *
+ * The method (DuoAttention) splits each layer's KV heads in two:
+ *   retrieval heads keep every token in a full, contiguous cache;
+ *   streaming heads keep a constant-length cache of the first S tokens
+ *   ("attention sinks") plus the most recent W tokens, as a ring buffer.
+ * Sources: "DuoAttention: Dual Retrieval & Streaming Heads Guide",
+ * section 2 ("Retrieval Heads vs. Streaming Heads", "DuoAttention Cache
+ * Partitioning Mechanics" and its memory equation); "Attention Variants and
+ * KV-Cache Compression", section "When Is Reuse Exact?" (chunk mask rule,
+ * positions kept after eviction); "Attention Variants and Memory
+ * Efficiency", sections "Multi-Query and Grouped-Query Attention" and
+ * "Sliding-Window and Mixed Attention" (window rule, ring buffer).
+ *
+ * Conventions shared by every call
+ *   - All tensors are dense, row-major, on the device of the handle, unless
+ *     marked "host".  bf16 tensors are passed as uint16_t bit patterns.
+ *   - B = batch, Hq = query heads, n_kv = KV heads, G = Hq / n_kv,
+ *     d = head_dim, S = sink, W = window.  Query head h reads KV head h / G.
+ *   - The caller owns every device buffer and stream.  The library never
+ *     allocates or frees device memory and never synchronises, except
+ *     duo_kv_read_status (documented below).  Calls are asynchronous on the
+ *     given stream (NULL = the legacy default stream).
+ *   - Sequence lengths live on the device and are passed on every call; the
+ *     library keeps no per-sequence state besides the cache contents.
+ *   - q and K are already position-encoded (e.g. RoPE) by the caller, each
+ *     at the token's original position; the library applies no positional
+ *     encoding.  Ring slots keep each token's original position.
+ *   - Return value: DUO_OK (0) or a negative DUO_ERR_* code.  On an error
+ *     nothing was launched.  Errors found by kernels (a length beyond the
+ *     capacity, an empty sequence, a pipeline wait that timed out) set bits
+ *     of a device status word instead; see duo_kv_read_status.
+ */
+#ifndef DUO_KV_H
+#define DUO_KV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define DUO_API __attribute__((visibility("default")))
+#else
+#define DUO_API
+#endif
+
+/* A cudaStream_t. */
+typedef struct CUstream_st* duo_stream_t;
+
+/* Return codes. */
+enum {
+    DUO_OK = 0,
+    DUO_ERR_INVALID_ARG = -1,   /* null pointer, out-of-range index or size   */
+    DUO_ERR_UNSUPPORTED = -2,   /* shape the library is not built for:        */
+                                /* head_dim not 64 or 128, G not 1/2/4/8,      */
+                                /* n_kv > 64                                   */
+    DUO_ERR_BUFFER_TOO_SMALL = -3,  /* device buffer smaller than required    */
+    DUO_ERR_WORKSPACE = -4,     /* workspace missing or too small              */
+    DUO_ERR_CUDA = -5,          /* a CUDA runtime call or launch failed        */
+    DUO_ERR_ALIGNMENT = -6      /* a device pointer is not 16-byte aligned     */
+                                /* (dev_buf: 256-byte)                         */
+};
+
+/* Bits of the device status word (set by kernels, never cleared by them). */
+enum {
+    DUO_STATUS_OVER_CAPACITY = 1,   /* a retrieval row index >= capacity:     */
+                                    /* the row was not written / read          */
+    DUO_STATUS_EMPTY_SEQUENCE = 2,  /* decode with len[b] < 1: output zeroed  */
+    DUO_STATUS_WAIT_TIMEOUT = 4,    /* a pipeline wait exceeded its limit:     */
+                                    /* the output of that launch is invalid    */
+    DUO_STATUS_BAD_LENGTH = 8       /* negative length or append count         */
+};
+
+/* Cache shape.  retrieval_mask is a HOST array [num_layers][num_kv_heads],
+ * 1 = retrieval head, 0 = streaming head: the binary head mask of the
+ * DuoAttention guide, section 3 item 4 ("Binarization"), given per KV head
+ * (with GQA a KV head is retrieval if any query head of its group needs it,
+ * the guide's deployment checklist item 2).  It is copied during
+ * duo_kv_alloc and not kept.  capacity = rows reserved per retrieval head
+ * per sequence (the maximum length).  Constraints: num_layers, batch,
+ * num_q_heads, num_kv_heads >= 1; num_q_heads % num_kv_heads == 0;
+ * head_dim in {64, 128}; sink >= 0; window >= 1; capacity >= 1. */
+typedef struct {
+    int32_t num_layers;
+    int32_t batch;
+    int32_t num_q_heads;
+    int32_t num_kv_heads;
+    int32_t head_dim;
+    int32_t sink;
+    int32_t window;
+    int64_t capacity;
+    const uint8_t* retrieval_mask;
+} duo_kv_desc;
+
+/* Opaque host-side handle (host memory only). */
+typedef struct duo_kv duo_kv;
+
+/* Device views of one layer's cache (for verification and for callers that
+ * manage the cache themselves).  Layouts:
+ *   k_retrieval, v_retrieval: [B][n_retrieval][capacity][d]  bf16
+ *   k_streaming, v_streaming: [B][n_streaming][S + W][d]     bf16
+ *   positions:                [B][S + W] int32, original position of the
+ *                             token in each streaming slot, -1 = empty
+ *                             (shared by all streaming heads of the layer).
+ * Streaming slot of token p: p if p < S, else S + (p - S) mod W.
+ * head_rank[g] = index of KV head g among the layer's retrieval heads (if
+ * retrieval) or among its streaming heads (if streaming); is_retrieval[g]
+ * is the mask entry. */
+typedef struct {
+    uint16_t* k_retrieval;
+    uint16_t* v_retrieval;
+    uint16_t* k_streaming;
+    uint16_t* v_streaming;
+    int32_t* positions;
+    int32_t n_retrieval;
+    int32_t n_streaming;
+    int32_t head_rank[64];
+    uint8_t is_retrieval[64];
+} duo_kv_layer_view;
+
+/* Bytes of device memory a cache of this shape needs (host arithmetic only,
+ * no CUDA call).  *cache_bytes (optional) receives the K/V part alone:
+ *   sum over layers of 2 * 2 * d * B * (n_r(l) * capacity + n_s(l) * (S+W)),
+ * the DuoAttention guide's memory equation (section 2) times the batch,
+ * with T = capacity and R = n_r / n_kv per layer.  The rest is the position
+ * tables, a status word and 256-byte alignment padding. */
+DUO_API int duo_kv_required_bytes(const duo_kv_desc* desc, size_t* total_bytes, size_t* cache_bytes);
+
+/* Lay a cache out in dev_buf (caller-allocated device memory of buf_bytes,
+ * 256-byte aligned, on the current device), set every position to -1 and
+ * the status word to 0 (two memsets on `stream`), and return a handle.
+ * Queries the current device's SM count once.  Errors: INVALID_ARG,
+ * UNSUPPORTED, BUFFER_TOO_SMALL, ALIGNMENT, CUDA. */
+DUO_API int duo_kv_alloc(const duo_kv_desc* desc, void* dev_buf, size_t buf_bytes,
+                 duo_stream_t stream, duo_kv** out);
+
+/* Release the host handle.  dev_buf stays the caller's.  NULL is a no-op. */
+DUO_API int duo_kv_free(duo_kv* kv);
+
+/* Fill *out with the device views of `layer`.  Host only. */
+DUO_API int duo_kv_layer_view_get(const duo_kv* kv, int32_t layer, duo_kv_layer_view* out);
+
+/* Append tokens to one layer's cache (append + evict).
+ *   k_new, v_new: [B][n_kv][n_new_max][d] bf16, token i of sequence b sits
+ *                 at absolute position len_before[b] + i;
+ *   len_before:   device int32 [B], tokens already appended to that layer;
+ *   n_new:        device int32 [B] tokens to append per sequence
+ *                 (<= n_new_max), or NULL = n_new_max for every sequence.
+ * Retrieval head: token p goes to row p (p >= capacity sets
+ * DUO_STATUS_OVER_CAPACITY and is dropped).  Streaming head: of the appended
+ * tokens only those the ring still holds afterwards are written -- p < S or
+ * p >= len_before + n_new - W -- to slot p (p < S) or S + (p - S) mod W, and
+ * positions[b][slot] = p; when len_before[b] == 0 the slots this call does
+ * not fill are reset to -1.  Following the DuoAttention guide's simulation
+ * (append_token) and the sliding-window ring of "Attention Variants and
+ * Memory Efficiency"; the result equals appending the tokens one at a time.
+ * Decode order per layer: append the new token, then duo_decode_attn.
+ * Prefill order per layer: duo_prefill_attn on the chunk, then append it. */
+DUO_API int duo_kv_append(duo_kv* kv, int32_t layer, const uint16_t* k_new, const uint16_t* v_new,
+                  const int32_t* len_before, const int32_t* n_new, int32_t n_new_max,
+                  duo_stream_t stream);
+
+/* Workspace bytes duo_decode_attn needs (host only). */
+DUO_API int duo_decode_workspace_bytes(const duo_kv* kv, size_t* bytes);
+
+/* Decode attention for one layer, every sequence and query head at once.
+ *   q:    [B][Hq][d] bf16, the query of each sequence's newest token;
+ *   len:  device int32 [B], tokens held after this step's append (>= 1);
+ *         the query sits at position t = len[b] - 1;
+ *   scale: softmax scale (typically 1/sqrt(d));
+ *   out:  [B][Hq][d] fp32, softmax(scale * q.K^T) V over the head's keys:
+ *         retrieval head: all positions 0..t; streaming head: positions
+ *         j <= t with j < S or j >= t - W + 1 (the sinks and the window);
+ *   lse:  optional [B][Hq] fp32, natural log of the softmax denominator;
+ *   workspace: device scratch of >= duo_decode_workspace_bytes bytes
+ *         (no initialisation needed; overlapping calls must not share it).
+ * Split-K over each head's keys with a log-sum-exp merge; the result does
+ * not depend on how the keys are split beyond rounding. */
+DUO_API int duo_decode_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const int32_t* len,
+                    float scale, float* out, float* lse, void* workspace, size_t workspace_bytes,
+                    duo_stream_t stream);
+
+/* Workspace bytes duo_prefill_attn needs for chunks of up to `chunk` rows. */
+DUO_API int duo_prefill_workspace_bytes(const duo_kv* kv, int32_t chunk, size_t* bytes);
+
+/* Chunked-prefill attention for one layer (before the chunk is appended).
+ *   q:          [B][Hq][chunk][d] bf16, rows at positions prefix[b] + i;
+ *   k_chunk, v_chunk: [B][n_kv][chunk][d] bf16, the chunk's own keys/values;
+ *   prefix_len: device int32 [B], tokens already in the cache (P);
+ *   out:        [B][Hq][chunk][d] fp32.
+ * Row i reads keys at positions j <= P + i ("Attention Variants and
+ * KV-Cache Compression", "When Is Reuse Exact?"): retrieval heads all of
+ * them (prefix from the cache, the rest from k_chunk); streaming heads only
+ * j < S or j >= P + i - W + 1 (the sinks and the window, read from the ring
+ * and from k_chunk).  The DuoAttention guide's "Hardware-Fused Prefill":
+ * dense causal attention for retrieval heads, block-sparse sink + local
+ * attention for streaming heads.  Requirements: chunk >= 1; for streaming
+ * heads prefix_len[b] must equal the tokens appended so far. */
+DUO_API int duo_prefill_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const uint16_t* k_chunk,
+                     const uint16_t* v_chunk, const int32_t* prefix_len, int32_t chunk,
+                     float scale, float* out, void* workspace, size_t workspace_bytes,
+                     duo_stream_t stream);
+
+/* Read the device status word into *status (host).  This call
+ * synchronises `stream`.  If clear != 0 the word is reset to 0 afterwards. */
+DUO_API int duo_kv_read_status(duo_kv* kv, int32_t* status, int32_t clear, duo_stream_t stream);
+
+/* Override the number of CTAs the decode kernel splits the keys over
+ * (0 = one persistent wave, the default).  For tests of split invariance;
+ * the workspace requirement grows with it. */
+DUO_API int duo_kv_set_decode_ctas(duo_kv* kv, int32_t ctas);
+
+/* Static text for a return code. */
+DUO_API const char* duo_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DUO_KV_H */

@@ -181,28 +181,32 @@ def attend(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float):
     return (e @ v) / z, m + math.log(z)
 
 
-def decode_attention(q, k_hist, v_hist, lens_after, mask, sink, window, scale):
+def decode_attention(q, k_hist, v_hist, lens_after, mask, sink, window, scale, pairs=None):
     """One decode step of one layer.
 
     q: [B][Hq][d] (the newest token's query per sequence);
-    k_hist(b, g) / v_hist(b, g): callables returning the full history
-    [lens_after[b]][d] of KV head g of sequence b (tokens 0 .. T_b-1);
+    k_hist(b, g) / v_hist(b, g): callables returning the history of KV head g
+    of sequence b as an array indexable by position (at least lens_after[b]
+    rows: tokens 0 .. T_b-1);
     mask: [n_kv], 1 = retrieval head.  Query position t = T_b - 1.
+    pairs: optional iterable of (b, h) to evaluate; the rest stay NaN.
     Returns out [B][Hq][d] and lse [B][Hq] (float64)."""
     q = np.asarray(q, dtype=np.float64)
     B, hq, d = q.shape
     n_kv = len(mask)
-    out = np.zeros((B, hq, d))
-    lse = np.zeros((B, hq))
+    out = np.full((B, hq, d), np.nan)
+    lse = np.full((B, hq), np.nan)
+    todo = {(b, h) for b in range(B) for h in range(hq)} if pairs is None else set(pairs)
     for b in range(B):
         t = int(lens_after[b]) - 1
         for g in range(n_kv):
+            heads = [h for h in range(hq) if kv_head_of(h, hq, n_kv) == g and (b, h) in todo]
+            if not heads:
+                continue
             keys = np.arange(t + 1) if mask[g] else keep_set(t, sink, window)
-            K = np.asarray(k_hist(b, g), dtype=np.float64)[keys]
-            V = np.asarray(v_hist(b, g), dtype=np.float64)[keys]
-            for h in range(hq):
-                if kv_head_of(h, hq, n_kv) != g:
-                    continue
+            K = np.asarray(k_hist(b, g)[keys], dtype=np.float64)
+            V = np.asarray(v_hist(b, g)[keys], dtype=np.float64)
+            for h in heads:
                 out[b, h], lse[b, h] = attend(q[b, h], K, V, scale)
     return out, lse
 

@@ -1,0 +1,126 @@
+"""C ABI checks that need no GPU: the library loads, exports every function
+include/duo_kv.h declares, sizes caches by the method's memory equation, and
+rejects bad arguments before touching CUDA."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import duo_workloads as W
+from oracle import duo_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _lib():
+    from head_wise_kv_b200 import _lib as L
+    return L
+
+
+def declared_functions():
+    names = []
+    for f in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if f.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", f)).read()
+            names += re.findall(r"^DUO_API\s+[\w\s\*]*?\b(duo_\w+)\s*\(", src, flags=re.M)
+    return names
+
+
+def test_library_exports_every_declared_function():
+    L = _lib()
+    names = declared_functions()
+    assert len(names) >= 12
+    raw = ctypes.CDLL(L.LIB_PATH)
+    for n in names:
+        assert hasattr(raw, n), f"{n} declared in include/ but not exported"
+    assert set(L.EXPORTED) <= set(names)
+
+
+def _desc(L, layers=2, B=3, hq=32, n_kv=8, d=128, S=64, Wn=256, cap=1000, mask=None):
+    if mask is None:
+        mask = np.zeros((layers, n_kv), np.uint8)
+        mask[:, ::2] = 1
+    return L.make_desc(layers, B, hq, n_kv, d, S, Wn, cap, np.asarray(mask, np.uint8).tobytes())
+
+
+@pytest.mark.parametrize("cfg", ["tiny", "mha32k", "gqa128k", "mtok", "prefill64k"])
+def test_cache_bytes_follow_memory_equation(cfg):
+    """The K/V bytes the library lays out equal the batch times the Duo memory
+    equation (oracle) with T = capacity and the per-layer retrieval counts."""
+    L = _lib()
+    w = W.WORKLOADS[cfg]
+    masks = W.retrieval_masks(w)
+    cap = W.capacity(w)
+    d, keep = L.make_desc(w.layers, w.batch, w.hq, w.n_kv, w.d, w.sink, w.window, cap, masks.tobytes())
+    total, cache = L.duo_kv_required_bytes(d)
+    want = w.batch * O.duo_cache_bytes(w.layers, w.n_kv, w.d, cap, w.sink, w.window, masks.sum(1).tolist())
+    assert cache == want
+    pos_bytes = w.layers * w.batch * (w.sink + w.window) * 4
+    assert want + pos_bytes <= total <= want + pos_bytes + 256 * (6 * w.layers + 1)
+
+
+def test_guide_example_bytes():
+    """80 layers, 8 KV heads (2 retrieval), d=128, T=128,000, S=32, W=128:
+    the guide's 32,120-token effective context times the dense bytes per token."""
+    L = _lib()
+    mask = np.zeros((80, 8), np.uint8)
+    mask[:, :2] = 1
+    d, keep = _desc(L, layers=80, B=1, hq=64, n_kv=8, d=128, S=32, Wn=128, cap=128000, mask=mask)
+    assert L.duo_kv_required_bytes(d)[1] == 10525081600
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("head_dim", 96, -2), ("head_dim", 256, -2), ("window", 0, -1), ("sink", -1, -1),
+    ("num_q_heads", 24, -2), ("num_q_heads", 30, -1), ("capacity", 0, -1), ("num_kv_heads", 0, -1),
+    ("batch", 0, -1), ("num_layers", 0, -1), ("capacity", 1 << 40, -1),
+])
+def test_rejects_bad_shapes(field, value, code):
+    L = _lib()
+    d, keep = _desc(L)
+    setattr(d, field, value)
+    with pytest.raises(L.DuoError) as e:
+        L.duo_kv_required_bytes(d)
+    assert e.value.code == code
+
+
+def test_rejects_more_than_64_kv_heads():
+    L = _lib()
+    d, keep = _desc(L, hq=128, n_kv=128, mask=np.zeros((2, 128), np.uint8))
+    with pytest.raises(L.DuoError) as e:
+        L.duo_kv_required_bytes(d)
+    assert e.value.code == L.DUO_ERR_UNSUPPORTED
+
+
+def test_alloc_argument_checks_before_cuda():
+    L = _lib()
+    d, keep = _desc(L)
+    total, _ = L.duo_kv_required_bytes(d)
+    with pytest.raises(L.DuoError) as e:
+        L.duo_kv_alloc(d, 0, total, 0)
+    assert e.value.code == L.DUO_ERR_INVALID_ARG
+    with pytest.raises(L.DuoError) as e:
+        L.duo_kv_alloc(d, 0x1000 + 16, total, 0)        # not 256-byte aligned
+    assert e.value.code == L.DUO_ERR_ALIGNMENT
+    with pytest.raises(L.DuoError) as e:
+        L.duo_kv_alloc(d, 0x100000, total - 1, 0)       # too small
+    assert e.value.code == L.DUO_ERR_BUFFER_TOO_SMALL
+
+
+def test_null_handle_calls_fail_cleanly():
+    L = _lib()
+    for fn, args in [(L.duo_kv_append, (None, 0, 16, 16, 16, None, 1, None)),
+                     (L.duo_decode_attn, (None, 0, 16, 16, 0.1, 16, None, 16, 1 << 20, None)),
+                     (L.duo_prefill_attn, (None, 0, 16, 16, 16, 16, 8, 0.1, 16, None, 0, None))]:
+        with pytest.raises(L.DuoError) as e:
+            fn(*args)
+        assert e.value.code == L.DUO_ERR_INVALID_ARG
+    assert L._c_free(None) == 0
+
+
+def test_strerror_covers_codes():
+    L = _lib()
+    for c in range(0, -7, -1):
+        assert L.duo_strerror(c) != "unknown error"
+    assert L.duo_strerror(-99) == "unknown error"
