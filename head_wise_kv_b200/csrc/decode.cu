@@ -196,6 +196,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     }
     build_prefix(p, bpre);
     __syncthreads();
+    // The merge kernel may be scheduled now; it waits (griddepcontrol.wait)
+    // for this grid's completion before it reads any partial.
+    asm volatile("griddepcontrol.launch_dependents;");
 
     const int64_t total = bpre[p.B];
     if (total == 0) return;
@@ -450,7 +453,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 
 // Merge the partials of segments that more than one CTA touched, and handle
 // empty / over-capacity sequences.  One CTA per segment, one warp per query
-// head of the group.
+// head of the group.  Launched as a programmatic dependent of the attention
+// kernel: everything before griddepcontrol.wait overlaps its tail.
 template <int D, int G>
 __global__ void __launch_bounds__(32 * G) merge_kernel(const __grid_constant__ DecodeParams p) {
     extern __shared__ int32_t bpre[];
@@ -461,40 +465,63 @@ __global__ void __launch_bounds__(32 * G) merge_kernel(const __grid_constant__ D
     const int h = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int qh = g * G + h;
     const int L = p.len[b];
+    float* out = p.out + (size_t(b) * p.hq + qh) * D;
+    const int64_t total = bpre[p.B];
+    const int nbr = blocks_of(rows_r(L, p.cap)), nbs = blocks_of(rows_s(L, p.S, p.W));
+    const int64_t seg_gb = bpre[b] + int64_t(p.r_before[g]) * nbr + int64_t(g - p.r_before[g]) * nbs;
+    const int seg_nb = p.is_r[g] ? nbr : nbs;
+    const int c0 = L < 1 ? 0 : cta_owner(seg_gb, total, p.num_ctas);
+    const int c1 = L < 1 ? 0 : cta_owner(seg_gb + seg_nb - 1, total, p.num_ctas);
+    const bool dense = total >= p.num_ctas;   // then no CTA range is empty
+
+    // wait for the attention kernel's partials (and its writes of `out`)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
     if (threadIdx.x == 0 && g == 0) {
         if (L < 0) set_status(p.status, DUO_STATUS_BAD_LENGTH);
         if (int64_t(L) > p.cap && p.n_r > 0) set_status(p.status, DUO_STATUS_OVER_CAPACITY);
         if (L < 1) set_status(p.status, DUO_STATUS_EMPTY_SEQUENCE);
     }
-    float* out = p.out + (size_t(b) * p.hq + qh) * D;
     if (L < 1) {
         for (int x = lane; x < D; x += 32) out[x] = 0.f;
         if (lane == 0 && p.lse != nullptr) p.lse[size_t(b) * p.hq + qh] = -CUDART_INF_F;
         return;
     }
-    const int64_t total = bpre[p.B];
-    const int nbr = blocks_of(rows_r(L, p.cap)), nbs = blocks_of(rows_s(L, p.S, p.W));
-    const int64_t seg_gb = bpre[b] + int64_t(p.r_before[g]) * nbr + int64_t(g - p.r_before[g]) * nbs;
-    const int seg_nb = p.is_r[g] ? nbr : nbs;
-    const int c0 = cta_owner(seg_gb, total, p.num_ctas);
-    const int c1 = cta_owner(seg_gb + seg_nb - 1, total, p.num_ctas);
     if (c0 == c1) return;
+
+    // lanes own pieces: max and weighted sum of the (max, sum) pairs.  CTAs
+    // with an empty range (fewer blocks than CTAs) wrote nothing: skipped.
     float M = kNegBig;
-    for (int c = c0; c <= c1; ++c) M = fmaxf(M, p.ws_ml[((size_t(seg) + c) * G + h) * 2]);
+    for (int c = c0 + lane; c <= c1; c += 32) {
+        if (!dense && cta_start(c + 1, total, p.num_ctas) == cta_start(c, total, p.num_ctas)) continue;
+        M = fmaxf(M, p.ws_ml[((size_t(seg) + c) * G + h) * 2]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float Lsum = 0.f;
+    for (int c = c0 + lane; c <= c1; c += 32) {
+        if (!dense && cta_start(c + 1, total, p.num_ctas) == cta_start(c, total, p.num_ctas)) continue;
+        const size_t slot = size_t(seg) + c;
+        Lsum += p.ws_ml[(slot * G + h) * 2 + 1] * fast_exp2(p.ws_ml[(slot * G + h) * 2] - M);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, o);
+
     float acc[D / 32];
 #pragma unroll
     for (int j = 0; j < D / 32; ++j) acc[j] = 0.f;
+#pragma unroll 4
     for (int c = c0; c <= c1; ++c) {
+        if (!dense && cta_start(c + 1, total, p.num_ctas) == cta_start(c, total, p.num_ctas)) continue;
         const size_t slot = size_t(seg) + c;
         const float f = fast_exp2(p.ws_ml[(slot * G + h) * 2] - M);
-        Lsum += p.ws_ml[(slot * G + h) * 2 + 1] * f;
         const float* src = p.ws_o + (slot * G + h) * D;
 #pragma unroll
         for (int j = 0; j < D / 32; ++j) acc[j] += src[lane + 32 * j] * f;
     }
+    const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
 #pragma unroll
-    for (int j = 0; j < D / 32; ++j) out[lane + 32 * j] = Lsum > 0.f ? acc[j] / Lsum : 0.f;
+    for (int j = 0; j < D / 32; ++j) out[lane + 32 * j] = acc[j] * inv;
     if (lane == 0 && p.lse != nullptr)
         p.lse[size_t(b) * p.hq + qh] =
             Lsum > 0.f ? (M + __log2f(Lsum)) * 0.69314718055994530942f : -CUDART_INF_F;
@@ -510,7 +537,18 @@ cudaError_t launch_t(const DecodeParams& p, cudaStream_t s) {
     decode_kernel<D, G><<<p.num_ctas, kThreads, smem, s>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    merge_kernel<D, G><<<p.B * p.n_kv, 32 * G, size_t(p.B + 1) * 4, s>>>(p);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(p.B * p.n_kv));
+    cfg.blockDim = dim3(32 * G);
+    cfg.dynamicSmemBytes = size_t(p.B + 1) * 4;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, merge_kernel<D, G>, p);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -31,6 +31,7 @@ def _run_steps(w, steps, lens0=None, ctas=None, layer=0, pairs=None, check_every
     cache = _mk(w, int(lens0.max()) + steps)
     if ctas is not None:
         cache.set_decode_ctas(ctas)
+    cache._ws.fill_(0xFF)   # NaN canary: a read of an unwritten workspace slot fails parity
     hist = History(w)
     fill(cache, hist, layer, lens0, dev)
     mask = W.retrieval_mask(w, layer)
