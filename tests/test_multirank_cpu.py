@@ -1,0 +1,47 @@
+"""Multi-rank host logic of bench.py on CPU (gloo, world size 2): each rank
+takes its own slice of the global batch (weak scaling, no data exchange), and
+the timing reduction is the max over ranks."""
+import os
+import socket
+
+import numpy as np
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out_dir):
+    import sys
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import bench
+    r, w, _ = bench.dist_init()
+    assert (r, w) == (rank, world)
+    base, gw, lens = bench.rank_workload(rank, world)
+    t = bench.max_over_ranks(10.0 + rank, world, "cpu")
+    bench.barrier(world)
+    np.save(os.path.join(out_dir, f"r{rank}.npy"), np.concatenate([lens, [t]]))
+    import torch.distributed as dist
+    dist.destroy_process_group()
+
+
+def test_two_ranks_shard_batch_and_reduce_max(tmp_path):
+    world = 2
+    mp.start_processes(_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    r0, r1 = (np.load(tmp_path / f"r{r}.npy") for r in range(world))
+    import duo_workloads as W
+    base = W.WORKLOADS["gqa128k"]
+    full = W.context_lengths(W.scaled(base, batch=base.batch * world))
+    # rank r holds sequences 8r .. 8r+7 of the global batch; per-GPU work is fixed
+    assert np.array_equal(r0[:-1], full[:8]) and np.array_equal(r1[:-1], full[8:])
+    # the single-GPU workload is rank 0's slice
+    assert np.array_equal(r0[:-1], W.context_lengths(base))
+    assert r0[-1] == r1[-1] == 11.0
