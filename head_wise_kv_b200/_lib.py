@@ -38,8 +38,9 @@ EXPORTED = (
     "duo_kv_required_bytes", "duo_kv_alloc", "duo_kv_free", "duo_kv_layer_view_get",
     "duo_kv_append", "duo_decode_workspace_bytes", "duo_decode_attn",
     "duo_prefill_workspace_bytes", "duo_prefill_attn", "duo_kv_read_status",
-    "duo_kv_set_decode_ctas", "duo_strerror",
+    "duo_kv_set_decode_ctas", "duo_strerror", "duo_decode_attn_static_ws",
 )
+DUO_STATIC_WS_BYTES = 4 << 20
 
 
 class duo_kv_desc(ctypes.Structure):
@@ -89,6 +90,7 @@ _c_view = _sig("duo_kv_layer_view_get", [_P, _I32, ctypes.POINTER(duo_kv_layer_v
 _c_append = _sig("duo_kv_append", [_P, _I32, _P, _P, _P, _P, _I32, _P])
 _c_dec_ws = _sig("duo_decode_workspace_bytes", [_P, ctypes.POINTER(_SZ)])
 _c_decode = _sig("duo_decode_attn", [_P, _I32, _P, _P, ctypes.c_float, _P, _P, _P, _SZ, _P])
+_c_decode_static = _sig("duo_decode_attn_static_ws", [_P, _I32, _P, _P, ctypes.c_float, _P, _P, _P])
 _c_pre_ws = _sig("duo_prefill_workspace_bytes", [_P, _I32, ctypes.POINTER(_SZ)])
 _c_prefill = _sig("duo_prefill_attn", [_P, _I32, _P, _P, _P, _P, _I32, ctypes.c_float, _P, _P, _SZ, _P])
 _c_status = _sig("duo_kv_read_status", [_P, ctypes.POINTER(_I32), _I32, _P])
@@ -155,6 +157,10 @@ def duo_decode_workspace_bytes(handle) -> int:
 def duo_decode_attn(handle, layer, q, length, scale, out, lse, workspace, workspace_bytes, stream) -> None:
     _check(_c_decode(handle, layer, q, length, scale, out, lse, workspace, workspace_bytes, stream),
            "duo_decode_attn")
+
+
+def duo_decode_attn_static_ws(handle, layer, q, length, scale, out, lse, stream) -> None:
+    _check(_c_decode_static(handle, layer, q, length, scale, out, lse, stream), "duo_decode_attn_static_ws")
 
 
 def duo_prefill_workspace_bytes(handle, chunk) -> int:

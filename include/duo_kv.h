@@ -185,6 +185,32 @@ DUO_API int duo_decode_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const 
                     float scale, float* out, float* lse, void* workspace, size_t workspace_bytes,
                     duo_stream_t stream);
 
+/* Bytes of device scratch built into the library for
+ * duo_decode_attn_static_ws (a file-scope __device__ array). */
+#define DUO_STATIC_WS_BYTES (4u << 20)
+
+/* Decode attention exactly as duo_decode_attn, for callers that cannot
+ * allocate device memory: a plugin whose host program owns all device
+ * memory and passes it only its inputs and outputs, or a serving loop that
+ * must not call cudaMalloc (it can synchronise the device and can fail with
+ * out-of-memory in the middle of a request).  Instead of a caller workspace
+ * the call uses the library's own DUO_STATIC_WS_BYTES (4 MiB) scratch array,
+ * which every GPU that loads the library holds until the process exits; the
+ * call itself allocates nothing.
+ *   - Limit: duo_decode_workspace_bytes(kv) must be <= DUO_STATIC_WS_BYTES,
+ *     otherwise DUO_ERR_WORKSPACE is returned and nothing is launched.
+ *   - The handle's device must be the current device (else INVALID_ARG).
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) and caches it; make that first call before any
+ *     stream capture begins.
+ *   - All calls on a device share the one array: calls whose kernels can
+ *     overlap on the GPU (e.g. on unordered streams) race and corrupt each
+ *     other's results.  Leftover contents from earlier calls do no harm.
+ * The pages describe no counterpart of this entry point; it only changes
+ * where the scratch memory comes from. */
+DUO_API int duo_decode_attn_static_ws(duo_kv* kv, int32_t layer, const uint16_t* q, const int32_t* len,
+                                      float scale, float* out, float* lse, duo_stream_t stream);
+
 /* Workspace bytes duo_prefill_attn needs for chunks of up to `chunk` rows. */
 DUO_API int duo_prefill_workspace_bytes(const duo_kv* kv, int32_t chunk, size_t* bytes);
 
