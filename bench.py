@@ -322,6 +322,91 @@ def run_ours(args, rank, world, local):
     return res, (gw, lens0, mask, first_b)
 
 
+# ---------------------------------------------------------------- chunked prefill
+def prefill_pairs(prompt, chunk, n_r_q, n_s_q, S, Wn):
+    """Mask-valid (query, key) pairs of a chunked prefill: retrieval query heads
+    see every key j <= t, streaming query heads min(t+1, S+W) keys."""
+    pairs = 0
+    for P in range(0, prompt, chunk):
+        C = min(chunk, prompt - P)
+        pairs += n_r_q * (P * C + C * (C + 1) // 2)
+        t = np.arange(P, P + C, dtype=np.int64)
+        pairs += n_s_q * int(np.minimum(t + 1, S + Wn).sum())
+    return pairs
+
+
+def bf16_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["bf16_tflops"]), float(j.get("bf16_tflops_sustained", j["bf16_tflops"])), "measured"
+    return 1590.0, 1400.0, "fallback"
+
+
+def run_prefill(local, reps=3):
+    """The 64K-token prompt in 16 chunks of 4096, attention then append per
+    chunk (one layer, GQA 32q/8kv, 4 retrieval KV heads, S=64, W=1024)."""
+    from head_wise_kv_b200 import DuoKVCache
+
+    dev = torch.device("cuda", local)
+    w = W.WORKLOADS["prefill64k"]
+    mask = W.retrieval_mask(w, 0)
+    G = w.hq // w.n_kv
+    C, n_chunks = w.chunk, w.prompt // w.chunk
+    cache = DuoKVCache(1, 1, w.hq, w.n_kv, w.d, w.sink, w.window, w.prompt, mask[None], device=dev)
+    q = torch.empty(w.hq, w.prompt, w.d, dtype=torch.bfloat16)
+    k = torch.empty(w.n_kv, w.prompt, w.d, dtype=torch.bfloat16)
+    v = torch.empty_like(k)
+    for h in range(w.hq):
+        q[h] = W.tokens(w, 0, 0, h, W.TENSOR_Q, 0, w.prompt)
+    for g in range(w.n_kv):
+        k[g] = W.tokens(w, 0, 0, g, W.TENSOR_K, 0, w.prompt)
+        v[g] = W.tokens(w, 0, 0, g, W.TENSOR_V, 0, w.prompt)
+    dq = [q[:, c * C:(c + 1) * C].contiguous()[None].to(dev) for c in range(n_chunks)]
+    dk = [k[:, c * C:(c + 1) * C].contiguous()[None].to(dev) for c in range(n_chunks)]
+    dv = [v[:, c * C:(c + 1) * C].contiguous()[None].to(dev) for c in range(n_chunks)]
+    pre = [torch.tensor([c * C], dtype=torch.int32, device=dev) for c in range(n_chunks)]
+    out = torch.empty(1, w.hq, C, w.d, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * n_chunks + 1)] for _ in range(reps + 1)]
+    for r in range(reps + 1):     # repetition 0 is the warm-up
+        e = ev[r]
+        e[0].record(stream)
+        for c in range(n_chunks):
+            cache.prefill(0, dq[c], dk[c], dv[c], pre[c], w.scale, out=out)
+            e[2 * c + 1].record(stream)
+            cache.append(0, dk[c], dv[c], pre[c])
+            e[2 * c + 2].record(stream)
+    torch.cuda.synchronize()
+    assert cache.status() == 0, "device status set during the prefill benchmark"
+    attn_ms, total_ms = [], []
+    for r in range(1, reps + 1):
+        e = ev[r]
+        attn_ms.append(sum(e[2 * c].elapsed_time(e[2 * c + 1]) for c in range(n_chunks)))
+        total_ms.append(e[0].elapsed_time(e[-1]))
+    n_r_q = int(mask.sum()) * G
+    pairs = prefill_pairs(w.prompt, C, n_r_q, w.hq - n_r_q, w.sink, w.window)
+    flops = 4 * w.d * pairs
+    a_ms = statistics.median(attn_ms)
+    tflops = flops / (a_ms * 1e-3) / 1e12
+    burst, sustained, kind = bf16_peaks()
+    cache.close()
+    return {
+        "workload": "prefill64k: 65536-token prompt in 16 chunks of 4096, GQA 32q/8kv d=128, 4/8 KV heads "
+                    "retrieval (causal), 4 streaming (sink 64 + window 1024)",
+        "attn_ms": round(a_ms, 3),
+        "total_ms_with_append": round(statistics.median(total_ms), 3),
+        "useful_flops": int(flops),
+        "useful_tflops": round(tflops, 1),
+        "roofline": {"bound": "tensor", "kernel": "prefill_kernel (tcgen05)", "achieved": round(tflops, 1),
+                     "peak": sustained, "peak_kind": f"{kind} sustained bf16", "unit": "TFLOP/s",
+                     "frac": round(tflops / sustained, 4), "frac_of_burst": round(tflops / burst, 4),
+                     "traffic": None},
+        "gpu_launches": 2 * n_chunks * reps,
+    }
+
+
 # ---------------------------------------------------------------- oracle timing
 def oracle_step_sample(gw, lens0, mask, first_b, seqs):
     """Time the fp64 oracle on one full layer-step of the given sequences
@@ -419,14 +504,21 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=64)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the chunked-prefill measurement")
+    ap.add_argument("--only", choices=["decode", "prefill"], default=None,
+                    help="measure one path only (profiling runs)")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
     rank, world, local = dist_init()
     try:
         if args.impl == "reference":
             res = run_reference(args, rank, world)
+        elif args.only == "prefill":
+            res = {"metric": "chunked prefill attention", "prefill": run_prefill(local)} if rank == 0 else None
         else:
             res, ctx = run_ours(args, rank, world, local)
+            if world == 1 and not args.no_prefill and args.only != "decode":
+                res["prefill"] = run_prefill(local)
             if rank == 0 and world == 1 and not args.no_cpu_baseline:
                 res["cpu_baseline"] = cpu_baseline(ctx)
         if rank == 0 and res is not None:

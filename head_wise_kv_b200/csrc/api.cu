@@ -5,6 +5,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <algorithm>
 #include <new>
 
 #include "duo_internal.cuh"
@@ -234,18 +235,59 @@ int duo_decode_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const int32_t*
 
 int duo_prefill_workspace_bytes(const duo_kv* kv, int32_t chunk, size_t* bytes) {
     if (!kv || !bytes || chunk < 1) return DUO_ERR_INVALID_ARG;
-    *bytes = 0;
+    *bytes = 0;   // the prefill kernel keeps all its state on chip
     return DUO_OK;
 }
 
 int duo_prefill_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const uint16_t* k_chunk,
                      const uint16_t* v_chunk, const int32_t* prefix_len, int32_t chunk, float scale,
                      float* out, void* workspace, size_t workspace_bytes, duo_stream_t stream) {
+    (void)workspace;
+    (void)workspace_bytes;
     if (!kv || layer < 0 || layer >= kv->desc.num_layers || !q || !k_chunk || !v_chunk || !prefix_len ||
         !out || chunk < 1)
         return DUO_ERR_INVALID_ARG;
-    (void)scale; (void)workspace; (void)workspace_bytes; (void)stream;
-    return DUO_ERR_UNSUPPORTED;
+    if (!(scale > 0.f) || scale != scale) return DUO_ERR_INVALID_ARG;
+    if (kv->desc.head_dim != 128) return DUO_ERR_UNSUPPORTED;
+    const duo_kv_desc& d = kv->desc;
+    if (duo::prefill_smem_bytes(d.sink, d.window) > 227 * 1024) return DUO_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k_chunk) || !aligned16(v_chunk) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(prefix_len) & 3))
+        return DUO_ERR_ALIGNMENT;
+    const duo::LayerLayout& L = kv->layers[layer];
+    const int64_t SW = int64_t(d.sink) + d.window;
+    // tile coordinates are 32-bit row indices
+    const int64_t rows_max = std::max({int64_t(d.batch) * d.num_q_heads * chunk,
+                                       int64_t(d.batch) * d.num_kv_heads * chunk,
+                                       int64_t(d.batch) * L.n_r * d.capacity + 128,
+                                       int64_t(d.batch) * L.n_s * SW + 128});
+    if (rows_max >= (int64_t(1) << 31)) return DUO_ERR_UNSUPPORTED;
+    duo::PrefillLaunch a;
+    a.q = q;
+    a.k_chunk = k_chunk;
+    a.v_chunk = v_chunk;
+    a.kr = kv->base + L.off_kr;
+    a.vr = kv->base + L.off_vr;
+    a.ks = kv->base + L.off_ks;
+    a.vs = kv->base + L.off_vs;
+    a.prefix = prefix_len;
+    a.pos = reinterpret_cast<const int32_t*>(kv->base + L.off_pos);
+    a.out = out;
+    a.status = kv->status;
+    a.cap = d.capacity;
+    a.B = d.batch;
+    a.hq = d.num_q_heads;
+    a.n_kv = d.num_kv_heads;
+    a.C = chunk;
+    a.S = d.sink;
+    a.W = d.window;
+    a.n_r = L.n_r;
+    a.n_s = L.n_s;
+    a.scale = scale;
+    a.timeout_ns = kWaitLimitNs;
+    memcpy(a.rank, L.rank, sizeof a.rank);
+    memcpy(a.is_r, L.is_r, sizeof a.is_r);
+    return duo::launch_prefill(a, stream);
 }
 
 int duo_kv_read_status(duo_kv* kv, int32_t* status, int32_t clear, duo_stream_t stream) {

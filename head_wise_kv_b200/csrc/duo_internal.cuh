@@ -77,11 +77,33 @@ struct AppendParams {
     uint8_t is_r[kMaxKvHeads];
 };
 
+struct PrefillLaunch {
+    const void* q;
+    const void* k_chunk;
+    const void* v_chunk;
+    const void* kr;
+    const void* vr;
+    const void* ks;
+    const void* vs;
+    const int32_t* prefix;
+    const int32_t* pos;
+    float* out;
+    int32_t* status;
+    int64_t cap;
+    int B, hq, n_kv, C, S, W, n_r, n_s;
+    float scale;
+    unsigned long long timeout_ns;
+    int32_t rank[kMaxKvHeads];
+    uint8_t is_r[kMaxKvHeads];
+};
+
 // Host-side launchers (defined in the kernel translation units).
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 int decode_ctas_default(int num_sms, int d, int group);
 size_t decode_workspace_bytes(int slots, int d, int group);
 cudaError_t launch_decode(const DecodeParams& p, int d, int group, cudaStream_t s);
+size_t prefill_smem_bytes(int S, int W);
+int launch_prefill(const PrefillLaunch& a, cudaStream_t s);   // returns a DUO_* code
 
 // ----------------------------------------------------------------- device helpers
 #ifdef __CUDACC__

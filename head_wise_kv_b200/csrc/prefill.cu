@@ -1,0 +1,597 @@
+// Chunked-prefill attention on the 5th-generation tensor cores (tcgen05).
+//
+// A chunk of C query rows that follows P cached tokens: row i sits at
+// position P + i and reads keys j <= P + i ("Attention Variants and KV-Cache
+// Compression", "When Is Reuse Exact?").  Retrieval heads read all of them
+// (dense causal attention: the cached prefix from the retrieval cache, the
+// rest from the chunk's own K/V); streaming heads read only the sinks and the
+// window (j < S or j >= P + i - W + 1), block-sparse: only the ring's sink
+// slots, its window slots (for the first W-1 rows) and the chunk tiles that
+// meet the band are visited ("Hardware-Fused Prefill" in the DuoAttention
+// guide: dense attention for retrieval heads, a block-sparse sliding-window
+// kernel for streaming heads).
+//
+// One CTA = one (sequence, query head, 128-row query tile); 8 warps:
+//   warp 0     TMA producer: Q once, then K/V tiles (128 keys x 128 dims, two
+//              128-byte-swizzled slabs each) into a 2-stage ring
+//   warp 1     allocates TMEM; one lane issues tcgen05.mma:
+//                S_j = Q K_j^T   (bf16 x bf16 -> fp32, M=N=128, 8 x K16)
+//                O  += P_j V_j   (fp16 x fp16 -> fp32, V MN-major)
+//              S is double-buffered in TMEM so S_{j+1} overlaps softmax_j
+//   warps 2-3  convert each V tile in place bf16 -> fp16 (exact for
+//              |v| < 65504) and zero key rows past the valid range
+//   warps 4-7  softmax, one query row per thread (TMEM lane = row): masked
+//              scores, running max with lazy rescaling (O is rescaled only
+//              when the max grows by more than 2^8), P_j as fp16 into a
+//              swizzled shared tile, final O / l to global memory.
+// P is fp16 rather than bf16: rounding P to bf16 alone costs ~1e-3 relative
+// error in the output, fp16 ~1.5e-4.
+//
+// Every mbarrier wait is bounded; on a timeout the CTA sets
+// DUO_STATUS_WAIT_TIMEOUT, stops, waits (bounded) for its own copies and
+// MMAs in flight, frees TMEM and exits.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <math_constants.h>
+#include <stdint.h>
+
+#include "duo_internal.cuh"
+
+namespace duo {
+
+namespace {
+
+constexpr int kBM = 128;   // query rows per CTA
+constexpr int kBN = 128;   // keys per tile
+constexpr int kHD = 128;   // head dim (prefill is built for d = 128)
+constexpr int kThreads = 256;
+constexpr uint32_t kSlab = 128 * 128;        // bytes: 128 rows x 64 bf16
+constexpr uint32_t kTile = 2 * kSlab;        // 32 KB: 128 rows x 128 bf16
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO = 256;
+constexpr float kNegBig = -1.0e30f;
+constexpr float kRescaleThreshold = 8.0f;    // log2 units
+
+// Instruction descriptors (kind::f16, fp32 accumulate, M = 128, N = 128).
+// bits: [4,6) D format (1 = f32), [7,10) A format, [10,13) B format
+// (0 = f16, 1 = bf16), 15 A major, 16 B major (1 = MN-major),
+// [17,23) N >> 3, [24,29) M >> 4.
+constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kBN >> 3) << 17) |
+                              (uint32_t(kBM >> 4) << 24);
+constexpr uint32_t kIdescPV = (1u << 4) | (0u << 7) | (0u << 10) | (1u << 16) | (uint32_t(kHD >> 3) << 17) |
+                              (uint32_t(kBM >> 4) << 24);
+
+struct PrefillParams {
+    CUtensorMap tm_q, tm_kc, tm_vc, tm_kr, tm_vr, tm_ks, tm_vs;
+    const int32_t* prefix;
+    const int32_t* pos;     // this layer's [B][S+W] position table
+    float* out;
+    int32_t* status;
+    int64_t cap;
+    int B, hq, n_kv, G, C, n_qt, S, W, n_r, n_s;
+    float scale_log2;
+    unsigned long long timeout_ns;
+    int32_t rank[kMaxKvHeads];
+    uint8_t is_r[kMaxKvHeads];
+};
+
+// ------------------------------------------------------------------ PTX helpers
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = uint64_t((saddr >> 4) & 0x3FFFu);
+    d |= uint64_t((lbo >> 4) & 0x3FFFu) << 16;
+    d |= uint64_t((sbo >> 4) & 0x3FFFu) << 32;
+    d |= uint64_t(1) << 46;   // descriptor version (sm_100)
+    d |= uint64_t(2) << 61;   // 128-byte swizzle
+    return d;
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+          "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+        "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+        "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+// One 128-row x 128-dim bf16 tile = two 64-dim slabs (x = 0 and x = 64).
+__device__ __forceinline__ void tma_tile(uint32_t dst, const CUtensorMap* map, int row, uint32_t bar) {
+    tma_load_2d(dst, map, 0, row, bar);
+    tma_load_2d(dst + kSlab, map, 64, row, bar);
+}
+
+// ------------------------------------------------------------------ key tiles
+enum : int { kSrcCache = 0, kSrcSink = 1, kSrcWindow = 2, kSrcChunk = 3 };
+
+struct KeyTile {
+    int src;       // kSrc*
+    int row0;      // first row in its source (cache row, ring slot offset, chunk row)
+    int nvalid;    // rows of the tile that hold keys
+    bool masked;   // needs the element mask
+};
+
+// The key tiles one CTA visits, in order.  Computed identically by every role.
+struct Plan {
+    bool retr;
+    int P, i0, i1, C, S, W;
+    int n_a;           // cache tiles (retrieval) or sink tiles (streaming)
+    int n_w;           // window tiles (streaming)
+    int nw_rows;       // filled window slots
+    int c0_lo, c0_hi, c1_lo, c1_hi;   // chunk tile ranges (inclusive; empty if lo > hi)
+    int n;
+
+    __device__ void init(bool is_retrieval, int P_, int i0_, int C_, int S_, int W_) {
+        retr = is_retrieval;
+        P = P_; i0 = i0_; C = C_; S = S_; W = W_;
+        i1 = min(i0 + kBM, C);
+        const int hi = (i1 - 1) / kBN;
+        n_w = 0; nw_rows = 0;
+        c1_lo = 1; c1_hi = 0;
+        if (retr) {
+            n_a = (P + kBN - 1) / kBN;
+            c0_lo = 0; c0_hi = hi;
+        } else {
+            const int sinks = min(S, P);
+            n_a = (sinks + kBN - 1) / kBN;
+            if (P > S && i0 <= W - 2) {
+                nw_rows = min(P - S, W);
+                n_w = (nw_rows + kBN - 1) / kBN;
+            }
+            const int lo = max(0, i0 - W + 1) / kBN;
+            if (P < S) {
+                const int sc = min((min(S - P, C) - 1) / kBN, hi);
+                if (sc + 1 >= lo) { c0_lo = 0; c0_hi = hi; }
+                else { c0_lo = 0; c0_hi = sc; c1_lo = lo; c1_hi = hi; }
+            } else {
+                c0_lo = lo; c0_hi = hi;
+            }
+        }
+        n = n_a + n_w + (c0_hi - c0_lo + 1) + (c1_hi >= c1_lo ? c1_hi - c1_lo + 1 : 0);
+    }
+
+    __device__ KeyTile get(int j) const {
+        KeyTile t;
+        if (j < n_a) {
+            t.src = retr ? kSrcCache : kSrcSink;
+            t.row0 = j * kBN;
+            const int lim = retr ? P : min(S, P);
+            t.nvalid = min(kBN, lim - t.row0);
+            t.masked = t.nvalid < kBN;
+            return t;
+        }
+        j -= n_a;
+        if (j < n_w) {
+            t.src = kSrcWindow;
+            t.row0 = j * kBN;
+            t.nvalid = min(kBN, nw_rows - t.row0);
+            t.masked = true;
+            return t;
+        }
+        j -= n_w;
+        const int n0 = c0_hi - c0_lo + 1;
+        const int k = j < n0 ? c0_lo + j : c1_lo + (j - n0);
+        t.src = kSrcChunk;
+        t.row0 = k * kBN;
+        t.nvalid = min(kBN, C - t.row0);
+        t.masked = !retr || t.nvalid < kBN || t.row0 + kBN - 1 > i0;
+        return t;
+    }
+};
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ bool timed_wait(uint32_t bar, uint32_t parity, const PrefillParams& p,
+                                           volatile int* abort_flag) {
+    if (*abort_flag) return false;
+    if (mbar_wait(bar, parity, p.timeout_ns)) return true;
+    set_status(p.status, DUO_STATUS_WAIT_TIMEOUT);
+    *abort_flag = 1;
+    return false;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_constant__ PrefillParams p) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sQ = smem_addr(smem);
+    const uint32_t sK0 = sQ + kTile, sK1 = sQ + 2 * kTile;
+    const uint32_t sV0 = sQ + 3 * kTile, sV1 = sQ + 4 * kTile;
+    const uint32_t sP = sQ + 5 * kTile;
+    unsigned char* sP_gen = smem + 5 * kTile;
+    unsigned char* sV_gen0 = smem + 3 * kTile;
+    int32_t* spos = reinterpret_cast<int32_t*>(smem + 6 * kTile);
+
+    __shared__ __align__(8) uint64_t bar_q, kv_full[2], kv_empty[2], v_conv[2], s_full[2], s_free[2], p_full,
+        o_done, mma_fin;
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int abort_sh;
+    volatile int* abort_flag = &abort_sh;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // ---------------------------------------------------------------- work item
+    const int per_qt = p.B * p.hq;
+    const int qt = p.n_qt - 1 - int(blockIdx.x) / per_qt;   // heaviest query tiles first
+    const int rem = int(blockIdx.x) % per_qt;
+    const int h = rem % p.hq, b = rem / p.hq;
+    const int g = h / p.G;
+    const int i0 = qt * kBM;
+    const int P = p.prefix[b];
+    const bool retr = p.is_r[g] != 0;
+    Plan plan;
+    plan.init(retr, P < 0 ? 0 : P, i0, p.C, p.S, p.W);
+
+    if (threadIdx.x == 0) {
+        mbar_init(smem_addr(&bar_q), 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(smem_addr(&kv_full[s]), 1);
+            mbar_init(smem_addr(&kv_empty[s]), 1);
+            mbar_init(smem_addr(&v_conv[s]), 2);
+            mbar_init(smem_addr(&s_full[s]), 1);
+            mbar_init(smem_addr(&s_free[s]), 4);
+        }
+        mbar_init(smem_addr(&p_full), 4);
+        mbar_init(smem_addr(&o_done), 1);
+        mbar_init(smem_addr(&mma_fin), 1);
+        abort_sh = (P < 0) ? 1 : 0;
+        if (P < 0) set_status(p.status, DUO_STATUS_BAD_LENGTH);
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_addr(&tmem_base_sh)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (!retr && threadIdx.x >= 128) {   // position table of the ring (window masks)
+        const int SW = p.S + p.W;
+        for (int s = threadIdx.x - 128; s < SW; s += 128) spos[s] = p.pos[size_t(b) * SW + s];
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_sh;
+
+    const int kv_rank = p.rank[g];
+    const int SW = p.S + p.W;
+
+    if (warp == 0) {
+        // ============================================================ TMA producer
+        if (lane == 0) {
+            mbar_arrive_expect_tx(smem_addr(&bar_q), kTile);
+            tma_tile(sQ, &p.tm_q, (b * p.hq + h) * p.C + i0, smem_addr(&bar_q));
+            int issued = 0;
+            for (int j = 0; j < plan.n; ++j) {
+                const int st = j & 1;
+                if (!timed_wait(smem_addr(&kv_empty[st]), ((j >> 1) & 1) ^ 1, p, abort_flag)) break;
+                const KeyTile kt = plan.get(j);
+                const CUtensorMap *mk, *mv;
+                int row;
+                if (kt.src == kSrcCache) {
+                    mk = &p.tm_kr; mv = &p.tm_vr;
+                    row = int((int64_t(b) * p.n_r + kv_rank) * p.cap + kt.row0);
+                } else if (kt.src == kSrcChunk) {
+                    mk = &p.tm_kc; mv = &p.tm_vc;
+                    row = (b * p.n_kv + g) * p.C + kt.row0;
+                } else {
+                    mk = &p.tm_ks; mv = &p.tm_vs;
+                    row = (b * p.n_s + kv_rank) * SW + (kt.src == kSrcWindow ? p.S : 0) + kt.row0;
+                }
+                const uint32_t bar = smem_addr(&kv_full[st]);
+                mbar_arrive_expect_tx(bar, 2 * kTile);
+                tma_tile(st ? sK1 : sK0, mk, row, bar);
+                tma_tile(st ? sV1 : sV0, mv, row, bar);
+                ++issued;
+            }
+            // do not leave while copies may still land in this CTA's shared memory
+            mbar_wait(smem_addr(&bar_q), 0, p.timeout_ns);
+            for (int k = 0; k < 2 && k < issued; ++k) {
+                const int j = issued - 1 - k;
+                mbar_wait(smem_addr(&kv_full[j & 1]), (j >> 1) & 1, p.timeout_ns);
+            }
+        }
+    } else if (warp == 1) {
+        // ============================================================ MMA issuer
+        if (lane == 0) {
+            bool ok = timed_wait(smem_addr(&bar_q), 0, p, abort_flag);
+            tc_fence_after();
+            auto issue_s = [&](int j) -> bool {
+                const int st = j & 1;
+                if (!timed_wait(smem_addr(&kv_full[st]), (j >> 1) & 1, p, abort_flag)) return false;
+                if (!timed_wait(smem_addr(&s_free[st]), ((j >> 1) & 1) ^ 1, p, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t sk = st ? sK1 : sK0;
+#pragma unroll
+                for (int k = 0; k < kHD / 16; ++k) {
+                    const uint32_t off = (k >> 2) * kSlab + (k & 3) * 32;
+                    umma_f16(tmem + (st ? kTmemS1 : kTmemS0), smem_desc(sQ + off, 16, 1024),
+                             smem_desc(sk + off, 16, 1024), kIdescQK, k > 0);
+                }
+                umma_commit(smem_addr(&s_full[st]));
+                return true;
+            };
+            if (ok) ok = issue_s(0);
+            for (int j = 0; ok && j < plan.n; ++j) {
+                if (j + 1 < plan.n && !issue_s(j + 1)) { ok = false; break; }
+                if (!timed_wait(smem_addr(&p_full), j & 1, p, abort_flag)) { ok = false; break; }
+                if (!timed_wait(smem_addr(&v_conv[j & 1]), (j >> 1) & 1, p, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t sv = (j & 1) ? sV1 : sV0;
+#pragma unroll
+                for (int k = 0; k < kBN / 16; ++k) {
+                    umma_f16(tmem + kTmemO, smem_desc(sP + (k >> 2) * kSlab + (k & 3) * 32, 16, 1024),
+                             smem_desc(sv + k * 2048, kSlab, 1024), kIdescPV, (j > 0 || k > 0) ? 1u : 0u);
+                }
+                umma_commit(smem_addr(&kv_empty[j & 1]));
+                umma_commit(smem_addr(&o_done));
+            }
+            // all MMAs issued by this thread have completed before TMEM is freed
+            umma_commit(smem_addr(&mma_fin));
+            mbar_wait(smem_addr(&mma_fin), 0, p.timeout_ns);
+        }
+    } else if (warp < 4) {
+        // ============================================================ V converter
+        const int t = threadIdx.x - 64;   // 0..63
+        for (int j = 0; j < plan.n; ++j) {
+            const int st = j & 1;
+            if (!timed_wait(smem_addr(&kv_full[st]), (j >> 1) & 1, p, abort_flag)) break;
+            const int nvalid = plan.get(j).nvalid;
+            uint4* v = reinterpret_cast<uint4*>(sV_gen0 + st * kTile);
+#pragma unroll 4
+            for (int c = t; c < int(kTile / 16); c += 64) {
+                const int row = (c % (kSlab / 16)) / 8;   // 8 chunks of 16 B per 128-byte row
+                uint4 x = v[c];
+                if (row >= nvalid) {
+                    x = make_uint4(0, 0, 0, 0);
+                } else {
+                    const float2 a = bf2_to_f2(x.x), bb = bf2_to_f2(x.y), cc = bf2_to_f2(x.z), dd = bf2_to_f2(x.w);
+                    x.x = pack_half2(a.x, a.y);
+                    x.y = pack_half2(bb.x, bb.y);
+                    x.z = pack_half2(cc.x, cc.y);
+                    x.w = pack_half2(dd.x, dd.y);
+                }
+                v[c] = x;
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&v_conv[st]));
+        }
+    } else {
+        // ============================================================ softmax
+        const int wq = warp & 3;                 // TMEM lane quarter of this warp
+        const int r = wq * 32 + lane;            // query row within the tile
+        const int i = i0 + r;                    // chunk row
+        const int tpos = plan.P + i;             // absolute position
+        const uint32_t lane_off = uint32_t(wq * 32) << 16;
+        float m = kNegBig, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < plan.n; ++j) {
+            const int st = j & 1;
+            if (!timed_wait(smem_addr(&s_full[st]), (j >> 1) & 1, p, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            float s[kBN];
+            {
+                uint32_t u[32];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    tmem_ld32(tmem + lane_off + (st ? kTmemS1 : kTmemS0) + c * 32, u);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) s[c * 32 + x] = __uint_as_float(u[x]) * p.scale_log2;
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&s_free[st]));
+
+            const KeyTile kt = plan.get(j);
+            if (kt.masked) {
+#pragma unroll
+                for (int c = 0; c < kBN; ++c) {
+                    bool keep = c < kt.nvalid;
+                    if (kt.src == kSrcWindow) {
+                        keep = keep && spos[p.S + kt.row0 + c] >= tpos - p.W + 1;
+                    } else if (kt.src == kSrcChunk) {
+                        const int jj = kt.row0 + c;
+                        keep = keep && jj <= i && (plan.retr || plan.P + jj < p.S || jj >= i - p.W + 1);
+                    }
+                    s[c] = keep ? s[c] : -CUDART_INF_F;
+                }
+            }
+            float mt = s[0];
+#pragma unroll
+            for (int c = 1; c < kBN; ++c) mt = fmaxf(mt, s[c]);
+            const bool grow = mt > m + kRescaleThreshold;
+            const float m_new = grow ? mt : m;
+            const float alpha = fast_exp2(m - m_new);   // 1 when the max is kept
+            float lt = 0.f;
+#pragma unroll
+            for (int c = 0; c < kBN; ++c) {
+                s[c] = fast_exp2(s[c] - m_new);
+                lt += s[c];
+            }
+            l = l * alpha + lt;
+            m = m_new;
+            // P_j reuses the shared tile of P_{j-1}, and a rescale touches O:
+            // both need PV_{j-1} to have completed.
+            if (j > 0) {
+                if (!timed_wait(smem_addr(&o_done), (j - 1) & 1, p, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, grow)) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t u[32];
+                        const uint32_t ta = tmem + lane_off + kTmemO + c * 32;
+                        tmem_ld32(ta, u);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int x = 0; x < 32; ++x) u[x] = __float_as_uint(__uint_as_float(u[x]) * alpha);
+                        tmem_st32(ta, u);
+                    }
+                    tmem_wait_st();
+                }
+            }
+            // P row as fp16, 128-byte swizzled K-major tile (two 64-key slabs)
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                const int slab = q >> 3, ch = q & 7;
+                uint4 w;
+                w.x = pack_half2(s[q * 8 + 0], s[q * 8 + 1]);
+                w.y = pack_half2(s[q * 8 + 2], s[q * 8 + 3]);
+                w.z = pack_half2(s[q * 8 + 4], s[q * 8 + 5]);
+                w.w = pack_half2(s[q * 8 + 6], s[q * 8 + 7]);
+                *reinterpret_cast<uint4*>(sP_gen + slab * kSlab + r * 128 + ((ch ^ (r & 7)) * 16)) = w;
+            }
+            fence_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&p_full));
+        }
+        // epilogue: O / l
+        if (ok && timed_wait(smem_addr(&o_done), (plan.n - 1) & 1, p, abort_flag)) {
+            tc_fence_after();
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            float* dst = p.out + ((size_t(b) * p.hq + h) * p.C + i) * kHD;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t u[32];
+                tmem_ld32(tmem + lane_off + kTmemO + c * 32, u);
+                tmem_wait_ld();
+                if (i < p.C) {
+#pragma unroll
+                    for (int x = 0; x < 32; x += 4)
+                        *reinterpret_cast<float4*>(dst + c * 32 + x) =
+                            make_float4(__uint_as_float(u[x]) * inv, __uint_as_float(u[x + 1]) * inv,
+                                        __uint_as_float(u[x + 2]) * inv, __uint_as_float(u[x + 3]) * inv);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    }
+    return fn;
+}
+
+// 2-D bf16 map over `rows` rows of 128 elements; box 64 x 128 rows, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {uint64_t(kHD), rows < 1 ? 1 : rows};
+    cuuint64_t strides[1] = {uint64_t(kHD) * 2};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+size_t prefill_smem_bytes(int S, int W) { return 6 * size_t(kTile) + size_t(S + W) * 4 + 1024; }
+
+int launch_prefill(const PrefillLaunch& a, cudaStream_t s) {
+    PrefillParams p;
+    memset(&p, 0, sizeof p);
+    const int SW = a.S + a.W;
+    if (!make_map(&p.tm_q, a.q, uint64_t(a.B) * a.hq * a.C) ||
+        !make_map(&p.tm_kc, a.k_chunk, uint64_t(a.B) * a.n_kv * a.C) ||
+        !make_map(&p.tm_vc, a.v_chunk, uint64_t(a.B) * a.n_kv * a.C) ||
+        !make_map(&p.tm_kr, a.kr, uint64_t(a.B) * a.n_r * a.cap) ||
+        !make_map(&p.tm_vr, a.vr, uint64_t(a.B) * a.n_r * a.cap) ||
+        !make_map(&p.tm_ks, a.ks, uint64_t(a.B) * a.n_s * SW) ||
+        !make_map(&p.tm_vs, a.vs, uint64_t(a.B) * a.n_s * SW))
+        return DUO_ERR_CUDA;
+    p.prefix = a.prefix;
+    p.pos = a.pos;
+    p.out = a.out;
+    p.status = a.status;
+    p.cap = a.cap;
+    p.B = a.B; p.hq = a.hq; p.n_kv = a.n_kv; p.G = a.hq / a.n_kv; p.C = a.C;
+    p.n_qt = (a.C + kBM - 1) / kBM;
+    p.S = a.S; p.W = a.W; p.n_r = a.n_r; p.n_s = a.n_s;
+    p.scale_log2 = a.scale * 1.4426950408889634f;
+    p.timeout_ns = a.timeout_ns;
+    memcpy(p.rank, a.rank, sizeof p.rank);
+    memcpy(p.is_r, a.is_r, sizeof p.is_r);
+    const size_t smem = prefill_smem_bytes(a.S, a.W);
+    cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return DUO_ERR_CUDA;
+    const int64_t grid = int64_t(p.n_qt) * a.B * a.hq;
+    if (grid > 0x7fffffff) return DUO_ERR_UNSUPPORTED;
+    prefill_kernel<<<unsigned(grid), kThreads, smem, s>>>(p);
+    return cudaGetLastError() == cudaSuccess ? DUO_OK : DUO_ERR_CUDA;
+}
+
+}  // namespace duo
