@@ -11,7 +11,7 @@
 // guide: dense attention for retrieval heads, a block-sparse sliding-window
 // kernel for streaming heads).
 //
-// One CTA = one (sequence, query head, 128-row query tile); 8 warps:
+// One CTA = one (sequence, query head, 128-row query tile); 12 warps:
 //   warp 0     TMA producer: Q once, then K/V tiles (128 keys x 128 dims, two
 //              128-byte-swizzled slabs each) into a 2-stage ring
 //   warp 1     allocates TMEM; one lane issues tcgen05.mma:
@@ -20,10 +20,10 @@
 //              S is double-buffered in TMEM so S_{j+1} overlaps softmax_j
 //   warps 2-3  convert each V tile in place bf16 -> fp16 (exact for
 //              |v| < 65504) and zero key rows past the valid range
-//   warps 4-7  softmax, one query row per thread (TMEM lane = row): masked
-//              scores, running max with lazy rescaling (O is rescaled only
-//              when the max grows by more than 2^8), P_j as fp16 into a
-//              swizzled shared tile, final O / l to global memory.
+//   warps 4-11 softmax, two threads per query row (TMEM lane = row, one
+//              64-key half each): masked scores, running max with lazy
+//              rescaling (O is rescaled only when the max grows by more than
+//              2^8), P_j as fp16 into a swizzled shared tile, final O / l.
 // P is fp16 rather than bf16: rounding P to bf16 alone costs ~1e-3 relative
 // error in the output, fp16 ~1.5e-4.
 //
@@ -45,7 +45,7 @@ namespace {
 constexpr int kBM = 128;   // query rows per CTA
 constexpr int kBN = 128;   // keys per tile
 constexpr int kHD = 128;   // head dim (prefill is built for d = 128)
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;   // 12 warps: TMA, MMA, 2 V converters, 8 softmax
 constexpr uint32_t kSlab = 128 * 128;        // bytes: 128 rows x 64 bf16
 constexpr uint32_t kTile = 2 * kSlab;        // 32 KB: 128 rows x 128 bf16
 constexpr uint32_t kTmemCols = 512;
@@ -116,6 +116,10 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
           "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
           "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld32p(uint32_t taddr, uint32_t* r) {
+    tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(r));
 }
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
@@ -224,6 +228,15 @@ struct Plan {
     }
 };
 
+// Bit c set for every c in [lo, hi] within 0..31.
+__device__ __forceinline__ uint32_t range_bits(int lo, int hi) {
+    lo = max(lo, 0);
+    hi = min(hi, 31);
+    if (lo > hi) return 0u;
+    const uint32_t upto = hi == 31 ? 0xffffffffu : ((2u << hi) - 1u);
+    return upto & ~((1u << lo) - 1u);
+}
+
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
     __half2 h = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&h);
@@ -238,6 +251,31 @@ __device__ __forceinline__ bool timed_wait(uint32_t bar, uint32_t parity, const 
     return false;
 }
 
+// Lane 0 waits on the mbarrier for the warp (fewer shared-memory polls).
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const PrefillParams& p,
+                                          volatile int* abort_flag) {
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0) ok = timed_wait(bar, parity, p, abort_flag) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
+}
+
+// Barrier over the 256 softmax threads that also ORs a flag across them, so
+// every softmax warp takes the same exit decision.
+__device__ __forceinline__ bool softmax_barrier_any(bool flag) {
+    uint32_t out;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\t"
+        "setp.ne.u32 pi, %1, 0;\n\t"
+        "bar.red.or.pred po, 1, 256, pi;\n\t"
+        "selp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(out)
+        : "r"(uint32_t(flag))
+        : "memory");
+    return out != 0;
+}
+
 __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_constant__ PrefillParams p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -248,11 +286,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     const uint32_t sP = sQ + 5 * kTile;
     unsigned char* sP_gen = smem + 5 * kTile;
     unsigned char* sV_gen0 = smem + 3 * kTile;
-    int32_t* spos = reinterpret_cast<int32_t*>(smem + 6 * kTile);
 
     __shared__ __align__(8) uint64_t bar_q, kv_full[2], kv_empty[2], v_conv[2], s_full[2], s_free[2], p_full,
         o_done, mma_fin;
     __shared__ uint32_t tmem_base_sh;
+    __shared__ float red_max[2][2][kBM];   // [tile parity][column half][row]
+    __shared__ float red_l[2][kBM];        // [column half][row] final row sums
     __shared__ int abort_sh;
     volatile int* abort_flag = &abort_sh;
 
@@ -277,9 +316,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             mbar_init(smem_addr(&kv_empty[s]), 1);
             mbar_init(smem_addr(&v_conv[s]), 2);
             mbar_init(smem_addr(&s_full[s]), 1);
-            mbar_init(smem_addr(&s_free[s]), 4);
+            mbar_init(smem_addr(&s_free[s]), 8);
         }
-        mbar_init(smem_addr(&p_full), 4);
+        mbar_init(smem_addr(&p_full), 8);
         mbar_init(smem_addr(&o_done), 1);
         mbar_init(smem_addr(&mma_fin), 1);
         abort_sh = (P < 0) ? 1 : 0;
@@ -292,10 +331,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                      "r"(kTmemCols)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-    }
-    if (!retr && threadIdx.x >= 128) {   // position table of the ring (window masks)
-        const int SW = p.S + p.W;
-        for (int s = threadIdx.x - 128; s < SW; s += 128) spos[s] = p.pos[size_t(b) * SW + s];
     }
     tc_fence_before();
     __syncthreads();
@@ -408,111 +443,148 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         }
     } else {
         // ============================================================ softmax
-        const int wq = warp & 3;                 // TMEM lane quarter of this warp
+        // 8 warps, two per scheduler: warp w owns the TMEM lane quarter w % 4
+        // (32 query rows) and the column half hf of every S tile (64 keys), of
+        // the P tile (one swizzled slab) and of O (64 dims).  The two halves of
+        // a row agree on the tile maximum through shared memory once per tile.
+        const int wq = warp & 3;
+        const int hf = (warp - 4) >> 2;
         const int r = wq * 32 + lane;            // query row within the tile
         const int i = i0 + r;                    // chunk row
         const int tpos = plan.P + i;             // absolute position
+        const int cb = hf * 64;                  // first key column of this half
         const uint32_t lane_off = uint32_t(wq * 32) << 16;
         float m = kNegBig, l = 0.f;
         bool ok = true;
         for (int j = 0; j < plan.n; ++j) {
             const int st = j & 1;
-            if (!timed_wait(smem_addr(&s_full[st]), (j >> 1) & 1, p, abort_flag)) { ok = false; break; }
-            tc_fence_after();
-            float s[kBN];
-            {
-                uint32_t u[32];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    tmem_ld32(tmem + lane_off + (st ? kTmemS1 : kTmemS0) + c * 32, u);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int x = 0; x < 32; ++x) s[c * 32 + x] = __uint_as_float(u[x]) * p.scale_log2;
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&s_free[st]));
+            const bool got = warp_wait(smem_addr(&s_full[st]), (j >> 1) & 1, p, abort_flag);
+            float s[64];   // raw scores of this half row, then probabilities
+            float mx = -CUDART_INF_F;
+            if (got) {
+                tc_fence_after();
+                uint32_t* u = reinterpret_cast<uint32_t*>(s);
+                const uint32_t ta = tmem + lane_off + (st ? kTmemS1 : kTmemS0) + cb;
+                tmem_ld32p(ta, u);
+                tmem_ld32p(ta + 32, u + 32);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_addr(&s_free[st]));
 
-            const KeyTile kt = plan.get(j);
-            if (kt.masked) {
-#pragma unroll
-                for (int c = 0; c < kBN; ++c) {
-                    bool keep = c < kt.nvalid;
-                    if (kt.src == kSrcWindow) {
-                        keep = keep && spos[p.S + kt.row0 + c] >= tpos - p.W + 1;
-                    } else if (kt.src == kSrcChunk) {
-                        const int jj = kt.row0 + c;
-                        keep = keep && jj <= i && (plan.retr || plan.P + jj < p.S || jj >= i - p.W + 1);
+                const KeyTile kt = plan.get(j);
+                if (kt.masked) {
+                    // Every mask is: c <= hi and (aL <= c <= aH or bL <= c <= bH),
+                    // with c the key's column in the tile.
+                    int hi = kt.nvalid - 1, aL = 0, aH = kBN, bL = kBN, bH = -1;
+                    if (kt.src == kSrcChunk) {
+                        // causal (key j <= row i); streaming heads also need j in
+                        // the window (j >= i-W+1) or a sink (P + j < S)
+                        hi = min(hi, i - kt.row0);
+                        if (!plan.retr) {
+                            aL = i - p.W + 1 - kt.row0;
+                            bL = 0;
+                            bH = p.S - plan.P - kt.row0 - 1;
+                        }
+                    } else if (kt.src == kSrcWindow) {
+                        // Window slot k holds the position the append rule gave it:
+                        // the ring's newest slot kn = (P-1-S) mod W (nw-1 before it
+                        // wraps) holds P-1; positions fall by one per slot going
+                        // back and wrap once.  Positions >= t-W+1: two intervals.
+                        const bool full = plan.P - p.S >= p.W;
+                        const int kn = full ? (plan.P - 1 - p.S) % p.W : plan.nw_rows - 1;
+                        aL = (tpos - p.W + 1) - (plan.P - 1) + kn - kt.row0;
+                        aH = kn - kt.row0;
+                        bL = max(aL + p.W, aH + 1);
+                        bH = full ? p.W - 1 - kt.row0 : -1;
                     }
-                    s[c] = keep ? s[c] : -CUDART_INF_F;
-                }
-            }
-            float mt = s[0];
 #pragma unroll
-            for (int c = 1; c < kBN; ++c) mt = fmaxf(mt, s[c]);
+                    for (int q = 0; q < 2; ++q) {
+                        const int o = cb + q * 32;
+                        const uint32_t keep = (range_bits(aL - o, aH - o) | range_bits(bL - o, bH - o)) &
+                                              range_bits(0, hi - o);
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) s[q * 32 + c] = (keep >> c) & 1u ? s[q * 32 + c] : -CUDART_INF_F;
+                    }
+                }
+                float t8[8];
+#pragma unroll
+                for (int x = 0; x < 8; ++x) t8[x] = s[x];
+#pragma unroll
+                for (int c = 8; c < 64; ++c) t8[c & 7] = fmaxf(t8[c & 7], s[c]);
+                mx = fmaxf(fmaxf(fmaxf(t8[0], t8[1]), fmaxf(t8[2], t8[3])),
+                           fmaxf(fmaxf(t8[4], t8[5]), fmaxf(t8[6], t8[7])));
+            }
+            // exchange the half-row maxima; the barrier also agrees on aborting
+            red_max[st][hf][r] = mx;
+            if (softmax_barrier_any(!got || *abort_flag)) { ok = false; break; }
+            mx = fmaxf(red_max[st][0][r], red_max[st][1][r]);
+
+            const float mt = mx * p.scale_log2;          // scale > 0 keeps the order
             const bool grow = mt > m + kRescaleThreshold;
             const float m_new = grow ? mt : m;
             const float alpha = fast_exp2(m - m_new);   // 1 when the max is kept
-            float lt = 0.f;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            uint32_t ph[32];   // probabilities as packed fp16 pairs
 #pragma unroll
-            for (int c = 0; c < kBN; ++c) {
-                s[c] = fast_exp2(s[c] - m_new);
-                lt += s[c];
+            for (int c = 0; c < 64; c += 2) {
+                const float e0 = fast_exp2(fmaf(s[c], p.scale_log2, -m_new));
+                const float e1 = fast_exp2(fmaf(s[c + 1], p.scale_log2, -m_new));
+                acc[(c >> 1) & 3] += e0 + e1;
+                ph[c / 2] = pack_half2(e0, e1);
             }
-            l = l * alpha + lt;
+            l = l * alpha + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
             m = m_new;
             // P_j reuses the shared tile of P_{j-1}, and a rescale touches O:
             // both need PV_{j-1} to have completed.
             if (j > 0) {
-                if (!timed_wait(smem_addr(&o_done), (j - 1) & 1, p, abort_flag)) { ok = false; break; }
+                if (!warp_wait(smem_addr(&o_done), (j - 1) & 1, p, abort_flag)) continue;   // next barrier exits
                 tc_fence_after();
-                if (__any_sync(0xffffffffu, grow)) {
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t u[32];
-                        const uint32_t ta = tmem + lane_off + kTmemO + c * 32;
-                        tmem_ld32(ta, u);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int x = 0; x < 32; ++x) u[x] = __float_as_uint(__uint_as_float(u[x]) * alpha);
-                        tmem_st32(ta, u);
-                    }
-                    tmem_wait_st();
-                }
             }
-            // P row as fp16, 128-byte swizzled K-major tile (two 64-key slabs)
+            // this half of the P row: slab hf of the 128-byte swizzled K-major tile
 #pragma unroll
-            for (int q = 0; q < 16; ++q) {
-                const int slab = q >> 3, ch = q & 7;
-                uint4 w;
-                w.x = pack_half2(s[q * 8 + 0], s[q * 8 + 1]);
-                w.y = pack_half2(s[q * 8 + 2], s[q * 8 + 3]);
-                w.z = pack_half2(s[q * 8 + 4], s[q * 8 + 5]);
-                w.w = pack_half2(s[q * 8 + 6], s[q * 8 + 7]);
-                *reinterpret_cast<uint4*>(sP_gen + slab * kSlab + r * 128 + ((ch ^ (r & 7)) * 16)) = w;
+            for (int ch = 0; ch < 8; ++ch)
+                *reinterpret_cast<uint4*>(sP_gen + hf * kSlab + r * 128 + ((ch ^ (r & 7)) * 16)) =
+                    make_uint4(ph[ch * 4 + 0], ph[ch * 4 + 1], ph[ch * 4 + 2], ph[ch * 4 + 3]);
+            if (j > 0 && __any_sync(0xffffffffu, grow)) {
+#pragma unroll 1
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t u[32];
+                    const uint32_t ta = tmem + lane_off + kTmemO + cb + c * 32;
+                    tmem_ld32(ta, u);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) u[x] = __float_as_uint(__uint_as_float(u[x]) * alpha);
+                    tmem_st32(ta, u);
+                }
+                tmem_wait_st();
             }
             fence_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_addr(&p_full));
         }
-        // epilogue: O / l
-        if (ok && timed_wait(smem_addr(&o_done), (plan.n - 1) & 1, p, abort_flag)) {
-            tc_fence_after();
-            const float inv = l > 0.f ? 1.f / l : 0.f;
-            float* dst = p.out + ((size_t(b) * p.hq + h) * p.C + i) * kHD;
+        // epilogue: O / (l of both halves)
+        if (ok) {
+            const bool got = warp_wait(smem_addr(&o_done), (plan.n - 1) & 1, p, abort_flag);
+            red_l[hf][r] = l;
+            if (!softmax_barrier_any(!got)) {
+                tc_fence_after();
+                const float lt = red_l[0][r] + red_l[1][r];
+                const float inv = lt > 0.f ? 1.f / lt : 0.f;
+                float* dst = p.out + ((size_t(b) * p.hq + h) * p.C + i) * kHD + cb;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t u[32];
-                tmem_ld32(tmem + lane_off + kTmemO + c * 32, u);
-                tmem_wait_ld();
-                if (i < p.C) {
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t u[32];
+                    tmem_ld32(tmem + lane_off + kTmemO + cb + c * 32, u);
+                    tmem_wait_ld();
+                    if (i < p.C) {
 #pragma unroll
-                    for (int x = 0; x < 32; x += 4)
-                        *reinterpret_cast<float4*>(dst + c * 32 + x) =
-                            make_float4(__uint_as_float(u[x]) * inv, __uint_as_float(u[x + 1]) * inv,
-                                        __uint_as_float(u[x + 2]) * inv, __uint_as_float(u[x + 3]) * inv);
+                        for (int x = 0; x < 32; x += 4)
+                            *reinterpret_cast<float4*>(dst + c * 32 + x) =
+                                make_float4(__uint_as_float(u[x]) * inv, __uint_as_float(u[x + 1]) * inv,
+                                            __uint_as_float(u[x + 2]) * inv, __uint_as_float(u[x + 3]) * inv);
+                    }
                 }
             }
         }
@@ -559,7 +631,11 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows) {
 
 }  // namespace
 
-size_t prefill_smem_bytes(int S, int W) { return 6 * size_t(kTile) + size_t(S + W) * 4 + 1024; }
+size_t prefill_smem_bytes(int S, int W) {
+    (void)S;
+    (void)W;
+    return 6 * size_t(kTile) + 1024;
+}
 
 int launch_prefill(const PrefillLaunch& a, cudaStream_t s) {
     PrefillParams p;
