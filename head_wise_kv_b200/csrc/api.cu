@@ -233,17 +233,25 @@ int duo_decode_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const int32_t*
     return cuda_err(duo::launch_decode(p, D, G, stream));
 }
 
+static size_t prefill_ws(const duo_kv* kv, int32_t chunk) {
+    int n_r = 0, n_s = 0;
+    for (const duo::LayerLayout& L : kv->layers) {
+        n_r = std::max(n_r, L.n_r);
+        n_s = std::max(n_s, L.n_s);
+    }
+    const duo_kv_desc& d = kv->desc;
+    return duo::prefill_workspace_bytes(d.batch, d.num_kv_heads, n_r, n_s, d.capacity, d.sink, d.window, chunk);
+}
+
 int duo_prefill_workspace_bytes(const duo_kv* kv, int32_t chunk, size_t* bytes) {
     if (!kv || !bytes || chunk < 1) return DUO_ERR_INVALID_ARG;
-    *bytes = 0;   // the prefill kernel keeps all its state on chip
+    *bytes = prefill_ws(kv, chunk);
     return DUO_OK;
 }
 
 int duo_prefill_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const uint16_t* k_chunk,
                      const uint16_t* v_chunk, const int32_t* prefix_len, int32_t chunk, float scale,
                      float* out, void* workspace, size_t workspace_bytes, duo_stream_t stream) {
-    (void)workspace;
-    (void)workspace_bytes;
     if (!kv || layer < 0 || layer >= kv->desc.num_layers || !q || !k_chunk || !v_chunk || !prefix_len ||
         !out || chunk < 1)
         return DUO_ERR_INVALID_ARG;
@@ -254,13 +262,15 @@ int duo_prefill_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const uint16_
     if (!aligned16(q) || !aligned16(k_chunk) || !aligned16(v_chunk) || !aligned16(out) ||
         (reinterpret_cast<uintptr_t>(prefix_len) & 3))
         return DUO_ERR_ALIGNMENT;
+    if (!workspace || workspace_bytes < prefill_ws(kv, chunk)) return DUO_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return DUO_ERR_ALIGNMENT;
     const duo::LayerLayout& L = kv->layers[layer];
     const int64_t SW = int64_t(d.sink) + d.window;
     // tile coordinates are 32-bit row indices
     const int64_t rows_max = std::max({int64_t(d.batch) * d.num_q_heads * chunk,
                                        int64_t(d.batch) * d.num_kv_heads * chunk,
-                                       int64_t(d.batch) * L.n_r * d.capacity + 128,
-                                       int64_t(d.batch) * L.n_s * SW + 128});
+                                       int64_t(d.batch) * L.n_r * (d.capacity + 256),
+                                       int64_t(d.batch) * L.n_s * (SW + 256)});
     if (rows_max >= (int64_t(1) << 31)) return DUO_ERR_UNSUPPORTED;
     duo::PrefillLaunch a;
     a.q = q;
@@ -271,8 +281,8 @@ int duo_prefill_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const uint16_
     a.ks = kv->base + L.off_ks;
     a.vs = kv->base + L.off_vs;
     a.prefix = prefix_len;
-    a.pos = reinterpret_cast<const int32_t*>(kv->base + L.off_pos);
     a.out = out;
+    a.workspace = workspace;
     a.status = kv->status;
     a.cap = d.capacity;
     a.B = d.batch;

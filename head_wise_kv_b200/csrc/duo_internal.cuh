@@ -86,9 +86,9 @@ struct PrefillLaunch {
     const void* ks;
     const void* vs;
     const int32_t* prefix;
-    const int32_t* pos;
     float* out;
     int32_t* status;
+    void* workspace;        // fp16 value copies, prefill_workspace_bytes(...) bytes
     int64_t cap;
     int B, hq, n_kv, C, S, W, n_r, n_s;
     float scale;
@@ -103,6 +103,7 @@ int decode_ctas_default(int num_sms, int d, int group);
 size_t decode_workspace_bytes(int slots, int d, int group);
 cudaError_t launch_decode(const DecodeParams& p, int d, int group, cudaStream_t s);
 size_t prefill_smem_bytes(int S, int W);
+size_t prefill_workspace_bytes(int B, int n_kv, int n_r, int n_s, int64_t cap, int S, int W, int C);
 int launch_prefill(const PrefillLaunch& a, cudaStream_t s);   // returns a DUO_* code
 
 // ----------------------------------------------------------------- device helpers

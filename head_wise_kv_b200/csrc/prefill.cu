@@ -11,21 +11,26 @@
 // guide: dense attention for retrieval heads, a block-sparse sliding-window
 // kernel for streaming heads).
 //
-// One CTA = one (sequence, query head, 128-row query tile); 12 warps:
-//   warp 0     TMA producer: Q once, then K/V tiles (128 keys x 128 dims, two
-//              128-byte-swizzled slabs each) into a 2-stage ring
-//   warp 1     allocates TMEM; one lane issues tcgen05.mma:
-//                S_j = Q K_j^T   (bf16 x bf16 -> fp32, M=N=128, 8 x K16)
-//                O  += P_j V_j   (fp16 x fp16 -> fp32, V MN-major)
-//              S is double-buffered in TMEM so S_{j+1} overlaps softmax_j
-//   warps 2-3  convert each V tile in place bf16 -> fp16 (exact for
-//              |v| < 65504) and zero key rows past the valid range
-//   warps 4-11 softmax, two threads per query row (TMEM lane = row, one
-//              64-key half each): masked scores, running max with lazy
-//              rescaling (O is rescaled only when the max grows by more than
-//              2^8), P_j as fp16 into a swizzled shared tile, final O / l.
-// P is fp16 rather than bf16: rounding P to bf16 alone costs ~1e-3 relative
-// error in the output, fp16 ~1.5e-4.
+// Two launches per call:
+//  1. convert_v_kernel writes an fp16 copy of every V row the attention can
+//     read (cached prefix, ring slots, the chunk) into the caller's workspace,
+//     zeroing tile tails.  P is multiplied in fp16 rather than bf16 (rounding
+//     P to bf16 alone costs ~1.5e-3 relative error in the output, fp16
+//     ~2e-4), and one tcgen05 MMA needs both operands in the same type; this
+//     way each V row is converted once per call instead of once per CTA.
+//  2. prefill_kernel, one CTA per (sequence, query head, 128-row query tile),
+//     11 warps:
+//       warp 0      TMA: Q once, then K tiles (bf16, 128 keys x 128 dims as
+//                   two 128-byte-swizzled slabs) into a 3-stage ring
+//       warp 1      allocates TMEM; one lane issues tcgen05.mma:
+//                     S_j  = Q K_j^T  (bf16, SS form, M = N = 128, 8 x K16)
+//                     O   += P_j V_j  (fp16, TS form: P from TMEM, V MN-major)
+//                   S is double-buffered in TMEM so S_{j+1} overlaps softmax_j
+//       warp 2      TMA: fp16 V tiles into a 2-stage ring
+//       warps 3-10  softmax, two threads per query row (TMEM lane = row, one
+//                   64-key half each): masked scores, running max with lazy
+//                   rescaling (O rescaled only when the max grows by more
+//                   than 2^8), P_j as packed fp16 written to TMEM, O / l.
 //
 // Every mbarrier wait is bounded; on a timeout the CTA sets
 // DUO_STATUS_WAIT_TIMEOUT, stops, waits (bounded) for its own copies and
@@ -35,6 +40,7 @@
 #include <cuda_runtime.h>
 #include <math_constants.h>
 #include <stdint.h>
+#include <string.h>
 
 #include "duo_internal.cuh"
 
@@ -45,11 +51,13 @@ namespace {
 constexpr int kBM = 128;   // query rows per CTA
 constexpr int kBN = 128;   // keys per tile
 constexpr int kHD = 128;   // head dim (prefill is built for d = 128)
-constexpr int kThreads = 384;   // 12 warps: TMA, MMA, 2 V converters, 8 softmax
-constexpr uint32_t kSlab = 128 * 128;        // bytes: 128 rows x 64 bf16
-constexpr uint32_t kTile = 2 * kSlab;        // 32 KB: 128 rows x 128 bf16
+constexpr int kThreads = 352;   // 11 warps: K TMA, MMA, V TMA, 8 softmax
+constexpr int kSoftmaxWarp0 = 3;
+constexpr int kKStages = 3, kVStages = 2;
+constexpr uint32_t kSlab = 128 * 128;        // bytes: 128 rows x 64 16-bit elements
+constexpr uint32_t kTile = 2 * kSlab;        // 32 KB: 128 rows x 128 16-bit elements
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO = 256;
+constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO = 256, kTmemP = 384;
 constexpr float kNegBig = -1.0e30f;
 constexpr float kRescaleThreshold = 8.0f;    // log2 units
 
@@ -63,15 +71,29 @@ constexpr uint32_t kIdescPV = (1u << 4) | (0u << 7) | (0u << 10) | (1u << 16) | 
                               (uint32_t(kBM >> 4) << 24);
 
 struct PrefillParams {
-    CUtensorMap tm_q, tm_kc, tm_vc, tm_kr, tm_vr, tm_ks, tm_vs;
+    CUtensorMap tm_q, tm_kc, tm_kr, tm_ks;      // bf16: queries, chunk / retrieval / ring keys
+    CUtensorMap tm_vc, tm_vr, tm_vs;            // fp16 copies of the values (workspace)
     const int32_t* prefix;
-    const int32_t* pos;     // this layer's [B][S+W] position table
     float* out;
     int32_t* status;
     int64_t cap;
-    int B, hq, n_kv, G, C, n_qt, S, W, n_r, n_s;
+    int B, hq, n_kv, G, C, n_qt, S, W, n_r, n_s, LR, LS;
     float scale_log2;
     unsigned long long timeout_ns;
+    int32_t rank[kMaxKvHeads];
+    uint8_t is_r[kMaxKvHeads];
+};
+
+struct ConvertParams {
+    const uint16_t* vr;     // bf16 caches and chunk
+    const uint16_t* vs;
+    const uint16_t* vc;
+    uint16_t* v16r;         // fp16 copies: [B][n_r][LR][d], [B][n_s][LS][d], [B][n_kv][C][d]
+    uint16_t* v16s;
+    uint16_t* v16c;
+    const int32_t* prefix;
+    int64_t cap;
+    int B, n_kv, n_r, n_s, S, W, C, LR, LS;
     int32_t rank[kMaxKvHeads];
     uint8_t is_r[kMaxKvHeads];
 };
@@ -103,7 +125,6 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
@@ -148,6 +169,17 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
 __device__ __forceinline__ void tma_tile(uint32_t dst, const CUtensorMap* map, int row, uint32_t bar) {
     tma_load_2d(dst, map, 0, row, bar);
     tma_load_2d(dst + kSlab, map, 64, row, bar);
+}
+
+// O += P V with A = P read from TMEM (TS form), B = V from shared memory.
+__device__ __forceinline__ void umma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(tmem_d), "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
 }
 
 // ------------------------------------------------------------------ key tiles
@@ -276,19 +308,64 @@ __device__ __forceinline__ bool softmax_barrier_any(bool flag) {
     return out != 0;
 }
 
+// ------------------------------------------------------------------ V -> fp16
+// One thread per 16-byte piece (8 values).  blockIdx.y = b * n_kv + g;
+// blockIdx.z = 0: the head's cached rows, 1: its chunk rows.  Rows that hold
+// no key (past the prefix or the filled ring slots) up to the end of the
+// last tile the attention reads are written as zeros, so masked columns
+// always meet finite values.
+__global__ void __launch_bounds__(256) convert_v_kernel(const __grid_constant__ ConvertParams c) {
+    const int bg = blockIdx.y;
+    const int b = bg / c.n_kv, g = bg % c.n_kv;
+    const int P = max(c.prefix[b], 0);
+    const uint16_t* src;
+    uint16_t* dst;
+    int64_t n_conv, n_rows;
+    if (blockIdx.z == 1) {
+        src = c.vc + size_t(bg) * c.C * kHD;
+        dst = c.v16c + size_t(bg) * c.C * kHD;
+        n_conv = n_rows = c.C;
+    } else if (c.is_r[g]) {
+        const size_t r = size_t(b) * c.n_r + c.rank[g];
+        src = c.vr + r * size_t(c.cap) * kHD;
+        dst = c.v16r + r * size_t(c.LR) * kHD;
+        n_conv = min(int64_t(P), c.cap);
+        n_rows = (n_conv + kBN - 1) / kBN * kBN;          // tail of the last prefix tile
+    } else {
+        const size_t r = size_t(b) * c.n_s + c.rank[g];
+        src = c.vs + r * size_t(c.S + c.W) * kHD;
+        dst = c.v16s + r * size_t(c.LS) * kHD;
+        n_conv = min(P, c.S + c.W);                         // filled slots
+        n_rows = c.LS;
+    }
+    const int64_t pieces = n_rows * (kHD / 8);
+    for (int64_t x = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; x < pieces;
+         x += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t row = x / (kHD / 8);
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (row < n_conv) {
+            const uint4 w = *reinterpret_cast<const uint4*>(src + x * 8);
+            const float2 a = bf2_to_f2(w.x), bb = bf2_to_f2(w.y), cc = bf2_to_f2(w.z), dd = bf2_to_f2(w.w);
+            v.x = pack_half2(a.x, a.y);
+            v.y = pack_half2(bb.x, bb.y);
+            v.z = pack_half2(cc.x, cc.y);
+            v.w = pack_half2(dd.x, dd.y);
+        }
+        *reinterpret_cast<uint4*>(dst + x * 8) = v;
+    }
+}
+
+// ------------------------------------------------------------------ attention
 __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_constant__ PrefillParams p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sQ = smem_addr(smem);
-    const uint32_t sK0 = sQ + kTile, sK1 = sQ + 2 * kTile;
-    const uint32_t sV0 = sQ + 3 * kTile, sV1 = sQ + 4 * kTile;
-    const uint32_t sP = sQ + 5 * kTile;
-    unsigned char* sP_gen = smem + 5 * kTile;
-    unsigned char* sV_gen0 = smem + 3 * kTile;
+    const uint32_t sK = sQ + kTile;                    // kKStages tiles
+    const uint32_t sV = sK + kKStages * kTile;         // kVStages tiles
 
-    __shared__ __align__(8) uint64_t bar_q, kv_full[2], kv_empty[2], v_conv[2], s_full[2], s_free[2], p_full,
-        o_done, mma_fin;
+    __shared__ __align__(8) uint64_t bar_q, k_full[kKStages], k_empty[kKStages], v_full[kVStages],
+        v_empty[kVStages], s_full[2], s_free[2], p_full, o_done, mma_fin;
     __shared__ uint32_t tmem_base_sh;
     __shared__ float red_max[2][2][kBM];   // [tile parity][column half][row]
     __shared__ float red_l[2][kBM];        // [column half][row] final row sums
@@ -311,10 +388,15 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
 
     if (threadIdx.x == 0) {
         mbar_init(smem_addr(&bar_q), 1);
+        for (int s = 0; s < kKStages; ++s) {
+            mbar_init(smem_addr(&k_full[s]), 1);
+            mbar_init(smem_addr(&k_empty[s]), 1);
+        }
+        for (int s = 0; s < kVStages; ++s) {
+            mbar_init(smem_addr(&v_full[s]), 1);
+            mbar_init(smem_addr(&v_empty[s]), 1);
+        }
         for (int s = 0; s < 2; ++s) {
-            mbar_init(smem_addr(&kv_full[s]), 1);
-            mbar_init(smem_addr(&kv_empty[s]), 1);
-            mbar_init(smem_addr(&v_conv[s]), 2);
             mbar_init(smem_addr(&s_full[s]), 1);
             mbar_init(smem_addr(&s_free[s]), 8);
         }
@@ -336,43 +418,48 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base_sh;
-
     const int kv_rank = p.rank[g];
-    const int SW = p.S + p.W;
 
-    if (warp == 0) {
-        // ============================================================ TMA producer
+    if (warp == 0 || warp == 2) {
+        // ============================================================ TMA producers
         if (lane == 0) {
-            mbar_arrive_expect_tx(smem_addr(&bar_q), kTile);
-            tma_tile(sQ, &p.tm_q, (b * p.hq + h) * p.C + i0, smem_addr(&bar_q));
+            const bool is_k = warp == 0;
+            const int stages = is_k ? kKStages : kVStages;
+            uint64_t* full = is_k ? k_full : v_full;
+            uint64_t* empty = is_k ? k_empty : v_empty;
+            const uint32_t base = is_k ? sK : sV;
+            if (is_k) {
+                mbar_arrive_expect_tx(smem_addr(&bar_q), kTile);
+                tma_tile(sQ, &p.tm_q, (b * p.hq + h) * p.C + i0, smem_addr(&bar_q));
+            }
             int issued = 0;
             for (int j = 0; j < plan.n; ++j) {
-                const int st = j & 1;
-                if (!timed_wait(smem_addr(&kv_empty[st]), ((j >> 1) & 1) ^ 1, p, abort_flag)) break;
+                const int st = j % stages;
+                if (!timed_wait(smem_addr(&empty[st]), ((j / stages) & 1) ^ 1, p, abort_flag)) break;
                 const KeyTile kt = plan.get(j);
-                const CUtensorMap *mk, *mv;
+                const CUtensorMap* map;
                 int row;
                 if (kt.src == kSrcCache) {
-                    mk = &p.tm_kr; mv = &p.tm_vr;
-                    row = int((int64_t(b) * p.n_r + kv_rank) * p.cap + kt.row0);
+                    map = is_k ? &p.tm_kr : &p.tm_vr;
+                    row = int((int64_t(b) * p.n_r + kv_rank) * (is_k ? p.cap : int64_t(p.LR)) + kt.row0);
                 } else if (kt.src == kSrcChunk) {
-                    mk = &p.tm_kc; mv = &p.tm_vc;
+                    map = is_k ? &p.tm_kc : &p.tm_vc;
                     row = (b * p.n_kv + g) * p.C + kt.row0;
                 } else {
-                    mk = &p.tm_ks; mv = &p.tm_vs;
-                    row = (b * p.n_s + kv_rank) * SW + (kt.src == kSrcWindow ? p.S : 0) + kt.row0;
+                    map = is_k ? &p.tm_ks : &p.tm_vs;
+                    row = (b * p.n_s + kv_rank) * (is_k ? p.S + p.W : p.LS) + (kt.src == kSrcWindow ? p.S : 0) +
+                          kt.row0;
                 }
-                const uint32_t bar = smem_addr(&kv_full[st]);
-                mbar_arrive_expect_tx(bar, 2 * kTile);
-                tma_tile(st ? sK1 : sK0, mk, row, bar);
-                tma_tile(st ? sV1 : sV0, mv, row, bar);
+                const uint32_t bar = smem_addr(&full[st]);
+                mbar_arrive_expect_tx(bar, kTile);
+                tma_tile(base + st * kTile, map, row, bar);
                 ++issued;
             }
             // do not leave while copies may still land in this CTA's shared memory
-            mbar_wait(smem_addr(&bar_q), 0, p.timeout_ns);
-            for (int k = 0; k < 2 && k < issued; ++k) {
+            if (is_k) mbar_wait(smem_addr(&bar_q), 0, p.timeout_ns);
+            for (int k = 0; k < stages && k < issued; ++k) {
                 const int j = issued - 1 - k;
-                mbar_wait(smem_addr(&kv_full[j & 1]), (j >> 1) & 1, p.timeout_ns);
+                mbar_wait(smem_addr(&full[j % stages]), (j / stages) & 1, p.timeout_ns);
             }
         }
     } else if (warp == 1) {
@@ -381,78 +468,54 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             bool ok = timed_wait(smem_addr(&bar_q), 0, p, abort_flag);
             tc_fence_after();
             auto issue_s = [&](int j) -> bool {
-                const int st = j & 1;
-                if (!timed_wait(smem_addr(&kv_full[st]), (j >> 1) & 1, p, abort_flag)) return false;
-                if (!timed_wait(smem_addr(&s_free[st]), ((j >> 1) & 1) ^ 1, p, abort_flag)) return false;
+                const int ks = j % kKStages, sb = j & 1;
+                if (!timed_wait(smem_addr(&k_full[ks]), (j / kKStages) & 1, p, abort_flag)) return false;
+                if (!timed_wait(smem_addr(&s_free[sb]), ((j >> 1) & 1) ^ 1, p, abort_flag)) return false;
                 tc_fence_after();
-                const uint32_t sk = st ? sK1 : sK0;
+                const uint32_t sk = sK + ks * kTile;
 #pragma unroll
                 for (int k = 0; k < kHD / 16; ++k) {
                     const uint32_t off = (k >> 2) * kSlab + (k & 3) * 32;
-                    umma_f16(tmem + (st ? kTmemS1 : kTmemS0), smem_desc(sQ + off, 16, 1024),
+                    umma_f16(tmem + (sb ? kTmemS1 : kTmemS0), smem_desc(sQ + off, 16, 1024),
                              smem_desc(sk + off, 16, 1024), kIdescQK, k > 0);
                 }
-                umma_commit(smem_addr(&s_full[st]));
+                umma_commit(smem_addr(&s_full[sb]));
+                umma_commit(smem_addr(&k_empty[ks]));
                 return true;
             };
             if (ok) ok = issue_s(0);
             for (int j = 0; ok && j < plan.n; ++j) {
                 if (j + 1 < plan.n && !issue_s(j + 1)) { ok = false; break; }
+                const int vs = j % kVStages;
                 if (!timed_wait(smem_addr(&p_full), j & 1, p, abort_flag)) { ok = false; break; }
-                if (!timed_wait(smem_addr(&v_conv[j & 1]), (j >> 1) & 1, p, abort_flag)) { ok = false; break; }
+                if (!timed_wait(smem_addr(&v_full[vs]), (j / kVStages) & 1, p, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t sv = (j & 1) ? sV1 : sV0;
+                const uint32_t sv = sV + vs * kTile;
 #pragma unroll
                 for (int k = 0; k < kBN / 16; ++k) {
-                    umma_f16(tmem + kTmemO, smem_desc(sP + (k >> 2) * kSlab + (k & 3) * 32, 16, 1024),
-                             smem_desc(sv + k * 2048, kSlab, 1024), kIdescPV, (j > 0 || k > 0) ? 1u : 0u);
+                    // A = P_j columns [8k, 8k+8) of the TMEM P region (16 keys, fp16 pairs)
+                    umma_f16_ts(tmem + kTmemO, tmem + kTmemP + k * 8, smem_desc(sv + k * 2048, kSlab, 1024),
+                                kIdescPV, (j > 0 || k > 0) ? 1u : 0u);
                 }
-                umma_commit(smem_addr(&kv_empty[j & 1]));
+                umma_commit(smem_addr(&v_empty[vs]));
                 umma_commit(smem_addr(&o_done));
             }
             // all MMAs issued by this thread have completed before TMEM is freed
             umma_commit(smem_addr(&mma_fin));
             mbar_wait(smem_addr(&mma_fin), 0, p.timeout_ns);
         }
-    } else if (warp < 4) {
-        // ============================================================ V converter
-        const int t = threadIdx.x - 64;   // 0..63
-        for (int j = 0; j < plan.n; ++j) {
-            const int st = j & 1;
-            if (!timed_wait(smem_addr(&kv_full[st]), (j >> 1) & 1, p, abort_flag)) break;
-            const int nvalid = plan.get(j).nvalid;
-            uint4* v = reinterpret_cast<uint4*>(sV_gen0 + st * kTile);
-#pragma unroll 4
-            for (int c = t; c < int(kTile / 16); c += 64) {
-                const int row = (c % (kSlab / 16)) / 8;   // 8 chunks of 16 B per 128-byte row
-                uint4 x = v[c];
-                if (row >= nvalid) {
-                    x = make_uint4(0, 0, 0, 0);
-                } else {
-                    const float2 a = bf2_to_f2(x.x), bb = bf2_to_f2(x.y), cc = bf2_to_f2(x.z), dd = bf2_to_f2(x.w);
-                    x.x = pack_half2(a.x, a.y);
-                    x.y = pack_half2(bb.x, bb.y);
-                    x.z = pack_half2(cc.x, cc.y);
-                    x.w = pack_half2(dd.x, dd.y);
-                }
-                v[c] = x;
-            }
-            fence_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&v_conv[st]));
-        }
     } else {
         // ============================================================ softmax
         // 8 warps, two per scheduler: warp w owns the TMEM lane quarter w % 4
         // (32 query rows) and the column half hf of every S tile (64 keys), of
-        // the P tile (one swizzled slab) and of O (64 dims).  The two halves of
-        // a row agree on the tile maximum through shared memory once per tile.
+        // the P tile (32 TMEM columns of fp16 pairs) and of O (64 dims).  The
+        // two halves of a row agree on the tile maximum once per tile.
         const int wq = warp & 3;
-        const int hf = (warp - 4) >> 2;
+        const int hf = (warp - kSoftmaxWarp0) >> 2;
         const int r = wq * 32 + lane;            // query row within the tile
         const int i = i0 + r;                    // chunk row
         const int tpos = plan.P + i;             // absolute position
-        const int cb = hf * 64;                  // first key column of this half
+        const int cb = hf * 64;                  // first key column (and O dim) of this half
         const uint32_t lane_off = uint32_t(wq * 32) << 16;
         float m = kNegBig, l = 0.f;
         bool ok = true;
@@ -535,17 +598,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             }
             l = l * alpha + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
             m = m_new;
-            // P_j reuses the shared tile of P_{j-1}, and a rescale touches O:
-            // both need PV_{j-1} to have completed.
+            // P_j overwrites P_{j-1} in TMEM, and a rescale touches O: both
+            // need PV_{j-1} to have completed.
             if (j > 0) {
                 if (!warp_wait(smem_addr(&o_done), (j - 1) & 1, p, abort_flag)) continue;   // next barrier exits
                 tc_fence_after();
             }
-            // this half of the P row: slab hf of the 128-byte swizzled K-major tile
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch)
-                *reinterpret_cast<uint4*>(sP_gen + hf * kSlab + r * 128 + ((ch ^ (r & 7)) * 16)) =
-                    make_uint4(ph[ch * 4 + 0], ph[ch * 4 + 1], ph[ch * 4 + 2], ph[ch * 4 + 3]);
+            tmem_st32(tmem + lane_off + kTmemP + hf * 32, *reinterpret_cast<const uint32_t(*)[32]>(ph));
             if (j > 0 && __any_sync(0xffffffffu, grow)) {
 #pragma unroll 1
                 for (int c = 0; c < 2; ++c) {
@@ -557,9 +616,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                     for (int x = 0; x < 32; ++x) u[x] = __float_as_uint(__uint_as_float(u[x]) * alpha);
                     tmem_st32(ta, u);
                 }
-                tmem_wait_st();
             }
-            fence_async_smem();
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_addr(&p_full));
@@ -616,51 +674,88 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2-D bf16 map over `rows` rows of 128 elements; box 64 x 128 rows, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows) {
+// 2-D map of 16-bit elements over `rows` rows of 128; box 64 x 128 rows, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, CUtensorMapDataType type) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     cuuint64_t dims[2] = {uint64_t(kHD), rows < 1 ? 1 : rows};
     cuuint64_t strides[1] = {uint64_t(kHD) * 2};
     cuuint32_t box[2] = {64, 128};
     cuuint32_t estr[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    return enc(m, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Rows per head of the fp16 value copies (whole tiles plus one spare tile).
+int rows_r(int64_t cap) { return int((cap + kBN - 1) / kBN * kBN + kBN); }
+int rows_s(int S, int W) { return (S + W + kBN - 1) / kBN * kBN + kBN; }
 
 }  // namespace
 
 size_t prefill_smem_bytes(int S, int W) {
     (void)S;
     (void)W;
-    return 6 * size_t(kTile) + 1024;
+    return (1 + kKStages + kVStages) * size_t(kTile) + 1024;
+}
+
+size_t prefill_workspace_bytes(int B, int n_kv, int n_r, int n_s, int64_t cap, int S, int W, int C) {
+    const size_t row = size_t(kHD) * 2;
+    return align256(size_t(B) * n_r * rows_r(cap) * row) + align256(size_t(B) * n_s * rows_s(S, W) * row) +
+           align256(size_t(B) * n_kv * C * row);
 }
 
 int launch_prefill(const PrefillLaunch& a, cudaStream_t s) {
+    const int LR = rows_r(a.cap), LS = rows_s(a.S, a.W);
+    const size_t row = size_t(kHD) * 2;
+    char* ws = static_cast<char*>(a.workspace);
+    uint16_t* v16r = reinterpret_cast<uint16_t*>(ws);
+    uint16_t* v16s = reinterpret_cast<uint16_t*>(ws + align256(size_t(a.B) * a.n_r * LR * row));
+    uint16_t* v16c = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(v16s) +
+                                                 align256(size_t(a.B) * a.n_s * LS * row));
+
     PrefillParams p;
     memset(&p, 0, sizeof p);
     const int SW = a.S + a.W;
-    if (!make_map(&p.tm_q, a.q, uint64_t(a.B) * a.hq * a.C) ||
-        !make_map(&p.tm_kc, a.k_chunk, uint64_t(a.B) * a.n_kv * a.C) ||
-        !make_map(&p.tm_vc, a.v_chunk, uint64_t(a.B) * a.n_kv * a.C) ||
-        !make_map(&p.tm_kr, a.kr, uint64_t(a.B) * a.n_r * a.cap) ||
-        !make_map(&p.tm_vr, a.vr, uint64_t(a.B) * a.n_r * a.cap) ||
-        !make_map(&p.tm_ks, a.ks, uint64_t(a.B) * a.n_s * SW) ||
-        !make_map(&p.tm_vs, a.vs, uint64_t(a.B) * a.n_s * SW))
+    const CUtensorMapDataType BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, F16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    if (!make_map(&p.tm_q, a.q, uint64_t(a.B) * a.hq * a.C, BF) ||
+        !make_map(&p.tm_kc, a.k_chunk, uint64_t(a.B) * a.n_kv * a.C, BF) ||
+        !make_map(&p.tm_kr, a.kr, uint64_t(a.B) * a.n_r * a.cap, BF) ||
+        !make_map(&p.tm_ks, a.ks, uint64_t(a.B) * a.n_s * SW, BF) ||
+        !make_map(&p.tm_vc, v16c, uint64_t(a.B) * a.n_kv * a.C, F16) ||
+        !make_map(&p.tm_vr, v16r, uint64_t(a.B) * a.n_r * LR, F16) ||
+        !make_map(&p.tm_vs, v16s, uint64_t(a.B) * a.n_s * LS, F16))
         return DUO_ERR_CUDA;
     p.prefix = a.prefix;
-    p.pos = a.pos;
     p.out = a.out;
     p.status = a.status;
     p.cap = a.cap;
     p.B = a.B; p.hq = a.hq; p.n_kv = a.n_kv; p.G = a.hq / a.n_kv; p.C = a.C;
     p.n_qt = (a.C + kBM - 1) / kBM;
-    p.S = a.S; p.W = a.W; p.n_r = a.n_r; p.n_s = a.n_s;
+    p.S = a.S; p.W = a.W; p.n_r = a.n_r; p.n_s = a.n_s; p.LR = LR; p.LS = LS;
     p.scale_log2 = a.scale * 1.4426950408889634f;
     p.timeout_ns = a.timeout_ns;
     memcpy(p.rank, a.rank, sizeof p.rank);
     memcpy(p.is_r, a.is_r, sizeof p.is_r);
+
+    ConvertParams c;
+    memset(&c, 0, sizeof c);
+    c.vr = static_cast<const uint16_t*>(a.vr);
+    c.vs = static_cast<const uint16_t*>(a.vs);
+    c.vc = static_cast<const uint16_t*>(a.v_chunk);
+    c.v16r = v16r; c.v16s = v16s; c.v16c = v16c;
+    c.prefix = a.prefix;
+    c.cap = a.cap;
+    c.B = a.B; c.n_kv = a.n_kv; c.n_r = a.n_r; c.n_s = a.n_s; c.S = a.S; c.W = a.W; c.C = a.C;
+    c.LR = LR; c.LS = LS;
+    memcpy(c.rank, a.rank, sizeof c.rank);
+    memcpy(c.is_r, a.is_r, sizeof c.is_r);
+    if (int64_t(a.B) * a.n_kv > 65535) return DUO_ERR_UNSUPPORTED;
+    convert_v_kernel<<<dim3(64, unsigned(a.B * a.n_kv), 2), 256, 0, s>>>(c);
+    if (cudaGetLastError() != cudaSuccess) return DUO_ERR_CUDA;
+
     const size_t smem = prefill_smem_bytes(a.S, a.W);
     cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return DUO_ERR_CUDA;

@@ -211,22 +211,29 @@ DUO_API int duo_decode_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const 
 DUO_API int duo_decode_attn_static_ws(duo_kv* kv, int32_t layer, const uint16_t* q, const int32_t* len,
                                       float scale, float* out, float* lse, duo_stream_t stream);
 
-/* Workspace bytes duo_prefill_attn needs for chunks of up to `chunk` rows. */
+/* Workspace bytes duo_prefill_attn needs for chunks of up to `chunk` rows
+ * (host only): fp16 copies of the values one call reads -- the retrieval
+ * heads' cached rows, the streaming rings and the chunk. */
 DUO_API int duo_prefill_workspace_bytes(const duo_kv* kv, int32_t chunk, size_t* bytes);
 
 /* Chunked-prefill attention for one layer (before the chunk is appended).
  *   q:          [B][Hq][chunk][d] bf16, rows at positions prefix[b] + i;
  *   k_chunk, v_chunk: [B][n_kv][chunk][d] bf16, the chunk's own keys/values;
  *   prefix_len: device int32 [B], tokens already in the cache (P);
- *   out:        [B][Hq][chunk][d] fp32.
+ *   out:        [B][Hq][chunk][d] fp32;
+ *   workspace:  device scratch of >= duo_prefill_workspace_bytes(kv, chunk)
+ *               bytes, 256-byte aligned (no initialisation; calls that may
+ *               overlap must not share it).
  * Row i reads keys at positions j <= P + i ("Attention Variants and
  * KV-Cache Compression", "When Is Reuse Exact?"): retrieval heads all of
  * them (prefix from the cache, the rest from k_chunk); streaming heads only
  * j < S or j >= P + i - W + 1 (the sinks and the window, read from the ring
  * and from k_chunk).  The DuoAttention guide's "Hardware-Fused Prefill":
  * dense causal attention for retrieval heads, block-sparse sink + local
- * attention for streaming heads.  Requirements: chunk >= 1; for streaming
- * heads prefix_len[b] must equal the tokens appended so far. */
+ * attention for streaming heads.  Products of probabilities and values run
+ * in fp16 (fp32 accumulation), so |v| must stay below 65504.  Requirements:
+ * head_dim 128 (else UNSUPPORTED); chunk >= 1; prefix_len[b] must equal the
+ * tokens appended so far (the ring state is derived from it). */
 DUO_API int duo_prefill_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const uint16_t* k_chunk,
                      const uint16_t* v_chunk, const int32_t* prefix_len, int32_t chunk,
                      float scale, float* out, void* workspace, size_t workspace_bytes,
