@@ -46,6 +46,9 @@ constexpr int kConsumerWarps = 7;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kBlk = 16;         // partition granularity in tokens
 constexpr float kNegBig = -1.0e30f;   // finite "minus infinity" for running maxima
+constexpr float kRescaleThreshold = 8.0f;   // log2 units: probabilities stay <= 2^8
+
+constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x >> 1); }
 
 template <int D, int G>
 struct Cfg {
@@ -58,6 +61,14 @@ struct Cfg {
     static constexpr int RED_STRIDE = D + 4;                     // floats; keeps float4 alignment
     static constexpr int RED_FLOATS = kConsumerWarps * G * RED_STRIDE;
     static constexpr size_t SMEM = size_t(2) * kStages * STAGE_BYTES + RED_FLOATS * 4 + 1024;
+    // reduce-scatter of the V = STEPS * G partial dot products of one tile
+    // over the LPT lanes of a token group: RS halving rounds leave KEEP
+    // complete scores per lane (all-reduce rounds finish when V < LPT)
+    static constexpr int V = STEPS * G;
+    static constexpr int LOG_LPT = ilog2(LPT);
+    static constexpr int LOG_V = ilog2(V);
+    static constexpr int RS = LOG_V < LOG_LPT ? LOG_V : LOG_LPT;
+    static constexpr int KEEP = V >> RS;
     static_assert(STEPS * TPW * kConsumerWarps == kTile, "tile must be whole warp steps");
     static_assert(STAGE_BYTES % 1024 == 0, "stage buffers stay 1024-byte aligned");
 };
@@ -149,6 +160,54 @@ __device__ __forceinline__ Piece locate(const DecodeParams& p, const int32_t* bp
     pc.tok1 = t1 < rows ? t1 : rows;
     pc.whole = (gb == pc.seg_gb) && (pc.end_gb == seg_end);
     return pc;
+}
+
+// First of the KEEP score indices (step * G + head) lane li of its token group
+// holds after the reduce-scatter.
+template <class C>
+__device__ __forceinline__ int rs_first(int li) {
+    int lo = 0;
+#pragma unroll
+    for (int k = 0; k < C::RS; ++k)
+        if (li & (C::LPT >> (k + 1))) lo += C::V >> (k + 1);
+    return lo;
+}
+
+// Lane (within the token group) holding score index v after the reduce-scatter.
+template <class C>
+__host__ __device__ constexpr int rs_lane(int v) {
+    int lane = 0;
+    const int base = v - v % C::KEEP;
+    for (int k = 0; k < C::RS; ++k)
+        if ((base >> (C::LOG_V - 1 - k)) & 1) lane += C::LPT >> (k + 1);
+    return lane;
+}
+
+// Sum x[0..V) over the LPT lanes of each token group; lane li keeps the
+// complete values of indices rs_first(li) .. + KEEP in x[0..KEEP).
+template <class C>
+__device__ __forceinline__ void reduce_scatter(float (&x)[C::V], int li) {
+#pragma unroll
+    for (int k = 0; k < C::RS; ++k) {
+        const int o = C::LPT >> (k + 1);
+        const int half = C::V >> (k + 1);
+        const bool upper = (li & o) != 0;
+#pragma unroll
+        for (int i = 0; i < half; ++i) {
+            const float send = upper ? x[i] : x[half + i];
+            const float keep = upper ? x[half + i] : x[i];
+            x[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+#pragma unroll
+    for (int k = C::RS; k < C::LOG_LPT; ++k) x[0] += __shfl_xor_sync(0xffffffffu, x[0], C::LPT >> (k + 1));
+}
+
+// Every lane of a token group receives all V values the group holds.
+template <class C>
+__device__ __forceinline__ void gather_group(const float (&held)[C::KEEP], float (&all)[C::V], int group_lane0) {
+#pragma unroll
+    for (int v = 0; v < C::V; ++v) all[v] = __shfl_sync(0xffffffffu, held[v % C::KEEP], group_lane0 + rs_lane<C>(v));
 }
 
 template <int D>
@@ -254,6 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     uint32_t it = 0;
     bool aborted = false;
     const uint32_t sK0 = smem_addr(sK), sV0 = smem_addr(sV);
+    const int lo_idx = rs_first<C>(li);   // first (step * G + head) score this lane owns
 
     for (int64_t gb = gb_begin; gb < gb_end;) {
         const Piece pc = locate(p, bpre, gb, gb_end);
@@ -276,6 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
         float2 o2[G][C::NCL * 4];
         float m[G], l[G];
+        float mv[C::KEEP];   // m of the head of each score this lane owns
 #pragma unroll
         for (int h = 0; h < G; ++h) {
             m[h] = kNegBig;
@@ -283,6 +344,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 #pragma unroll
             for (int j = 0; j < C::NCL * 4; ++j) o2[h][j] = make_float2(0.f, 0.f);
         }
+#pragma unroll
+        for (int e = 0; e < C::KEEP; ++e) mv[e] = kNegBig;
 
         for (int64_t t = pc.tok0; t < pc.tok1 && !aborted; t += kTile, ++it) {
             const int rows = int(pc.tok1 - t < kTile ? pc.tok1 - t : kTile);
@@ -303,7 +366,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             const uint32_t kbase = sK0 + st * C::STAGE_BYTES;
             const uint32_t vbase = sV0 + st * C::STAGE_BYTES;
 
-            float sc[C::STEPS][G];
+            // partial dot products of this lane's dims, all steps and heads
+            float x[C::V];
 #pragma unroll
             for (int s = 0; s < C::STEPS; ++s) {
                 const int row = (s * kConsumerWarps + warp) * C::TPW + grp;
@@ -324,33 +388,56 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                     }
                 }
 #pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    float x = acc[h].x + acc[h].y;
-#pragma unroll
-                    for (int o = 1; o < C::LPT; o <<= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-                    sc[s][h] = row < rows ? x * p.scale_log2 : -CUDART_INF_F;
-                }
+                for (int h = 0; h < G; ++h) x[s * G + h] = acc[h].x + acc[h].y;
             }
-            // online softmax: one rescale per tile
+            // complete scores: each lane owns KEEP of the group's (step, head) pairs
+            reduce_scatter<C>(x, li);
+            float sc[C::KEEP];
+            bool need = false;
 #pragma unroll
-            for (int h = 0; h < G; ++h) {
-                float mt = sc[0][h];
+            for (int e = 0; e < C::KEEP; ++e) {
+                const int idx = lo_idx + e;
+                const int row = ((idx / G) * kConsumerWarps + warp) * C::TPW + grp;
+                sc[e] = row < rows ? x[e] * p.scale_log2 : -CUDART_INF_F;
+                need |= sc[e] > mv[e] + kRescaleThreshold;
+            }
+            // Lazy rescaling: the running max only moves when a score exceeds it
+            // by more than 2^8 (first tile of a piece, then rarely), so the
+            // probabilities stay <= 256 and the common path exchanges nothing.
+            if (__any_sync(0xffffffffu, need)) {
+                float all[C::V];
+                gather_group<C>(sc, all, grp * C::LPT);
 #pragma unroll
-                for (int s = 1; s < C::STEPS; ++s) mt = fmaxf(mt, sc[s][h]);
-                if (mt > m[h]) {
-                    const float a = fast_exp2(m[h] - mt);
-                    m[h] = mt;
+                for (int h = 0; h < G; ++h) {
+                    float mt = all[h];
+#pragma unroll
+                    for (int s = 1; s < C::STEPS; ++s) mt = fmaxf(mt, all[s * G + h]);
+                    const float mn = fmaxf(m[h], mt);
+                    const float a = fast_exp2(m[h] - mn);
+                    m[h] = mn;
                     l[h] *= a;
                     const float2 a2 = make_float2(a, a);
 #pragma unroll
                     for (int j = 0; j < C::NCL * 4; ++j) o2[h][j] = fmul2(o2[h][j], a2);
                 }
 #pragma unroll
-                for (int s = 0; s < C::STEPS; ++s) {
-                    sc[s][h] = fast_exp2(sc[s][h] - m[h]);
-                    l[h] += sc[s][h];
+                for (int e = 0; e < C::KEEP; ++e) {
+                    const int hh = (lo_idx + e) % G;
+                    float mm = m[0];
+#pragma unroll
+                    for (int h = 1; h < G; ++h) mm = hh == h ? m[h] : mm;
+                    mv[e] = mm;
                 }
             }
+            float pe[C::KEEP];
+#pragma unroll
+            for (int e = 0; e < C::KEEP; ++e) pe[e] = fast_exp2(sc[e] - mv[e]);
+            float pa[C::V];
+            gather_group<C>(pe, pa, grp * C::LPT);
+#pragma unroll
+            for (int h = 0; h < G; ++h)
+#pragma unroll
+                for (int s = 0; s < C::STEPS; ++s) l[h] += pa[s * G + h];
 #pragma unroll
             for (int s = 0; s < C::STEPS; ++s) {
                 const int row = (s * kConsumerWarps + warp) * C::TPW + grp;
@@ -362,7 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                         const float2 v2 = bf2_to_f2(vv.z), v3 = bf2_to_f2(vv.w);
 #pragma unroll
                         for (int h = 0; h < G; ++h) {
-                            const float2 pp = make_float2(sc[s][h], sc[s][h]);
+                            const float2 pp = make_float2(pa[s * G + h], pa[s * G + h]);
                             o2[h][k * 4 + 0] = ffma2(pp, v0, o2[h][k * 4 + 0]);
                             o2[h][k * 4 + 1] = ffma2(pp, v1, o2[h][k * 4 + 1]);
                             o2[h][k * 4 + 2] = ffma2(pp, v2, o2[h][k * 4 + 2]);
