@@ -31,6 +31,10 @@ import duo_workloads as W  # noqa: E402
 METRIC = "mixed-head decode attn: µs/layer-step, achieved HBM GB/s (% of B200 peak)"
 WORKLOAD = "gqa128k"
 FALLBACK_HBM_GBS = 6650.0
+# DRAM read + write bytes per launch of decode_kernel<128,4> on this workload,
+# from the ncu capture summarised in profiles/decode_kernel_gqa128k.md.  Must be
+# reset to None whenever the decode kernel changes.
+DECODE_TRAFFIC_BYTES = 1118949000 + 3422720
 
 
 # ---------------------------------------------------------------- helpers
@@ -311,7 +315,8 @@ def run_ours(args, rank, world, local):
             "peak_kind": peak_kind,
             "unit": "GB/s",
             "frac": round(achieved / hbm_peak, 4),
-            "traffic": None,
+            "traffic": DECODE_TRAFFIC_BYTES,
+            "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch",
         },
         "e2e": {"value": round(e2e_ms * 1e3 / K, 3), "unit": "us/layer-step",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
