@@ -269,6 +269,20 @@ __device__ __forceinline__ uint32_t range_bits(int lo, int hi) {
     return upto & ~((1u << lo) - 1u);
 }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+    unsigned long long av = *reinterpret_cast<unsigned long long*>(&a);
+    unsigned long long bv = *reinterpret_cast<unsigned long long*>(&b);
+    unsigned long long dv;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(dv) : "l"(av), "l"(bv));
+    return *reinterpret_cast<float2*>(&dv);
+}
+
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
     __half2 h = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&h);
@@ -574,9 +588,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
 #pragma unroll
                 for (int x = 0; x < 8; ++x) t8[x] = s[x];
 #pragma unroll
-                for (int c = 8; c < 64; ++c) t8[c & 7] = fmaxf(t8[c & 7], s[c]);
-                mx = fmaxf(fmaxf(fmaxf(t8[0], t8[1]), fmaxf(t8[2], t8[3])),
-                           fmaxf(fmaxf(t8[4], t8[5]), fmaxf(t8[6], t8[7])));
+                for (int c = 8; c < 64; c += 2) t8[(c >> 1) & 7] = fmax3(t8[(c >> 1) & 7], s[c], s[c + 1]);
+                mx = fmax3(fmax3(t8[0], t8[1], t8[2]), fmax3(t8[3], t8[4], t8[5]), fmaxf(t8[6], t8[7]));
             }
             // exchange the half-row maxima; the barrier also agrees on aborting
             red_max[st][hf][r] = mx;
@@ -587,16 +600,21 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             const bool grow = mt > m + kRescaleThreshold;
             const float m_new = grow ? mt : m;
             const float alpha = fast_exp2(m - m_new);   // 1 when the max is kept
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                             make_float2(0.f, 0.f)};
             uint32_t ph[32];   // probabilities as packed fp16 pairs
+            const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+            const float2 nm2 = make_float2(-m_new, -m_new);
 #pragma unroll
             for (int c = 0; c < 64; c += 2) {
-                const float e0 = fast_exp2(fmaf(s[c], p.scale_log2, -m_new));
-                const float e1 = fast_exp2(fmaf(s[c + 1], p.scale_log2, -m_new));
-                acc[(c >> 1) & 3] += e0 + e1;
-                ph[c / 2] = pack_half2(e0, e1);
+                const float2 x = ffma2(make_float2(s[c], s[c + 1]), sc2, nm2);
+                const float2 e = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+                acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], e);
+                ph[c / 2] = pack_half2(e.x, e.y);
             }
-            l = l * alpha + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
+            const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
+            const float2 at = fadd2(a01, a23);
+            l = l * alpha + (at.x + at.y);
             m = m_new;
             // P_j overwrites P_{j-1} in TMEM, and a rescale touches O: both
             // need PV_{j-1} to have completed.
