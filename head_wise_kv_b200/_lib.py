@@ -39,6 +39,7 @@ EXPORTED = (
     "duo_kv_append", "duo_decode_workspace_bytes", "duo_decode_attn",
     "duo_prefill_workspace_bytes", "duo_prefill_attn", "duo_kv_read_status",
     "duo_kv_set_decode_ctas", "duo_strerror", "duo_decode_attn_static_ws",
+    "duo_kv_append_rows", "duo_decode_attn_rows", "duo_lse_merge", "duo_alpha_blend",
 )
 DUO_STATIC_WS_BYTES = 4 << 20
 
@@ -91,6 +92,10 @@ _c_append = _sig("duo_kv_append", [_P, _I32, _P, _P, _P, _P, _I32, _P])
 _c_dec_ws = _sig("duo_decode_workspace_bytes", [_P, ctypes.POINTER(_SZ)])
 _c_decode = _sig("duo_decode_attn", [_P, _I32, _P, _P, ctypes.c_float, _P, _P, _P, _SZ, _P])
 _c_decode_static = _sig("duo_decode_attn_static_ws", [_P, _I32, _P, _P, ctypes.c_float, _P, _P, _P])
+_c_append_rows = _sig("duo_kv_append_rows", [_P, _I32, _P, _P, _P, _P, _I32, _P, _P, _P])
+_c_decode_rows = _sig("duo_decode_attn_rows", [_P, _I32, _P, _P, _P, _P, ctypes.c_float, _P, _P, _P, _SZ, _P])
+_c_lse_merge = _sig("duo_lse_merge", [_I32, _I32, _I32, _P, _P, _P, _P, _P])
+_c_blend = _sig("duo_alpha_blend", [_I32, _I32, _I32, _P, _P, _P, _P, _P])
 _c_pre_ws = _sig("duo_prefill_workspace_bytes", [_P, _I32, ctypes.POINTER(_SZ)])
 _c_prefill = _sig("duo_prefill_attn", [_P, _I32, _P, _P, _P, _P, _I32, ctypes.c_float, _P, _P, _SZ, _P])
 _c_status = _sig("duo_kv_read_status", [_P, ctypes.POINTER(_I32), _I32, _P])
@@ -161,6 +166,26 @@ def duo_decode_attn(handle, layer, q, length, scale, out, lse, workspace, worksp
 
 def duo_decode_attn_static_ws(handle, layer, q, length, scale, out, lse, stream) -> None:
     _check(_c_decode_static(handle, layer, q, length, scale, out, lse, stream), "duo_decode_attn_static_ws")
+
+
+def duo_kv_append_rows(handle, layer, k_new, v_new, len_before, n_new, n_new_max, r_pos_begin, r_pos_end,
+                       stream) -> None:
+    _check(_c_append_rows(handle, layer, k_new, v_new, len_before, n_new, n_new_max, r_pos_begin, r_pos_end,
+                          stream), "duo_kv_append_rows")
+
+
+def duo_decode_attn_rows(handle, layer, q, r_begin, r_end, s_len, scale, out, lse, workspace, workspace_bytes,
+                         stream) -> None:
+    _check(_c_decode_rows(handle, layer, q, r_begin, r_end, s_len, scale, out, lse, workspace, workspace_bytes,
+                          stream), "duo_decode_attn_rows")
+
+
+def duo_lse_merge(parts, rows, d, part_out, part_lse, out, lse, stream) -> None:
+    _check(_c_lse_merge(parts, rows, d, part_out, part_lse, out, lse, stream), "duo_lse_merge")
+
+
+def duo_alpha_blend(batch, num_q_heads, d, alpha, full_out, stream_out, out, stream) -> None:
+    _check(_c_blend(batch, num_q_heads, d, alpha, full_out, stream_out, out, stream), "duo_alpha_blend")
 
 
 def duo_prefill_workspace_bytes(handle, chunk) -> int:

@@ -109,6 +109,37 @@ class DuoKVCache:
         np_ = _need(n_new, "n_new", torch.int32, (self.B,), self.device) if n_new is not None else None
         L.duo_kv_append(self.handle, layer, kp, vp, lp, np_, n, _stream(self.device))
 
+    def append_rows(self, layer: int, k_new, v_new, len_before, r_pos_begin, r_pos_end, n_new=None):
+        """append() for a cache whose retrieval rows hold positions
+        [r_pos_begin[b], r_pos_end[b]) (int32 [B] each) from row 0."""
+        n = k_new.shape[2]
+        shp = (self.B, self.n_kv, n, self.d)
+        kp = _need(k_new, "k_new", torch.bfloat16, shp, self.device)
+        vp = _need(v_new, "v_new", torch.bfloat16, shp, self.device)
+        lp = _need(len_before, "len_before", torch.int32, (self.B,), self.device)
+        bp = _need(r_pos_begin, "r_pos_begin", torch.int32, (self.B,), self.device)
+        ep = _need(r_pos_end, "r_pos_end", torch.int32, (self.B,), self.device)
+        np_ = _need(n_new, "n_new", torch.int32, (self.B,), self.device) if n_new is not None else None
+        L.duo_kv_append_rows(self.handle, layer, kp, vp, lp, np_, n, bp, ep, _stream(self.device))
+
+    def decode_rows(self, layer: int, q, r_end, scale: float, r_begin=None, s_len=None, out=None, lse=None):
+        """Decode over retrieval rows [r_begin, r_end) and streaming slots
+        [0, s_len) (int32 [B] each; r_begin / s_len optional).  Returns
+        (out [B][Hq][d], lse [B][Hq]) fp32."""
+        qp = _need(q, "q", torch.bfloat16, (self.B, self.hq, self.d), self.device)
+        ep = _need(r_end, "r_end", torch.int32, (self.B,), self.device)
+        bp = _need(r_begin, "r_begin", torch.int32, (self.B,), self.device) if r_begin is not None else None
+        sp = _need(s_len, "s_len", torch.int32, (self.B,), self.device) if s_len is not None else None
+        if out is None:
+            out = torch.empty(self.B, self.hq, self.d, dtype=torch.float32, device=self.device)
+        if lse is None:
+            lse = torch.empty(self.B, self.hq, dtype=torch.float32, device=self.device)
+        op = _need(out, "out", torch.float32, (self.B, self.hq, self.d), self.device)
+        lp = _need(lse, "lse", torch.float32, (self.B, self.hq), self.device)
+        L.duo_decode_attn_rows(self.handle, layer, qp, bp, ep, sp, float(scale), op, lp, self._ws.data_ptr(),
+                               self._ws.numel(), _stream(self.device))
+        return out, lse
+
     def decode(self, layer: int, q, lengths, scale: float, out=None, lse=None, want_lse=False):
         """q: bf16 [B][Hq][d]; lengths: int32 [B] after this step's append.
         Returns fp32 out [B][Hq][d] (and lse [B][Hq] if asked)."""
@@ -140,3 +171,40 @@ class DuoKVCache:
         L.duo_prefill_attn(self.handle, layer, qp, kp, vp, pp, C, float(scale), op, ws.data_ptr(), ws.numel(),
                            _stream(self.device))
         return out
+
+
+def lse_merge(part_out, part_lse, out=None, lse=None):
+    """Combine attention over disjoint key sets: part_out fp32 [R][..., d],
+    part_lse fp32 [R][...] (same leading shape) -> (out [..., d], lse [...])."""
+    R = part_out.shape[0]
+    d = part_out.shape[-1]
+    rows = part_lse[0].numel()
+    dev = part_out.device
+    if part_out.dtype != torch.float32 or part_lse.dtype != torch.float32:
+        raise TypeError("lse_merge takes fp32 tensors")
+    if not (part_out.is_contiguous() and part_lse.is_contiguous()):
+        raise ValueError("lse_merge takes contiguous tensors")
+    if part_out.numel() != R * rows * d or part_lse.shape[0] != R:
+        raise ValueError("part_out must be [R][rows][d] and part_lse [R][rows]")
+    if out is None:
+        out = torch.empty(part_out.shape[1:], dtype=torch.float32, device=dev)
+    if lse is None:
+        lse = torch.empty(part_lse.shape[1:], dtype=torch.float32, device=dev)
+    L.duo_lse_merge(R, rows, d, part_out.data_ptr(), part_lse.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                    _stream(dev))
+    return out, lse
+
+
+def alpha_blend(alpha, full_out, stream_out, out=None):
+    """out = alpha[h] * full_out + (1 - alpha[h]) * stream_out, tensors
+    [B][Hq][d] fp32, alpha fp32 [Hq]."""
+    B, hq, d = full_out.shape
+    dev = full_out.device
+    ap = _need(alpha, "alpha", torch.float32, (hq,), dev)
+    fp = _need(full_out, "full_out", torch.float32, (B, hq, d), dev)
+    sp = _need(stream_out, "stream_out", torch.float32, (B, hq, d), dev)
+    if out is None:
+        out = torch.empty_like(full_out)
+    op = _need(out, "out", torch.float32, (B, hq, d), dev)
+    L.duo_alpha_blend(B, hq, d, ap, fp, sp, op, _stream(dev))
+    return out

@@ -139,9 +139,9 @@ int duo_kv_layer_view_get(const duo_kv* kv, int32_t layer, duo_kv_layer_view* ou
     return DUO_OK;
 }
 
-int duo_kv_append(duo_kv* kv, int32_t layer, const uint16_t* k_new, const uint16_t* v_new,
-                  const int32_t* len_before, const int32_t* n_new, int32_t n_new_max,
-                  duo_stream_t stream) {
+static int append_impl(duo_kv* kv, int32_t layer, const uint16_t* k_new, const uint16_t* v_new,
+                       const int32_t* len_before, const int32_t* n_new, int32_t n_new_max,
+                       const int32_t* r_pos_begin, const int32_t* r_pos_end, duo_stream_t stream) {
     if (!kv || layer < 0 || layer >= kv->desc.num_layers || n_new_max < 0) return DUO_ERR_INVALID_ARG;
     if (n_new_max == 0) return DUO_OK;
     if (!k_new || !v_new || !len_before) return DUO_ERR_INVALID_ARG;
@@ -149,7 +149,11 @@ int duo_kv_append(duo_kv* kv, int32_t layer, const uint16_t* k_new, const uint16
         (reinterpret_cast<uintptr_t>(n_new) & 3))
         return DUO_ERR_ALIGNMENT;
     const duo::LayerLayout& L = kv->layers[layer];
+    if ((reinterpret_cast<uintptr_t>(r_pos_begin) & 3) || (reinterpret_cast<uintptr_t>(r_pos_end) & 3))
+        return DUO_ERR_ALIGNMENT;
     duo::AppendParams p;
+    p.r_pos_begin = r_pos_begin;
+    p.r_pos_end = r_pos_end;
     p.k_new = k_new;
     p.v_new = v_new;
     p.len_before = len_before;
@@ -174,6 +178,19 @@ int duo_kv_append(duo_kv* kv, int32_t layer, const uint16_t* k_new, const uint16
     return cuda_err(duo::launch_append(p, stream));
 }
 
+int duo_kv_append(duo_kv* kv, int32_t layer, const uint16_t* k_new, const uint16_t* v_new,
+                  const int32_t* len_before, const int32_t* n_new, int32_t n_new_max,
+                  duo_stream_t stream) {
+    return append_impl(kv, layer, k_new, v_new, len_before, n_new, n_new_max, nullptr, nullptr, stream);
+}
+
+int duo_kv_append_rows(duo_kv* kv, int32_t layer, const uint16_t* k_new, const uint16_t* v_new,
+                       const int32_t* len_before, const int32_t* n_new, int32_t n_new_max,
+                       const int32_t* r_pos_begin, const int32_t* r_pos_end, duo_stream_t stream) {
+    if (!r_pos_begin || !r_pos_end) return DUO_ERR_INVALID_ARG;
+    return append_impl(kv, layer, k_new, v_new, len_before, n_new, n_new_max, r_pos_begin, r_pos_end, stream);
+}
+
 static int decode_slots(const duo_kv* kv) {
     const int ctas = kv->decode_ctas > 0 ? kv->decode_ctas
                                          : duo::decode_ctas_default(kv->num_sms, kv->desc.head_dim,
@@ -188,10 +205,14 @@ int duo_decode_workspace_bytes(const duo_kv* kv, size_t* bytes) {
     return DUO_OK;
 }
 
-int duo_decode_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const int32_t* len, float scale,
-                    float* out, float* lse, void* workspace, size_t workspace_bytes,
-                    duo_stream_t stream) {
-    if (!kv || layer < 0 || layer >= kv->desc.num_layers || !q || !len || !out) return DUO_ERR_INVALID_ARG;
+static int decode_impl(duo_kv* kv, int32_t layer, const uint16_t* q, const int32_t* len, const int32_t* r_begin,
+                       const int32_t* r_end, const int32_t* s_len, float scale, float* out, float* lse,
+                       void* workspace, size_t workspace_bytes, duo_stream_t stream) {
+    if (!kv || layer < 0 || layer >= kv->desc.num_layers || !q || (!len && !r_end) || !out)
+        return DUO_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(r_begin) & 3) || (reinterpret_cast<uintptr_t>(r_end) & 3) ||
+        (reinterpret_cast<uintptr_t>(s_len) & 3))
+        return DUO_ERR_ALIGNMENT;
     if (!(scale > 0.f) || scale != scale) return DUO_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(out) || (reinterpret_cast<uintptr_t>(len) & 3) ||
         (reinterpret_cast<uintptr_t>(lse) & 3))
@@ -210,6 +231,9 @@ int duo_decode_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const int32_t*
     p.vs = reinterpret_cast<const uint16_t*>(kv->base + L.off_vs);
     p.q = q;
     p.len = len;
+    p.r_begin = r_begin;
+    p.r_end = r_end;
+    p.s_len = s_len;
     p.out = out;
     p.lse = lse;
     p.ws_o = static_cast<float*>(workspace);
@@ -231,6 +255,44 @@ int duo_decode_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const int32_t*
     memcpy(p.r_before, L.r_before, sizeof p.r_before);
     memcpy(p.is_r, L.is_r, sizeof p.is_r);
     return cuda_err(duo::launch_decode(p, D, G, stream));
+}
+
+int duo_decode_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const int32_t* len, float scale,
+                    float* out, float* lse, void* workspace, size_t workspace_bytes,
+                    duo_stream_t stream) {
+    if (!len) return DUO_ERR_INVALID_ARG;
+    return decode_impl(kv, layer, q, len, nullptr, nullptr, nullptr, scale, out, lse, workspace, workspace_bytes,
+                       stream);
+}
+
+int duo_decode_attn_rows(duo_kv* kv, int32_t layer, const uint16_t* q, const int32_t* r_begin,
+                         const int32_t* r_end, const int32_t* s_len, float scale, float* out, float* lse,
+                         void* workspace, size_t workspace_bytes, duo_stream_t stream) {
+    if (!r_end) return DUO_ERR_INVALID_ARG;
+    return decode_impl(kv, layer, q, nullptr, r_begin, r_end, s_len, scale, out, lse, workspace, workspace_bytes,
+                       stream);
+}
+
+int duo_lse_merge(int32_t parts, int32_t rows, int32_t d, const float* part_out, const float* part_lse, float* out,
+                  float* lse, duo_stream_t stream) {
+    if (parts < 1 || rows < 0 || d < 1 || !part_out || !part_lse || !out) return DUO_ERR_INVALID_ARG;
+    if (rows == 0) return DUO_OK;
+    if ((reinterpret_cast<uintptr_t>(part_out) & 3) || (reinterpret_cast<uintptr_t>(part_lse) & 3) ||
+        (reinterpret_cast<uintptr_t>(out) & 3) || (reinterpret_cast<uintptr_t>(lse) & 3))
+        return DUO_ERR_ALIGNMENT;
+    return cuda_err(duo::launch_lse_merge(parts, rows, d, part_out, part_lse, out, lse, stream));
+}
+
+int duo_alpha_blend(int32_t batch, int32_t num_q_heads, int32_t d, const float* alpha, const float* full_out,
+                    const float* stream_out, float* out, duo_stream_t stream) {
+    if (batch < 0 || num_q_heads < 1 || d < 1 || !alpha || !full_out || !stream_out || !out)
+        return DUO_ERR_INVALID_ARG;
+    const int64_t n = int64_t(batch) * num_q_heads * d;
+    if (n == 0) return DUO_OK;
+    if ((reinterpret_cast<uintptr_t>(alpha) & 3) || (reinterpret_cast<uintptr_t>(full_out) & 3) ||
+        (reinterpret_cast<uintptr_t>(stream_out) & 3) || (reinterpret_cast<uintptr_t>(out) & 3))
+        return DUO_ERR_ALIGNMENT;
+    return cuda_err(duo::launch_blend(n, num_q_heads, d, alpha, full_out, stream_out, out, stream));
 }
 
 static size_t prefill_ws(const duo_kv* kv, int32_t chunk) {

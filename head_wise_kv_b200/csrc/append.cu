@@ -17,6 +17,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <climits>
+
 #include "duo_internal.cuh"
 
 namespace duo {
@@ -64,13 +66,19 @@ __global__ void __launch_bounds__(kThreads) append_kernel(const __grid_constant_
 
     const size_t src = ((size_t(b) * p.n_kv + g) * p.n_new_max + i) * D + part * 8;
     if (p.is_r[g]) {
-        if (pos >= p.cap) {
+        // a cache may hold only a slice [r_pos_begin, r_pos_end) of the
+        // positions in its retrieval rows (sequence split over devices)
+        const int64_t lo = p.r_pos_begin ? p.r_pos_begin[b] : 0;
+        const int64_t hi = p.r_pos_end ? p.r_pos_end[b] : INT64_MAX;
+        if (pos < lo || pos >= hi) return;
+        const int64_t row = pos - lo;
+        if (row >= p.cap) {
             if (part == 0) set_status(p.status, DUO_STATUS_OVER_CAPACITY);
             return;
         }
         const uint4 kv = *reinterpret_cast<const uint4*>(p.k_new + src);
         const uint4 vv = *reinterpret_cast<const uint4*>(p.v_new + src);
-        const size_t dst = ((size_t(b) * p.n_r + p.rank[g]) * size_t(p.cap) + pos) * D + part * 8;
+        const size_t dst = ((size_t(b) * p.n_r + p.rank[g]) * size_t(p.cap) + row) * D + part * 8;
         *reinterpret_cast<uint4*>(p.kr + dst) = kv;
         *reinterpret_cast<uint4*>(p.vr + dst) = vv;
     } else if (survives) {

@@ -84,6 +84,32 @@ __device__ __forceinline__ int64_t rows_s(int len, int S, int W) {
     return r < S + W ? r : S + W;
 }
 
+// Rows each segment of sequence b reads: retrieval rows [r0, r0 + nr) of its
+// cache, streaming slots [0, ns) of its ring.
+struct SeqRows {
+    int64_t r0, nr, ns;
+};
+
+__device__ __forceinline__ SeqRows seq_rows(const DecodeParams& p, int b) {
+    SeqRows x;
+    if (p.r_end == nullptr) {
+        const int L = p.len[b];
+        x.r0 = 0;
+        x.nr = rows_r(L, p.cap);
+        x.ns = rows_s(L, p.S, p.W);
+    } else {
+        int64_t r0 = p.r_begin ? p.r_begin[b] : 0;
+        r0 = r0 < 0 ? 0 : (r0 > p.cap ? p.cap : r0);
+        int64_t r1 = p.r_end[b];
+        r1 = r1 < r0 ? r0 : (r1 > p.cap ? p.cap : r1);
+        x.r0 = r0;
+        x.nr = r1 - r0;
+        int64_t ns = p.s_len ? p.s_len[b] : 0;
+        x.ns = ns < 0 ? 0 : (ns > p.S + p.W ? p.S + p.W : ns);
+    }
+    return x;
+}
+
 // Fill bpre[0..B] (shared) with the running count of 16-token blocks per
 // sequence; warp 0 does a chunked shuffle scan.  Caller syncs afterwards.
 __device__ void build_prefix(const DecodeParams& p, int32_t* bpre) {
@@ -95,8 +121,8 @@ __device__ void build_prefix(const DecodeParams& p, int32_t* bpre) {
         const int b = base + lane;
         int c = 0;
         if (b < p.B) {
-            const int L = p.len[b];
-            c = p.n_r * blocks_of(rows_r(L, p.cap)) + p.n_s * blocks_of(rows_s(L, p.S, p.W));
+            const SeqRows x = seq_rows(p, b);
+            c = p.n_r * blocks_of(x.nr) + p.n_s * blocks_of(x.ns);
         }
         int x = c;
 #pragma unroll
@@ -119,6 +145,7 @@ __device__ __forceinline__ int cta_owner(int64_t gb, int64_t total, int64_t n) {
 
 struct Piece {
     int b, g, seg;          // sequence, KV head, segment index b * n_kv + g
+    int64_t row0;           // first cache row of the segment (retrieval row ranges)
     int64_t seg_gb;         // first global block of the segment
     int seg_nb;             // blocks in the segment
     int64_t tok0, tok1;     // token rows of this piece inside the segment
@@ -137,8 +164,8 @@ __device__ __forceinline__ Piece locate(const DecodeParams& p, const int32_t* bp
         if (bpre[mid] <= gb) lo = mid; else hi = mid;
     }
     pc.b = lo;
-    const int L = p.len[lo];
-    const int64_t rr = rows_r(L, p.cap), rs = rows_s(L, p.S, p.W);
+    const SeqRows x = seq_rows(p, lo);
+    const int64_t rr = x.nr, rs = x.ns;
     const int nbr = blocks_of(rr), nbs = blocks_of(rs);
     const int64_t local = gb - bpre[lo];
     int g = 0;
@@ -150,6 +177,7 @@ __device__ __forceinline__ Piece locate(const DecodeParams& p, const int32_t* bp
     }
     pc.g = g;
     pc.seg = lo * p.n_kv + g;
+    pc.row0 = p.is_r[g] ? x.r0 : 0;
     pc.seg_nb = p.is_r[g] ? nbr : nbs;
     pc.seg_gb = bpre[lo] + start;
     const int64_t seg_end = pc.seg_gb + pc.seg_nb;
@@ -211,11 +239,11 @@ __device__ __forceinline__ void gather_group(const float (&held)[C::KEEP], float
 }
 
 template <int D>
-__device__ __forceinline__ void seg_ptrs(const DecodeParams& p, int b, int g, const uint16_t*& k,
+__device__ __forceinline__ void seg_ptrs(const DecodeParams& p, int b, int g, int64_t row0, const uint16_t*& k,
                                          const uint16_t*& v) {
     const int r = p.rank[g];
     if (p.is_r[g]) {
-        const size_t off = (size_t(b) * p.n_r + r) * size_t(p.cap) * D;
+        const size_t off = ((size_t(b) * p.n_r + r) * size_t(p.cap) + size_t(row0)) * D;
         k = p.kr + off;
         v = p.vr + off;
     } else {
@@ -275,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         for (int64_t gb = gb_begin; gb < gb_end && ok;) {
             const Piece pc = locate(p, bpre, gb, gb_end);
             const uint16_t *kp, *vp;
-            seg_ptrs<D>(p, pc.b, pc.g, kp, vp);
+            seg_ptrs<D>(p, pc.b, pc.g, pc.row0, kp, vp);
             for (int64_t t = pc.tok0; t < pc.tok1; t += kTile, ++it) {
                 const int rows = int(pc.tok1 - t < kTile ? pc.tok1 - t : kTile);
                 const int st = it % kStages;
@@ -551,26 +579,27 @@ __global__ void __launch_bounds__(32 * G) merge_kernel(const __grid_constant__ D
     const int b = seg / p.n_kv, g = seg % p.n_kv;
     const int h = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int qh = g * G + h;
-    const int L = p.len[b];
     float* out = p.out + (size_t(b) * p.hq + qh) * D;
     const int64_t total = bpre[p.B];
-    const int nbr = blocks_of(rows_r(L, p.cap)), nbs = blocks_of(rows_s(L, p.S, p.W));
+    const SeqRows x = seq_rows(p, b);
+    const int nbr = blocks_of(x.nr), nbs = blocks_of(x.ns);
     const int64_t seg_gb = bpre[b] + int64_t(p.r_before[g]) * nbr + int64_t(g - p.r_before[g]) * nbs;
     const int seg_nb = p.is_r[g] ? nbr : nbs;
-    const int c0 = L < 1 ? 0 : cta_owner(seg_gb, total, p.num_ctas);
-    const int c1 = L < 1 ? 0 : cta_owner(seg_gb + seg_nb - 1, total, p.num_ctas);
+    const int c0 = seg_nb < 1 ? 0 : cta_owner(seg_gb, total, p.num_ctas);
+    const int c1 = seg_nb < 1 ? 0 : cta_owner(seg_gb + seg_nb - 1, total, p.num_ctas);
     const bool dense = total >= p.num_ctas;   // then no CTA range is empty
 
     // wait for the attention kernel's partials (and its writes of `out`)
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
-    if (threadIdx.x == 0 && g == 0) {
+    if (p.r_end == nullptr && threadIdx.x == 0 && g == 0) {
+        const int L = p.len[b];
         if (L < 0) set_status(p.status, DUO_STATUS_BAD_LENGTH);
         if (int64_t(L) > p.cap && p.n_r > 0) set_status(p.status, DUO_STATUS_OVER_CAPACITY);
         if (L < 1) set_status(p.status, DUO_STATUS_EMPTY_SEQUENCE);
     }
-    if (L < 1) {
-        for (int x = lane; x < D; x += 32) out[x] = 0.f;
+    if (seg_nb < 1) {   // no key: zero output, lse = -inf (contributes nothing to a merge)
+        for (int xx = lane; xx < D; xx += 32) out[xx] = 0.f;
         if (lane == 0 && p.lse != nullptr) p.lse[size_t(b) * p.hq + qh] = -CUDART_INF_F;
         return;
     }

@@ -44,7 +44,10 @@ struct DecodeParams {
     const uint16_t* ks;
     const uint16_t* vs;
     const uint16_t* q;
-    const int32_t* len;
+    const int32_t* len;       // classic mode: rows = min(len, cap) and min(len, S+W)
+    const int32_t* r_begin;   // row-range mode (r_end != null): retrieval rows
+    const int32_t* r_end;     //   [r_begin[b], r_end[b]) (r_begin may be null = 0),
+    const int32_t* s_len;     //   streaming slots [0, s_len[b]) (null = none)
     float* out;
     float* lse;
     float* ws_o;      // [slots][G][D]  partial outputs (unnormalised)
@@ -61,6 +64,8 @@ struct DecodeParams {
 };
 
 struct AppendParams {
+    const int32_t* r_pos_begin;   // optional: retrieval rows hold positions
+    const int32_t* r_pos_end;     //   [r_pos_begin[b], r_pos_end[b]) at rows from 0
     const uint16_t* k_new;
     const uint16_t* v_new;
     const int32_t* len_before;
@@ -102,6 +107,10 @@ cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 int decode_ctas_default(int num_sms, int d, int group);
 size_t decode_workspace_bytes(int slots, int d, int group);
 cudaError_t launch_decode(const DecodeParams& p, int d, int group, cudaStream_t s);
+cudaError_t launch_lse_merge(int parts, int rows, int d, const float* part_out, const float* part_lse, float* out,
+                             float* lse, cudaStream_t s);
+cudaError_t launch_blend(int64_t n, int hq, int d, const float* alpha, const float* full, const float* strm,
+                         float* out, cudaStream_t s);
 size_t prefill_smem_bytes(int S, int W);
 size_t prefill_workspace_bytes(int B, int n_kv, int n_r, int n_s, int64_t cap, int S, int W, int C);
 int launch_prefill(const PrefillLaunch& a, cudaStream_t s);   // returns a DUO_* code

@@ -165,6 +165,18 @@ DUO_API int duo_kv_append(duo_kv* kv, int32_t layer, const uint16_t* k_new, cons
                   const int32_t* len_before, const int32_t* n_new, int32_t n_new_max,
                   duo_stream_t stream);
 
+/* duo_kv_append for a cache whose retrieval rows hold only a slice of each
+ * sequence's positions, [r_pos_begin[b], r_pos_end[b]) (device int32 [B]),
+ * stored from row 0: position p goes to row p - r_pos_begin[b]; positions
+ * outside the slice are not written to retrieval heads.  Streaming heads and
+ * the position table are updated exactly as by duo_kv_append (positions are
+ * absolute).  This is the storage of a sequence split over devices: each
+ * device appends every token, its retrieval heads keep their own slice.  Not
+ * on the pages (their plan has one device); see duo_decode_attn_rows. */
+DUO_API int duo_kv_append_rows(duo_kv* kv, int32_t layer, const uint16_t* k_new, const uint16_t* v_new,
+                               const int32_t* len_before, const int32_t* n_new, int32_t n_new_max,
+                               const int32_t* r_pos_begin, const int32_t* r_pos_end, duo_stream_t stream);
+
 /* Workspace bytes duo_decode_attn needs (host only). */
 DUO_API int duo_decode_workspace_bytes(const duo_kv* kv, size_t* bytes);
 
@@ -184,6 +196,42 @@ DUO_API int duo_decode_workspace_bytes(const duo_kv* kv, size_t* bytes);
 DUO_API int duo_decode_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const int32_t* len,
                     float scale, float* out, float* lse, void* workspace, size_t workspace_bytes,
                     duo_stream_t stream);
+
+/* Decode attention over chosen rows.  Like duo_decode_attn, except that
+ * the keys come from explicit row ranges instead of the sequence length:
+ *   retrieval heads: cache rows [r_begin[b], r_end[b]) (r_begin may be NULL
+ *     = 0; both device int32 [B], clamped to [0, capacity]);
+ *   streaming heads: ring slots [0, s_len[b]) (device int32 [B], clamped to
+ *     S + W; NULL = no slots).
+ * A head with no rows gets out = 0 and lse = -inf, so it contributes nothing
+ * to duo_lse_merge.  No status bits are set by this call.  Two uses:
+ *   - sequence split over devices: each device holds a slice of every
+ *     retrieval head (duo_kv_append_rows) and decodes rows [0, slice); one
+ *     device also passes s_len for the streaming heads; the partial (out,
+ *     lse) are exchanged and combined with duo_lse_merge;
+ *   - the streaming part of the gated forward on a full cache: sinks = rows
+ *     [0, S) and window = rows [t-W+1, t+1) of each head, merged with
+ *     duo_lse_merge (see duo_alpha_blend). */
+DUO_API int duo_decode_attn_rows(duo_kv* kv, int32_t layer, const uint16_t* q, const int32_t* r_begin,
+                                 const int32_t* r_end, const int32_t* s_len, float scale, float* out, float* lse,
+                                 void* workspace, size_t workspace_bytes, duo_stream_t stream);
+
+/* Combine attention results over disjoint key sets: for each of `rows`
+ * rows, out = sum_r exp(lse_r - LSE) part_out[r], LSE = log sum_r exp(lse_r).
+ *   part_out: device fp32 [parts][rows][d]; part_lse: [parts][rows] (natural
+ *   log of each part's softmax denominator; -inf = the part saw no key);
+ *   out: [rows][d]; lse: optional [rows].  Rows where every part is -inf get
+ *   out = 0, lse = -inf.  Exact up to rounding (the softmax over a union is
+ *   the log-sum-exp weighted mix of the softmaxes over its parts). */
+DUO_API int duo_lse_merge(int32_t parts, int32_t rows, int32_t d, const float* part_out, const float* part_lse,
+                          float* out, float* lse, duo_stream_t stream);
+
+/* Gated attention of the DuoAttention guide's head identification (section
+ * 3, item 2): out = alpha[h] * full_out + (1 - alpha[h]) * stream_out for
+ * query head h.  alpha: device fp32 [num_q_heads]; full_out, stream_out,
+ * out: [batch][num_q_heads][d] fp32 (out may alias either input). */
+DUO_API int duo_alpha_blend(int32_t batch, int32_t num_q_heads, int32_t d, const float* alpha,
+                            const float* full_out, const float* stream_out, float* out, duo_stream_t stream);
 
 /* Bytes of device scratch built into the library for
  * duo_decode_attn_static_ws (a file-scope __device__ array). */

@@ -43,7 +43,7 @@ import numpy as np
 __all__ = [
     "kv_cache_bytes", "duo_effective_context", "duo_cache_bytes", "duo_slots",
     "StreamingCache", "ring_positions", "keep_set", "key_mask", "kv_head_of",
-    "attend", "decode_attention", "prefill_attention", "brute_force_attention",
+    "attend", "decode_attention", "prefill_attention", "brute_force_attention", "blended_decode",
 ]
 
 
@@ -209,6 +209,18 @@ def decode_attention(q, k_hist, v_hist, lens_after, mask, sink, window, scale, p
             for h in heads:
                 out[b, h], lse[b, h] = attend(q[b, h], K, V, scale)
     return out, lse
+
+
+def blended_decode(q, k_hist, v_hist, lens_after, n_kv, alpha, sink, window, scale):
+    """Gated attention of head identification (DuoAttention guide, section 3
+    "Automated Head Identification", item 2): for each query head h,
+    alpha[h] * FullAttn + (1 - alpha[h]) * StreamAttn, where FullAttn reads
+    every key 0..t of the head's full history and StreamAttn only the sinks
+    and the recent window of that same history.  Returns [B][Hq][d] float64."""
+    alpha = np.asarray(alpha, dtype=np.float64)[None, :, None]
+    full, _ = decode_attention(q, k_hist, v_hist, lens_after, np.ones(n_kv, np.uint8), sink, window, scale)
+    strm, _ = decode_attention(q, k_hist, v_hist, lens_after, np.zeros(n_kv, np.uint8), sink, window, scale)
+    return alpha * full + (1.0 - alpha) * strm
 
 
 def prefill_attention(q, k_hist, v_hist, prefix, mask, sink, window, scale,

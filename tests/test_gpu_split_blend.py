@@ -1,0 +1,137 @@
+"""Row-range decode, log-sum-exp merge and the gated (alpha-blended) forward
+through the C ABI, against the fp64 oracle.
+
+* Sequence split: R caches (one per device in a real deployment; here R
+  independent caches on one GPU, none waiting on another) each hold a slice
+  of every sequence's retrieval history; their partial (out, lse) merge to the
+  single-device result.
+* Gated forward: on a cache whose heads all keep full history, the streaming
+  attention is two row ranges (sinks, recent window) merged, then blended
+  with full attention per query head.
+"""
+import numpy as np
+import pytest
+import torch
+
+import duo_workloads as W
+from _harness import History, assert_close
+from oracle import duo_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+
+def _dev():
+    return torch.device("cuda", 0)
+
+
+def _cache(w, cap, mask):
+    from head_wise_kv_b200 import DuoKVCache
+    return DuoKVCache(1, w.batch, w.hq, w.n_kv, w.d, w.sink, w.window, cap, mask[None], device=_dev())
+
+
+def _history(w, T):
+    k = torch.zeros(w.batch, w.n_kv, T, w.d, dtype=torch.bfloat16)
+    v = torch.zeros_like(k)
+    return k, v
+
+
+def _fill_rows(cache, w, lens, lo, hi, dev):
+    """Append tokens 0..lens[b]-1 of every sequence (one bulk call with
+    per-sequence counts); retrieval rows keep positions [lo[b], hi[b])."""
+    T = int(max(lens))
+    k = torch.zeros(w.batch, w.n_kv, T, w.d, dtype=torch.bfloat16)
+    v = torch.zeros_like(k)
+    for b in range(w.batch):
+        for g in range(w.n_kv):
+            k[b, g, :lens[b]] = W.tokens(w, 0, b, g, W.TENSOR_K, 0, int(lens[b]))
+            v[b, g, :lens[b]] = W.tokens(w, 0, b, g, W.TENSOR_V, 0, int(lens[b]))
+    i32 = lambda a: torch.tensor(np.asarray(a, dtype=np.int32), device=dev)
+    cache.append_rows(0, k.to(dev), v.to(dev), i32([0] * w.batch), i32(lo), i32(hi), n_new=i32(lens))
+
+
+def _oracle_full(w, q, lens, mask):
+    hist = History(w)
+
+    def kh(b, g):
+        return hist.kv(0, b, g, W.TENSOR_K, int(lens[b])).float().numpy()
+
+    def vh(b, g):
+        return hist.kv(0, b, g, W.TENSOR_V, int(lens[b])).float().numpy()
+    return kh, vh
+
+
+@pytest.mark.parametrize("R,cap", [(2, 1600), (3, 1100), (4, 1024)])
+def test_sequence_split_decode_merges_to_full_result(R, cap):
+    from head_wise_kv_b200 import seqsplit
+    from head_wise_kv_b200.cache import lse_merge
+    w = W.scaled(W.WORKLOADS["gqa128k"], batch=2, t0_range=None, t0=0, sink=16, window=64)
+    dev = _dev()
+    mask = W.retrieval_mask(w, 0)
+    lens = np.array([2900, 1301])            # after this step's append
+    caches = [_cache(w, cap, mask) for _ in range(R)]
+    for r, c in enumerate(caches):
+        lo, hi = seqsplit.slice_bounds(cap, r)
+        _fill_rows(c, w, lens, [lo] * w.batch, [hi] * w.batch, dev)
+    q = W.decode_q(w, 0, lens)
+    L = torch.from_numpy(lens.astype(np.int32)).to(dev)
+    outs, lses = [], []
+    for r, c in enumerate(caches):
+        rows = seqsplit.local_rows(L, cap, r)
+        s_len = L if r == R - 1 else torch.zeros_like(L)
+        o, l = c.decode_rows(0, q.to(dev), rows, w.scale, s_len=s_len)
+        outs.append(o)
+        lses.append(l)
+    out, lse = lse_merge(torch.stack(outs), torch.stack(lses))
+    kh, vh = _oracle_full(w, q, lens, mask)
+    ref, ref_lse = O.decode_attention(q.double().numpy(), kh, vh, lens, mask, w.sink, w.window, w.scale)
+    assert_close(out.cpu().double().numpy(), ref, f"split over {R}")
+    assert np.abs(lse.cpu().double().numpy() - ref_lse).max() < 1e-3
+    for c in caches:
+        assert c.status() == 0
+        c.close()
+
+
+@pytest.mark.parametrize("lens", [[700, 90], [79, 12], [5, 300]])
+def test_gated_forward_matches_oracle(lens):
+    from head_wise_kv_b200.cache import alpha_blend, lse_merge
+    w = W.scaled(W.WORKLOADS["gqa128k"], batch=2, hq=8, n_kv=4, t0_range=None, t0=0, sink=16, window=64)
+    dev = _dev()
+    lens = np.array(lens)
+    full_mask = np.ones(w.n_kv, np.uint8)         # identification keeps every head's full history
+    cache = _cache(w, int(lens.max()), full_mask)
+    _fill_rows(cache, w, lens, [0] * w.batch, [1 << 30] * w.batch, dev)
+    q = W.decode_q(w, 0, lens).to(dev)
+    L = torch.from_numpy(lens.astype(np.int32)).to(dev)
+    full = cache.decode(0, q, L, w.scale)
+    S, Wn = w.sink, w.window
+    sink_end = torch.clamp(L, max=S)
+    win_begin = torch.clamp(L - Wn, min=S)
+    o_s, l_s = cache.decode_rows(0, q, sink_end, w.scale)
+    o_w, l_w = cache.decode_rows(0, q, L, w.scale, r_begin=win_begin)
+    strm, _ = lse_merge(torch.stack([o_s, o_w]), torch.stack([l_s, l_w]))
+    alpha = torch.from_numpy(np.random.default_rng(3).uniform(0, 1, w.hq).astype(np.float32)).to(dev)
+    out = alpha_blend(alpha, full, strm)
+    kh, vh = _oracle_full(w, q.cpu(), lens, full_mask)
+    ref = O.blended_decode(q.cpu().double().numpy(), kh, vh, lens, w.n_kv, alpha.cpu().double().numpy(), S, Wn,
+                           w.scale)
+    assert_close(out.cpu().double().numpy(), ref, "gated forward")
+    cache.close()
+
+
+def test_lse_merge_ignores_empty_parts():
+    from head_wise_kv_b200.cache import lse_merge
+    dev = _dev()
+    rng = np.random.default_rng(4)
+    o = torch.from_numpy(rng.standard_normal((3, 5, 64)).astype(np.float32)).to(dev)
+    l = torch.from_numpy(rng.standard_normal((3, 5)).astype(np.float32)).to(dev)
+    l[1] = float("-inf")
+    o[1] = float("nan")                            # an empty part's output is never read
+    l[:, 4] = float("-inf")                        # a row no part saw
+    out, lse = lse_merge(o, l)
+    ll = l.cpu().double().numpy()
+    oo = o.cpu().double().numpy()
+    for row in range(4):
+        wts = np.exp(ll[[0, 2], row] - np.logaddexp(ll[0, row], ll[2, row]))
+        np.testing.assert_allclose(out[row].cpu().numpy(), wts[0] * oo[0, row] + wts[1] * oo[2, row], rtol=1e-5,
+                                   atol=1e-6)
+    assert torch.all(out[4] == 0) and lse[4].item() == float("-inf")

@@ -391,3 +391,44 @@ def test_planted_missing_scale_is_caught(monkeypatch):
 def test_planted_size_factor_error_is_caught(monkeypatch):
     monkeypatch.setattr(O, "kv_cache_bytes", lambda L, n, d, T, elem_bytes=2: elem_bytes * L * n * d * T)
     assert _fails(test_dense_sizes_match_printed_values)
+
+
+# ------------------------------------------------------------------ gated forward, split sums
+def test_blended_decode_reduces_to_full_and_streaming_and_is_linear():
+    """alpha = 1 is full attention (every head retrieval), alpha = 0 is the
+    sink + window attention (every head streaming), and the gate mixes the two
+    linearly (DuoAttention guide, section 3, item 2)."""
+    rng = np.random.default_rng(21)
+    B, hq, n_kv, d, T = 2, 8, 4, 16, 70
+    K, V = _hist(rng, B, n_kv, T, d)
+    q = _rand(rng, B, hq, d)
+    kh, vh = (lambda b, g: K[b, g]), (lambda b, g: V[b, g])
+    lens = [T, T - 20]
+    full, _ = O.decode_attention(q, kh, vh, lens, np.ones(n_kv, np.uint8), 4, 16, 0.3)
+    strm, _ = O.decode_attention(q, kh, vh, lens, np.zeros(n_kv, np.uint8), 4, 16, 0.3)
+    np.testing.assert_allclose(O.blended_decode(q, kh, vh, lens, n_kv, np.ones(hq), 4, 16, 0.3), full,
+                               rtol=1e-14, atol=1e-14)
+    np.testing.assert_allclose(O.blended_decode(q, kh, vh, lens, n_kv, np.zeros(hq), 4, 16, 0.3), strm,
+                               rtol=1e-14, atol=1e-14)
+    a = rng.uniform(0, 1, hq)
+    mix = O.blended_decode(q, kh, vh, lens, n_kv, a, 4, 16, 0.3)
+    np.testing.assert_allclose(mix, a[None, :, None] * full + (1 - a[None, :, None]) * strm, rtol=1e-13,
+                               atol=1e-14)
+    assert np.abs(full - strm).max() > 1e-3
+
+
+def test_attention_over_a_union_is_the_lse_weighted_mix_of_its_parts():
+    """The identity sequence-split decode and the two-range streaming
+    attention rely on: softmax attention over disjoint key sets joined by
+    their log-sum-exps equals attention over the union (brute force)."""
+    rng = np.random.default_rng(22)
+    d, T = 8, 40
+    q, k, v = _rand(rng, d), _rand(rng, T, d), _rand(rng, T, d)
+    cuts = [0, 7, 8, 25, 40]
+    parts = [O.attend(q, k[a:b], v[a:b], 0.4) for a, b in zip(cuts[:-1], cuts[1:])]
+    lse = np.array([p[1] for p in parts])
+    LSE = np.log(np.exp(lse - lse.max()).sum()) + lse.max()
+    mixed = sum(np.exp(l - LSE) * o for o, l in parts)
+    want, want_lse = O.brute_force_attention(q, k, v, list(range(T)), 0.4)
+    np.testing.assert_allclose(mixed, want, rtol=1e-12, atol=1e-13)
+    assert LSE == pytest.approx(want_lse, rel=1e-13)
