@@ -34,7 +34,7 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM read + write bytes per launch of decode_kernel<128,4> on this workload,
 # from the ncu capture summarised in profiles/decode_kernel_gqa128k.md.  Must be
 # reset to None whenever the decode kernel changes.
-DECODE_TRAFFIC_BYTES = 1119041000 + 3481088
+DECODE_TRAFFIC_BYTES = None
 
 
 # ---------------------------------------------------------------- helpers

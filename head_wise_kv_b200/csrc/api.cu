@@ -112,6 +112,17 @@ int duo_kv_alloc(const duo_kv_desc* desc, void* dev_buf, size_t buf_bytes, duo_s
         delete h;
         return DUO_ERR_CUDA;
     }
+    if (desc->head_dim == 128) {
+        h->maps.resize(h->layers.size());
+        for (size_t l = 0; l < h->layers.size(); ++l) {
+            const duo::LayerLayout& L = h->layers[l];
+            if (!duo::make_decode_maps(&h->maps[l], h->base + L.off_kr, h->base + L.off_vr, h->base + L.off_ks,
+                                       h->base + L.off_vs, desc->batch, L.n_r, L.n_s, desc->capacity, int(SW))) {
+                delete h;
+                return DUO_ERR_CUDA;
+            }
+        }
+    }
     *out = h;
     return DUO_OK;
 }
@@ -225,6 +236,13 @@ static int decode_impl(duo_kv* kv, int32_t layer, const uint16_t* q, const int32
     if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return DUO_ERR_ALIGNMENT;
     const duo::LayerLayout& L = kv->layers[layer];
     duo::DecodeParams p;
+    memset(&p, 0, sizeof p);
+    if (!kv->maps.empty()) {
+        p.tm_kr = kv->maps[layer].kr;
+        p.tm_vr = kv->maps[layer].vr;
+        p.tm_ks = kv->maps[layer].ks;
+        p.tm_vs = kv->maps[layer].vs;
+    }
     p.kr = reinterpret_cast<const uint16_t*>(kv->base + L.off_kr);
     p.vr = reinterpret_cast<const uint16_t*>(kv->base + L.off_vr);
     p.ks = reinterpret_cast<const uint16_t*>(kv->base + L.off_ks);

@@ -30,6 +30,7 @@
 #include <math_constants.h>
 #include <stdint.h>
 
+#include "decode_sched.cuh"
 #include "duo_internal.cuh"
 
 namespace duo {
@@ -44,7 +45,6 @@ constexpr int kTile = 56;        // rows per pipeline stage
 constexpr int kStages = 4;
 constexpr int kConsumerWarps = 7;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr int kBlk = 16;         // partition granularity in tokens
 constexpr float kNegBig = -1.0e30f;   // finite "minus infinity" for running maxima
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: probabilities stay <= 2^8
 
@@ -72,123 +72,6 @@ struct Cfg {
     static_assert(STEPS * TPW * kConsumerWarps == kTile, "tile must be whole warp steps");
     static_assert(STAGE_BYTES % 1024 == 0, "stage buffers stay 1024-byte aligned");
 };
-
-__device__ __forceinline__ int blocks_of(int64_t rows) { return int((rows + kBlk - 1) / kBlk); }
-
-__device__ __forceinline__ int64_t rows_r(int len, int64_t cap) {
-    int64_t r = len < 0 ? 0 : len;
-    return r < cap ? r : cap;
-}
-__device__ __forceinline__ int64_t rows_s(int len, int S, int W) {
-    int64_t r = len < 0 ? 0 : len;
-    return r < S + W ? r : S + W;
-}
-
-// Rows each segment of sequence b reads: retrieval rows [r0, r0 + nr) of its
-// cache, streaming slots [0, ns) of its ring.
-struct SeqRows {
-    int64_t r0, nr, ns;
-};
-
-__device__ __forceinline__ SeqRows seq_rows(const DecodeParams& p, int b) {
-    SeqRows x;
-    if (p.r_end == nullptr) {
-        const int L = p.len[b];
-        x.r0 = 0;
-        x.nr = rows_r(L, p.cap);
-        x.ns = rows_s(L, p.S, p.W);
-    } else {
-        int64_t r0 = p.r_begin ? p.r_begin[b] : 0;
-        r0 = r0 < 0 ? 0 : (r0 > p.cap ? p.cap : r0);
-        int64_t r1 = p.r_end[b];
-        r1 = r1 < r0 ? r0 : (r1 > p.cap ? p.cap : r1);
-        x.r0 = r0;
-        x.nr = r1 - r0;
-        int64_t ns = p.s_len ? p.s_len[b] : 0;
-        x.ns = ns < 0 ? 0 : (ns > p.S + p.W ? p.S + p.W : ns);
-    }
-    return x;
-}
-
-// Fill bpre[0..B] (shared) with the running count of 16-token blocks per
-// sequence; warp 0 does a chunked shuffle scan.  Caller syncs afterwards.
-__device__ void build_prefix(const DecodeParams& p, int32_t* bpre) {
-    if (threadIdx.x >= 32) return;
-    const int lane = threadIdx.x;
-    int run = 0;
-    if (lane == 0) bpre[0] = 0;
-    for (int base = 0; base < p.B; base += 32) {
-        const int b = base + lane;
-        int c = 0;
-        if (b < p.B) {
-            const SeqRows x = seq_rows(p, b);
-            c = p.n_r * blocks_of(x.nr) + p.n_s * blocks_of(x.ns);
-        }
-        int x = c;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += y;
-        }
-        if (b < p.B) bpre[b + 1] = run + x;
-        run += __shfl_sync(0xffffffffu, x, 31);
-    }
-}
-
-// First block index owned by CTA c when `total` blocks are split over n CTAs.
-__device__ __forceinline__ int64_t cta_start(int64_t c, int64_t total, int64_t n) { return c * total / n; }
-// CTA that owns block gb.
-__device__ __forceinline__ int cta_owner(int64_t gb, int64_t total, int64_t n) {
-    int64_t c = ((gb + 1) * n - 1) / total;
-    return int(c < n - 1 ? c : n - 1);
-}
-
-struct Piece {
-    int b, g, seg;          // sequence, KV head, segment index b * n_kv + g
-    int64_t row0;           // first cache row of the segment (retrieval row ranges)
-    int64_t seg_gb;         // first global block of the segment
-    int seg_nb;             // blocks in the segment
-    int64_t tok0, tok1;     // token rows of this piece inside the segment
-    int64_t end_gb;         // global block after the piece
-    bool whole;             // the piece is the whole segment
-};
-
-// Locate the piece that starts at global block gb (gb < range end).
-__device__ __forceinline__ Piece locate(const DecodeParams& p, const int32_t* bpre, int64_t gb,
-                                        int64_t range_end) {
-    Piece pc;
-    // b = last index with bpre[b] <= gb  (binary search over B + 1 entries)
-    int lo = 0, hi = p.B;   // invariant: bpre[lo] <= gb < bpre[hi]
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (bpre[mid] <= gb) lo = mid; else hi = mid;
-    }
-    pc.b = lo;
-    const SeqRows x = seq_rows(p, lo);
-    const int64_t rr = x.nr, rs = x.ns;
-    const int nbr = blocks_of(rr), nbs = blocks_of(rs);
-    const int64_t local = gb - bpre[lo];
-    int g = 0;
-    int64_t start = 0;
-    for (; g < p.n_kv; ++g) {
-        start = int64_t(p.r_before[g]) * nbr + int64_t(g - p.r_before[g]) * nbs;
-        const int nb = p.is_r[g] ? nbr : nbs;
-        if (local < start + nb) break;
-    }
-    pc.g = g;
-    pc.seg = lo * p.n_kv + g;
-    pc.row0 = p.is_r[g] ? x.r0 : 0;
-    pc.seg_nb = p.is_r[g] ? nbr : nbs;
-    pc.seg_gb = bpre[lo] + start;
-    const int64_t seg_end = pc.seg_gb + pc.seg_nb;
-    pc.end_gb = seg_end < range_end ? seg_end : range_end;
-    const int64_t rows = p.is_r[g] ? rr : rs;
-    pc.tok0 = (gb - pc.seg_gb) * kBlk;
-    const int64_t t1 = (pc.end_gb - pc.seg_gb) * kBlk;
-    pc.tok1 = t1 < rows ? t1 : rows;
-    pc.whole = (gb == pc.seg_gb) && (pc.end_gb == seg_end);
-    return pc;
-}
 
 // First of the KEEP score indices (step * G + head) lane li of its token group
 // holds after the reduce-scatter.
@@ -644,15 +527,7 @@ __global__ void __launch_bounds__(32 * G) merge_kernel(const __grid_constant__ D
 }
 
 template <int D, int G>
-cudaError_t launch_t(const DecodeParams& p, cudaStream_t s) {
-    using C = Cfg<D, G>;
-    const size_t smem = C::SMEM + size_t(p.B + 1) * 4;
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         int(smem));
-    if (e != cudaSuccess) return e;
-    decode_kernel<D, G><<<p.num_ctas, kThreads, smem, s>>>(p);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+cudaError_t launch_merge(const DecodeParams& p, cudaStream_t s) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(unsigned(p.B * p.n_kv));
     cfg.blockDim = dim3(32 * G);
@@ -663,9 +538,28 @@ cudaError_t launch_t(const DecodeParams& p, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, merge_kernel<D, G>, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, merge_kernel<D, G>, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
+}
+
+// Attention (CUDA-core kernel for d = 64, tensor-core kernel for d = 128),
+// then the merge as its programmatic dependent.
+template <int D, int G>
+cudaError_t launch_t(const DecodeParams& p, cudaStream_t s) {
+    cudaError_t e;
+    if constexpr (D == 128) {
+        e = launch_decode_tc(p, G, s);
+    } else {
+        using C = Cfg<D, G>;
+        const size_t smem = C::SMEM + size_t(p.B + 1) * 4;
+        e = cudaFuncSetAttribute(decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e != cudaSuccess) return e;
+        decode_kernel<D, G><<<p.num_ctas, kThreads, smem, s>>>(p);
+        e = cudaGetLastError();
+    }
+    if (e != cudaSuccess) return e;
+    return launch_merge<D, G>(p, s);
 }
 
 }  // namespace

@@ -1,0 +1,139 @@
+// Split-K work partition shared by the decode kernels.
+//
+// Every (sequence b, KV head g) pair is a *segment* of keys: the retrieval
+// rows or the filled ring slots it reads.  All segments are laid end to end
+// in blocks of 16 tokens and a persistent grid of C CTAs takes C equal
+// contiguous ranges of that axis; a CTA walks its range piece by piece (a
+// piece = the part of one segment inside the range).  Partial results go to
+// workspace slot (segment + CTA), unique because moving along the axis
+// crosses either a segment or a CTA boundary.
+#pragma once
+
+#include <stdint.h>
+
+#include "duo_internal.cuh"
+
+namespace duo {
+namespace {
+
+constexpr int kBlk = 16;   // partition granularity in tokens
+
+__device__ __forceinline__ int blocks_of(int64_t rows) { return int((rows + kBlk - 1) / kBlk); }
+
+__device__ __forceinline__ int64_t rows_r(int len, int64_t cap) {
+    int64_t r = len < 0 ? 0 : len;
+    return r < cap ? r : cap;
+}
+__device__ __forceinline__ int64_t rows_s(int len, int S, int W) {
+    int64_t r = len < 0 ? 0 : len;
+    return r < S + W ? r : S + W;
+}
+
+// Rows each segment of sequence b reads: retrieval rows [r0, r0 + nr) of its
+// cache, streaming slots [0, ns) of its ring.
+struct SeqRows {
+    int64_t r0, nr, ns;
+};
+
+__device__ __forceinline__ SeqRows seq_rows(const DecodeParams& p, int b) {
+    SeqRows x;
+    if (p.r_end == nullptr) {
+        const int L = p.len[b];
+        x.r0 = 0;
+        x.nr = rows_r(L, p.cap);
+        x.ns = rows_s(L, p.S, p.W);
+    } else {
+        int64_t r0 = p.r_begin ? p.r_begin[b] : 0;
+        r0 = r0 < 0 ? 0 : (r0 > p.cap ? p.cap : r0);
+        int64_t r1 = p.r_end[b];
+        r1 = r1 < r0 ? r0 : (r1 > p.cap ? p.cap : r1);
+        x.r0 = r0;
+        x.nr = r1 - r0;
+        int64_t ns = p.s_len ? p.s_len[b] : 0;
+        x.ns = ns < 0 ? 0 : (ns > p.S + p.W ? p.S + p.W : ns);
+    }
+    return x;
+}
+
+// Fill bpre[0..B] (shared) with the running count of 16-token blocks per
+// sequence; warp 0 does a chunked shuffle scan.  Caller syncs afterwards.
+__device__ void build_prefix(const DecodeParams& p, int32_t* bpre) {
+    if (threadIdx.x >= 32) return;
+    const int lane = threadIdx.x;
+    int run = 0;
+    if (lane == 0) bpre[0] = 0;
+    for (int base = 0; base < p.B; base += 32) {
+        const int b = base + lane;
+        int c = 0;
+        if (b < p.B) {
+            const SeqRows x = seq_rows(p, b);
+            c = p.n_r * blocks_of(x.nr) + p.n_s * blocks_of(x.ns);
+        }
+        int x = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (b < p.B) bpre[b + 1] = run + x;
+        run += __shfl_sync(0xffffffffu, x, 31);
+    }
+}
+
+// First block index owned by CTA c when `total` blocks are split over n CTAs.
+__device__ __forceinline__ int64_t cta_start(int64_t c, int64_t total, int64_t n) { return c * total / n; }
+// CTA that owns block gb.
+__device__ __forceinline__ int cta_owner(int64_t gb, int64_t total, int64_t n) {
+    int64_t c = ((gb + 1) * n - 1) / total;
+    return int(c < n - 1 ? c : n - 1);
+}
+
+struct Piece {
+    int b, g, seg;          // sequence, KV head, segment index b * n_kv + g
+    int64_t row0;           // first cache row of the segment (retrieval row ranges)
+    int64_t seg_gb;         // first global block of the segment
+    int seg_nb;             // blocks in the segment
+    int64_t tok0, tok1;     // token rows of this piece inside the segment
+    int64_t end_gb;         // global block after the piece
+    bool whole;             // the piece is the whole segment
+};
+
+// Locate the piece that starts at global block gb (gb < range end).
+__device__ __forceinline__ Piece locate(const DecodeParams& p, const int32_t* bpre, int64_t gb,
+                                        int64_t range_end) {
+    Piece pc;
+    // b = last index with bpre[b] <= gb  (binary search over B + 1 entries)
+    int lo = 0, hi = p.B;   // invariant: bpre[lo] <= gb < bpre[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (bpre[mid] <= gb) lo = mid; else hi = mid;
+    }
+    pc.b = lo;
+    const SeqRows x = seq_rows(p, lo);
+    const int64_t rr = x.nr, rs = x.ns;
+    const int nbr = blocks_of(rr), nbs = blocks_of(rs);
+    const int64_t local = gb - bpre[lo];
+    int g = 0;
+    int64_t start = 0;
+    for (; g < p.n_kv; ++g) {
+        start = int64_t(p.r_before[g]) * nbr + int64_t(g - p.r_before[g]) * nbs;
+        const int nb = p.is_r[g] ? nbr : nbs;
+        if (local < start + nb) break;
+    }
+    pc.g = g;
+    pc.seg = lo * p.n_kv + g;
+    pc.row0 = p.is_r[g] ? x.r0 : 0;
+    pc.seg_nb = p.is_r[g] ? nbr : nbs;
+    pc.seg_gb = bpre[lo] + start;
+    const int64_t seg_end = pc.seg_gb + pc.seg_nb;
+    pc.end_gb = seg_end < range_end ? seg_end : range_end;
+    const int64_t rows = p.is_r[g] ? rr : rs;
+    pc.tok0 = (gb - pc.seg_gb) * kBlk;
+    const int64_t t1 = (pc.end_gb - pc.seg_gb) * kBlk;
+    pc.tok1 = t1 < rows ? t1 : rows;
+    pc.whole = (gb == pc.seg_gb) && (pc.end_gb == seg_end);
+    return pc;
+}
+
+}  // namespace
+}  // namespace duo

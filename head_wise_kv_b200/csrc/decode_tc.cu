@@ -1,0 +1,561 @@
+// Mixed-head decode attention on the 5th-generation tensor cores (d = 128).
+//
+// Same work as decode.cu (DuoAttention guide, section 2: retrieval KV heads
+// read their full cache, streaming KV heads their sink + window ring) and the
+// same split-K partition (decode_sched.cuh), but the two contractions of a
+// key tile run as tcgen05 MMAs instead of CUDA-core FMAs:
+//
+//   S^T = K_tile Q^T      M = 128 keys, N = 16, K = d = 128    (bf16 x bf16)
+//   O^T += V_tile^T P^T   M = d = 128,  N = 16, K = 128 keys   (bf16 x bf16)
+//
+// N = 16 holds the G query heads that share the KV head ("Multi-Query and
+// Grouped-Query Attention": one K/V tile feeds all of them).  For the second
+// product each probability is split into two bf16 terms, P = P_hi + P_lo
+// (columns h and G + h of P^T), so P keeps ~16 significant bits although the
+// MMA takes it in bf16; the two output columns are added in the epilogue.
+// Decode at G <= 8 is bound by HBM, not by the tensor cores (they run at a
+// small fraction of their peak here): moving the dot products off the
+// CUDA cores is what lets the kernel stream K/V at the memory's rate, since
+// the FMA version issues ~40 warp instructions per 512-byte token.
+//
+// One persistent CTA per SM, 7 warps:
+//   warp 0     stages each piece's q rows into shared memory (K-major,
+//              128-byte swizzle) and, one lane, issues the TMA loads of the
+//              K tiles (3-D tensor maps over [head][row][dim], rows past the
+//              cache read as zeros) into a 3-stage ring, L2 evict-first
+//   warp 6     the same for the V tiles, into their own ring: a K buffer is
+//              released as soon as its S product has completed, a V buffer
+//              once its PV product has, so neither waits on the other
+//   warp 1     allocates TMEM (S^T double-buffered, O^T) and, one lane,
+//              issues the MMAs from an event loop: S_j as soon as K_j and an
+//              S buffer are there, PV_j as soon as P_j is, so the softmax of
+//              tile j overlaps the products of its neighbours
+//   warps 2-5  softmax: thread = TMEM lane = key row of the tile; running max
+//              per head in the log2 domain with lazy rescaling (O^T rescaled
+//              in TMEM only when a tile's max exceeds it by more than 2^8);
+//              P^T written to shared memory; per-piece epilogue (thread = the
+//              output dimension) writes `out` or the workspace partial.
+//
+// Every mbarrier wait is bounded; on a timeout the CTA sets
+// DUO_STATUS_WAIT_TIMEOUT, stops, waits (bounded) for its copies and MMAs in
+// flight, frees TMEM and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math_constants.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "decode_sched.cuh"
+#include "duo_internal.cuh"
+#include "tcgen05.cuh"
+
+namespace duo {
+
+namespace {
+
+constexpr int kD = 128;                       // head dim
+constexpr int kT = 128;                       // keys per tile
+constexpr int kN = 16;                        // MMA N (query-head columns)
+constexpr int kThreads = 224;
+constexpr int kSoftWarp0 = 2;              // softmax warps 2-5
+constexpr int kVWarp = 6;
+constexpr uint32_t kSlab = 128 * 128;         // 128 rows x 64 bf16: one dim-half of a tile
+constexpr uint32_t kTileBytes = 2 * kSlab;    // 32 KB: one of K or V
+constexpr uint32_t kSmall = kN * kD * 2;      // 4 KB: the q or P^T operand (16 rows)
+constexpr uint32_t kTmemCols = 128;
+constexpr uint32_t kTmemS0 = 0, kTmemS1 = 32, kTmemO = 64;
+constexpr float kNegBig = -1.0e30f;
+constexpr float kRescaleThreshold = 8.0f;     // log2 units: probabilities stay <= 2^8
+
+constexpr uint32_t kIdescQK = idesc_f16(kT, kN, true, false, false);   // A = K (K-major), B = q (K-major)
+constexpr uint32_t kIdescPV = idesc_f16(kD, kN, true, true, false);    // A = V^T (MN-major), B = P^T
+
+// Byte offset of 16-byte chunk c (0..15, along the 128 dims or keys) of row
+// r (0..15) in a 16-row K-major operand with 128-byte swizzle: two 2 KB
+// halves (dims / keys 0-63 and 64-127), each two 8-row groups of 1 KB.
+__device__ __forceinline__ uint32_t small_off(int r, int c) {
+    return uint32_t((c >> 3) * 2048 + (r >> 3) * 1024 + (r & 7) * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+__device__ __forceinline__ int tiles_of(const Piece& pc) { return int((pc.tok1 - pc.tok0 + kT - 1) / kT); }
+
+// Position in the CTA's sequence of tiles: piece `pi` (its locate() result
+// in pc), tile t of its nt.
+struct TileCursor {
+    Piece pc;
+    int pi, t, nt;
+    bool valid;
+
+    __device__ void start(const DecodeParams& p, const int32_t* bpre, int64_t gb_begin, int64_t gb_end) {
+        pi = 0;
+        t = 0;
+        valid = gb_begin < gb_end;
+        if (valid) {
+            pc = locate(p, bpre, gb_begin, gb_end);
+            nt = tiles_of(pc);
+        }
+    }
+    __device__ void advance(const DecodeParams& p, const int32_t* bpre, int64_t gb_end) {
+        if (++t < nt) return;
+        t = 0;
+        ++pi;
+        valid = pc.end_gb < gb_end;
+        if (valid) {
+            pc = locate(p, bpre, pc.end_gb, gb_end);
+            nt = tiles_of(pc);
+        }
+    }
+};
+
+__device__ __forceinline__ bool timed_wait(uint32_t bar, uint32_t parity, const DecodeParams& p,
+                                           volatile int* abort_flag) {
+    if (*abort_flag) return false;
+    if (mbar_wait(bar, parity, p.timeout_ns)) return true;
+    set_status(p.status, DUO_STATUS_WAIT_TIMEOUT);
+    *abort_flag = 1;
+    return false;
+}
+
+// Lane 0 waits for the warp.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const DecodeParams& p,
+                                          volatile int* abort_flag) {
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0) ok = timed_wait(bar, parity, p, abort_flag) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
+}
+
+// Barrier over the 128 softmax threads that ORs a flag across them.
+__device__ __forceinline__ bool softmax_barrier_any(bool flag) {
+    uint32_t out;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\t"
+        "setp.ne.u32 pi, %1, 0;\n\t"
+        "bar.red.or.pred po, 1, 128, pi;\n\t"
+        "selp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(out)
+        : "r"(uint32_t(flag))
+        : "memory");
+    return out != 0;
+}
+
+__device__ __forceinline__ uint16_t bf16_bits(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
+
+template <int G>
+__global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_constant__ DecodeParams p) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int nst = p.stages;
+    const uint32_t sK = smem_addr(smem);                  // nst K tiles
+    const uint32_t sV = sK + nst * kTileBytes;            // nst V tiles
+    const uint32_t sQ = sV + nst * kTileBytes;            // 2 q operands (piece parity)
+    const uint32_t sP = sQ + 2 * kSmall;                  // 2 P^T operands (tile parity)
+    int32_t* bpre = reinterpret_cast<int32_t*>(smem + 2 * nst * kTileBytes + 4 * kSmall);
+
+    constexpr int kMaxStages = 3;
+    __shared__ __align__(8) uint64_t full_k[kMaxStages], full_v[kMaxStages], empty_k[kMaxStages],
+        empty_v[kMaxStages], q_full[2],
+        q_empty[2], s_full[2], s_free[2], p_full[2], p_free[2], mma_fin;
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ float red_max[2][4][G];
+    __shared__ float red_l[4][G];
+    __shared__ int abort_sh;
+    volatile int* abort_flag = &abort_sh;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < nst; ++s) {
+            mbar_init(smem_addr(&full_k[s]), 1);
+            mbar_init(smem_addr(&full_v[s]), 1);
+            mbar_init(smem_addr(&empty_k[s]), 1);
+            mbar_init(smem_addr(&empty_v[s]), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(smem_addr(&q_full[s]), 1);
+            mbar_init(smem_addr(&q_empty[s]), 1);
+            mbar_init(smem_addr(&s_full[s]), 1);
+            mbar_init(smem_addr(&s_free[s]), 4);
+            mbar_init(smem_addr(&p_full[s]), 4);
+            mbar_init(smem_addr(&p_free[s]), 1);
+        }
+        mbar_init(smem_addr(&mma_fin), 1);
+        abort_sh = 0;
+        fence_mbar_init();
+    }
+    // q and P^T rows past the heads in use stay zero (their S / O columns are never read)
+    for (uint32_t o = threadIdx.x * 16; o < 4 * kSmall; o += kThreads * 16) st_shared_v4(sQ + o, make_uint4(0, 0, 0, 0));
+    fence_proxy_async_smem();
+    if (warp == 1) tmem_alloc(smem_addr(&tmem_base_sh), kTmemCols);
+    build_prefix(p, bpre);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    // The merge kernel may be scheduled now; it waits (griddepcontrol.wait)
+    // for this grid's completion before it reads any partial.
+    asm volatile("griddepcontrol.launch_dependents;");
+    const uint32_t tmem = tmem_base_sh;
+
+    const int64_t total = bpre[p.B];
+    const int64_t n = p.num_ctas;
+    const int64_t gb_begin = total > 0 ? cta_start(blockIdx.x, total, n) : 0;
+    const int64_t gb_end = total > 0 ? cta_start(blockIdx.x + 1, total, n) : 0;
+
+    if (gb_begin < gb_end) {
+        if (warp == 0) {
+            // ======================================================== q + TMA producer
+            const uint64_t policy = l2_evict_first_policy();
+            uint32_t it = 0;   // tiles issued (lane 0)
+            bool ok = true;
+            int pi = 0;
+            for (int64_t gb = gb_begin; ok && gb < gb_end; ++pi) {
+                const Piece pc = locate(p, bpre, gb, gb_end);
+                gb = pc.end_gb;
+                if (!warp_wait(smem_addr(&q_empty[pi & 1]), ((pi >> 1) & 1) ^ 1, p, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const uint16_t* qb = p.q + (size_t(pc.b) * p.hq + size_t(pc.g) * G) * kD;
+                const uint32_t qs = sQ + (pi & 1) * kSmall;
+                for (int c = lane; c < G * 16; c += 32) {
+                    const int h = c >> 4, c16 = c & 15;
+                    st_shared_v4(qs + small_off(h, c16), *reinterpret_cast<const uint4*>(qb + h * kD + c16 * 8));
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(smem_addr(&q_full[pi & 1]));
+                    const bool retr = p.is_r[pc.g] != 0;
+                    const CUtensorMap* mk = retr ? &p.tm_kr : &p.tm_ks;
+                    const int z = retr ? pc.b * p.n_r + p.rank[pc.g] : pc.b * p.n_s + p.rank[pc.g];
+                    for (int64_t t = pc.tok0; t < pc.tok1; t += kT, ++it) {
+                        const int st = int(it % uint32_t(nst));
+                        if (!timed_wait(smem_addr(&empty_k[st]), ((it / nst) & 1) ^ 1, p, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        const int y = int(pc.row0 + t);
+                        const uint32_t fk = smem_addr(&full_k[st]);
+                        mbar_arrive_expect_tx(fk, kTileBytes);
+                        tma_load_3d(sK + st * kTileBytes, mk, 0, y, z, fk, policy);
+                        tma_load_3d(sK + st * kTileBytes + kSlab, mk, 64, y, z, fk, policy);
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            }
+            if (lane == 0) {
+                // do not leave while copies may still land in this CTA's shared memory
+                for (uint32_t k = 0; k < uint32_t(nst) && k < it; ++k) {
+                    const uint32_t last = it - 1 - k;
+                    mbar_wait(smem_addr(&full_k[last % nst]), (last / nst) & 1, p.timeout_ns);
+                }
+            }
+        } else if (warp == kVWarp) {
+            // ======================================================== V producer
+            if (lane == 0) {
+                const uint64_t policy = l2_evict_first_policy();
+                uint32_t it = 0;
+                bool ok = true;
+                for (int64_t gb = gb_begin; ok && gb < gb_end;) {
+                    const Piece pc = locate(p, bpre, gb, gb_end);
+                    gb = pc.end_gb;
+                    const bool retr = p.is_r[pc.g] != 0;
+                    const CUtensorMap* mv = retr ? &p.tm_vr : &p.tm_vs;
+                    const int z = retr ? pc.b * p.n_r + p.rank[pc.g] : pc.b * p.n_s + p.rank[pc.g];
+                    for (int64_t t = pc.tok0; t < pc.tok1; t += kT, ++it) {
+                        const int st = int(it % uint32_t(nst));
+                        if (!timed_wait(smem_addr(&empty_v[st]), ((it / nst) & 1) ^ 1, p, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        const int y = int(pc.row0 + t);
+                        const uint32_t fv = smem_addr(&full_v[st]);
+                        mbar_arrive_expect_tx(fv, kTileBytes);
+                        tma_load_3d(sV + st * kTileBytes, mv, 0, y, z, fv, policy);
+                        tma_load_3d(sV + st * kTileBytes + kSlab, mv, 64, y, z, fv, policy);
+                    }
+                }
+                for (uint32_t k = 0; k < uint32_t(nst) && k < it; ++k) {
+                    const uint32_t last = it - 1 - k;
+                    mbar_wait(smem_addr(&full_v[last % nst]), (last / nst) & 1, p.timeout_ns);
+                }
+            }
+        } else if (warp == 1) {
+            // ======================================================== MMA issuer
+            // An event loop over two cursors: S_j needs K_j and a free S buffer,
+            // PV_j needs P_j; whichever is ready goes first, so that PV_j (and
+            // with it the release of stage j) never waits on the arrival of
+            // K_{j+1}.
+            if (lane == 0) {
+                TileCursor cq, cv;   // next S tile, next PV tile
+                cq.start(p, bpre, gb_begin, gb_end);
+                cv.start(p, bpre, gb_begin, gb_end);
+                uint32_t jq = 0, jv = 0;
+                bool ok = true;
+                unsigned long long last = global_ns();
+                while (ok && cv.valid) {
+                    bool progressed = false;
+                    if (cq.valid) {
+                        const int st = int(jq % uint32_t(nst));
+                        if ((cq.t > 0 || mbar_test_wait(smem_addr(&q_full[cq.pi & 1]), (cq.pi >> 1) & 1)) &&
+                            mbar_test_wait(smem_addr(&full_k[st]), (jq / nst) & 1) &&
+                            mbar_test_wait(smem_addr(&s_free[jq & 1]), ((jq >> 1) & 1) ^ 1)) {
+                            tc_fence_after();
+                            const uint32_t sk = sK + st * kTileBytes, sq = sQ + (cq.pi & 1) * kSmall;
+#pragma unroll
+                            for (int k = 0; k < kD / 16; ++k) {
+                                const uint32_t off = (k >> 2) * kSlab + (k & 3) * 32;
+                                const uint32_t qoff = (k >> 2) * 2048 + (k & 3) * 32;
+                                umma_f16(tmem + ((jq & 1) ? kTmemS1 : kTmemS0), smem_desc(sk + off, 16, 1024),
+                                         smem_desc(sq + qoff, 16, 1024), kIdescQK, k > 0 ? 1u : 0u);
+                            }
+                            umma_commit(smem_addr(&s_full[jq & 1]));
+                            umma_commit(smem_addr(&empty_k[st]));
+                            if (cq.t == cq.nt - 1) umma_commit(smem_addr(&q_empty[cq.pi & 1]));
+                            ++jq;
+                            cq.advance(p, bpre, gb_end);
+                            progressed = true;
+                        }
+                    }
+                    if (jv < jq) {
+                        const int st = int(jv % uint32_t(nst));
+                        if (mbar_test_wait(smem_addr(&p_full[jv & 1]), (jv >> 1) & 1) &&
+                            mbar_test_wait(smem_addr(&full_v[st]), (jv / nst) & 1)) {
+                            tc_fence_after();
+                            const uint32_t sv = sV + st * kTileBytes, sp = sP + (jv & 1) * kSmall;
+#pragma unroll
+                            for (int k = 0; k < kT / 16; ++k)
+                                umma_f16(tmem + kTmemO, smem_desc(sv + k * 2048, kSlab, 1024),
+                                         smem_desc(sp + (k >> 2) * 2048 + (k & 3) * 32, 16, 1024), kIdescPV,
+                                         (cv.t > 0 || k > 0) ? 1u : 0u);
+                            umma_commit(smem_addr(&empty_v[st]));
+                            umma_commit(smem_addr(&p_free[jv & 1]));
+                            ++jv;
+                            cv.advance(p, bpre, gb_end);
+                            progressed = true;
+                        }
+                    }
+                    if (progressed) {
+                        last = global_ns();
+                    } else if (*abort_flag) {
+                        ok = false;
+                    } else if (global_ns() - last > p.timeout_ns) {
+                        set_status(p.status, DUO_STATUS_WAIT_TIMEOUT);
+                        *abort_flag = 1;
+                        ok = false;
+                    }
+                }
+                // every MMA issued by this thread has completed before TMEM is freed
+                umma_commit(smem_addr(&mma_fin));
+                mbar_wait(smem_addr(&mma_fin), 0, p.timeout_ns);
+            }
+        } else {
+            // ======================================================== softmax + epilogue
+            const int sw = warp - kSoftWarp0;              // 0..3
+            const int sub = warp & 3;                      // TMEM lane quarter this warp may access
+            const int row = sub * 32 + lane;               // key row of S^T; output dim of O^T
+            const uint32_t lane_off = uint32_t(sub * 32) << 16;
+            uint32_t j = 0;
+            bool ok = true;
+            for (int64_t gb = gb_begin; ok && gb < gb_end;) {
+                const Piece pc = locate(p, bpre, gb, gb_end);
+                gb = pc.end_gb;
+                float m[G], l[G];
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    m[h] = kNegBig;
+                    l[h] = 0.f;
+                }
+                const int nt = tiles_of(pc);
+                const int64_t rows_total = pc.tok1 - pc.tok0;
+                for (int t = 0; t < nt; ++t, ++j) {
+                    const uint32_t sb = j & 1;
+                    const int st = int(j % uint32_t(nst));
+                    const bool got = warp_wait(smem_addr(&s_full[sb]), (j >> 1) & 1, p, abort_flag);
+                    float s[G];
+                    if (got) {
+                        tc_fence_after();
+                        uint32_t u[G];
+                        tmem_ldn<G>(tmem + lane_off + (sb ? kTmemS1 : kTmemS0), u);
+                        tmem_wait_ld();
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(smem_addr(&s_free[sb]));
+#pragma unroll
+                        for (int h = 0; h < G; ++h) s[h] = __uint_as_float(u[h]);
+                    }
+                    const int64_t left = rows_total - int64_t(t) * kT;
+                    const int valid_rows = int(left < kT ? left : kT);
+                    const bool valid = got && row < valid_rows;
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        s[h] = valid ? s[h] * p.scale_log2 : -CUDART_INF_F;
+                        const float mx = warp_max_f32(s[h]);
+                        if (lane == 0) red_max[sb][sw][h] = mx;
+                    }
+                    // the barrier also agrees on aborting
+                    if (softmax_barrier_any(!got || *abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    bool grow_any = false;
+                    float alpha[G];
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        const float mt = fmaxf(fmaxf(red_max[sb][0][h], red_max[sb][1][h]),
+                                               fmaxf(red_max[sb][2][h], red_max[sb][3][h]));
+                        const bool grow = mt > m[h] + kRescaleThreshold;
+                        const float mn = grow ? mt : m[h];
+                        alpha[h] = fast_exp2(m[h] - mn);   // 1 when the max is kept
+                        m[h] = mn;
+                        l[h] *= alpha[h];
+                        grow_any |= grow;
+                    }
+                    // P^T buffer sb is free once PV_{j-2} has completed
+                    if (!warp_wait(smem_addr(&p_free[sb]), ((j >> 1) & 1) ^ 1, p, abort_flag)) continue;
+                    const uint32_t pb = sP + sb * kSmall + (row & 7) * 2;   // key `row` of P^T
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        const float pr = fast_exp2(s[h] - m[h]);   // 0 for rows outside the piece
+                        l[h] += pr;
+                        const uint16_t hi = bf16_bits(pr);
+                        const uint16_t lo = bf16_bits(pr - __uint_as_float(uint32_t(hi) << 16));
+                        st_shared_u16(pb + small_off(h, row >> 3), hi);
+                        st_shared_u16(pb + small_off(G + h, row >> 3), lo);
+                    }
+                    if (valid_rows < kT) {
+                        // Rows past the piece get P = 0; clear their V rows too, so
+                        // that whatever the memory there holds adds exactly 0.
+                        if (!warp_wait(smem_addr(&full_v[st]), (j / nst) & 1, p, abort_flag)) continue;
+                        if (row >= valid_rows) {
+                            const uint32_t vr = sV + st * kTileBytes + row * 128;
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) {
+                                st_shared_v4(vr + c * 16, make_uint4(0, 0, 0, 0));
+                                st_shared_v4(vr + kSlab + c * 16, make_uint4(0, 0, 0, 0));
+                            }
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    if (t > 0 && grow_any) {
+                        // rescale O^T (rows = dims) once PV_{j-1} has landed
+                        if (!warp_wait(smem_addr(&p_free[(j - 1) & 1]), ((j - 1) >> 1) & 1, p, abort_flag)) continue;
+                        tc_fence_after();
+                        uint32_t u[2 * G];
+                        tmem_ldn<2 * G>(tmem + lane_off + kTmemO, u);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int h = 0; h < G; ++h) {
+                            u[h] = __float_as_uint(__uint_as_float(u[h]) * alpha[h]);
+                            u[G + h] = __float_as_uint(__uint_as_float(u[G + h]) * alpha[h]);
+                        }
+                        tmem_stn<2 * G>(tmem + lane_off + kTmemO, u);
+                        tmem_wait_st();
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_addr(&p_full[sb]));
+                }
+                if (!ok) break;
+
+                // ---- epilogue: O^T of the piece is final once PV of its last tile landed
+                const uint32_t jl = j - 1;
+                const bool got = warp_wait(smem_addr(&p_free[jl & 1]), (jl >> 1) & 1, p, abort_flag);
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    float x = l[h];
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+                    if (lane == 0) red_l[sw][h] = x;
+                }
+                if (softmax_barrier_any(!got || *abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t u[2 * G];
+                tmem_ldn<2 * G>(tmem + lane_off + kTmemO, u);
+                tmem_wait_ld();
+                tc_fence_before();
+                const int d = row;
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    const float o = __uint_as_float(u[h]) + __uint_as_float(u[G + h]);
+                    const float L = red_l[0][h] + red_l[1][h] + red_l[2][h] + red_l[3][h];
+                    const int qh = pc.g * G + h;
+                    if (pc.whole) {
+                        p.out[(size_t(pc.b) * p.hq + qh) * kD + d] = L > 0.f ? o / L : 0.f;
+                        if (d == 0 && p.lse != nullptr)
+                            p.lse[size_t(pc.b) * p.hq + qh] =
+                                L > 0.f ? (m[h] + __log2f(L)) * 0.69314718055994530942f : -CUDART_INF_F;
+                    } else {
+                        const size_t slot = size_t(pc.seg) + blockIdx.x;
+                        p.ws_o[(slot * G + h) * kD + d] = o;
+                        if (d == 0) {
+                            p.ws_ml[(slot * G + h) * 2 + 0] = m[h];
+                            p.ws_ml[(slot * G + h) * 2 + 1] = L;
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+template <int G>
+cudaError_t launch_g(const DecodeParams& p, cudaStream_t s) {
+    DecodeParams q = p;
+    const size_t fixed = 4 * size_t(kSmall) + size_t(p.B + 1) * 4 + 1024;
+    q.stages = fixed + 3 * 2 * size_t(kTileBytes) <= size_t(227) * 1024 ? 3 : 2;
+    const size_t smem = fixed + size_t(q.stages) * 2 * kTileBytes;
+    if (smem > size_t(227) * 1024) return cudaErrorInvalidConfiguration;
+    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    decode_tc_kernel<G><<<p.num_ctas, kThreads, smem, s>>>(q);
+    return cudaGetLastError();
+}
+
+// 3-D map [heads][rows][128 dims] of bf16, box 64 dims x 128 rows x 1 head, 128-byte swizzle.
+bool make_map3(CUtensorMap* m, const void* base, uint64_t rows, uint64_t heads) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {uint64_t(kD), rows < 1 ? 1 : rows, heads < 1 ? 1 : heads};
+    cuuint64_t strides[2] = {uint64_t(kD) * 2, (rows < 1 ? 1 : rows) * uint64_t(kD) * 2};
+    cuuint32_t box[3] = {64, uint32_t(kT), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool make_decode_maps(DecodeMaps* m, const void* kr, const void* vr, const void* ks, const void* vs, int B, int n_r,
+                      int n_s, int64_t cap, int SW) {
+    return make_map3(&m->kr, kr, uint64_t(cap), uint64_t(B) * n_r) &&
+           make_map3(&m->vr, vr, uint64_t(cap), uint64_t(B) * n_r) &&
+           make_map3(&m->ks, ks, uint64_t(SW), uint64_t(B) * n_s) &&
+           make_map3(&m->vs, vs, uint64_t(SW), uint64_t(B) * n_s);
+}
+
+cudaError_t launch_decode_tc(const DecodeParams& p, int group, cudaStream_t s) {
+    switch (group) {
+        case 1: return launch_g<1>(p, s);
+        case 2: return launch_g<2>(p, s);
+        case 4: return launch_g<4>(p, s);
+        case 8: return launch_g<8>(p, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace duo

@@ -2,6 +2,7 @@
 // Not part of the C ABI (include/duo_kv.h is).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -22,6 +23,12 @@ struct LayerLayout {
     uint8_t is_r[kMaxKvHeads];
 };
 
+// TMA descriptors of one layer's caches for the tensor-core decode
+// ([head][row][dim] bf16, 128-row boxes).
+struct DecodeMaps {
+    CUtensorMap kr, vr, ks, vs;
+};
+
 }  // namespace duo
 
 struct duo_kv {
@@ -33,12 +40,14 @@ struct duo_kv {
     int device = 0;
     int num_sms = 0;
     int decode_ctas = 0;                    // 0 = default persistent wave
+    std::vector<duo::DecodeMaps> maps;      // per layer (head_dim 128 only)
 };
 
 namespace duo {
 
 // ----------------------------------------------------------------- launch params
 struct DecodeParams {
+    CUtensorMap tm_kr, tm_vr, tm_ks, tm_vs;   // tensor-core kernel (head_dim 128)
     const uint16_t* kr;
     const uint16_t* vr;
     const uint16_t* ks;
@@ -56,6 +65,7 @@ struct DecodeParams {
     int64_t cap;
     int B, n_kv, hq, n_r, n_s, S, W;
     int num_ctas;
+    int stages;               // tensor-core kernel pipeline depth (set by its launcher)
     float scale_log2;
     unsigned long long timeout_ns;
     int32_t rank[kMaxKvHeads];
@@ -107,6 +117,9 @@ cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 int decode_ctas_default(int num_sms, int d, int group);
 size_t decode_workspace_bytes(int slots, int d, int group);
 cudaError_t launch_decode(const DecodeParams& p, int d, int group, cudaStream_t s);
+cudaError_t launch_decode_tc(const DecodeParams& p, int group, cudaStream_t s);   // attention only
+bool make_decode_maps(DecodeMaps* m, const void* kr, const void* vr, const void* ks, const void* vs, int B, int n_r,
+                      int n_s, int64_t cap, int SW);
 cudaError_t launch_lse_merge(int parts, int rows, int d, const float* part_out, const float* part_lse, float* out,
                              float* lse, cudaStream_t s);
 cudaError_t launch_blend(int64_t n, int hq, int d, const float* alpha, const float* full, const float* strm,
@@ -143,6 +156,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Non-blocking probe of an mbarrier phase (never suspends the thread).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(bar), "r"(parity)

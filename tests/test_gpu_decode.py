@@ -106,7 +106,10 @@ def test_streaming_slot_order_does_not_matter():
     views["positions"].copy_(views["positions"][:, perm].clone())
     b = cache.decode(0, q, lens, w.scale)
     m, r = errors(b.cpu().numpy(), a.cpu().numpy())
-    assert m < 1e-5 and r < 1e-6
+    # Up to rounding: the probabilities enter the PV product as a sum of two
+    # bf16 terms (~2^-16 relative), and the running max that scales them
+    # depends on which keys the first tile holds.
+    assert m < 1e-4 and r < 2e-5
 
 
 def test_empty_and_over_capacity_status():
