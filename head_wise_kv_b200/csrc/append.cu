@@ -29,6 +29,9 @@ constexpr int kThreads = 256;
 
 template <int D>
 __global__ void __launch_bounds__(kThreads) append_kernel(const __grid_constant__ AppendParams p) {
+    // A decode launched next as a programmatic dependent may start its
+    // set-up now; it waits (griddepcontrol.wait) for this grid's writes.
+    asm volatile("griddepcontrol.launch_dependents;");
     constexpr int TPR = D / 8;   // threads per row, 16 bytes each
     const int64_t rows_total = int64_t(p.B) * p.n_kv * p.n_new_max;
     const int64_t item = (int64_t(blockIdx.x) * kThreads + threadIdx.x) / TPR;

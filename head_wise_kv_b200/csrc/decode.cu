@@ -150,7 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     __shared__ __align__(8) uint64_t empty_bar[kStages];
     __shared__ int abort_flag;
 
-    // bpre lives after the reduction buffer; sized B + 1 by the launcher
+    // the sequence table lives after the reduction buffer; sized by the launcher
     int32_t* bpre = reinterpret_cast<int32_t*>(red + C::RED_FLOATS);
 
     const int warp = threadIdx.x >> 5;
@@ -531,7 +531,7 @@ cudaError_t launch_merge(const DecodeParams& p, cudaStream_t s) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(unsigned(p.B * p.n_kv));
     cfg.blockDim = dim3(32 * G);
-    cfg.dynamicSmemBytes = size_t(p.B + 1) * 4;
+    cfg.dynamicSmemBytes = seq_table_bytes(p.B);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -552,7 +552,7 @@ cudaError_t launch_t(const DecodeParams& p, cudaStream_t s) {
         e = launch_decode_tc(p, G, s);
     } else {
         using C = Cfg<D, G>;
-        const size_t smem = C::SMEM + size_t(p.B + 1) * 4;
+        const size_t smem = C::SMEM + seq_table_bytes(p.B);
         e = cudaFuncSetAttribute(decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         if (e != cudaSuccess) return e;
         decode_kernel<D, G><<<p.num_ctas, kThreads, smem, s>>>(p);

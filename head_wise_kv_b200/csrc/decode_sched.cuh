@@ -55,8 +55,14 @@ __device__ __forceinline__ SeqRows seq_rows(const DecodeParams& p, int b) {
     return x;
 }
 
-// Fill bpre[0..B] (shared) with the running count of 16-token blocks per
-// sequence; warp 0 does a chunked shuffle scan.  Caller syncs afterwards.
+// Shared-memory sequence table built once per launch: int32 words
+// [0, B]  running count of 16-token blocks per sequence (prefix),
+// then three arrays of B: first retrieval row, retrieval rows, ring slots.
+// Locating a piece then reads shared memory only (a global read of the
+// lengths costs microseconds while the kernel saturates HBM).
+__host__ __device__ constexpr size_t seq_table_bytes(int B) { return (size_t(B + 1) + 3 * size_t(B)) * 4; }
+
+// Fill the table (shared); warp 0 does a chunked shuffle scan.  Caller syncs afterwards.
 __device__ void build_prefix(const DecodeParams& p, int32_t* bpre) {
     if (threadIdx.x >= 32) return;
     const int lane = threadIdx.x;
@@ -68,6 +74,10 @@ __device__ void build_prefix(const DecodeParams& p, int32_t* bpre) {
         if (b < p.B) {
             const SeqRows x = seq_rows(p, b);
             c = p.n_r * blocks_of(x.nr) + p.n_s * blocks_of(x.ns);
+            int32_t* rows = bpre + p.B + 1;
+            rows[b] = int32_t(x.r0);
+            rows[p.B + b] = int32_t(x.nr);
+            rows[2 * p.B + b] = int32_t(x.ns);
         }
         int x = c;
 #pragma unroll
@@ -109,8 +119,8 @@ __device__ __forceinline__ Piece locate(const DecodeParams& p, const int32_t* bp
         if (bpre[mid] <= gb) lo = mid; else hi = mid;
     }
     pc.b = lo;
-    const SeqRows x = seq_rows(p, lo);
-    const int64_t rr = x.nr, rs = x.ns;
+    const int32_t* tab = bpre + p.B + 1;
+    const int64_t r0 = tab[lo], rr = tab[p.B + lo], rs = tab[2 * p.B + lo];
     const int nbr = blocks_of(rr), nbs = blocks_of(rs);
     const int64_t local = gb - bpre[lo];
     int g = 0;
@@ -122,7 +132,7 @@ __device__ __forceinline__ Piece locate(const DecodeParams& p, const int32_t* bp
     }
     pc.g = g;
     pc.seg = lo * p.n_kv + g;
-    pc.row0 = p.is_r[g] ? x.r0 : 0;
+    pc.row0 = p.is_r[g] ? r0 : 0;
     pc.seg_nb = p.is_r[g] ? nbr : nbs;
     pc.seg_gb = bpre[lo] + start;
     const int64_t seg_end = pc.seg_gb + pc.seg_nb;

@@ -18,11 +18,12 @@
 // CUDA cores is what lets the kernel stream K/V at the memory's rate, since
 // the FMA version issues ~40 warp instructions per 512-byte token.
 //
-// One persistent CTA per SM, 7 warps:
-//   warp 0     stages each piece's q rows into shared memory (K-major,
-//              128-byte swizzle) and, one lane, issues the TMA loads of the
-//              K tiles (3-D tensor maps over [head][row][dim], rows past the
-//              cache read as zeros) into a 3-stage ring, L2 evict-first
+// One persistent CTA per SM, 12 warps:
+//   warp 7     stages each piece's q rows into shared memory (K-major,
+//              128-byte swizzle), up to two pieces ahead
+//   warp 0     one lane issues the TMA loads of the K tiles (3-D tensor
+//              maps over [head][row][dim], rows past the cache read as
+//              zeros) into a 3-stage ring, L2 evict-first
 //   warp 6     the same for the V tiles, into their own ring: a K buffer is
 //              released as soon as its S product has completed, a V buffer
 //              once its PV product has, so neither waits on the other
@@ -33,8 +34,12 @@
 //   warps 2-5  softmax: thread = TMEM lane = key row of the tile; running max
 //              per head in the log2 domain with lazy rescaling (O^T rescaled
 //              in TMEM only when a tile's max exceeds it by more than 2^8);
-//              P^T written to shared memory; per-piece epilogue (thread = the
-//              output dimension) writes `out` or the workspace partial.
+//              P^T written to shared memory; at the end of a piece, the row
+//              sums and the max go to the epilogue through shared memory
+//   warps 8-11 epilogue (thread = output dim): O^T is double-buffered in TMEM
+//              by piece parity, so a piece's tail (its last V tile and PV)
+//              never holds up the softmax of the next; writes `out` or the
+//              workspace partial.
 //
 // Every mbarrier wait is bounded; on a timeout the CTA sets
 // DUO_STATUS_WAIT_TIMEOUT, stops, waits (bounded) for its copies and MMAs in
@@ -57,14 +62,16 @@ namespace {
 constexpr int kD = 128;                       // head dim
 constexpr int kT = 128;                       // keys per tile
 constexpr int kN = 16;                        // MMA N (query-head columns)
-constexpr int kThreads = 224;
+constexpr int kThreads = 384;
 constexpr int kSoftWarp0 = 2;              // softmax warps 2-5
 constexpr int kVWarp = 6;
+constexpr int kQWarp = 7;
+constexpr int kEpiWarp0 = 8;               // epilogue warps 8-11
 constexpr uint32_t kSlab = 128 * 128;         // 128 rows x 64 bf16: one dim-half of a tile
 constexpr uint32_t kTileBytes = 2 * kSlab;    // 32 KB: one of K or V
 constexpr uint32_t kSmall = kN * kD * 2;      // 4 KB: the q or P^T operand (16 rows)
 constexpr uint32_t kTmemCols = 128;
-constexpr uint32_t kTmemS0 = 0, kTmemS1 = 32, kTmemO = 64;
+constexpr uint32_t kTmemS0 = 0, kTmemS1 = 32, kTmemO0 = 64;   // O^T of piece pi at kTmemO0 + 32 (pi & 1)
 constexpr float kNegBig = -1.0e30f;
 constexpr float kRescaleThreshold = 8.0f;     // log2 units: probabilities stay <= 2^8
 
@@ -158,10 +165,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     constexpr int kMaxStages = 3;
     __shared__ __align__(8) uint64_t full_k[kMaxStages], full_v[kMaxStages], empty_k[kMaxStages],
         empty_v[kMaxStages], q_full[2],
-        q_empty[2], s_full[2], s_free[2], p_full[2], p_free[2], mma_fin;
+        q_empty[2], s_full[2], s_free[2], p_full[2], p_free[2], o_full[2], o_empty[2], epi_full[2], mma_fin;
     __shared__ uint32_t tmem_base_sh;
     __shared__ float red_max[2][4][G];
-    __shared__ float red_l[4][G];
+    __shared__ float red_l[2][4][G];   // [piece parity][softmax warp][head] row sums
+    __shared__ float epi_m[2][G];      // [piece parity][head] running max
     __shared__ int abort_sh;
     volatile int* abort_flag = &abort_sh;
 
@@ -181,6 +189,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             mbar_init(smem_addr(&s_free[s]), 4);
             mbar_init(smem_addr(&p_full[s]), 4);
             mbar_init(smem_addr(&p_free[s]), 1);
+            mbar_init(smem_addr(&o_full[s]), 1);
+            mbar_init(smem_addr(&o_empty[s]), 4);
+            mbar_init(smem_addr(&epi_full[s]), 4);
         }
         mbar_init(smem_addr(&mma_fin), 1);
         abort_sh = 0;
@@ -190,6 +201,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     for (uint32_t o = threadIdx.x * 16; o < 4 * kSmall; o += kThreads * 16) st_shared_v4(sQ + o, make_uint4(0, 0, 0, 0));
     fence_proxy_async_smem();
     if (warp == 1) tmem_alloc(smem_addr(&tmem_base_sh), kTmemCols);
+    if (threadIdx.x == 32) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tm_kr)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tm_vr)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tm_ks)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tm_vs)) : "memory");
+    }
+    // Launched as a programmatic dependent: everything above overlaps the
+    // previous kernel in the stream; nothing it writes is read before this.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     build_prefix(p, bpre);
     tc_fence_before();
     __syncthreads();
@@ -206,28 +226,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
 
     if (gb_begin < gb_end) {
         if (warp == 0) {
-            // ======================================================== q + TMA producer
-            const uint64_t policy = l2_evict_first_policy();
-            uint32_t it = 0;   // tiles issued (lane 0)
-            bool ok = true;
-            int pi = 0;
-            for (int64_t gb = gb_begin; ok && gb < gb_end; ++pi) {
-                const Piece pc = locate(p, bpre, gb, gb_end);
-                gb = pc.end_gb;
-                if (!warp_wait(smem_addr(&q_empty[pi & 1]), ((pi >> 1) & 1) ^ 1, p, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                const uint16_t* qb = p.q + (size_t(pc.b) * p.hq + size_t(pc.g) * G) * kD;
-                const uint32_t qs = sQ + (pi & 1) * kSmall;
-                for (int c = lane; c < G * 16; c += 32) {
-                    const int h = c >> 4, c16 = c & 15;
-                    st_shared_v4(qs + small_off(h, c16), *reinterpret_cast<const uint4*>(qb + h * kD + c16 * 8));
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(smem_addr(&q_full[pi & 1]));
+            // ======================================================== K producer
+            if (lane == 0) {
+                const uint64_t policy = l2_evict_first_policy();
+                uint32_t it = 0;
+                bool ok = true;
+                for (int64_t gb = gb_begin; ok && gb < gb_end;) {
+                    const Piece pc = locate(p, bpre, gb, gb_end);
+                    gb = pc.end_gb;
                     const bool retr = p.is_r[pc.g] != 0;
                     const CUtensorMap* mk = retr ? &p.tm_kr : &p.tm_ks;
                     const int z = retr ? pc.b * p.n_r + p.rank[pc.g] : pc.b * p.n_s + p.rank[pc.g];
@@ -244,14 +250,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                         tma_load_3d(sK + st * kTileBytes + kSlab, mk, 64, y, z, fk, policy);
                     }
                 }
-                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            }
-            if (lane == 0) {
                 // do not leave while copies may still land in this CTA's shared memory
                 for (uint32_t k = 0; k < uint32_t(nst) && k < it; ++k) {
                     const uint32_t last = it - 1 - k;
                     mbar_wait(smem_addr(&full_k[last % nst]), (last / nst) & 1, p.timeout_ns);
                 }
+            }
+        } else if (warp == kQWarp) {
+            // ======================================================== q staging
+            // Runs up to two pieces ahead of the S products (two q buffers).
+            int pi = 0;
+            for (int64_t gb = gb_begin; gb < gb_end; ++pi) {
+                const Piece pc = locate(p, bpre, gb, gb_end);
+                gb = pc.end_gb;
+                if (!warp_wait(smem_addr(&q_empty[pi & 1]), ((pi >> 1) & 1) ^ 1, p, abort_flag)) break;
+                const uint16_t* qb = p.q + (size_t(pc.b) * p.hq + size_t(pc.g) * G) * kD;
+                const uint32_t qs = sQ + (pi & 1) * kSmall;
+                for (int c = lane; c < G * 16; c += 32) {
+                    const int h = c >> 4, c16 = c & 15;
+                    st_shared_v4(qs + small_off(h, c16), *reinterpret_cast<const uint4*>(qb + h * kD + c16 * 8));
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_addr(&q_full[pi & 1]));
             }
         } else if (warp == kVWarp) {
             // ======================================================== V producer
@@ -323,16 +344,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                     if (jv < jq) {
                         const int st = int(jv % uint32_t(nst));
                         if (mbar_test_wait(smem_addr(&p_full[jv & 1]), (jv >> 1) & 1) &&
-                            mbar_test_wait(smem_addr(&full_v[st]), (jv / nst) & 1)) {
+                            mbar_test_wait(smem_addr(&full_v[st]), (jv / nst) & 1) &&
+                            (cv.t > 0 || mbar_test_wait(smem_addr(&o_empty[cv.pi & 1]), ((cv.pi >> 1) & 1) ^ 1))) {
                             tc_fence_after();
                             const uint32_t sv = sV + st * kTileBytes, sp = sP + (jv & 1) * kSmall;
 #pragma unroll
                             for (int k = 0; k < kT / 16; ++k)
-                                umma_f16(tmem + kTmemO, smem_desc(sv + k * 2048, kSlab, 1024),
+                                umma_f16(tmem + kTmemO0 + (cv.pi & 1) * 32, smem_desc(sv + k * 2048, kSlab, 1024),
                                          smem_desc(sp + (k >> 2) * 2048 + (k & 3) * 32, 16, 1024), kIdescPV,
                                          (cv.t > 0 || k > 0) ? 1u : 0u);
                             umma_commit(smem_addr(&empty_v[st]));
                             umma_commit(smem_addr(&p_free[jv & 1]));
+                            if (cv.t == cv.nt - 1) umma_commit(smem_addr(&o_full[cv.pi & 1]));
                             ++jv;
                             cv.advance(p, bpre, gb_end);
                             progressed = true;
@@ -352,17 +375,65 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                 umma_commit(smem_addr(&mma_fin));
                 mbar_wait(smem_addr(&mma_fin), 0, p.timeout_ns);
             }
+        } else if (warp >= kEpiWarp0) {
+            // ======================================================== epilogue
+            // thread = output dim (TMEM lane of O^T); O^T of piece pi is final
+            // once the MMA thread's o_full commit for it has landed.
+            const int sub = warp & 3;
+            const int d = sub * 32 + lane;
+            const uint32_t lane_off = uint32_t(sub * 32) << 16;
+            int pi = 0;
+            for (int64_t gb = gb_begin; gb < gb_end; ++pi) {
+                const Piece pc = locate(p, bpre, gb, gb_end);
+                gb = pc.end_gb;
+                if (!warp_wait(smem_addr(&epi_full[pi & 1]), (pi >> 1) & 1, p, abort_flag) ||
+                    !warp_wait(smem_addr(&o_full[pi & 1]), (pi >> 1) & 1, p, abort_flag))
+                    break;
+                tc_fence_after();
+                uint32_t u[2 * G];
+                tmem_ldn<2 * G>(tmem + lane_off + kTmemO0 + (pi & 1) * 32, u);
+                tmem_wait_ld();
+                float L[G], M[G];
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    L[h] = red_l[pi & 1][0][h] + red_l[pi & 1][1][h] + red_l[pi & 1][2][h] + red_l[pi & 1][3][h];
+                    M[h] = epi_m[pi & 1][h];
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_addr(&o_empty[pi & 1]));
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    const float o = __uint_as_float(u[h]) + __uint_as_float(u[G + h]);
+                    const int qh = pc.g * G + h;
+                    if (pc.whole) {
+                        p.out[(size_t(pc.b) * p.hq + qh) * kD + d] = L[h] > 0.f ? o / L[h] : 0.f;
+                        if (d == 0 && p.lse != nullptr)
+                            p.lse[size_t(pc.b) * p.hq + qh] =
+                                L[h] > 0.f ? (M[h] + __log2f(L[h])) * 0.69314718055994530942f : -CUDART_INF_F;
+                    } else {
+                        const size_t slot = size_t(pc.seg) + blockIdx.x;
+                        p.ws_o[(slot * G + h) * kD + d] = o;
+                        if (d == 0) {
+                            p.ws_ml[(slot * G + h) * 2 + 0] = M[h];
+                            p.ws_ml[(slot * G + h) * 2 + 1] = L[h];
+                        }
+                    }
+                }
+            }
         } else {
-            // ======================================================== softmax + epilogue
+            // ======================================================== softmax
             const int sw = warp - kSoftWarp0;              // 0..3
             const int sub = warp & 3;                      // TMEM lane quarter this warp may access
             const int row = sub * 32 + lane;               // key row of S^T; output dim of O^T
             const uint32_t lane_off = uint32_t(sub * 32) << 16;
             uint32_t j = 0;
             bool ok = true;
-            for (int64_t gb = gb_begin; ok && gb < gb_end;) {
+            int pi = 0;
+            for (int64_t gb = gb_begin; ok && gb < gb_end; ++pi) {
                 const Piece pc = locate(p, bpre, gb, gb_end);
                 gb = pc.end_gb;
+                const uint32_t tmem_o = tmem + lane_off + kTmemO0 + (pi & 1) * 32;
                 float m[G], l[G];
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
@@ -445,14 +516,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                         if (!warp_wait(smem_addr(&p_free[(j - 1) & 1]), ((j - 1) >> 1) & 1, p, abort_flag)) continue;
                         tc_fence_after();
                         uint32_t u[2 * G];
-                        tmem_ldn<2 * G>(tmem + lane_off + kTmemO, u);
+                        tmem_ldn<2 * G>(tmem_o, u);
                         tmem_wait_ld();
 #pragma unroll
                         for (int h = 0; h < G; ++h) {
                             u[h] = __float_as_uint(__uint_as_float(u[h]) * alpha[h]);
                             u[G + h] = __float_as_uint(__uint_as_float(u[G + h]) * alpha[h]);
                         }
-                        tmem_stn<2 * G>(tmem + lane_off + kTmemO, u);
+                        tmem_stn<2 * G>(tmem_o, u);
                         tmem_wait_st();
                     }
                     tc_fence_before();
@@ -461,45 +532,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                 }
                 if (!ok) break;
 
-                // ---- epilogue: O^T of the piece is final once PV of its last tile landed
-                const uint32_t jl = j - 1;
-                const bool got = warp_wait(smem_addr(&p_free[jl & 1]), (jl >> 1) & 1, p, abort_flag);
+                // ---- hand the piece to the epilogue warps (per-warp row sums and
+                // the max) and go on with the next piece at once
+                if (!warp_wait(smem_addr(&o_empty[pi & 1]), ((pi >> 1) & 1) ^ 1, p, abort_flag)) continue;
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
                     float x = l[h];
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-                    if (lane == 0) red_l[sw][h] = x;
-                }
-                if (softmax_barrier_any(!got || *abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                uint32_t u[2 * G];
-                tmem_ldn<2 * G>(tmem + lane_off + kTmemO, u);
-                tmem_wait_ld();
-                tc_fence_before();
-                const int d = row;
-#pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    const float o = __uint_as_float(u[h]) + __uint_as_float(u[G + h]);
-                    const float L = red_l[0][h] + red_l[1][h] + red_l[2][h] + red_l[3][h];
-                    const int qh = pc.g * G + h;
-                    if (pc.whole) {
-                        p.out[(size_t(pc.b) * p.hq + qh) * kD + d] = L > 0.f ? o / L : 0.f;
-                        if (d == 0 && p.lse != nullptr)
-                            p.lse[size_t(pc.b) * p.hq + qh] =
-                                L > 0.f ? (m[h] + __log2f(L)) * 0.69314718055994530942f : -CUDART_INF_F;
-                    } else {
-                        const size_t slot = size_t(pc.seg) + blockIdx.x;
-                        p.ws_o[(slot * G + h) * kD + d] = o;
-                        if (d == 0) {
-                            p.ws_ml[(slot * G + h) * 2 + 0] = m[h];
-                            p.ws_ml[(slot * G + h) * 2 + 1] = L;
-                        }
+                    if (lane == 0) {
+                        red_l[pi & 1][sw][h] = x;
+                        if (sw == 0) epi_m[pi & 1][h] = m[h];
                     }
                 }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_addr(&epi_full[pi & 1]));
             }
         }
     }
@@ -515,13 +562,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
 template <int G>
 cudaError_t launch_g(const DecodeParams& p, cudaStream_t s) {
     DecodeParams q = p;
-    const size_t fixed = 4 * size_t(kSmall) + size_t(p.B + 1) * 4 + 1024;
+    const size_t fixed = 4 * size_t(kSmall) + seq_table_bytes(p.B) + 1024;
     q.stages = fixed + 3 * 2 * size_t(kTileBytes) <= size_t(227) * 1024 ? 3 : 2;
     const size_t smem = fixed + size_t(q.stages) * 2 * kTileBytes;
     if (smem > size_t(227) * 1024) return cudaErrorInvalidConfiguration;
     cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
-    decode_tc_kernel<G><<<p.num_ctas, kThreads, smem, s>>>(q);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(p.num_ctas));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<G>, q);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
