@@ -309,7 +309,7 @@ def run_ours(args, rank, world, local):
         "decode_us": round(1e3 * dec_avg_ms, 3),
         "roofline": {
             "bound": "hbm",
-            "kernel": "decode (split-K attention + LSE merge launch pair)",
+            "kernel": "decode_tc_kernel (split-K tcgen05 attention with the log-sum-exp merge in-kernel)",
             "achieved": round(achieved, 1),
             "peak": hbm_peak,
             "peak_kind": peak_kind,
@@ -320,7 +320,7 @@ def run_ours(args, rank, world, local):
         },
         "e2e": {"value": round(e2e_ms * 1e3 / K, 3), "unit": "us/layer-step",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
-        "gpu_launches": 3 * K,
+        "gpu_launches": 2 * K,          # append + decode per layer-step
         "clocks": clk.summary(),
     }
     cache.close()

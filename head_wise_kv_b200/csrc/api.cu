@@ -35,9 +35,15 @@ int check_desc(const duo_kv_desc* d) {
     return DUO_OK;
 }
 
-// Layout: [status 256 B] then per layer [Kr][Vr][Ks][Vs][pos], each 256-aligned.
+// Bytes of the head of the buffer: status word, then the decode merge
+// counters (one int32 per (sequence, KV head)).
+size_t header_bytes(const duo_kv_desc* d) {
+    return kAlign + align_up(size_t(d->batch) * d->num_kv_heads * 4);
+}
+
+// Layout: [status 256 B][merge counters] then per layer [Kr][Vr][Ks][Vs][pos], each 256-aligned.
 size_t plan_layout(const duo_kv_desc* d, std::vector<duo::LayerLayout>* layers, size_t* cache_bytes) {
-    size_t off = kAlign;   // status word
+    size_t off = header_bytes(d);
     size_t cache = 0;
     const size_t D = size_t(d->head_dim), B = size_t(d->batch), SW = size_t(d->sink) + d->window;
     for (int l = 0; l < d->num_layers; ++l) {
@@ -99,12 +105,13 @@ int duo_kv_alloc(const duo_kv_desc* desc, void* dev_buf, size_t buf_bytes, duo_s
     h->base = static_cast<char*>(dev_buf);
     h->bytes = need;
     h->status = reinterpret_cast<int32_t*>(h->base);
+    h->seg_count = reinterpret_cast<int32_t*>(h->base + kAlign);
     if (cudaGetDevice(&h->device) != cudaSuccess ||
         cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess) {
         delete h;
         return DUO_ERR_CUDA;
     }
-    cudaError_t e = cudaMemsetAsync(h->status, 0, kAlign, stream);
+    cudaError_t e = cudaMemsetAsync(h->status, 0, header_bytes(desc), stream);
     const size_t SW = size_t(desc->sink) + desc->window;
     for (size_t l = 0; l < h->layers.size() && e == cudaSuccess; ++l)
         e = cudaMemsetAsync(h->base + h->layers[l].off_pos, 0xff, size_t(desc->batch) * SW * 4, stream);
@@ -258,6 +265,7 @@ static int decode_impl(duo_kv* kv, int32_t layer, const uint16_t* q, const int32
     p.ws_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                        ((size_t(slots) * G * D * 4 + 255) & ~size_t(255)));
     p.status = kv->status;
+    p.seg_count = kv->seg_count;
     p.cap = kv->desc.capacity;
     p.B = kv->desc.batch;
     p.n_kv = kv->desc.num_kv_heads;
@@ -385,6 +393,9 @@ int duo_kv_read_status(duo_kv* kv, int32_t* status, int32_t clear, duo_stream_t 
     cudaError_t e = cudaMemcpyAsync(status, kv->status, sizeof(int32_t), cudaMemcpyDeviceToHost, stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
     if (e == cudaSuccess && clear) e = cudaMemsetAsync(kv->status, 0, sizeof(int32_t), stream);
+    // a decode that gave up on a wait may have left merge counters behind
+    if (e == cudaSuccess && clear && (*status & DUO_STATUS_WAIT_TIMEOUT))
+        e = cudaMemsetAsync(kv->seg_count, 0, size_t(kv->desc.batch) * kv->desc.num_kv_heads * 4, stream);
     return cuda_err(e);
 }
 

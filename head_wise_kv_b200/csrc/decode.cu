@@ -531,7 +531,7 @@ cudaError_t launch_merge(const DecodeParams& p, cudaStream_t s) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(unsigned(p.B * p.n_kv));
     cfg.blockDim = dim3(32 * G);
-    cfg.dynamicSmemBytes = seq_table_bytes(p.B);
+    cfg.dynamicSmemBytes = seq_table_bytes(p.B, p.n_kv);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -543,23 +543,22 @@ cudaError_t launch_merge(const DecodeParams& p, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-// Attention (CUDA-core kernel for d = 64, tensor-core kernel for d = 128),
-// then the merge as its programmatic dependent.
+// d = 128: the tensor-core kernel, which merges its partials itself.
+// d = 64: the CUDA-core kernel, then the merge as its programmatic dependent.
 template <int D, int G>
 cudaError_t launch_t(const DecodeParams& p, cudaStream_t s) {
-    cudaError_t e;
     if constexpr (D == 128) {
-        e = launch_decode_tc(p, G, s);
+        return launch_decode_tc(p, G, s);
     } else {
         using C = Cfg<D, G>;
-        const size_t smem = C::SMEM + seq_table_bytes(p.B);
-        e = cudaFuncSetAttribute(decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        const size_t smem = C::SMEM + seq_table_bytes(p.B, p.n_kv);
+        cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         if (e != cudaSuccess) return e;
         decode_kernel<D, G><<<p.num_ctas, kThreads, smem, s>>>(p);
         e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        return launch_merge<D, G>(p, s);
     }
-    if (e != cudaSuccess) return e;
-    return launch_merge<D, G>(p, s);
 }
 
 }  // namespace

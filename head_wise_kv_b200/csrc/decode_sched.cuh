@@ -55,12 +55,23 @@ __device__ __forceinline__ SeqRows seq_rows(const DecodeParams& p, int b) {
     return x;
 }
 
-// Shared-memory sequence table built once per launch: int32 words
+// Shared-memory table built once per launch: int32 words
 // [0, B]  running count of 16-token blocks per sequence (prefix),
-// then three arrays of B: first retrieval row, retrieval rows, ring slots.
-// Locating a piece then reads shared memory only (a global read of the
-// lengths costs microseconds while the kernel saturates HBM).
-__host__ __device__ constexpr size_t seq_table_bytes(int B) { return (size_t(B + 1) + 3 * size_t(B)) * 4; }
+// then three arrays of B: first retrieval row, retrieval rows, ring slots,
+// then per KV head: retrieval heads before it (n_kv + 1 words) and its
+// rank with the retrieval flag in the sign bit (n_kv words).
+// Locating a piece then reads shared memory only: a global read of the
+// lengths, or an indexed read of the launch parameters that misses the
+// constant cache, costs microseconds while the kernel saturates HBM.
+__host__ __device__ constexpr size_t seq_table_bytes(int B, int n_kv) {
+    return (size_t(B + 1) + 3 * size_t(B) + 2 * size_t(n_kv) + 1) * 4;
+}
+
+// Units a segment of nb blocks takes on the partition axis: its blocks,
+// preceded by `weight` blocks that hold no keys when it has any.  The weight
+// stands for the fixed cost of starting a piece, so that a CTA whose range
+// starts many segments gets fewer keys (0 = partition by keys alone).
+__device__ __forceinline__ int seg_units(int nb, int weight) { return nb > 0 ? nb + weight : 0; }
 
 // Fill the table (shared); warp 0 does a chunked shuffle scan.  Caller syncs afterwards.
 __device__ void build_prefix(const DecodeParams& p, int32_t* bpre) {
@@ -73,7 +84,7 @@ __device__ void build_prefix(const DecodeParams& p, int32_t* bpre) {
         int c = 0;
         if (b < p.B) {
             const SeqRows x = seq_rows(p, b);
-            c = p.n_r * blocks_of(x.nr) + p.n_s * blocks_of(x.ns);
+            c = p.n_r * seg_units(blocks_of(x.nr), p.seg_weight) + p.n_s * seg_units(blocks_of(x.ns), p.seg_weight);
             int32_t* rows = bpre + p.B + 1;
             rows[b] = int32_t(x.r0);
             rows[p.B + b] = int32_t(x.nr);
@@ -87,6 +98,12 @@ __device__ void build_prefix(const DecodeParams& p, int32_t* bpre) {
         }
         if (b < p.B) bpre[b + 1] = run + x;
         run += __shfl_sync(0xffffffffu, x, 31);
+    }
+    int32_t* hb = bpre + 4 * p.B + 1;
+    int32_t* hr = hb + p.n_kv + 1;
+    for (int g = lane; g <= p.n_kv; g += 32) {
+        hb[g] = p.r_before[g];
+        if (g < p.n_kv) hr[g] = p.rank[g] | (p.is_r[g] ? int32_t(0x80000000u) : 0);
     }
 }
 
@@ -106,6 +123,8 @@ struct Piece {
     int64_t tok0, tok1;     // token rows of this piece inside the segment
     int64_t end_gb;         // global block after the piece
     bool whole;             // the piece is the whole segment
+    bool retr;              // KV head g is a retrieval head
+    int rank;               // g's index among the layer's retrieval or streaming heads
 };
 
 // Locate the piece that starts at global block gb (gb < range end).
@@ -122,27 +141,47 @@ __device__ __forceinline__ Piece locate(const DecodeParams& p, const int32_t* bp
     const int32_t* tab = bpre + p.B + 1;
     const int64_t r0 = tab[lo], rr = tab[p.B + lo], rs = tab[2 * p.B + lo];
     const int nbr = blocks_of(rr), nbs = blocks_of(rs);
+    const int ur = seg_units(nbr, p.seg_weight), us = seg_units(nbs, p.seg_weight);
     const int64_t local = gb - bpre[lo];
+    const int32_t* hb = bpre + 4 * p.B + 1;
+    const int32_t* hr = hb + p.n_kv + 1;
     int g = 0;
     int64_t start = 0;
+    bool retr = false;
     for (; g < p.n_kv; ++g) {
-        start = int64_t(p.r_before[g]) * nbr + int64_t(g - p.r_before[g]) * nbs;
-        const int nb = p.is_r[g] ? nbr : nbs;
-        if (local < start + nb) break;
+        start = int64_t(hb[g]) * ur + int64_t(g - hb[g]) * us;
+        retr = hr[g] < 0;
+        if (local < start + (retr ? ur : us)) break;
     }
     pc.g = g;
+    pc.retr = retr;
+    pc.rank = hr[g] & 0x7fffffff;
     pc.seg = lo * p.n_kv + g;
-    pc.row0 = p.is_r[g] ? r0 : 0;
-    pc.seg_nb = p.is_r[g] ? nbr : nbs;
-    pc.seg_gb = bpre[lo] + start;
+    pc.row0 = retr ? r0 : 0;
+    pc.seg_nb = retr ? nbr : nbs;
+    pc.seg_gb = bpre[lo] + start + (pc.seg_nb > 0 ? p.seg_weight : 0);   // first block with keys
     const int64_t seg_end = pc.seg_gb + pc.seg_nb;
     pc.end_gb = seg_end < range_end ? seg_end : range_end;
-    const int64_t rows = p.is_r[g] ? rr : rs;
-    pc.tok0 = (gb - pc.seg_gb) * kBlk;
+    const int64_t rows = retr ? rr : rs;
+    pc.tok0 = gb > pc.seg_gb ? (gb - pc.seg_gb) * kBlk : 0;
     const int64_t t1 = (pc.end_gb - pc.seg_gb) * kBlk;
     pc.tok1 = t1 < rows ? t1 : rows;
-    pc.whole = (gb == pc.seg_gb) && (pc.end_gb == seg_end);
+    if (pc.tok1 < pc.tok0) pc.tok1 = pc.tok0;   // the range ends before the segment's first key
+    pc.whole = (gb <= pc.seg_gb) && (pc.end_gb == seg_end);
     return pc;
+}
+
+// The next piece that holds keys, starting at global block gb (advanced
+// past it); false when the range has none left.  With a segment weight a
+// range may start or end inside a weight, which gives a piece without keys.
+__device__ __forceinline__ bool next_piece(const DecodeParams& p, const int32_t* bpre, int64_t& gb,
+                                           int64_t range_end, Piece& pc) {
+    while (gb < range_end) {
+        pc = locate(p, bpre, gb, range_end);
+        gb = pc.end_gb;
+        if (pc.tok1 > pc.tok0) return true;
+    }
+    return false;
 }
 
 }  // namespace

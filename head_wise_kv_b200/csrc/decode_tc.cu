@@ -38,8 +38,14 @@
 //              sums and the max go to the epilogue through shared memory
 //   warps 8-11 epilogue (thread = output dim): O^T is double-buffered in TMEM
 //              by piece parity, so a piece's tail (its last V tile and PV)
-//              never holds up the softmax of the next; writes `out` or the
-//              workspace partial.
+//              never holds up the softmax of the next.  A piece that is a
+//              whole segment is written to `out`; otherwise the partial
+//              (o, max, sum) goes to the workspace and the last CTA to finish
+//              a part of that segment (a per-segment arrival counter, reset
+//              by that CTA) merges the parts by log-sum-exp, so no second
+//              kernel is launched.
+//   warp 7 also writes the output of segments without keys and sets the
+//              length status bits.
 //
 // Every mbarrier wait is bounded; on a timeout the CTA sets
 // DUO_STATUS_WAIT_TIMEOUT, stops, waits (bounded) for its copies and MMAs in
@@ -74,6 +80,14 @@ constexpr uint32_t kTmemCols = 128;
 constexpr uint32_t kTmemS0 = 0, kTmemS1 = 32, kTmemO0 = 64;   // O^T of piece pi at kTmemO0 + 32 (pi & 1)
 constexpr float kNegBig = -1.0e30f;
 constexpr float kRescaleThreshold = 8.0f;     // log2 units: probabilities stay <= 2^8
+// Partition weight of a segment start in 16-token blocks: starting a piece
+// (its first tile's latency, the hand-over of the last one) costs about as
+// much time as streaming this many blocks.  Measured on the 128K GQA
+// workload: 0 -> 193 us, 8 -> 188, 16 -> 183, 24..48 -> 181.5-183, 64 -> 183.
+#ifndef DUO_DECODE_SEG_WEIGHT
+#define DUO_DECODE_SEG_WEIGHT 32
+#endif
+constexpr int kSegWeight = DUO_DECODE_SEG_WEIGHT;
 
 constexpr uint32_t kIdescQK = idesc_f16(kT, kN, true, false, false);   // A = K (K-major), B = q (K-major)
 constexpr uint32_t kIdescPV = idesc_f16(kD, kN, true, true, false);    // A = V^T (MN-major), B = P^T
@@ -87,31 +101,28 @@ __device__ __forceinline__ uint32_t small_off(int r, int c) {
 
 __device__ __forceinline__ int tiles_of(const Piece& pc) { return int((pc.tok1 - pc.tok0 + kT - 1) / kT); }
 
-// Position in the CTA's sequence of tiles: piece `pi` (its locate() result
-// in pc), tile t of its nt.
+// Position in the CTA's sequence of tiles: piece `pi` (pc), tile t of its
+// nt; gb is where the search for the next piece starts.
 struct TileCursor {
     Piece pc;
     int pi, t, nt;
     bool valid;
 
+    int64_t gb;
+
     __device__ void start(const DecodeParams& p, const int32_t* bpre, int64_t gb_begin, int64_t gb_end) {
         pi = 0;
         t = 0;
-        valid = gb_begin < gb_end;
-        if (valid) {
-            pc = locate(p, bpre, gb_begin, gb_end);
-            nt = tiles_of(pc);
-        }
+        gb = gb_begin;
+        valid = next_piece(p, bpre, gb, gb_end, pc);
+        if (valid) nt = tiles_of(pc);
     }
     __device__ void advance(const DecodeParams& p, const int32_t* bpre, int64_t gb_end) {
         if (++t < nt) return;
         t = 0;
         ++pi;
-        valid = pc.end_gb < gb_end;
-        if (valid) {
-            pc = locate(p, bpre, pc.end_gb, gb_end);
-            nt = tiles_of(pc);
-        }
+        valid = next_piece(p, bpre, gb, gb_end, pc);
+        if (valid) nt = tiles_of(pc);
     }
 };
 
@@ -134,19 +145,68 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const D
     return ok != 0;
 }
 
-// Barrier over the 128 softmax threads that ORs a flag across them.
-__device__ __forceinline__ bool softmax_barrier_any(bool flag) {
+// Lane 0 polls for the warp, napping between polls: for waits that span a
+// whole piece, so that the poll takes no issue slots from the warps on the
+// critical path.
+__device__ __forceinline__ bool warp_wait_lazy(uint32_t bar, uint32_t parity, const DecodeParams& p,
+                                               volatile int* abort_flag) {
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0) {
+        const unsigned long long t0 = global_ns();
+        while (!mbar_test_wait(bar, parity)) {
+            if (*abort_flag) {
+                ok = 0;
+                break;
+            }
+            if (global_ns() - t0 > p.timeout_ns) {
+                set_status(p.status, DUO_STATUS_WAIT_TIMEOUT);
+                *abort_flag = 1;
+                ok = 0;
+                break;
+            }
+            __nanosleep(256);
+        }
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
+}
+
+// CTAs that hold a piece of the segment starting at global block seg_gb
+// (seg_nb >= 1 blocks): [c0, c1], of which `n` have a non-empty range.
+struct Owners {
+    int c0, c1, n;
+};
+
+__device__ __forceinline__ Owners owners_of(int64_t seg_gb, int seg_nb, int64_t total, int64_t ctas) {
+    Owners o;
+    o.c0 = cta_owner(seg_gb, total, ctas);
+    o.c1 = cta_owner(seg_gb + seg_nb - 1, total, ctas);
+    if (total >= ctas) {
+        o.n = o.c1 - o.c0 + 1;   // no CTA range is empty
+    } else {
+        o.n = 0;
+        for (int c = o.c0; c <= o.c1; ++c) o.n += cta_start(c + 1, total, ctas) > cta_start(c, total, ctas);
+    }
+    return o;
+}
+
+// Barrier over 128 threads (named barrier `id`) that ORs a flag across
+// them, so that every participating warp takes the same exit decision.
+template <int id>
+__device__ __forceinline__ bool barrier_any(bool flag) {
     uint32_t out;
     asm volatile(
         "{\n\t.reg .pred pi, po;\n\t"
         "setp.ne.u32 pi, %1, 0;\n\t"
-        "bar.red.or.pred po, 1, 128, pi;\n\t"
+        "bar.red.or.pred po, %2, 128, pi;\n\t"
         "selp.u32 %0, 1, 0, po;\n\t}"
         : "=r"(out)
-        : "r"(uint32_t(flag))
+        : "r"(uint32_t(flag)), "n"(id)
         : "memory");
     return out != 0;
 }
+constexpr int kBarSoftmax = 1, kBarEpilogue = 2;
 
 __device__ __forceinline__ uint16_t bf16_bits(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
 
@@ -170,6 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     __shared__ float red_max[2][4][G];
     __shared__ float red_l[2][4][G];   // [piece parity][softmax warp][head] row sums
     __shared__ float epi_m[2][G];      // [piece parity][head] running max
+    __shared__ bool epi_last;          // this CTA is the last owner of the piece's segment
     __shared__ int abort_sh;
     volatile int* abort_flag = &abort_sh;
 
@@ -214,8 +275,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    // The merge kernel may be scheduled now; it waits (griddepcontrol.wait)
-    // for this grid's completion before it reads any partial.
+    // A following kernel launched as a programmatic dependent may be
+    // scheduled now; it waits (griddepcontrol.wait) for this grid's writes.
     asm volatile("griddepcontrol.launch_dependents;");
     const uint32_t tmem = tmem_base_sh;
 
@@ -232,11 +293,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                 uint32_t it = 0;
                 bool ok = true;
                 for (int64_t gb = gb_begin; ok && gb < gb_end;) {
-                    const Piece pc = locate(p, bpre, gb, gb_end);
-                    gb = pc.end_gb;
-                    const bool retr = p.is_r[pc.g] != 0;
-                    const CUtensorMap* mk = retr ? &p.tm_kr : &p.tm_ks;
-                    const int z = retr ? pc.b * p.n_r + p.rank[pc.g] : pc.b * p.n_s + p.rank[pc.g];
+                    Piece pc;
+                    if (!next_piece(p, bpre, gb, gb_end, pc)) break;
+                    const CUtensorMap* mk = pc.retr ? &p.tm_kr : &p.tm_ks;
+                    const int z = pc.b * (pc.retr ? p.n_r : p.n_s) + pc.rank;
                     for (int64_t t = pc.tok0; t < pc.tok1; t += kT, ++it) {
                         const int st = int(it % uint32_t(nst));
                         if (!timed_wait(smem_addr(&empty_k[st]), ((it / nst) & 1) ^ 1, p, abort_flag)) {
@@ -261,8 +321,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             // Runs up to two pieces ahead of the S products (two q buffers).
             int pi = 0;
             for (int64_t gb = gb_begin; gb < gb_end; ++pi) {
-                const Piece pc = locate(p, bpre, gb, gb_end);
-                gb = pc.end_gb;
+                Piece pc;
+                if (!next_piece(p, bpre, gb, gb_end, pc)) break;
                 if (!warp_wait(smem_addr(&q_empty[pi & 1]), ((pi >> 1) & 1) ^ 1, p, abort_flag)) break;
                 const uint16_t* qb = p.q + (size_t(pc.b) * p.hq + size_t(pc.g) * G) * kD;
                 const uint32_t qs = sQ + (pi & 1) * kSmall;
@@ -281,11 +341,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                 uint32_t it = 0;
                 bool ok = true;
                 for (int64_t gb = gb_begin; ok && gb < gb_end;) {
-                    const Piece pc = locate(p, bpre, gb, gb_end);
-                    gb = pc.end_gb;
-                    const bool retr = p.is_r[pc.g] != 0;
-                    const CUtensorMap* mv = retr ? &p.tm_vr : &p.tm_vs;
-                    const int z = retr ? pc.b * p.n_r + p.rank[pc.g] : pc.b * p.n_s + p.rank[pc.g];
+                    Piece pc;
+                    if (!next_piece(p, bpre, gb, gb_end, pc)) break;
+                    const CUtensorMap* mv = pc.retr ? &p.tm_vr : &p.tm_vs;
+                    const int z = pc.b * (pc.retr ? p.n_r : p.n_s) + pc.rank;
                     for (int64_t t = pc.tok0; t < pc.tok1; t += kT, ++it) {
                         const int st = int(it % uint32_t(nst));
                         if (!timed_wait(smem_addr(&empty_v[st]), ((it / nst) & 1) ^ 1, p, abort_flag)) {
@@ -369,6 +428,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                         set_status(p.status, DUO_STATUS_WAIT_TIMEOUT);
                         *abort_flag = 1;
                         ok = false;
+                    } else {
+                        __nanosleep(32);   // leave issue slots to the softmax warp on this scheduler
                     }
                 }
                 // every MMA issued by this thread has completed before TMEM is freed
@@ -384,11 +445,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             const uint32_t lane_off = uint32_t(sub * 32) << 16;
             int pi = 0;
             for (int64_t gb = gb_begin; gb < gb_end; ++pi) {
-                const Piece pc = locate(p, bpre, gb, gb_end);
-                gb = pc.end_gb;
-                if (!warp_wait(smem_addr(&epi_full[pi & 1]), (pi >> 1) & 1, p, abort_flag) ||
-                    !warp_wait(smem_addr(&o_full[pi & 1]), (pi >> 1) & 1, p, abort_flag))
-                    break;
+                Piece pc;
+                if (!next_piece(p, bpre, gb, gb_end, pc)) break;
+                const bool got = warp_wait_lazy(smem_addr(&epi_full[pi & 1]), (pi >> 1) & 1, p, abort_flag) &&
+                                 warp_wait_lazy(smem_addr(&o_full[pi & 1]), (pi >> 1) & 1, p, abort_flag);
+                if (barrier_any<kBarEpilogue>(!got)) break;
                 tc_fence_after();
                 uint32_t u[2 * G];
                 tmem_ldn<2 * G>(tmem + lane_off + kTmemO0 + (pi & 1) * 32, u);
@@ -402,24 +463,74 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_addr(&o_empty[pi & 1]));
+                if (pc.whole) {
 #pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    const float o = __uint_as_float(u[h]) + __uint_as_float(u[G + h]);
-                    const int qh = pc.g * G + h;
-                    if (pc.whole) {
+                    for (int h = 0; h < G; ++h) {
+                        const float o = __uint_as_float(u[h]) + __uint_as_float(u[G + h]);
+                        const int qh = pc.g * G + h;
                         p.out[(size_t(pc.b) * p.hq + qh) * kD + d] = L[h] > 0.f ? o / L[h] : 0.f;
                         if (d == 0 && p.lse != nullptr)
                             p.lse[size_t(pc.b) * p.hq + qh] =
                                 L[h] > 0.f ? (M[h] + __log2f(L[h])) * 0.69314718055994530942f : -CUDART_INF_F;
-                    } else {
-                        const size_t slot = size_t(pc.seg) + blockIdx.x;
-                        p.ws_o[(slot * G + h) * kD + d] = o;
+                    }
+                    continue;
+                }
+                // Part of a segment that other CTAs share: leave the partial in
+                // the workspace (slot = segment + CTA); the last of the owners to
+                // finish merges them all by log-sum-exp (fence, then count).
+                {
+                    const size_t slot = size_t(pc.seg) + blockIdx.x;
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        p.ws_o[(slot * G + h) * kD + d] = __uint_as_float(u[h]) + __uint_as_float(u[G + h]);
                         if (d == 0) {
                             p.ws_ml[(slot * G + h) * 2 + 0] = M[h];
                             p.ws_ml[(slot * G + h) * 2 + 1] = L[h];
                         }
                     }
                 }
+                __threadfence();
+                named_bar_sync(kBarEpilogue, 128);
+                const Owners ow = owners_of(pc.seg_gb, pc.seg_nb, total, n);
+                if (warp == kEpiWarp0 && lane == 0) {
+                    const int before = atomicAdd(&p.seg_count[pc.seg], 1);
+                    epi_last = before == ow.n - 1;
+                    __threadfence();
+                }
+                named_bar_sync(kBarEpilogue, 128);
+                if (!epi_last) continue;
+                float Mx[G], Ls[G], acc[G];
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    Mx[h] = kNegBig;
+                    Ls[h] = 0.f;
+                    acc[h] = 0.f;
+                }
+                for (int c = ow.c0; c <= ow.c1; ++c) {
+                    if (total < n && cta_start(c + 1, total, n) == cta_start(c, total, n)) continue;
+                    const size_t slot = size_t(pc.seg) + c;
+#pragma unroll
+                    for (int h = 0; h < G; ++h) Mx[h] = fmaxf(Mx[h], __ldcg(&p.ws_ml[(slot * G + h) * 2]));
+                }
+                for (int c = ow.c0; c <= ow.c1; ++c) {
+                    if (total < n && cta_start(c + 1, total, n) == cta_start(c, total, n)) continue;
+                    const size_t slot = size_t(pc.seg) + c;
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        const float f = fast_exp2(__ldcg(&p.ws_ml[(slot * G + h) * 2]) - Mx[h]);
+                        Ls[h] += __ldcg(&p.ws_ml[(slot * G + h) * 2 + 1]) * f;
+                        acc[h] += __ldcg(&p.ws_o[(slot * G + h) * kD + d]) * f;
+                    }
+                }
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    const int qh = pc.g * G + h;
+                    p.out[(size_t(pc.b) * p.hq + qh) * kD + d] = Ls[h] > 0.f ? acc[h] / Ls[h] : 0.f;
+                    if (d == 0 && p.lse != nullptr)
+                        p.lse[size_t(pc.b) * p.hq + qh] =
+                            Ls[h] > 0.f ? (Mx[h] + __log2f(Ls[h])) * 0.69314718055994530942f : -CUDART_INF_F;
+                }
+                if (d == 0) p.seg_count[pc.seg] = 0;   // every owner has counted: ready for the next launch
             }
         } else {
             // ======================================================== softmax
@@ -431,8 +542,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             bool ok = true;
             int pi = 0;
             for (int64_t gb = gb_begin; ok && gb < gb_end; ++pi) {
-                const Piece pc = locate(p, bpre, gb, gb_end);
-                gb = pc.end_gb;
+                Piece pc;
+                if (!next_piece(p, bpre, gb, gb_end, pc)) break;
                 const uint32_t tmem_o = tmem + lane_off + kTmemO0 + (pi & 1) * 32;
                 float m[G], l[G];
 #pragma unroll
@@ -468,7 +579,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                         if (lane == 0) red_max[sb][sw][h] = mx;
                     }
                     // the barrier also agrees on aborting
-                    if (softmax_barrier_any(!got || *abort_flag)) {
+                    if (barrier_any<kBarSoftmax>(!got || *abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -551,6 +662,28 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         }
     }
 
+    if (warp == kQWarp) {
+        // Segments without keys (an empty sequence, an empty row range) have
+        // no piece: their output is 0 with lse = -inf, which adds nothing to
+        // a later merge.  Length checks of the classic form set status bits.
+        const int32_t* tab = bpre + p.B + 1;
+        const int32_t* hr = bpre + 4 * p.B + 1 + p.n_kv + 1;
+        for (int seg = blockIdx.x; seg < p.B * p.n_kv; seg += gridDim.x) {
+            const int b = seg / p.n_kv, g = seg % p.n_kv;
+            const int32_t rows = hr[g] < 0 ? tab[p.B + b] : tab[2 * p.B + b];
+            if (rows == 0) {
+                for (int x = lane; x < G * kD; x += 32) p.out[(size_t(b) * p.hq + g * G) * kD + x] = 0.f;
+                if (lane < G && p.lse != nullptr) p.lse[size_t(b) * p.hq + g * G + lane] = -CUDART_INF_F;
+            }
+            if (p.r_end == nullptr && g == 0 && lane == 0) {
+                const int L = p.len[b];
+                if (L < 0) set_status(p.status, DUO_STATUS_BAD_LENGTH);
+                if (int64_t(L) > p.cap && p.n_r > 0) set_status(p.status, DUO_STATUS_OVER_CAPACITY);
+                if (L < 1) set_status(p.status, DUO_STATUS_EMPTY_SEQUENCE);
+            }
+        }
+    }
+
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -562,7 +695,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
 template <int G>
 cudaError_t launch_g(const DecodeParams& p, cudaStream_t s) {
     DecodeParams q = p;
-    const size_t fixed = 4 * size_t(kSmall) + seq_table_bytes(p.B) + 1024;
+    q.seg_weight = kSegWeight;
+    const size_t fixed = 4 * size_t(kSmall) + seq_table_bytes(p.B, p.n_kv) + 1024;
     q.stages = fixed + 3 * 2 * size_t(kTileBytes) <= size_t(227) * 1024 ? 3 : 2;
     const size_t smem = fixed + size_t(q.stages) * 2 * kTileBytes;
     if (smem > size_t(227) * 1024) return cudaErrorInvalidConfiguration;

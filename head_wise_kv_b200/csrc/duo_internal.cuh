@@ -37,6 +37,7 @@ struct duo_kv {
     char* base = nullptr;                   // caller's device buffer
     size_t bytes = 0;
     int32_t* status = nullptr;              // device status word
+    int32_t* seg_count = nullptr;           // device [B * n_kv] merge arrival counters (zero between launches)
     int device = 0;
     int num_sms = 0;
     int decode_ctas = 0;                    // 0 = default persistent wave
@@ -62,9 +63,11 @@ struct DecodeParams {
     float* ws_o;      // [slots][G][D]  partial outputs (unnormalised)
     float* ws_ml;     // [slots][G][2]  partial (max, sum) in the log2 domain
     int32_t* status;
+    int32_t* seg_count;       // tensor-core kernel: per-segment arrival counters for the in-kernel merge
     int64_t cap;
     int B, n_kv, hq, n_r, n_s, S, W;
     int num_ctas;
+    int seg_weight;           // partition weight of a segment start, in 16-token blocks (0 = none)
     int stages;               // tensor-core kernel pipeline depth (set by its launcher)
     float scale_log2;
     unsigned long long timeout_ns;
