@@ -31,10 +31,10 @@ import duo_workloads as W  # noqa: E402
 METRIC = "mixed-head decode attn: µs/layer-step, achieved HBM GB/s (% of B200 peak)"
 WORKLOAD = "gqa128k"
 FALLBACK_HBM_GBS = 6650.0
-# DRAM read + write bytes per launch of decode_kernel<128,4> on this workload,
-# from the ncu capture summarised in profiles/decode_kernel_gqa128k.md.  Must be
+# DRAM read + write bytes per launch of decode_tc_kernel<4> on this workload,
+# from the ncu capture summarised in profiles/decode_tc_kernel_gqa128k.md.  Must be
 # reset to None whenever the decode kernel changes.
-DECODE_TRAFFIC_BYTES = None
+DECODE_TRAFFIC_BYTES = 1126346000 + 3740672
 
 
 # ---------------------------------------------------------------- helpers

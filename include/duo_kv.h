@@ -128,12 +128,14 @@ typedef struct {
  *   sum over layers of 2 * 2 * d * B * (n_r(l) * capacity + n_s(l) * (S+W)),
  * the DuoAttention guide's memory equation (section 2) times the batch,
  * with T = capacity and R = n_r / n_kv per layer.  The rest is the position
- * tables, a status word and 256-byte alignment padding. */
+ * tables, a status word, one int32 merge counter per (sequence, KV head)
+ * for the decode kernel, and 256-byte alignment padding. */
 DUO_API int duo_kv_required_bytes(const duo_kv_desc* desc, size_t* total_bytes, size_t* cache_bytes);
 
 /* Lay a cache out in dev_buf (caller-allocated device memory of buf_bytes,
  * 256-byte aligned, on the current device), set every position to -1 and
- * the status word to 0 (two memsets on `stream`), and return a handle.
+ * the status word and merge counters to 0 (memsets on `stream`), build the
+ * decode kernel's TMA descriptors (head_dim 128), and return a handle.
  * Queries the current device's SM count once.  Errors: INVALID_ARG,
  * UNSUPPORTED, BUFFER_TOO_SMALL, ALIGNMENT, CUDA. */
 DUO_API int duo_kv_alloc(const duo_kv_desc* desc, void* dev_buf, size_t buf_bytes,
@@ -192,7 +194,11 @@ DUO_API int duo_decode_workspace_bytes(const duo_kv* kv, size_t* bytes);
  *   workspace: device scratch of >= duo_decode_workspace_bytes bytes
  *         (no initialisation needed; overlapping calls must not share it).
  * Split-K over each head's keys with a log-sum-exp merge; the result does
- * not depend on how the keys are split beyond rounding. */
+ * not depend on how the keys are split beyond rounding.  At head_dim 128
+ * the merge happens inside the one kernel launch, counted by the handle's
+ * per-(sequence, KV head) counters, which return to 0 when the launch ends:
+ * decode calls on one handle must therefore be ordered (one stream, or
+ * events), as they also share the status word. */
 DUO_API int duo_decode_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const int32_t* len,
                     float scale, float* out, float* lse, void* workspace, size_t workspace_bytes,
                     duo_stream_t stream);
@@ -288,7 +294,9 @@ DUO_API int duo_prefill_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const
                      duo_stream_t stream);
 
 /* Read the device status word into *status (host).  This call
- * synchronises `stream`.  If clear != 0 the word is reset to 0 afterwards. */
+ * synchronises `stream`.  If clear != 0 the word is reset to 0 afterwards,
+ * and if DUO_STATUS_WAIT_TIMEOUT was set, the decode merge counters too (a
+ * launch that gave up may have left them non-zero). */
 DUO_API int duo_kv_read_status(duo_kv* kv, int32_t* status, int32_t clear, duo_stream_t stream);
 
 /* Override the number of CTAs the decode kernel splits the keys over
