@@ -32,6 +32,22 @@ notes of the repository):
   * a decode query sits at t = T - 1, the token just appended; prefill row i
     of a chunk that follows P cached tokens sits at t = P + i.
 
+FP8 KV cache (DuoAttention guide, "Synergies with Low-Bit Quantization":
+cache elements stored in 8 bits instead of 16, a 2x footprint reduction).
+The pages fix neither the 8-bit format nor the scaling; readings taken:
+  * the format is FP8 E4M3 (OCP 8-bit floating point: sign, 4 exponent bits
+    with bias 7, 3 mantissa bits, subnormals, no infinities, code 0x7F/0xFF
+    NaN, largest finite magnitude 448);
+  * one scale per (layer, KV head) for keys and one for values, given by the
+    caller (static, no per-token metadata: exactly 2x, as the pages state);
+  * code = round-to-nearest-even E4M3 of fp32(x) / fp32(scale), computed in
+    fp32 (IEEE division), magnitudes above 448 saturating to 448; the stored
+    value stands for scale * E4M3(code);
+  * attention reads every cached key and value dequantized (decode: all of
+    them, the new token included, since it is appended first; chunked
+    prefill: the cached prefix dequantized, the chunk's own keys and values
+    as given, because they are attended before they are appended).
+
 Parity pins for every function live in ``tests/test_oracle_pins.py``.
 """
 from __future__ import annotations
@@ -44,6 +60,7 @@ __all__ = [
     "kv_cache_bytes", "duo_effective_context", "duo_cache_bytes", "duo_slots",
     "StreamingCache", "ring_positions", "keep_set", "key_mask", "kv_head_of",
     "attend", "decode_attention", "prefill_attention", "brute_force_attention", "blended_decode",
+    "E4M3_MAX", "e4m3_decode", "e4m3_encode", "quantize_kv", "dequantize_kv",
 ]
 
 
@@ -279,3 +296,55 @@ def brute_force_attention(q, k, v, keys, scale):
         for x in range(d):
             o[x] += wj * float(v[j][x])
     return [ox / z for ox in o], m + math.log(z)
+
+
+# ---------------------------------------------------------------- FP8 (E4M3) KV cache
+E4M3_MAX = 448.0
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """Value of each E4M3 byte, float64.  Bit 7 sign, bits 6..3 exponent e
+    (bias 7), bits 2..0 mantissa m: e = 0 gives (m / 8) * 2^-6, otherwise
+    (1 + m / 8) * 2^(e - 7); e = 15 with m = 7 is NaN (no infinities)."""
+    c = np.asarray(codes, dtype=np.int64) & 0xFF
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, (m / 8.0) * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    mag = np.where((e == 15) & (m == 7), np.nan, mag)
+    return sign * mag
+
+
+# the 127 non-negative finite values, codes 0x00 .. 0x7E, increasing
+_E4M3_POS = e4m3_decode(np.arange(0x7F))
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """E4M3 byte nearest to each value of x (round to nearest, ties to the
+    code with an even mantissa), magnitudes beyond 448 saturating to 448;
+    the sign is kept (a negative value that rounds to 0 gives 0x80); NaN
+    gives 0x7F.  x is taken as float64 (pass fp32 values for fp32 inputs)."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    hi = np.clip(np.searchsorted(_E4M3_POS, a, side="left"), 0, 0x7E)   # first value >= a
+    lo = np.clip(hi - 1, 0, 0x7E)
+    d_hi = np.abs(_E4M3_POS[hi] - a)
+    d_lo = np.abs(a - _E4M3_POS[lo])
+    pick = np.where(d_lo < d_hi, lo, hi)
+    pick = np.where(d_lo == d_hi, np.where(lo % 2 == 0, lo, hi), pick)   # tie: even code = even mantissa
+    pick = np.where(a >= E4M3_MAX, 0x7E, pick)
+    code = pick.astype(np.int64) | np.where(np.signbit(x), 0x80, 0)
+    code = np.where(np.isnan(x), 0x7F, code)
+    return code.astype(np.uint8)
+
+
+def quantize_kv(x, scale: float) -> np.ndarray:
+    """Cache codes of K or V values x (bf16 values, any shape) under one
+    scale: E4M3 of fp32(x) / fp32(scale), the quotient rounded once in fp32."""
+    q = np.asarray(x, dtype=np.float32) / np.float32(scale)
+    return e4m3_encode(q.astype(np.float64))
+
+
+def dequantize_kv(codes, scale: float) -> np.ndarray:
+    """Values the cache codes stand for: scale * E4M3(code), float64 (exact)."""
+    return float(np.float32(scale)) * e4m3_decode(codes)

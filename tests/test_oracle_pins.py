@@ -432,3 +432,78 @@ def test_attention_over_a_union_is_the_lse_weighted_mix_of_its_parts():
     want, want_lse = O.brute_force_attention(q, k, v, list(range(T)), 0.4)
     np.testing.assert_allclose(mixed, want, rtol=1e-12, atol=1e-13)
     assert LSE == pytest.approx(want_lse, rel=1e-13)
+
+
+# ------------------------------------------------------------------ FP8 (E4M3) KV codes
+def _torch_codes(x32):
+    """E4M3 bytes from torch's float8_e4m3fn conversion (a library routine)."""
+    return torch.from_numpy(np.asarray(x32, dtype=np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def test_e4m3_decode_closed_forms_and_library_table():
+    v = O.e4m3_decode([0x00, 0x01, 0x07, 0x08, 0x38, 0x3F, 0x7E, 0x80, 0xB8, 0xFE])
+    assert list(v) == [0.0, 2.0 ** -9, 7 * 2.0 ** -9, 2.0 ** -6, 1.0, 1.875, 448.0, -0.0, -1.0, -448.0]
+    assert np.signbit(v[7])
+    assert np.isnan(O.e4m3_decode([0x7F, 0xFF])).all()
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    ours = O.e4m3_decode(codes)
+    assert np.array_equal(np.isnan(ours), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(ours[ok], ref[ok]) and np.array_equal(np.signbit(ours[ok]), np.signbit(ref[ok]))
+
+
+def test_e4m3_encode_matches_library_in_range():
+    rng = np.random.default_rng(11)
+    mag = np.exp2(rng.uniform(-13, np.log2(440.0), 20000))
+    x = (mag * rng.choice([-1.0, 1.0], mag.size)).astype(np.float32)
+    pos = O.e4m3_decode(np.arange(0x7E))
+    mids = ((pos[:-1] + pos[1:]) / 2).astype(np.float32)            # every tie between neighbours
+    x = np.concatenate([x, mids, -mids, np.float32([0.0, -0.0, 1e-30, -1e-30])])
+    assert np.array_equal(O.e4m3_encode(x.astype(np.float64)), _torch_codes(x))
+
+
+def test_e4m3_ties_saturation_nan_and_round_trip():
+    # ties go to the even mantissa
+    assert list(O.e4m3_encode([2.0 ** -10, 3 * 2.0 ** -10, 1.0625, 1.1875])) == [0x00, 0x02, 0x38, 0x3A]
+    # magnitudes beyond the largest finite value saturate to it, sign kept
+    assert list(O.e4m3_encode([448.0, 460.0, 464.0, 1e6, -1e6, np.inf])) == [0x7E] * 4 + [0xFE, 0x7E]
+    assert O.e4m3_encode([np.nan])[0] == 0x7F
+    finite = np.array([c for c in range(256) if c not in (0x7F, 0xFF)])
+    assert np.array_equal(O.e4m3_encode(O.e4m3_decode(finite)), finite.astype(np.uint8))
+
+
+def test_quantize_kv_is_one_fp32_division_then_e4m3():
+    rng = np.random.default_rng(12)
+    x = torch.randn(4096, dtype=torch.float32).to(torch.bfloat16).float().numpy()
+    for s in (1.0, 0.37, 3.0, 1 / 64):
+        q32 = (torch.from_numpy(x) / torch.tensor(s, dtype=torch.float32)).numpy()
+        assert np.array_equal(O.quantize_kv(x, s), _torch_codes(q32))
+        back = O.dequantize_kv(O.quantize_kv(x, s), s)
+        # relative error of E4M3 (3 mantissa bits) is at most 2^-4 above the subnormal range
+        big = np.abs(x / s) >= 2.0 ** -6
+        assert np.all(np.abs(back[big] - x[big]) <= 2.0 ** -4 * np.abs(x[big]) + 1e-12)
+
+
+def test_planted_e4m3_bias_error_is_caught(monkeypatch):
+    def wrong(codes):
+        c = np.asarray(codes, dtype=np.int64) & 0xFF
+        e = (c >> 3) & 0xF
+        m = (c & 0x7).astype(np.float64)
+        mag = np.where(e == 0, (m / 8.0) * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 8.0))   # bias 8
+        return np.where(c & 0x80, -1.0, 1.0) * np.where((e == 15) & (m == 7), np.nan, mag)
+    monkeypatch.setattr(O, "e4m3_decode", wrong)
+    with pytest.raises(AssertionError):
+        test_e4m3_decode_closed_forms_and_library_table()
+
+
+def test_planted_e4m3_ties_away_is_caught(monkeypatch):
+    real = O.e4m3_encode
+
+    def away(x):
+        x = np.asarray(x, dtype=np.float64)
+        nudged = x * (1 + 2.0 ** -40)          # ties resolve away from zero
+        return real(nudged)
+    monkeypatch.setattr(O, "e4m3_encode", away)
+    with pytest.raises(AssertionError):
+        test_e4m3_ties_saturation_nan_and_round_trip()
