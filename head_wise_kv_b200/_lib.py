@@ -28,6 +28,9 @@ DUO_ERR_WORKSPACE = -4
 DUO_ERR_CUDA = -5
 DUO_ERR_ALIGNMENT = -6
 
+DUO_KV_BF16 = 0
+DUO_KV_FP8_E4M3 = 1
+
 DUO_STATUS_OVER_CAPACITY = 1
 DUO_STATUS_EMPTY_SEQUENCE = 2
 DUO_STATUS_WAIT_TIMEOUT = 4
@@ -55,6 +58,9 @@ class duo_kv_desc(ctypes.Structure):
         ("window", ctypes.c_int32),
         ("capacity", ctypes.c_int64),
         ("retrieval_mask", ctypes.POINTER(ctypes.c_uint8)),
+        ("kv_dtype", ctypes.c_int32),
+        ("k_scale", ctypes.POINTER(ctypes.c_float)),
+        ("v_scale", ctypes.POINTER(ctypes.c_float)),
     ]
 
 
@@ -118,13 +124,23 @@ def duo_strerror(code: int) -> str:
     return _c_strerror(code).decode()
 
 
-def make_desc(num_layers, batch, num_q_heads, num_kv_heads, head_dim, sink, window, capacity, mask_u8):
-    """Build a duo_kv_desc; ``mask_u8`` is a host bytes-like [layers][n_kv] (kept
-    alive by the returned pair)."""
+def make_desc(num_layers, batch, num_q_heads, num_kv_heads, head_dim, sink, window, capacity, mask_u8,
+              kv_dtype=DUO_KV_BF16, k_scale=None, v_scale=None):
+    """Build a duo_kv_desc; ``mask_u8`` is a host bytes-like [layers][n_kv];
+    k_scale / v_scale optional float sequences [layers * n_kv] (FP8).  The
+    host arrays are kept alive by the returned pair."""
     buf = (ctypes.c_uint8 * len(mask_u8)).from_buffer_copy(bytes(mask_u8))
+    keep = [buf]
+
+    def floats(x):
+        if x is None:
+            return None
+        arr = (ctypes.c_float * len(x))(*[float(v) for v in x])
+        keep.append(arr)
+        return ctypes.cast(arr, ctypes.POINTER(ctypes.c_float))
     d = duo_kv_desc(num_layers, batch, num_q_heads, num_kv_heads, head_dim, sink, window, capacity,
-                    ctypes.cast(buf, ctypes.POINTER(ctypes.c_uint8)))
-    return d, buf
+                    ctypes.cast(buf, ctypes.POINTER(ctypes.c_uint8)), kv_dtype, floats(k_scale), floats(v_scale))
+    return d, keep
 
 
 def duo_kv_required_bytes(desc) -> tuple[int, int]:

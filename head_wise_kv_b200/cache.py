@@ -32,10 +32,12 @@ class DuoKVCache:
     """Mixed-head KV cache for ``num_layers`` layers and ``batch`` sequences.
 
     retrieval_mask: [num_layers][num_kv_heads] (1 = retrieval KV head).
+    kv_dtype: "bf16" or "fp8" (E4M3 codes; k_scale / v_scale per
+    [num_layers][num_kv_heads], default 1.0).
     """
 
     def __init__(self, num_layers, batch, num_q_heads, num_kv_heads, head_dim, sink, window, capacity,
-                 retrieval_mask, device="cuda"):
+                 retrieval_mask, device="cuda", kv_dtype="bf16", k_scale=None, v_scale=None):
         self.device = torch.device(device)
         if self.device.type != "cuda":
             raise ValueError("DuoKVCache lives on a CUDA device")
@@ -45,8 +47,20 @@ class DuoKVCache:
         self.mask = mask.copy()
         self.L, self.B, self.hq, self.n_kv, self.d = num_layers, batch, num_q_heads, num_kv_heads, head_dim
         self.S, self.W, self.cap = sink, window, capacity
-        self._desc, self._mask_buf = L.make_desc(num_layers, batch, num_q_heads, num_kv_heads, head_dim,
-                                                 sink, window, capacity, mask.tobytes())
+        if kv_dtype not in ("bf16", "fp8"):
+            raise ValueError("kv_dtype must be 'bf16' or 'fp8'")
+        self.kv_dtype = kv_dtype
+        self.fp8 = kv_dtype == "fp8"
+
+        def scales(x):
+            if x is None:
+                return np.ones((num_layers, num_kv_heads), dtype=np.float32)
+            return np.asarray(x, dtype=np.float32).reshape(num_layers, num_kv_heads)
+        self.k_scale, self.v_scale = scales(k_scale), scales(v_scale)
+        self._desc, self._mask_buf = L.make_desc(
+            num_layers, batch, num_q_heads, num_kv_heads, head_dim, sink, window, capacity, mask.tobytes(),
+            L.DUO_KV_FP8_E4M3 if self.fp8 else L.DUO_KV_BF16, self.k_scale.ravel().tolist(),
+            self.v_scale.ravel().tolist())
         self.total_bytes, self.cache_bytes = L.duo_kv_required_bytes(self._desc)
         with torch.cuda.device(self.device):
             self.buf = torch.empty(self.total_bytes, dtype=torch.uint8, device=self.device)
@@ -78,7 +92,8 @@ class DuoKVCache:
         return L.duo_kv_read_status(self.handle, clear, _stream(self.device))
 
     def layer_views(self, layer: int) -> dict:
-        """Torch views of one layer's cache regions (see duo_kv_layer_view)."""
+        """Torch views of one layer's cache regions (see duo_kv_layer_view):
+        bf16 tensors, or uint8 E4M3 codes for an FP8 cache."""
         v = L.duo_kv_layer_view_get(self.handle, layer)
         base = self.buf.data_ptr()
         B, d, SW, cap = self.B, self.d, self.S + self.W, self.cap
@@ -87,10 +102,14 @@ class DuoKVCache:
             off = ptr - base
             return self.buf[off:off + nbytes]
         nr, ns = v.n_retrieval, v.n_streaming
-        kr = region(v.k_retrieval, B * nr * cap * d * 2).view(torch.bfloat16).view(B, nr, cap, d)
-        vr = region(v.v_retrieval, B * nr * cap * d * 2).view(torch.bfloat16).view(B, nr, cap, d)
-        ks = region(v.k_streaming, B * ns * SW * d * 2).view(torch.bfloat16).view(B, ns, SW, d)
-        vs = region(v.v_streaming, B * ns * SW * d * 2).view(torch.bfloat16).view(B, ns, SW, d)
+        eb = 1 if self.fp8 else 2
+
+        def typed(t):
+            return t if self.fp8 else t.view(torch.bfloat16)
+        kr = typed(region(v.k_retrieval, B * nr * cap * d * eb)).view(B, nr, cap, d)
+        vr = typed(region(v.v_retrieval, B * nr * cap * d * eb)).view(B, nr, cap, d)
+        ks = typed(region(v.k_streaming, B * ns * SW * d * eb)).view(B, ns, SW, d)
+        vs = typed(region(v.v_streaming, B * ns * SW * d * eb)).view(B, ns, SW, d)
         pos = region(v.positions, B * SW * 4).view(torch.int32).view(B, SW)
         rank = [v.head_rank[g] for g in range(self.n_kv)]
         is_r = [bool(v.is_retrieval[g]) for g in range(self.n_kv)]

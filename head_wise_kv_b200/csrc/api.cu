@@ -31,6 +31,15 @@ int check_desc(const duo_kv_desc* d) {
     const int g = d->num_q_heads / d->num_kv_heads;
     if (g != 1 && g != 2 && g != 4 && g != 8) return DUO_ERR_UNSUPPORTED;
     if (d->num_kv_heads > duo::kMaxKvHeads) return DUO_ERR_UNSUPPORTED;
+    if (d->kv_dtype != DUO_KV_BF16 && d->kv_dtype != DUO_KV_FP8_E4M3) return DUO_ERR_INVALID_ARG;
+    if (d->kv_dtype == DUO_KV_FP8_E4M3) {
+        if (d->head_dim != 128) return DUO_ERR_UNSUPPORTED;
+        const size_t n = size_t(d->num_layers) * d->num_kv_heads;
+        for (const float* s : {d->k_scale, d->v_scale})
+            if (s)
+                for (size_t i = 0; i < n; ++i)
+                    if (!(s[i] > 0.f) || !(s[i] < 3.0e38f)) return DUO_ERR_INVALID_ARG;
+    }
     if (d->batch > 65536) return DUO_ERR_UNSUPPORTED;
     return DUO_OK;
 }
@@ -46,6 +55,7 @@ size_t plan_layout(const duo_kv_desc* d, std::vector<duo::LayerLayout>* layers, 
     size_t off = header_bytes(d);
     size_t cache = 0;
     const size_t D = size_t(d->head_dim), B = size_t(d->batch), SW = size_t(d->sink) + d->window;
+    const size_t E = d->kv_dtype == DUO_KV_FP8_E4M3 ? 1 : 2;   // bytes per cached element
     for (int l = 0; l < d->num_layers; ++l) {
         duo::LayerLayout L;
         memset(L.rank, 0, sizeof L.rank);
@@ -58,8 +68,8 @@ size_t plan_layout(const duo_kv_desc* d, std::vector<duo::LayerLayout>* layers, 
             L.rank[g] = r ? L.n_r++ : L.n_s++;
         }
         L.r_before[d->num_kv_heads] = L.n_r;
-        const size_t kr = B * L.n_r * size_t(d->capacity) * D * 2;
-        const size_t ks = B * L.n_s * SW * D * 2;
+        const size_t kr = B * L.n_r * size_t(d->capacity) * D * E;
+        const size_t ks = B * L.n_s * SW * D * E;
         L.off_kr = off; off = align_up(off + kr);
         L.off_vr = off; off = align_up(off + kr);
         L.off_ks = off; off = align_up(off + ks);
@@ -97,6 +107,17 @@ int duo_kv_alloc(const duo_kv_desc* desc, void* dev_buf, size_t buf_bytes, duo_s
     if (!h) return DUO_ERR_INVALID_ARG;
     h->desc = *desc;
     h->desc.retrieval_mask = nullptr;
+    h->desc.k_scale = h->desc.v_scale = nullptr;
+    h->fp8 = desc->kv_dtype == DUO_KV_FP8_E4M3;
+    {
+        const size_t n = size_t(desc->num_layers) * desc->num_kv_heads;
+        h->k_scale.assign(n, 1.f);
+        h->v_scale.assign(n, 1.f);
+        for (size_t i = 0; i < n; ++i) {
+            if (desc->k_scale) h->k_scale[i] = desc->k_scale[i];
+            if (desc->v_scale) h->v_scale[i] = desc->v_scale[i];
+        }
+    }
     const size_t need = plan_layout(desc, &h->layers, nullptr);
     if (buf_bytes < need) {
         delete h;
@@ -124,7 +145,8 @@ int duo_kv_alloc(const duo_kv_desc* desc, void* dev_buf, size_t buf_bytes, duo_s
         for (size_t l = 0; l < h->layers.size(); ++l) {
             const duo::LayerLayout& L = h->layers[l];
             if (!duo::make_decode_maps(&h->maps[l], h->base + L.off_kr, h->base + L.off_vr, h->base + L.off_ks,
-                                       h->base + L.off_vs, desc->batch, L.n_r, L.n_s, desc->capacity, int(SW))) {
+                                       h->base + L.off_vs, desc->batch, L.n_r, L.n_s, desc->capacity, int(SW),
+                                       h->fp8 != 0)) {
                 delete h;
                 return DUO_ERR_CUDA;
             }
@@ -170,6 +192,7 @@ static int append_impl(duo_kv* kv, int32_t layer, const uint16_t* k_new, const u
     if ((reinterpret_cast<uintptr_t>(r_pos_begin) & 3) || (reinterpret_cast<uintptr_t>(r_pos_end) & 3))
         return DUO_ERR_ALIGNMENT;
     duo::AppendParams p;
+    memset(&p, 0, sizeof p);
     p.r_pos_begin = r_pos_begin;
     p.r_pos_end = r_pos_end;
     p.k_new = k_new;
@@ -193,6 +216,11 @@ static int append_impl(duo_kv* kv, int32_t layer, const uint16_t* k_new, const u
     p.n_new_max = n_new_max;
     memcpy(p.rank, L.rank, sizeof p.rank);
     memcpy(p.is_r, L.is_r, sizeof p.is_r);
+    p.fp8 = kv->fp8;
+    for (int g = 0; g < kv->desc.num_kv_heads; ++g) {
+        p.k_scale[g] = kv->k_scale[size_t(layer) * kv->desc.num_kv_heads + g];
+        p.v_scale[g] = kv->v_scale[size_t(layer) * kv->desc.num_kv_heads + g];
+    }
     return cuda_err(duo::launch_append(p, stream));
 }
 
@@ -280,6 +308,11 @@ static int decode_impl(duo_kv* kv, int32_t layer, const uint16_t* q, const int32
     memcpy(p.rank, L.rank, sizeof p.rank);
     memcpy(p.r_before, L.r_before, sizeof p.r_before);
     memcpy(p.is_r, L.is_r, sizeof p.is_r);
+    p.fp8 = kv->fp8;
+    for (int g = 0; g < kv->desc.num_kv_heads; ++g) {
+        p.k_scale[g] = kv->k_scale[size_t(layer) * kv->desc.num_kv_heads + g];
+        p.v_scale[g] = kv->v_scale[size_t(layer) * kv->desc.num_kv_heads + g];
+    }
     return cuda_err(duo::launch_decode(p, D, G, stream));
 }
 
@@ -345,6 +378,7 @@ int duo_prefill_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const uint16_
         return DUO_ERR_INVALID_ARG;
     if (!(scale > 0.f) || scale != scale) return DUO_ERR_INVALID_ARG;
     if (kv->desc.head_dim != 128) return DUO_ERR_UNSUPPORTED;
+    if (kv->fp8) return DUO_ERR_UNSUPPORTED;   // FP8 prefix not read by the prefill kernel yet
     const duo_kv_desc& d = kv->desc;
     if (duo::prefill_smem_bytes(d.sink, d.window) > 227 * 1024) return DUO_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k_chunk) || !aligned16(v_chunk) || !aligned16(out) ||
@@ -361,6 +395,7 @@ int duo_prefill_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const uint16_
                                        int64_t(d.batch) * L.n_s * (SW + 256)});
     if (rows_max >= (int64_t(1) << 31)) return DUO_ERR_UNSUPPORTED;
     duo::PrefillLaunch a;
+    memset(&a, 0, sizeof a);
     a.q = q;
     a.k_chunk = k_chunk;
     a.v_chunk = v_chunk;
@@ -385,6 +420,11 @@ int duo_prefill_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const uint16_
     a.timeout_ns = kWaitLimitNs;
     memcpy(a.rank, L.rank, sizeof a.rank);
     memcpy(a.is_r, L.is_r, sizeof a.is_r);
+    a.fp8 = kv->fp8;
+    for (int g = 0; g < d.num_kv_heads; ++g) {
+        a.k_scale[g] = kv->k_scale[size_t(layer) * d.num_kv_heads + g];
+        a.v_scale[g] = kv->v_scale[size_t(layer) * d.num_kv_heads + g];
+    }
     return duo::launch_prefill(a, stream);
 }
 

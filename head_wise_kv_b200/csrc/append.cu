@@ -27,6 +27,30 @@ namespace {
 
 constexpr int kThreads = 256;
 
+// Eight bf16 values (16 bytes) -> their eight E4M3 codes of value / scale:
+// IEEE fp32 division, then round-to-nearest-even with saturation (the
+// conversion puts its first operand in the upper byte).
+__device__ __forceinline__ uint2 e4m3_codes(uint4 x, float scale) {
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    uint16_t c[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float lo = __fdiv_rn(__uint_as_float(w[i] << 16), scale);
+        const float hi = __fdiv_rn(__uint_as_float(w[i] & 0xffff0000u), scale);
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(c[i]) : "f"(hi), "f"(lo));
+    }
+    return make_uint2(uint32_t(c[0]) | (uint32_t(c[1]) << 16), uint32_t(c[2]) | (uint32_t(c[3]) << 16));
+}
+
+// Store 8 elements (16 bytes of bf16) at element offset `dst` of a cache:
+// as given, or as E4M3 codes (8 bytes).
+__device__ __forceinline__ void put8(const AppendParams& p, uint16_t* base, size_t dst, uint4 v, float scale) {
+    if (p.fp8)
+        *reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(base) + dst) = e4m3_codes(v, scale);
+    else
+        *reinterpret_cast<uint4*>(base + dst) = v;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads) append_kernel(const __grid_constant__ AppendParams p) {
     // A decode launched next as a programmatic dependent may start its
@@ -82,14 +106,14 @@ __global__ void __launch_bounds__(kThreads) append_kernel(const __grid_constant_
         const uint4 kv = *reinterpret_cast<const uint4*>(p.k_new + src);
         const uint4 vv = *reinterpret_cast<const uint4*>(p.v_new + src);
         const size_t dst = ((size_t(b) * p.n_r + p.rank[g]) * size_t(p.cap) + row) * D + part * 8;
-        *reinterpret_cast<uint4*>(p.kr + dst) = kv;
-        *reinterpret_cast<uint4*>(p.vr + dst) = vv;
+        put8(p, p.kr, dst, kv, p.k_scale[g]);
+        put8(p, p.vr, dst, vv, p.v_scale[g]);
     } else if (survives) {
         const uint4 kv = *reinterpret_cast<const uint4*>(p.k_new + src);
         const uint4 vv = *reinterpret_cast<const uint4*>(p.v_new + src);
         const size_t dst = ((size_t(b) * p.n_s + p.rank[g]) * SW + slot) * D + part * 8;
-        *reinterpret_cast<uint4*>(p.ks + dst) = kv;
-        *reinterpret_cast<uint4*>(p.vs + dst) = vv;
+        put8(p, p.ks, dst, kv, p.k_scale[g]);
+        put8(p, p.vs, dst, vv, p.v_scale[g]);
     }
 }
 

@@ -61,23 +61,20 @@
 #include "duo_internal.cuh"
 #include "tcgen05.cuh"
 
+#include <cuda_fp16.h>
+
 namespace duo {
 
 namespace {
 
 constexpr int kD = 128;                       // head dim
-constexpr int kT = 128;                       // keys per tile
-constexpr int kN = 16;                        // MMA N (query-head columns)
 constexpr int kThreads = 384;
 constexpr int kSoftWarp0 = 2;              // softmax warps 2-5
 constexpr int kVWarp = 6;
 constexpr int kQWarp = 7;
 constexpr int kEpiWarp0 = 8;               // epilogue warps 8-11
-constexpr uint32_t kSlab = 128 * 128;         // 128 rows x 64 bf16: one dim-half of a tile
-constexpr uint32_t kTileBytes = 2 * kSlab;    // 32 KB: one of K or V
-constexpr uint32_t kSmall = kN * kD * 2;      // 4 KB: the q or P^T operand (16 rows)
-constexpr uint32_t kTmemCols = 128;
-constexpr uint32_t kTmemS0 = 0, kTmemS1 = 32, kTmemO0 = 64;   // O^T of piece pi at kTmemO0 + 32 (pi & 1)
+constexpr uint32_t kSlab = 128 * 128;         // 128 rows x 64 bf16: one dim-half of a bf16 tile
+constexpr uint32_t kTileBytes = 32768;        // one K or V tile: 128 bf16 rows or 256 FP8 rows
 constexpr float kNegBig = -1.0e30f;
 constexpr float kRescaleThreshold = 8.0f;     // log2 units: probabilities stay <= 2^8
 // Partition weight of a segment start in 16-token blocks: starting a piece
@@ -89,8 +86,68 @@ constexpr float kRescaleThreshold = 8.0f;     // log2 units: probabilities stay 
 #endif
 constexpr int kSegWeight = DUO_DECODE_SEG_WEIGHT;
 
-constexpr uint32_t kIdescQK = idesc_f16(kT, kN, true, false, false);   // A = K (K-major), B = q (K-major)
-constexpr uint32_t kIdescPV = idesc_f16(kD, kN, true, true, false);    // A = V^T (MN-major), B = P^T
+// Shapes of the two element types.
+//   bf16: 128-key tiles; S^T one column per head (q as is); P as hi + lo
+//         bf16 terms, so O^T holds two columns per head.
+//   FP8:  256-key tiles (two 128-key halves of S^T); q and P each as a sum of
+//         four E4M3 terms (~16 significant bits), columns term * G + h; the
+//         products run as kind::f8f6f4 straight on the cached codes.
+template <int G, bool F8>
+struct Tr {
+    static constexpr int T = F8 ? 256 : 128;                       // keys per tile
+    static constexpr int HALVES = T / 128;                         // 128-key blocks of S^T
+    static constexpr int QT = F8 ? 4 : 1;                          // q terms
+    static constexpr int PT = F8 ? 4 : 2;                          // P terms
+    static constexpr int N = F8 ? ((4 * G + 15) / 16) * 16 : 16;   // MMA N
+    static constexpr uint32_t SB = HALVES * N < 32 ? 32 : HALVES * N;   // TMEM columns of one S buffer
+    static constexpr uint32_t OB = N < 32 ? 32 : N;                     // of one O buffer
+    static constexpr uint32_t S0 = 0, S1 = SB, O0 = 2 * SB;
+    static constexpr uint32_t RAW = 2 * SB + 2 * OB;
+    static constexpr uint32_t COLS = RAW <= 32 ? 32 : RAW <= 64 ? 64 : RAW <= 128 ? 128 : RAW <= 256 ? 256 : 512;
+    static constexpr uint32_t QB = 4096;                           // bytes of one q operand
+    static constexpr uint32_t PB = F8 ? N * 256 : 4096;            // bytes of one P^T operand
+    static constexpr uint32_t PHALF = F8 ? N * 128 : 2048;         // P^T bytes per K-half (128 / 64 keys)
+    // FP8: P enters the MMA as P' = 2^7 P with the running max kept within
+    // 2^1 of the tile maxima, so P' <= 256 < 448 and the E4M3 grid floor
+    // (2^-10 after four terms) sits 2^-17 below the largest probability;
+    // bf16 terms have no such floor (threshold 2^8, no offset).
+    static constexpr float THRESH = F8 ? 1.0f : kRescaleThreshold;    // log2 units
+    static constexpr float POFF = F8 ? 7.0f : 0.0f;                    // log2 of the P offset
+    static constexpr uint32_t IQK = idesc_f16(128, N, !F8, false, false);   // A = K (K-major), B = q
+    static constexpr uint32_t IPV = idesc_f16(kD, N, !F8, true, false);     // A = V^T (MN-major), B = P^T
+    static_assert(QT * G <= N && PT * G <= N, "terms must fit the MMA N");
+};
+
+// Two values -> two E4M3 codes (round to nearest even, saturating); the
+// first operand lands in the upper byte.
+__device__ __forceinline__ uint16_t e4m3x2(float hi, float lo) {
+    uint16_t c;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(c) : "f"(hi), "f"(lo));
+    return c;
+}
+
+// Two E4M3 codes -> their values (exact): .x from the low byte.
+__device__ __forceinline__ float2 e4m3x2_value(uint16_t c) {
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(c));
+    return make_float2(__half2float(__ushort_as_half(uint16_t(h2 & 0xffff))),
+                       __half2float(__ushort_as_half(uint16_t(h2 >> 16))));
+}
+
+// D (TMEM) (+)= A (smem, E4M3) * B (smem, E4M3), fp32 accumulate.
+__device__ __forceinline__ void umma_f8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void st_shared_u8(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared.b8 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
 
 // Byte offset of 16-byte chunk c (0..15, along the 128 dims or keys) of row
 // r (0..15) in a 16-row K-major operand with 128-byte swizzle: two 2 KB
@@ -99,10 +156,12 @@ __device__ __forceinline__ uint32_t small_off(int r, int c) {
     return uint32_t((c >> 3) * 2048 + (r >> 3) * 1024 + (r & 7) * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
 
-__device__ __forceinline__ int tiles_of(const Piece& pc) { return int((pc.tok1 - pc.tok0 + kT - 1) / kT); }
+template <int T>
+__device__ __forceinline__ int tiles_of(const Piece& pc) { return int((pc.tok1 - pc.tok0 + T - 1) / T); }
 
-// Position in the CTA's sequence of tiles: piece `pi` (pc), tile t of its
-// nt; gb is where the search for the next piece starts.
+// Position in the CTA's sequence of tiles (T keys each): piece `pi` (pc),
+// tile t of its nt; gb is where the search for the next piece starts.
+template <int T>
 struct TileCursor {
     Piece pc;
     int pi, t, nt;
@@ -115,14 +174,14 @@ struct TileCursor {
         t = 0;
         gb = gb_begin;
         valid = next_piece(p, bpre, gb, gb_end, pc);
-        if (valid) nt = tiles_of(pc);
+        if (valid) nt = tiles_of<T>(pc);
     }
     __device__ void advance(const DecodeParams& p, const int32_t* bpre, int64_t gb_end) {
         if (++t < nt) return;
         t = 0;
         ++pi;
         valid = next_piece(p, bpre, gb, gb_end, pc);
-        if (valid) nt = tiles_of(pc);
+        if (valid) nt = tiles_of<T>(pc);
     }
 };
 
@@ -210,8 +269,9 @@ constexpr int kBarSoftmax = 1, kBarEpilogue = 2;
 
 __device__ __forceinline__ uint16_t bf16_bits(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
 
-template <int G>
+template <int G, bool F8>
 __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_constant__ DecodeParams p) {
+    using C = Tr<G, F8>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -219,13 +279,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     const uint32_t sK = smem_addr(smem);                  // nst K tiles
     const uint32_t sV = sK + nst * kTileBytes;            // nst V tiles
     const uint32_t sQ = sV + nst * kTileBytes;            // 2 q operands (piece parity)
-    const uint32_t sP = sQ + 2 * kSmall;                  // 2 P^T operands (tile parity)
-    int32_t* bpre = reinterpret_cast<int32_t*>(smem + 2 * nst * kTileBytes + 4 * kSmall);
+    const uint32_t sP = sQ + 2 * C::QB;                   // 2 P^T operands (tile parity)
+    int32_t* bpre = reinterpret_cast<int32_t*>(smem + 2 * nst * kTileBytes + 2 * C::QB + 2 * C::PB);
 
     constexpr int kMaxStages = 3;
     __shared__ __align__(8) uint64_t full_k[kMaxStages], full_v[kMaxStages], empty_k[kMaxStages],
         empty_v[kMaxStages], q_full[2],
-        q_empty[2], s_full[2], s_free[2], p_full[2], p_free[2], o_full[2], o_empty[2], epi_full[2], mma_fin;
+        q_empty[2], s_full[2], s_free[2], p_full[2], p_free[2], o_full[2], o_empty[2], epi_full[2], mma_fin,
+        qs_full[4];
+    // FP8: 2^-a of each piece's q prescale, a ring of four (the q warp runs
+    // at most three pieces ahead of the softmax, see the q warp)
+    __shared__ float q_scale[4];
     __shared__ uint32_t tmem_base_sh;
     __shared__ float red_max[2][4][G];
     __shared__ float red_l[2][4][G];   // [piece parity][softmax warp][head] row sums
@@ -255,13 +319,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             mbar_init(smem_addr(&epi_full[s]), 4);
         }
         mbar_init(smem_addr(&mma_fin), 1);
+        for (int s = 0; s < 4; ++s) mbar_init(smem_addr(&qs_full[s]), 1);
         abort_sh = 0;
         fence_mbar_init();
     }
     // q and P^T rows past the heads in use stay zero (their S / O columns are never read)
-    for (uint32_t o = threadIdx.x * 16; o < 4 * kSmall; o += kThreads * 16) st_shared_v4(sQ + o, make_uint4(0, 0, 0, 0));
+    for (uint32_t o = threadIdx.x * 16; o < 2 * (C::QB + C::PB); o += kThreads * 16)
+        st_shared_v4(sQ + o, make_uint4(0, 0, 0, 0));
     fence_proxy_async_smem();
-    if (warp == 1) tmem_alloc(smem_addr(&tmem_base_sh), kTmemCols);
+    if (warp == 1) tmem_alloc(smem_addr(&tmem_base_sh), C::COLS);
     if (threadIdx.x == 32) {
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tm_kr)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tm_vr)) : "memory");
@@ -297,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                     if (!next_piece(p, bpre, gb, gb_end, pc)) break;
                     const CUtensorMap* mk = pc.retr ? &p.tm_kr : &p.tm_ks;
                     const int z = pc.b * (pc.retr ? p.n_r : p.n_s) + pc.rank;
-                    for (int64_t t = pc.tok0; t < pc.tok1; t += kT, ++it) {
+                    for (int64_t t = pc.tok0; t < pc.tok1; t += C::T, ++it) {
                         const int st = int(it % uint32_t(nst));
                         if (!timed_wait(smem_addr(&empty_k[st]), ((it / nst) & 1) ^ 1, p, abort_flag)) {
                             ok = false;
@@ -306,8 +372,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                         const int y = int(pc.row0 + t);
                         const uint32_t fk = smem_addr(&full_k[st]);
                         mbar_arrive_expect_tx(fk, kTileBytes);
-                        tma_load_3d(sK + st * kTileBytes, mk, 0, y, z, fk, policy);
-                        tma_load_3d(sK + st * kTileBytes + kSlab, mk, 64, y, z, fk, policy);
+                        if constexpr (F8) {
+                            tma_load_3d(sK + st * kTileBytes, mk, 0, y, z, fk, policy);   // 256 rows x 128 codes
+                        } else {
+                            tma_load_3d(sK + st * kTileBytes, mk, 0, y, z, fk, policy);
+                            tma_load_3d(sK + st * kTileBytes + kSlab, mk, 64, y, z, fk, policy);
+                        }
                     }
                 }
                 // do not leave while copies may still land in this CTA's shared memory
@@ -325,14 +395,83 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                 if (!next_piece(p, bpre, gb, gb_end, pc)) break;
                 if (!warp_wait(smem_addr(&q_empty[pi & 1]), ((pi >> 1) & 1) ^ 1, p, abort_flag)) break;
                 const uint16_t* qb = p.q + (size_t(pc.b) * p.hq + size_t(pc.g) * G) * kD;
-                const uint32_t qs = sQ + (pi & 1) * kSmall;
-                for (int c = lane; c < G * 16; c += 32) {
-                    const int h = c >> 4, c16 = c & 15;
-                    st_shared_v4(qs + small_off(h, c16), *reinterpret_cast<const uint4*>(qb + h * kD + c16 * 8));
+                const uint32_t qs = sQ + (pi & 1) * C::QB;
+                if constexpr (F8) {
+                    // q' = q * 2^a (exact) with max |q'| in [128, 256), then four
+                    // E4M3 terms, each the code of what the previous ones left:
+                    // q' = t0 + t1 + t2 + t3 + r, |r| ~ 2^-16 |q'|.  Row
+                    // term * G + h of the operand holds term `term` of head h.
+                    constexpr int kItems = (G * 8 + 31) / 32;   // (head, 16-dim chunk) per lane
+                    uint4 raw[kItems][2];
+                    float amax = 0.f;
+#pragma unroll
+                    for (int k = 0; k < kItems; ++k) {
+                        const int c = lane + 32 * k;
+                        raw[k][0] = raw[k][1] = make_uint4(0, 0, 0, 0);
+                        if (c < G * 8) {
+                            const uint16_t* src = qb + (c >> 3) * kD + (c & 7) * 16;
+                            raw[k][0] = *reinterpret_cast<const uint4*>(src);
+                            raw[k][1] = *reinterpret_cast<const uint4*>(src + 8);
+                        }
+                        const uint32_t w[8] = {raw[k][0].x, raw[k][0].y, raw[k][0].z, raw[k][0].w,
+                                               raw[k][1].x, raw[k][1].y, raw[k][1].z, raw[k][1].w};
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w[i] << 16)),
+                                                     fabsf(__uint_as_float(w[i] & 0xffff0000u))));
+                    }
+                    uint32_t abits;   // non-negative floats order like their bit patterns
+                    asm volatile("redux.sync.max.u32 %0, %1, 0xffffffff;" : "=r"(abits) : "r"(__float_as_uint(amax)));
+                    const int e = abits ? int((abits >> 23) & 0xff) - 127 : 0;
+                    const int a = e > 107 ? -100 : (e < -93 ? 100 : 7 - e);
+                    const float up = __uint_as_float(uint32_t(a + 127) << 23);   // 2^a
+#pragma unroll
+                    for (int k = 0; k < kItems; ++k) {
+                        const int c = lane + 32 * k;
+                        if (c >= G * 8) continue;
+                        const uint32_t w[8] = {raw[k][0].x, raw[k][0].y, raw[k][0].z, raw[k][0].w,
+                                               raw[k][1].x, raw[k][1].y, raw[k][1].z, raw[k][1].w};
+                        float y[16];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            y[2 * i] = __uint_as_float(w[i] << 16) * up;
+                            y[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u) * up;
+                        }
+#pragma unroll
+                        for (int term = 0; term < 4; ++term) {
+                            uint32_t pk[4];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const uint16_t c2 = e4m3x2(y[2 * i + 1], y[2 * i]);
+                                if (i & 1) pk[i >> 1] |= uint32_t(c2) << 16; else pk[i >> 1] = c2;
+                                if (term < 3) {
+                                    const float2 v = e4m3x2_value(c2);
+                                    y[2 * i] -= v.x;
+                                    y[2 * i + 1] -= v.y;
+                                }
+                            }
+                            st_shared_v4(qs + small_off(term * G + (c >> 3), c & 7), make_uint4(pk[0], pk[1], pk[2], pk[3]));
+                        }
+                    }
+                    // factor that turns the S columns' sum into q.k in cache
+                    // units times the key scale: 2^-a * k_scale
+                    if (lane == 0) q_scale[pi & 3] = __uint_as_float(uint32_t(127 - a) << 23) * p.k_scale[pc.g];
+                } else {
+                    for (int c = lane; c < G * 16; c += 32) {
+                        const int h = c >> 4, c16 = c & 15;
+                        st_shared_v4(qs + small_off(h, c16), *reinterpret_cast<const uint4*>(qb + h * kD + c16 * 8));
+                    }
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_addr(&q_full[pi & 1]));
+                if (lane == 0) {
+                    mbar_arrive(smem_addr(&q_full[pi & 1]));
+                    // Ring of four for the softmax: the q warp can stage piece
+                    // pi + 3 at most (it needs the last S product of pi + 1,
+                    // which needs the softmax past piece pi), so an entry and
+                    // its barrier phase are never reused before being read.
+                    if constexpr (F8) mbar_arrive(smem_addr(&qs_full[pi & 3]));
+                }
             }
         } else if (warp == kVWarp) {
             // ======================================================== V producer
@@ -345,7 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                     if (!next_piece(p, bpre, gb, gb_end, pc)) break;
                     const CUtensorMap* mv = pc.retr ? &p.tm_vr : &p.tm_vs;
                     const int z = pc.b * (pc.retr ? p.n_r : p.n_s) + pc.rank;
-                    for (int64_t t = pc.tok0; t < pc.tok1; t += kT, ++it) {
+                    for (int64_t t = pc.tok0; t < pc.tok1; t += C::T, ++it) {
                         const int st = int(it % uint32_t(nst));
                         if (!timed_wait(smem_addr(&empty_v[st]), ((it / nst) & 1) ^ 1, p, abort_flag)) {
                             ok = false;
@@ -354,8 +493,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                         const int y = int(pc.row0 + t);
                         const uint32_t fv = smem_addr(&full_v[st]);
                         mbar_arrive_expect_tx(fv, kTileBytes);
-                        tma_load_3d(sV + st * kTileBytes, mv, 0, y, z, fv, policy);
-                        tma_load_3d(sV + st * kTileBytes + kSlab, mv, 64, y, z, fv, policy);
+                        if constexpr (F8) {
+                            tma_load_3d(sV + st * kTileBytes, mv, 0, y, z, fv, policy);
+                        } else {
+                            tma_load_3d(sV + st * kTileBytes, mv, 0, y, z, fv, policy);
+                            tma_load_3d(sV + st * kTileBytes + kSlab, mv, 64, y, z, fv, policy);
+                        }
                     }
                 }
                 for (uint32_t k = 0; k < uint32_t(nst) && k < it; ++k) {
@@ -370,7 +513,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             // with it the release of stage j) never waits on the arrival of
             // K_{j+1}.
             if (lane == 0) {
-                TileCursor cq, cv;   // next S tile, next PV tile
+                TileCursor<C::T> cq, cv;   // next S tile, next PV tile
                 cq.start(p, bpre, gb_begin, gb_end);
                 cv.start(p, bpre, gb_begin, gb_end);
                 uint32_t jq = 0, jv = 0;
@@ -384,13 +527,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                             mbar_test_wait(smem_addr(&full_k[st]), (jq / nst) & 1) &&
                             mbar_test_wait(smem_addr(&s_free[jq & 1]), ((jq >> 1) & 1) ^ 1)) {
                             tc_fence_after();
-                            const uint32_t sk = sK + st * kTileBytes, sq = sQ + (cq.pi & 1) * kSmall;
+                            const uint32_t sk = sK + st * kTileBytes, sq = sQ + (cq.pi & 1) * C::QB;
+                            const uint32_t ts = tmem + ((jq & 1) ? C::S1 : C::S0);
+                            if constexpr (F8) {
+                                // two 128-key halves; K = d = 128 codes = one swizzled row, 4 x K32
 #pragma unroll
-                            for (int k = 0; k < kD / 16; ++k) {
-                                const uint32_t off = (k >> 2) * kSlab + (k & 3) * 32;
-                                const uint32_t qoff = (k >> 2) * 2048 + (k & 3) * 32;
-                                umma_f16(tmem + ((jq & 1) ? kTmemS1 : kTmemS0), smem_desc(sk + off, 16, 1024),
-                                         smem_desc(sq + qoff, 16, 1024), kIdescQK, k > 0 ? 1u : 0u);
+                                for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+                                    for (int k = 0; k < 4; ++k)
+                                        umma_f8(ts + hf * C::N, smem_desc(sk + hf * 16384 + k * 32, 16, 1024),
+                                                smem_desc(sq + k * 32, 16, 1024), C::IQK, k > 0 ? 1u : 0u);
+                            } else {
+#pragma unroll
+                                for (int k = 0; k < kD / 16; ++k) {
+                                    const uint32_t off = (k >> 2) * kSlab + (k & 3) * 32;
+                                    const uint32_t qoff = (k >> 2) * 2048 + (k & 3) * 32;
+                                    umma_f16(ts, smem_desc(sk + off, 16, 1024), smem_desc(sq + qoff, 16, 1024), C::IQK,
+                                             k > 0 ? 1u : 0u);
+                                }
                             }
                             umma_commit(smem_addr(&s_full[jq & 1]));
                             umma_commit(smem_addr(&empty_k[st]));
@@ -406,12 +560,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                             mbar_test_wait(smem_addr(&full_v[st]), (jv / nst) & 1) &&
                             (cv.t > 0 || mbar_test_wait(smem_addr(&o_empty[cv.pi & 1]), ((cv.pi >> 1) & 1) ^ 1))) {
                             tc_fence_after();
-                            const uint32_t sv = sV + st * kTileBytes, sp = sP + (jv & 1) * kSmall;
+                            const uint32_t sv = sV + st * kTileBytes, sp = sP + (jv & 1) * C::PB;
+                            const uint32_t to = tmem + C::O0 + (cv.pi & 1) * C::OB;
+                            if constexpr (F8) {
+                                // V^T MN-major: d = 128 codes is one 128-byte atom; 8 x K32 keys
 #pragma unroll
-                            for (int k = 0; k < kT / 16; ++k)
-                                umma_f16(tmem + kTmemO0 + (cv.pi & 1) * 32, smem_desc(sv + k * 2048, kSlab, 1024),
-                                         smem_desc(sp + (k >> 2) * 2048 + (k & 3) * 32, 16, 1024), kIdescPV,
-                                         (cv.t > 0 || k > 0) ? 1u : 0u);
+                                for (int k = 0; k < 8; ++k)
+                                    umma_f8(to, smem_desc(sv + k * 4096, 16, 1024),
+                                            smem_desc(sp + (k >> 2) * C::PHALF + (k & 3) * 32, 16, 1024), C::IPV,
+                                            (cv.t > 0 || k > 0) ? 1u : 0u);
+                            } else {
+#pragma unroll
+                                for (int k = 0; k < 128 / 16; ++k)
+                                    umma_f16(to, smem_desc(sv + k * 2048, kSlab, 1024),
+                                             smem_desc(sp + (k >> 2) * C::PHALF + (k & 3) * 32, 16, 1024), C::IPV,
+                                             (cv.t > 0 || k > 0) ? 1u : 0u);
+                            }
                             umma_commit(smem_addr(&empty_v[st]));
                             umma_commit(smem_addr(&p_free[jv & 1]));
                             if (cv.t == cv.nt - 1) umma_commit(smem_addr(&o_full[cv.pi & 1]));
@@ -451,14 +615,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                                  warp_wait_lazy(smem_addr(&o_full[pi & 1]), (pi >> 1) & 1, p, abort_flag);
                 if (barrier_any<kBarEpilogue>(!got)) break;
                 tc_fence_after();
-                uint32_t u[2 * G];
-                tmem_ldn<2 * G>(tmem + lane_off + kTmemO0 + (pi & 1) * 32, u);
+                uint32_t u[C::PT * G];
+                tmem_ldn<C::PT * G>(tmem + lane_off + C::O0 + (pi & 1) * C::OB, u);
                 tmem_wait_ld();
-                float L[G], M[G];
+                float L[G], M[G], o[G];
+                const float vs = F8 ? p.v_scale[pc.g] : 1.f;   // FP8: O^T is in value-code units
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    float x = 0.f;
+#pragma unroll
+                    for (int term = 0; term < C::PT; ++term) x += __uint_as_float(u[term * G + h]);
+                    o[h] = x * vs;
+                }
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
                     L[h] = red_l[pi & 1][0][h] + red_l[pi & 1][1][h] + red_l[pi & 1][2][h] + red_l[pi & 1][3][h];
-                    M[h] = epi_m[pi & 1][h];
+                    M[h] = epi_m[pi & 1][h] - C::POFF;   // sums are of P' = 2^POFF P
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -466,9 +638,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                 if (pc.whole) {
 #pragma unroll
                     for (int h = 0; h < G; ++h) {
-                        const float o = __uint_as_float(u[h]) + __uint_as_float(u[G + h]);
                         const int qh = pc.g * G + h;
-                        p.out[(size_t(pc.b) * p.hq + qh) * kD + d] = L[h] > 0.f ? o / L[h] : 0.f;
+                        p.out[(size_t(pc.b) * p.hq + qh) * kD + d] = L[h] > 0.f ? o[h] / L[h] : 0.f;
                         if (d == 0 && p.lse != nullptr)
                             p.lse[size_t(pc.b) * p.hq + qh] =
                                 L[h] > 0.f ? (M[h] + __log2f(L[h])) * 0.69314718055994530942f : -CUDART_INF_F;
@@ -482,7 +653,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                     const size_t slot = size_t(pc.seg) + blockIdx.x;
 #pragma unroll
                     for (int h = 0; h < G; ++h) {
-                        p.ws_o[(slot * G + h) * kD + d] = __uint_as_float(u[h]) + __uint_as_float(u[G + h]);
+                        p.ws_o[(slot * G + h) * kD + d] = o[h];
                         if (d == 0) {
                             p.ws_ml[(slot * G + h) * 2 + 0] = M[h];
                             p.ws_ml[(slot * G + h) * 2 + 1] = L[h];
@@ -536,7 +707,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             // ======================================================== softmax
             const int sw = warp - kSoftWarp0;              // 0..3
             const int sub = warp & 3;                      // TMEM lane quarter this warp may access
-            const int row = sub * 32 + lane;               // key row of S^T; output dim of O^T
+            const int row = sub * 32 + lane;               // key row of each 128-key S^T block
             const uint32_t lane_off = uint32_t(sub * 32) << 16;
             uint32_t j = 0;
             bool ok = true;
@@ -544,38 +715,57 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             for (int64_t gb = gb_begin; ok && gb < gb_end; ++pi) {
                 Piece pc;
                 if (!next_piece(p, bpre, gb, gb_end, pc)) break;
-                const uint32_t tmem_o = tmem + lane_off + kTmemO0 + (pi & 1) * 32;
+                const uint32_t tmem_o = tmem + lane_off + C::O0 + (pi & 1) * C::OB;
+                float sc = p.scale_log2;   // log2(e) * scale, per score
+                if constexpr (F8) {
+                    // (on failure the first tile's barrier below agrees on leaving)
+                    if (warp_wait(smem_addr(&qs_full[pi & 3]), (pi >> 2) & 1, p, abort_flag)) sc *= q_scale[pi & 3];
+                }
                 float m[G], l[G];
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
                     m[h] = kNegBig;
                     l[h] = 0.f;
                 }
-                const int nt = tiles_of(pc);
+                const int nt = tiles_of<C::T>(pc);
                 const int64_t rows_total = pc.tok1 - pc.tok0;
                 for (int t = 0; t < nt; ++t, ++j) {
                     const uint32_t sb = j & 1;
                     const int st = int(j % uint32_t(nst));
                     const bool got = warp_wait(smem_addr(&s_full[sb]), (j >> 1) & 1, p, abort_flag);
-                    float s[G];
+                    float s[C::HALVES][G];
                     if (got) {
                         tc_fence_after();
-                        uint32_t u[G];
-                        tmem_ldn<G>(tmem + lane_off + (sb ? kTmemS1 : kTmemS0), u);
+                        uint32_t u[C::HALVES][C::QT * G];
+#pragma unroll
+                        for (int hf = 0; hf < C::HALVES; ++hf)
+                            tmem_ldn<C::QT * G>(tmem + lane_off + (sb ? C::S1 : C::S0) + hf * C::N, u[hf]);
                         tmem_wait_ld();
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(smem_addr(&s_free[sb]));
 #pragma unroll
-                        for (int h = 0; h < G; ++h) s[h] = __uint_as_float(u[h]);
+                        for (int hf = 0; hf < C::HALVES; ++hf)
+#pragma unroll
+                            for (int h = 0; h < G; ++h) {
+                                float x = __uint_as_float(u[hf][h]);
+#pragma unroll
+                                for (int term = 1; term < C::QT; ++term) x += __uint_as_float(u[hf][term * G + h]);
+                                s[hf][h] = x;
+                            }
                     }
-                    const int64_t left = rows_total - int64_t(t) * kT;
-                    const int valid_rows = int(left < kT ? left : kT);
-                    const bool valid = got && row < valid_rows;
+                    const int64_t left = rows_total - int64_t(t) * C::T;
+                    const int valid_rows = int(left < C::T ? left : C::T);
 #pragma unroll
                     for (int h = 0; h < G; ++h) {
-                        s[h] = valid ? s[h] * p.scale_log2 : -CUDART_INF_F;
-                        const float mx = warp_max_f32(s[h]);
+                        float mx = -CUDART_INF_F;
+#pragma unroll
+                        for (int hf = 0; hf < C::HALVES; ++hf) {
+                            const bool valid = got && row + 128 * hf < valid_rows;
+                            s[hf][h] = valid ? s[hf][h] * sc : -CUDART_INF_F;
+                            mx = fmaxf(mx, s[hf][h]);
+                        }
+                        mx = warp_max_f32(mx);
                         if (lane == 0) red_max[sb][sw][h] = mx;
                     }
                     // the barrier also agrees on aborting
@@ -589,7 +779,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                     for (int h = 0; h < G; ++h) {
                         const float mt = fmaxf(fmaxf(red_max[sb][0][h], red_max[sb][1][h]),
                                                fmaxf(red_max[sb][2][h], red_max[sb][3][h]));
-                        const bool grow = mt > m[h] + kRescaleThreshold;
+                        const bool grow = mt > m[h] + C::THRESH;
                         const float mn = grow ? mt : m[h];
                         alpha[h] = fast_exp2(m[h] - mn);   // 1 when the max is kept
                         m[h] = mn;
@@ -598,26 +788,53 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                     }
                     // P^T buffer sb is free once PV_{j-2} has completed
                     if (!warp_wait(smem_addr(&p_free[sb]), ((j >> 1) & 1) ^ 1, p, abort_flag)) continue;
-                    const uint32_t pb = sP + sb * kSmall + (row & 7) * 2;   // key `row` of P^T
+                    if constexpr (F8) {
+                        // key `row` (+128) of P^T as four E4M3 terms, rows term * G + h
+                        const uint32_t pb = sP + sb * C::PB + (row & 15);
 #pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        const float pr = fast_exp2(s[h] - m[h]);   // 0 for rows outside the piece
-                        l[h] += pr;
-                        const uint16_t hi = bf16_bits(pr);
-                        const uint16_t lo = bf16_bits(pr - __uint_as_float(uint32_t(hi) << 16));
-                        st_shared_u16(pb + small_off(h, row >> 3), hi);
-                        st_shared_u16(pb + small_off(G + h, row >> 3), lo);
+                        for (int h = 0; h < G; ++h) {
+                            // P' = 2^7 exp2(s - m); 0 off-piece
+                            float r0 = fast_exp2(s[0][h] - m[h] + C::POFF), r1 = fast_exp2(s[1][h] - m[h] + C::POFF);
+                            l[h] += r0 + r1;
+#pragma unroll
+                            for (int term = 0; term < 4; ++term) {
+                                const uint16_t c2 = e4m3x2(r1, r0);
+                                const uint32_t off = small_off(term * G + h, row >> 4);
+                                st_shared_u8(pb + off, c2 & 0xffu);
+                                st_shared_u8(pb + C::PHALF + off, uint32_t(c2) >> 8);
+                                if (term < 3) {
+                                    const float2 v = e4m3x2_value(c2);
+                                    r0 -= v.x;
+                                    r1 -= v.y;
+                                }
+                            }
+                        }
+                    } else {
+                        const uint32_t pb = sP + sb * C::PB + (row & 7) * 2;   // key `row` of P^T
+#pragma unroll
+                        for (int h = 0; h < G; ++h) {
+                            const float pr = fast_exp2(s[0][h] - m[h]);   // 0 for rows outside the piece
+                            l[h] += pr;
+                            const uint16_t hi = bf16_bits(pr);
+                            const uint16_t lo = bf16_bits(pr - __uint_as_float(uint32_t(hi) << 16));
+                            st_shared_u16(pb + small_off(h, row >> 3), hi);
+                            st_shared_u16(pb + small_off(G + h, row >> 3), lo);
+                        }
                     }
-                    if (valid_rows < kT) {
+                    if (valid_rows < C::T) {
                         // Rows past the piece get P = 0; clear their V rows too, so
                         // that whatever the memory there holds adds exactly 0.
                         if (!warp_wait(smem_addr(&full_v[st]), (j / nst) & 1, p, abort_flag)) continue;
-                        if (row >= valid_rows) {
-                            const uint32_t vr = sV + st * kTileBytes + row * 128;
 #pragma unroll
-                            for (int c = 0; c < 8; ++c) {
-                                st_shared_v4(vr + c * 16, make_uint4(0, 0, 0, 0));
-                                st_shared_v4(vr + kSlab + c * 16, make_uint4(0, 0, 0, 0));
+                        for (int hf = 0; hf < C::HALVES; ++hf) {
+                            const int kr = row + 128 * hf;
+                            if (kr >= valid_rows) {
+                                const uint32_t vr = sV + st * kTileBytes + kr * 128;
+#pragma unroll
+                                for (int c = 0; c < 8; ++c) {
+                                    st_shared_v4(vr + c * 16, make_uint4(0, 0, 0, 0));
+                                    if constexpr (!F8) st_shared_v4(vr + kSlab + c * 16, make_uint4(0, 0, 0, 0));
+                                }
                             }
                         }
                     }
@@ -626,15 +843,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                         // rescale O^T (rows = dims) once PV_{j-1} has landed
                         if (!warp_wait(smem_addr(&p_free[(j - 1) & 1]), ((j - 1) >> 1) & 1, p, abort_flag)) continue;
                         tc_fence_after();
-                        uint32_t u[2 * G];
-                        tmem_ldn<2 * G>(tmem_o, u);
+                        uint32_t u[C::PT * G];
+                        tmem_ldn<C::PT * G>(tmem_o, u);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int h = 0; h < G; ++h) {
-                            u[h] = __float_as_uint(__uint_as_float(u[h]) * alpha[h]);
-                            u[G + h] = __float_as_uint(__uint_as_float(u[G + h]) * alpha[h]);
-                        }
-                        tmem_stn<2 * G>(tmem_o, u);
+                        for (int term = 0; term < C::PT; ++term)
+#pragma unroll
+                            for (int h = 0; h < G; ++h)
+                                u[term * G + h] = __float_as_uint(__uint_as_float(u[term * G + h]) * alpha[h]);
+                        tmem_stn<C::PT * G>(tmem_o, u);
                         tmem_wait_st();
                     }
                     tc_fence_before();
@@ -688,19 +905,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc(tmem, C::COLS);
     }
 }
 
-template <int G>
+template <int G, bool F8>
 cudaError_t launch_g(const DecodeParams& p, cudaStream_t s) {
+    using C = Tr<G, F8>;
     DecodeParams q = p;
     q.seg_weight = kSegWeight;
-    const size_t fixed = 4 * size_t(kSmall) + seq_table_bytes(p.B, p.n_kv) + 1024;
+    const size_t fixed = 2 * size_t(C::QB + C::PB) + seq_table_bytes(p.B, p.n_kv) + 1024;
     q.stages = fixed + 3 * 2 * size_t(kTileBytes) <= size_t(227) * 1024 ? 3 : 2;
     const size_t smem = fixed + size_t(q.stages) * 2 * kTileBytes;
     if (smem > size_t(227) * 1024) return cudaErrorInvalidConfiguration;
-    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    cudaError_t e =
+        cudaFuncSetAttribute(decode_tc_kernel<G, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(unsigned(p.num_ctas));
@@ -712,40 +931,52 @@ cudaError_t launch_g(const DecodeParams& p, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<G>, q);
+    e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<G, F8>, q);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
-// 3-D map [heads][rows][128 dims] of bf16, box 64 dims x 128 rows x 1 head, 128-byte swizzle.
-bool make_map3(CUtensorMap* m, const void* base, uint64_t rows, uint64_t heads) {
+// 3-D map over [heads][rows][128 dims] with 128-byte swizzle: bf16 in boxes
+// of 64 dims x 128 rows (two per tile), FP8 codes in boxes of 128 x 256 rows.
+bool make_map3(CUtensorMap* m, const void* base, uint64_t rows, uint64_t heads, bool fp8) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
-    cuuint64_t dims[3] = {uint64_t(kD), rows < 1 ? 1 : rows, heads < 1 ? 1 : heads};
-    cuuint64_t strides[2] = {uint64_t(kD) * 2, (rows < 1 ? 1 : rows) * uint64_t(kD) * 2};
-    cuuint32_t box[3] = {64, uint32_t(kT), 1};
+    const uint64_t eb = fp8 ? 1 : 2;
+    rows = rows < 1 ? 1 : rows;
+    cuuint64_t dims[3] = {uint64_t(kD), rows, heads < 1 ? 1 : heads};
+    cuuint64_t strides[2] = {uint64_t(kD) * eb, rows * uint64_t(kD) * eb};
+    cuuint32_t box[3] = {fp8 ? 128u : 64u, fp8 ? 256u : 128u, 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return enc(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base),
+               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
 
 bool make_decode_maps(DecodeMaps* m, const void* kr, const void* vr, const void* ks, const void* vs, int B, int n_r,
-                      int n_s, int64_t cap, int SW) {
-    return make_map3(&m->kr, kr, uint64_t(cap), uint64_t(B) * n_r) &&
-           make_map3(&m->vr, vr, uint64_t(cap), uint64_t(B) * n_r) &&
-           make_map3(&m->ks, ks, uint64_t(SW), uint64_t(B) * n_s) &&
-           make_map3(&m->vs, vs, uint64_t(SW), uint64_t(B) * n_s);
+                      int n_s, int64_t cap, int SW, bool fp8) {
+    return make_map3(&m->kr, kr, uint64_t(cap), uint64_t(B) * n_r, fp8) &&
+           make_map3(&m->vr, vr, uint64_t(cap), uint64_t(B) * n_r, fp8) &&
+           make_map3(&m->ks, ks, uint64_t(SW), uint64_t(B) * n_s, fp8) &&
+           make_map3(&m->vs, vs, uint64_t(SW), uint64_t(B) * n_s, fp8);
 }
 
 cudaError_t launch_decode_tc(const DecodeParams& p, int group, cudaStream_t s) {
-    switch (group) {
-        case 1: return launch_g<1>(p, s);
-        case 2: return launch_g<2>(p, s);
-        case 4: return launch_g<4>(p, s);
-        case 8: return launch_g<8>(p, s);
+    if (p.fp8) {
+        switch (group) {
+            case 1: return launch_g<1, true>(p, s);
+            case 2: return launch_g<2, true>(p, s);
+            case 4: return launch_g<4, true>(p, s);
+            case 8: return launch_g<8, true>(p, s);
+        }
+    } else {
+        switch (group) {
+            case 1: return launch_g<1, false>(p, s);
+            case 2: return launch_g<2, false>(p, s);
+            case 4: return launch_g<4, false>(p, s);
+            case 8: return launch_g<8, false>(p, s);
+        }
     }
     return cudaErrorInvalidValue;
 }

@@ -41,6 +41,8 @@ struct duo_kv {
     int device = 0;
     int num_sms = 0;
     int decode_ctas = 0;                    // 0 = default persistent wave
+    int fp8 = 0;                            // caches hold E4M3 codes
+    std::vector<float> k_scale, v_scale;    // [L][n_kv] (FP8)
     std::vector<duo::DecodeMaps> maps;      // per layer (head_dim 128 only)
 };
 
@@ -68,12 +70,14 @@ struct DecodeParams {
     int B, n_kv, hq, n_r, n_s, S, W;
     int num_ctas;
     int seg_weight;           // partition weight of a segment start, in 16-token blocks (0 = none)
+    int fp8;                  // caches hold E4M3 codes (tensor-core kernel only)
     int stages;               // tensor-core kernel pipeline depth (set by its launcher)
     float scale_log2;
     unsigned long long timeout_ns;
     int32_t rank[kMaxKvHeads];
     int32_t r_before[kMaxKvHeads + 1];
     uint8_t is_r[kMaxKvHeads];
+    float k_scale[kMaxKvHeads], v_scale[kMaxKvHeads];   // FP8: this layer's scales
 };
 
 struct AppendParams {
@@ -91,8 +95,10 @@ struct AppendParams {
     int32_t* status;
     int64_t cap;
     int B, n_kv, n_r, n_s, S, W, d, n_new_max;
+    int fp8;                      // store E4M3 codes of value / scale
     int32_t rank[kMaxKvHeads];
     uint8_t is_r[kMaxKvHeads];
+    float k_scale[kMaxKvHeads], v_scale[kMaxKvHeads];
 };
 
 struct PrefillLaunch {
@@ -109,6 +115,8 @@ struct PrefillLaunch {
     void* workspace;        // fp16 value copies, prefill_workspace_bytes(...) bytes
     int64_t cap;
     int B, hq, n_kv, C, S, W, n_r, n_s;
+    int fp8;                // cached prefix holds E4M3 codes
+    float k_scale[kMaxKvHeads], v_scale[kMaxKvHeads];
     float scale;
     unsigned long long timeout_ns;
     int32_t rank[kMaxKvHeads];
@@ -122,7 +130,7 @@ size_t decode_workspace_bytes(int slots, int d, int group);
 cudaError_t launch_decode(const DecodeParams& p, int d, int group, cudaStream_t s);
 cudaError_t launch_decode_tc(const DecodeParams& p, int group, cudaStream_t s);   // attention only
 bool make_decode_maps(DecodeMaps* m, const void* kr, const void* vr, const void* ks, const void* vs, int B, int n_r,
-                      int n_s, int64_t cap, int SW);
+                      int n_s, int64_t cap, int SW, bool fp8);
 cudaError_t launch_lse_merge(int parts, int rows, int d, const float* part_out, const float* part_lse, float* out,
                              float* lse, cudaStream_t s);
 cudaError_t launch_blend(int64_t n, int hq, int d, const float* alpha, const float* full, const float* strm,

@@ -133,8 +133,17 @@ __device__ __forceinline__ void tmem_ldn<16>(uint32_t taddr, uint32_t* r) {
         : "r"(taddr));
 }
 
+template <>
+__device__ __forceinline__ void tmem_ldn<32>(uint32_t taddr, uint32_t* r) {
+    tmem_ld32p(taddr, r);
+}
+
 template <int N>
 __device__ __forceinline__ void tmem_stn(uint32_t taddr, const uint32_t* r);
+template <>
+__device__ __forceinline__ void tmem_stn<32>(uint32_t taddr, const uint32_t* r) {
+    tmem_st32(taddr, *reinterpret_cast<const uint32_t(*)[32]>(r));
+}
 template <>
 __device__ __forceinline__ void tmem_stn<2>(uint32_t taddr, const uint32_t* r) {
     asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1,%2};" ::"r"(taddr), "r"(r[0]), "r"(r[1])

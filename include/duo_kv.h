@@ -76,6 +76,12 @@ enum {
     DUO_STATUS_BAD_LENGTH = 8       /* negative length or append count         */
 };
 
+/* Element type of the K/V caches. */
+enum {
+    DUO_KV_BF16 = 0,        /* bf16, as given                                  */
+    DUO_KV_FP8_E4M3 = 1     /* FP8 E4M3 codes with per-(layer, KV head) scales  */
+};
+
 /* Cache shape.  retrieval_mask is a HOST array [num_layers][num_kv_heads],
  * 1 = retrieval head, 0 = streaming head: the binary head mask of the
  * DuoAttention guide, section 3 item 4 ("Binarization"), given per KV head
@@ -84,7 +90,16 @@ enum {
  * duo_kv_alloc and not kept.  capacity = rows reserved per retrieval head
  * per sequence (the maximum length).  Constraints: num_layers, batch,
  * num_q_heads, num_kv_heads >= 1; num_q_heads % num_kv_heads == 0;
- * head_dim in {64, 128}; sink >= 0; window >= 1; capacity >= 1. */
+ * head_dim in {64, 128}; sink >= 0; window >= 1; capacity >= 1.
+ *
+ * kv_dtype = DUO_KV_FP8_E4M3 stores every cached key and value (retrieval
+ * and streaming heads) as one byte, halving the cache (the DuoAttention
+ * guide's "Synergies with Low-Bit Quantization": 8 instead of 16 bits per
+ * element).  The pages fix neither the format nor the scaling; this library
+ * stores code = E4M3(fp32(x) / fp32(scale)) (round to nearest even,
+ * saturating at 448) and reads scale * E4M3(code).  k_scale and v_scale are
+ * HOST arrays [num_layers][num_kv_heads] of finite positive scales (NULL =
+ * all 1.0), copied during duo_kv_alloc.  FP8 needs head_dim 128. */
 typedef struct {
     int32_t num_layers;
     int32_t batch;
@@ -95,15 +110,20 @@ typedef struct {
     int32_t window;
     int64_t capacity;
     const uint8_t* retrieval_mask;
+    int32_t kv_dtype;           /* DUO_KV_BF16 (0) or DUO_KV_FP8_E4M3 (1) */
+    const float* k_scale;       /* FP8 only, see above                     */
+    const float* v_scale;
 } duo_kv_desc;
 
 /* Opaque host-side handle (host memory only). */
 typedef struct duo_kv duo_kv;
 
 /* Device views of one layer's cache (for verification and for callers that
- * manage the cache themselves).  Layouts:
- *   k_retrieval, v_retrieval: [B][n_retrieval][capacity][d]  bf16
- *   k_streaming, v_streaming: [B][n_streaming][S + W][d]     bf16
+ * manage the cache themselves).  Layouts, in elements of the cache's
+ * kv_dtype (bf16 bit patterns, or one E4M3 byte each -- the pointers then
+ * address bytes):
+ *   k_retrieval, v_retrieval: [B][n_retrieval][capacity][d]
+ *   k_streaming, v_streaming: [B][n_streaming][S + W][d]
  *   positions:                [B][S + W] int32, original position of the
  *                             token in each streaming slot, -1 = empty
  *                             (shared by all streaming heads of the layer).
@@ -161,6 +181,7 @@ DUO_API int duo_kv_layer_view_get(const duo_kv* kv, int32_t layer, duo_kv_layer_
  * not fill are reset to -1.  Following the DuoAttention guide's simulation
  * (append_token) and the sliding-window ring of "Attention Variants and
  * Memory Efficiency"; the result equals appending the tokens one at a time.
+ * FP8 caches store each value's code (see duo_kv_desc) instead of its bits.
  * Decode order per layer: append the new token, then duo_decode_attn.
  * Prefill order per layer: duo_prefill_attn on the chunk, then append it. */
 DUO_API int duo_kv_append(duo_kv* kv, int32_t layer, const uint16_t* k_new, const uint16_t* v_new,

@@ -124,3 +124,46 @@ def test_strerror_covers_codes():
     for c in range(0, -7, -1):
         assert L.duo_strerror(c) != "unknown error"
     assert L.duo_strerror(-99) == "unknown error"
+
+
+@pytest.mark.parametrize("cfg", ["mha32k", "gqa128k", "mtok"])
+def test_fp8_cache_bytes_follow_memory_equation_at_one_byte(cfg):
+    """FP8 caches: the same memory equation with one byte per element
+    (the guide's 8 instead of 16 bits), i.e. half the bf16 bytes."""
+    L = _lib()
+    w = W.WORKLOADS[cfg]
+    masks = W.retrieval_masks(w)
+    cap = W.capacity(w)
+    d, keep = L.make_desc(w.layers, w.batch, w.hq, w.n_kv, w.d, w.sink, w.window, cap, masks.tobytes(),
+                          L.DUO_KV_FP8_E4M3)
+    _, cache = L.duo_kv_required_bytes(d)
+    want = w.batch * O.duo_cache_bytes(w.layers, w.n_kv, w.d, cap, w.sink, w.window, masks.sum(1).tolist(),
+                                       elem_bytes=1)
+    assert cache == want
+    d16, keep16 = L.make_desc(w.layers, w.batch, w.hq, w.n_kv, w.d, w.sink, w.window, cap, masks.tobytes())
+    assert 2 * cache == L.duo_kv_required_bytes(d16)[1]
+
+
+def test_fp8_descriptor_checks():
+    L = _lib()
+    n = 2 * 8
+    d, keep = _desc(L)
+    d.kv_dtype = 7
+    with pytest.raises(L.DuoError) as e:
+        L.duo_kv_required_bytes(d)
+    assert e.value.code == L.DUO_ERR_INVALID_ARG
+    d, keep = _desc(L, d=64, hq=8)
+    d.kv_dtype = L.DUO_KV_FP8_E4M3
+    with pytest.raises(L.DuoError) as e:
+        L.duo_kv_required_bytes(d)
+    assert e.value.code == L.DUO_ERR_UNSUPPORTED
+    for bad in (0.0, -1.0, float("nan"), float("inf")):
+        mask = np.zeros((2, 8), np.uint8)
+        d, keep = L.make_desc(2, 3, 32, 8, 128, 64, 256, 1000, mask.tobytes(), L.DUO_KV_FP8_E4M3,
+                              [1.0] * (n - 1) + [bad], None)
+        with pytest.raises(L.DuoError) as e:
+            L.duo_kv_required_bytes(d)
+        assert e.value.code == L.DUO_ERR_INVALID_ARG
+    d, keep = L.make_desc(2, 3, 32, 8, 128, 64, 256, 1000, np.zeros((2, 8), np.uint8).tobytes(),
+                          L.DUO_KV_FP8_E4M3, [0.5] * n, [2.0] * n)
+    assert L.duo_kv_required_bytes(d)[1] > 0
