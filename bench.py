@@ -327,6 +327,67 @@ def run_ours(args, rank, world, local):
     return res, (gw, lens0, mask, first_b)
 
 
+# ---------------------------------------------------------------- FP8 decode
+def run_fp8_decode(local, steps=512, warmup=16):
+    """The same layer-step (append of the new token + decode) on an FP8 E4M3
+    cache of the same workload (scales 1.0: the N(0,1) data sits well inside
+    E4M3's range).  Reports the decode launch against the HBM roofline at
+    one byte per cached element."""
+    from head_wise_kv_b200 import DuoKVCache
+    dev = torch.device("cuda", local)
+    base, gw, lens0 = rank_workload(0, 1)
+    mask = W.retrieval_mask(gw, 0)
+    cap = int(lens0.max()) + base.steps
+    B = base.batch
+    cache = DuoKVCache(1, B, base.hq, base.n_kv, base.d, base.sink, base.window, cap, mask[None], device=dev,
+                       kv_dtype="fp8")
+    fill_rank(cache, gw, lens0, 0, dev)
+    qs, ks, vs = step_inputs(gw, lens0, 0, base.steps)
+    dq = [q.to(dev) for q in qs]
+    dk = [k.to(dev) for k in ks]
+    dv = [v.to(dev) for v in vs]
+    lb = [torch.from_numpy((lens0 + s).astype(np.int32)).to(dev) for s in range(base.steps)]
+    la = [torch.from_numpy((lens0 + s + 1).astype(np.int32)).to(dev) for s in range(base.steps)]
+    out = torch.empty(B, base.hq, base.d, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for i in range(warmup):
+        s = i % base.steps
+        cache.append(0, dk[s], dv[s], lb[s])
+        cache.decode(0, dq[s], la[s], base.scale, out=out)
+    torch.cuda.synchronize()
+    assert cache.status() == 0, "device status set during the FP8 warm-up"
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        s = i % base.steps
+        ev[i][0].record(stream)
+        cache.append(0, dk[s], dv[s], lb[s])
+        ev[i][1].record(stream)
+        cache.decode(0, dq[s], la[s], base.scale, out=out)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    assert cache.status() == 0, "device status set during the FP8 timed region"
+    dec_ms = sum(ev[i][1].elapsed_time(ev[i][2]) for i in range(steps)) / steps
+    step_ms = ev[0][0].elapsed_time(ev[-1][2]) / steps
+    fp8_bytes = sum(kv_bytes(lens0 + (i % base.steps) + 1, mask, base.d, base.sink, base.window, cap)
+                    for i in range(steps)) / steps / 2
+    hbm_peak, peak_kind = peaks()
+    achieved = fp8_bytes / (dec_ms * 1e-3) / 1e9
+    cache.close()
+    return {
+        "workload": "gqa128k with an FP8 E4M3 cache (retrieval and streaming heads), append + decode per "
+                    "layer-step, 32 distinct steps cycled",
+        "steps": steps, "warmup": warmup,
+        "layer_step_us": round(step_ms * 1e3, 3),
+        "decode_us": round(dec_ms * 1e3, 3),
+        "kv_bytes_per_layer_step": int(fp8_bytes),
+        "roofline": {"bound": "hbm", "kernel": "decode_tc_kernel FP8 (kind::f8f6f4)", "achieved": round(achieved, 1),
+                     "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": round(achieved / hbm_peak, 4), "traffic": None},
+        "gpu_launches": 2 * steps,
+    }
+
+
 # ---------------------------------------------------------------- chunked prefill
 def prefill_pairs(prompt, chunk, n_r_q, n_s_q, S, Wn):
     """Mask-valid (query, key) pairs of a chunked prefill: retrieval query heads
@@ -517,8 +578,9 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the chunked-prefill measurement")
-    ap.add_argument("--only", choices=["decode", "prefill"], default=None,
+    ap.add_argument("--only", choices=["decode", "prefill", "fp8"], default=None,
                     help="measure one path only (profiling runs)")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the FP8-cache decode measurement")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
     rank, world, local = dist_init()
@@ -527,10 +589,15 @@ def main(argv=None):
             res = run_reference(args, rank, world)
         elif args.only == "prefill":
             res = {"metric": "chunked prefill attention", "prefill": run_prefill(local)} if rank == 0 else None
+        elif args.only == "fp8":
+            res = ({"metric": "FP8-cache decode", "decode_fp8": run_fp8_decode(local, args.steps, args.warmup)}
+                   if rank == 0 else None)
         else:
             res, ctx = run_ours(args, rank, world, local)
             if world == 1 and not args.no_prefill and args.only != "decode":
                 res["prefill"] = run_prefill(local)
+            if world == 1 and not args.no_fp8 and args.only != "decode":
+                res["decode_fp8"] = run_fp8_decode(local)
             if rank == 0 and world == 1 and not args.no_cpu_baseline:
                 res["cpu_baseline"] = cpu_baseline(ctx)
         if rank == 0 and res is not None:

@@ -361,7 +361,8 @@ static size_t prefill_ws(const duo_kv* kv, int32_t chunk) {
         n_s = std::max(n_s, L.n_s);
     }
     const duo_kv_desc& d = kv->desc;
-    return duo::prefill_workspace_bytes(d.batch, d.num_kv_heads, n_r, n_s, d.capacity, d.sink, d.window, chunk);
+    return duo::prefill_workspace_bytes(d.batch, d.num_kv_heads, n_r, n_s, d.capacity, d.sink, d.window, chunk,
+                                        kv->fp8 != 0);
 }
 
 int duo_prefill_workspace_bytes(const duo_kv* kv, int32_t chunk, size_t* bytes) {
@@ -378,8 +379,14 @@ int duo_prefill_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const uint16_
         return DUO_ERR_INVALID_ARG;
     if (!(scale > 0.f) || scale != scale) return DUO_ERR_INVALID_ARG;
     if (kv->desc.head_dim != 128) return DUO_ERR_UNSUPPORTED;
-    if (kv->fp8) return DUO_ERR_UNSUPPORTED;   // FP8 prefix not read by the prefill kernel yet
     const duo_kv_desc& d = kv->desc;
+    if (kv->fp8) {
+        // the prefix's probabilities are multiplied by the value scale in fp16
+        for (int g = 0; g < d.num_kv_heads; ++g) {
+            const float vs = kv->v_scale[size_t(layer) * d.num_kv_heads + g];
+            if (!(vs >= 1.0f / 256.0f && vs <= 128.0f)) return DUO_ERR_UNSUPPORTED;
+        }
+    }
     if (duo::prefill_smem_bytes(d.sink, d.window) > 227 * 1024) return DUO_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k_chunk) || !aligned16(v_chunk) || !aligned16(out) ||
         (reinterpret_cast<uintptr_t>(prefix_len) & 3))

@@ -85,6 +85,11 @@ constexpr float kRescaleThreshold = 8.0f;     // log2 units: probabilities stay 
 #define DUO_DECODE_SEG_WEIGHT 32
 #endif
 constexpr int kSegWeight = DUO_DECODE_SEG_WEIGHT;
+// FP8 streams twice the keys per byte, so a piece start costs twice the blocks.
+#ifndef DUO_DECODE_SEG_WEIGHT_FP8
+#define DUO_DECODE_SEG_WEIGHT_FP8 64
+#endif
+constexpr int kSegWeightF8 = DUO_DECODE_SEG_WEIGHT_FP8;
 
 // Shapes of the two element types.
 //   bf16: 128-key tiles; S^T one column per head (q as is); P as hi + lo
@@ -107,11 +112,14 @@ struct Tr {
     static constexpr uint32_t QB = 4096;                           // bytes of one q operand
     static constexpr uint32_t PB = F8 ? N * 256 : 4096;            // bytes of one P^T operand
     static constexpr uint32_t PHALF = F8 ? N * 128 : 2048;         // P^T bytes per K-half (128 / 64 keys)
-    // FP8: P enters the MMA as P' = 2^7 P with the running max kept within
-    // 2^1 of the tile maxima, so P' <= 256 < 448 and the E4M3 grid floor
-    // (2^-10 after four terms) sits 2^-17 below the largest probability;
-    // bf16 terms have no such floor (threshold 2^8, no offset).
-    static constexpr float THRESH = F8 ? 1.0f : kRescaleThreshold;    // log2 units
+    // FP8: P enters the MMA as P' = 2^7 P.  When a tile's max exceeds the
+    // running max m by more than 1.75, m moves to that max + 2 (headroom, so
+    // that the slowly growing max of a long sequence rarely forces another
+    // rescale); hence P' <= 2^8.75 < 448 and the E4M3 grid floor (2^-10
+    // after four terms) stays >= 2^-15 below the largest P'.  bf16 terms have
+    // no such floor: threshold 2^8, no offset, no headroom.
+    static constexpr float THRESH = F8 ? 1.75f : kRescaleThreshold;   // log2 units
+    static constexpr float HEAD = F8 ? 2.0f : 0.0f;
     static constexpr float POFF = F8 ? 7.0f : 0.0f;                    // log2 of the P offset
     static constexpr uint32_t IQK = idesc_f16(128, N, !F8, false, false);   // A = K (K-major), B = q
     static constexpr uint32_t IPV = idesc_f16(kD, N, !F8, true, false);     // A = V^T (MN-major), B = P^T
@@ -780,7 +788,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                         const float mt = fmaxf(fmaxf(red_max[sb][0][h], red_max[sb][1][h]),
                                                fmaxf(red_max[sb][2][h], red_max[sb][3][h]));
                         const bool grow = mt > m[h] + C::THRESH;
-                        const float mn = grow ? mt : m[h];
+                        const float mn = grow ? mt + C::HEAD : m[h];
                         alpha[h] = fast_exp2(m[h] - mn);   // 1 when the max is kept
                         m[h] = mn;
                         l[h] *= alpha[h];
@@ -913,7 +921,7 @@ template <int G, bool F8>
 cudaError_t launch_g(const DecodeParams& p, cudaStream_t s) {
     using C = Tr<G, F8>;
     DecodeParams q = p;
-    q.seg_weight = kSegWeight;
+    q.seg_weight = F8 ? kSegWeightF8 : kSegWeight;
     const size_t fixed = 2 * size_t(C::QB + C::PB) + seq_table_bytes(p.B, p.n_kv) + 1024;
     q.stages = fixed + 3 * 2 * size_t(kTileBytes) <= size_t(227) * 1024 ? 3 : 2;
     const size_t smem = fixed + size_t(q.stages) * 2 * kTileBytes;

@@ -112,7 +112,7 @@ struct PrefillLaunch {
     const int32_t* prefix;
     float* out;
     int32_t* status;
-    void* workspace;        // fp16 value copies, prefill_workspace_bytes(...) bytes
+    void* workspace;        // fp16 value copies (and bf16 key copies of an FP8 prefix), prefill_workspace_bytes(...) bytes
     int64_t cap;
     int B, hq, n_kv, C, S, W, n_r, n_s;
     int fp8;                // cached prefix holds E4M3 codes
@@ -136,7 +136,7 @@ cudaError_t launch_lse_merge(int parts, int rows, int d, const float* part_out, 
 cudaError_t launch_blend(int64_t n, int hq, int d, const float* alpha, const float* full, const float* strm,
                          float* out, cudaStream_t s);
 size_t prefill_smem_bytes(int S, int W);
-size_t prefill_workspace_bytes(int B, int n_kv, int n_r, int n_s, int64_t cap, int S, int W, int C);
+size_t prefill_workspace_bytes(int B, int n_kv, int n_r, int n_s, int64_t cap, int S, int W, int C, bool fp8);
 int launch_prefill(const PrefillLaunch& a, cudaStream_t s);   // returns a DUO_* code
 
 // ----------------------------------------------------------------- device helpers

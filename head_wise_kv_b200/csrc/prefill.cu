@@ -36,6 +36,7 @@
 // DUO_STATUS_WAIT_TIMEOUT, stops, waits (bounded) for its own copies and
 // MMAs in flight, frees TMEM and exits.
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <math_constants.h>
@@ -69,6 +70,7 @@ constexpr uint32_t kIdescPV = idesc_f16(kBM, kHD, false, false, true);
 
 struct PrefillParams {
     CUtensorMap tm_q, tm_kc, tm_kr, tm_ks;      // bf16: queries, chunk / retrieval / ring keys
+    CUtensorMap tm_kr16, tm_ks16;               // FP8 caches: bf16 copies of the cached keys' codes
     CUtensorMap tm_vc, tm_vr, tm_vs;            // fp16 copies of the values (workspace)
     const int32_t* prefix;
     float* out;
@@ -77,8 +79,10 @@ struct PrefillParams {
     int B, hq, n_kv, G, C, n_qt, S, W, n_r, n_s, LR, LS;
     float scale_log2;
     unsigned long long timeout_ns;
+    int fp8;                                    // cached keys / values are E4M3 codes
     int32_t rank[kMaxKvHeads];
     uint8_t is_r[kMaxKvHeads];
+    float k_scale[kMaxKvHeads], v_scale[kMaxKvHeads];
 };
 
 struct ConvertParams {
@@ -88,6 +92,11 @@ struct ConvertParams {
     uint16_t* v16r;         // fp16 copies: [B][n_r][LR][d], [B][n_s][LS][d], [B][n_kv][C][d]
     uint16_t* v16s;
     uint16_t* v16c;
+    const uint8_t* kr8;     // FP8 caches: key codes, and bf16 copies of them [B][n_r][LR][d], [B][n_s][LS][d]
+    const uint8_t* ks8;
+    uint16_t* k16r;
+    uint16_t* k16s;
+    int fp8;
     const int32_t* prefix;
     int64_t cap;
     int B, n_kv, n_r, n_s, S, W, C, LR, LS;
@@ -242,17 +251,46 @@ __device__ __forceinline__ bool softmax_barrier_any(bool flag) {
     return out != 0;
 }
 
-// ------------------------------------------------------------------ V -> fp16
-// One thread per 16-byte piece (8 values).  blockIdx.y = b * n_kv + g;
-// blockIdx.z = 0: the head's cached rows, 1: its chunk rows.  Rows that hold
-// no key (past the prefix or the filled ring slots) up to the end of the
-// last tile the attention reads are written as zeros, so masked columns
-// always meet finite values.
+// ------------------------------------------------------------------ V -> fp16 (and FP8 codes -> 16 bits)
+// Eight E4M3 codes -> their values as fp16 (exact: every E4M3 value is an
+// fp16 value), or as bf16 (also exact).
+__device__ __forceinline__ uint4 e4m3x8_to_f16(uint2 c) {
+    uint32_t h[4];
+    const uint16_t s[4] = {uint16_t(c.x & 0xffff), uint16_t(c.x >> 16), uint16_t(c.y & 0xffff), uint16_t(c.y >> 16)};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h[i]) : "h"(s[i]));
+    return make_uint4(h[0], h[1], h[2], h[3]);
+}
+
+__device__ __forceinline__ uint4 e4m3x8_to_bf16(uint2 c) {
+    const uint4 h = e4m3x8_to_f16(c);
+    const uint32_t w[4] = {h.x, h.y, h.z, h.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __half2 hh = *reinterpret_cast<const __half2*>(&w[i]);
+        const float2 f = __half22float2(hh);
+        const __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);
+        o[i] = *reinterpret_cast<const uint32_t*>(&b);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// One thread per 8 values (16 bytes of output).  blockIdx.y = b * n_kv + g;
+// blockIdx.z = 0: the head's cached value rows, 1: its chunk's value rows,
+// 2 (FP8 caches only): its cached key rows.  Values become fp16; cached
+// FP8 codes become their (unscaled) values, fp16 for V and bf16 for K -- the
+// scales are applied in the attention kernel.  Rows that hold no key (past
+// the prefix or the filled ring slots) up to the end of the last tile the
+// attention reads are written as zeros, so masked columns always meet
+// finite values.
 __global__ void __launch_bounds__(256) convert_v_kernel(const __grid_constant__ ConvertParams c) {
     const int bg = blockIdx.y;
     const int b = bg / c.n_kv, g = bg % c.n_kv;
     const int P = max(c.prefix[b], 0);
-    const uint16_t* src;
+    const bool keys = blockIdx.z == 2;
+    const uint16_t* src = nullptr;
+    const uint8_t* src8 = nullptr;
     uint16_t* dst;
     int64_t n_conv, n_rows;
     if (blockIdx.z == 1) {
@@ -261,14 +299,20 @@ __global__ void __launch_bounds__(256) convert_v_kernel(const __grid_constant__ 
         n_conv = n_rows = c.C;
     } else if (c.is_r[g]) {
         const size_t r = size_t(b) * c.n_r + c.rank[g];
-        src = c.vr + r * size_t(c.cap) * kHD;
-        dst = c.v16r + r * size_t(c.LR) * kHD;
+        if (c.fp8)
+            src8 = (keys ? c.kr8 : reinterpret_cast<const uint8_t*>(c.vr)) + r * size_t(c.cap) * kHD;
+        else
+            src = c.vr + r * size_t(c.cap) * kHD;
+        dst = (keys ? c.k16r : c.v16r) + r * size_t(c.LR) * kHD;
         n_conv = min(int64_t(P), c.cap);
         n_rows = (n_conv + kBN - 1) / kBN * kBN;          // tail of the last prefix tile
     } else {
         const size_t r = size_t(b) * c.n_s + c.rank[g];
-        src = c.vs + r * size_t(c.S + c.W) * kHD;
-        dst = c.v16s + r * size_t(c.LS) * kHD;
+        if (c.fp8)
+            src8 = (keys ? c.ks8 : reinterpret_cast<const uint8_t*>(c.vs)) + r * size_t(c.S + c.W) * kHD;
+        else
+            src = c.vs + r * size_t(c.S + c.W) * kHD;
+        dst = (keys ? c.k16s : c.v16s) + r * size_t(c.LS) * kHD;
         n_conv = min(P, c.S + c.W);                         // filled slots
         n_rows = c.LS;
     }
@@ -278,18 +322,24 @@ __global__ void __launch_bounds__(256) convert_v_kernel(const __grid_constant__ 
         const int64_t row = x / (kHD / 8);
         uint4 v = make_uint4(0, 0, 0, 0);
         if (row < n_conv) {
-            const uint4 w = *reinterpret_cast<const uint4*>(src + x * 8);
-            const float2 a = bf2_to_f2(w.x), bb = bf2_to_f2(w.y), cc = bf2_to_f2(w.z), dd = bf2_to_f2(w.w);
-            v.x = pack_half2(a.x, a.y);
-            v.y = pack_half2(bb.x, bb.y);
-            v.z = pack_half2(cc.x, cc.y);
-            v.w = pack_half2(dd.x, dd.y);
+            if (src8) {
+                const uint2 cc = *reinterpret_cast<const uint2*>(src8 + x * 8);
+                v = keys ? e4m3x8_to_bf16(cc) : e4m3x8_to_f16(cc);
+            } else {
+                const uint4 w = *reinterpret_cast<const uint4*>(src + x * 8);
+                const float2 a = bf2_to_f2(w.x), bb = bf2_to_f2(w.y), cc = bf2_to_f2(w.z), dd = bf2_to_f2(w.w);
+                v.x = pack_half2(a.x, a.y);
+                v.y = pack_half2(bb.x, bb.y);
+                v.z = pack_half2(cc.x, cc.y);
+                v.w = pack_half2(dd.x, dd.y);
+            }
         }
         *reinterpret_cast<uint4*>(dst + x * 8) = v;
     }
 }
 
 // ------------------------------------------------------------------ attention
+template <bool F8>
 __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_constant__ PrefillParams p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -369,15 +419,17 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 const KeyTile kt = plan.get(j);
                 const CUtensorMap* map;
                 int row;
+                // FP8 caches: cached keys come from their bf16 copies (rows LR / LS)
+                const bool copy = !is_k || p.fp8;
                 if (kt.src == kSrcCache) {
-                    map = is_k ? &p.tm_kr : &p.tm_vr;
-                    row = int((int64_t(b) * p.n_r + kv_rank) * (is_k ? p.cap : int64_t(p.LR)) + kt.row0);
+                    map = is_k ? (p.fp8 ? &p.tm_kr16 : &p.tm_kr) : &p.tm_vr;
+                    row = int((int64_t(b) * p.n_r + kv_rank) * (copy ? int64_t(p.LR) : p.cap) + kt.row0);
                 } else if (kt.src == kSrcChunk) {
                     map = is_k ? &p.tm_kc : &p.tm_vc;
                     row = (b * p.n_kv + g) * p.C + kt.row0;
                 } else {
-                    map = is_k ? &p.tm_ks : &p.tm_vs;
-                    row = (b * p.n_s + kv_rank) * (is_k ? p.S + p.W : p.LS) + (kt.src == kSrcWindow ? p.S : 0) +
+                    map = is_k ? (p.fp8 ? &p.tm_ks16 : &p.tm_ks) : &p.tm_vs;
+                    row = (b * p.n_s + kv_rank) * (copy ? p.LS : p.S + p.W) + (kt.src == kSrcWindow ? p.S : 0) +
                           kt.row0;
                 }
                 const uint32_t bar = smem_addr(&full[st]);
@@ -448,6 +500,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         const int cb = hf * 64;                  // first key column (and O dim) of this half
         const uint32_t lane_off = uint32_t(wq * 32) << 16;
         float m = kNegBig, l = 0.f;
+        // FP8 caches: a cached key's tile holds codes, so its scores take the
+        // key scale and its probabilities the value scale (the chunk's own
+        // keys and values are exact)
+        const float ksc = F8 ? p.k_scale[g] : 1.f;
+        const float lvs = F8 ? __log2f(p.v_scale[g]) : 0.f, ivs = F8 ? 1.f / p.v_scale[g] : 1.f;
         bool ok = true;
         for (int j = 0; j < plan.n; ++j) {
             const int st = j & 1;
@@ -512,15 +569,19 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             if (softmax_barrier_any(!got || *abort_flag)) { ok = false; break; }
             mx = fmaxf(red_max[st][0][r], red_max[st][1][r]);
 
-            const float mt = mx * p.scale_log2;          // scale > 0 keeps the order
+            const bool cached = F8 && j < plan.n_a + plan.n_w;   // tiles of the cache come first
+            const float fs = cached ? p.scale_log2 * ksc : p.scale_log2;   // score factor of this tile
+            const float mt = mx * fs;                    // factor > 0 keeps the order
             const bool grow = mt > m + kRescaleThreshold;
             const float m_new = grow ? mt : m;
             const float alpha = fast_exp2(m - m_new);   // 1 when the max is kept
             float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                              make_float2(0.f, 0.f)};
             uint32_t ph[32];   // probabilities as packed fp16 pairs
-            const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
-            const float2 nm2 = make_float2(-m_new, -m_new);
+            const float2 sc2 = make_float2(fs, fs);
+            // cached tiles of an FP8 cache: P times the value scale, via the exponent
+            const float off = cached ? lvs - m_new : -m_new;
+            const float2 nm2 = make_float2(off, off);
 #pragma unroll
             for (int c = 0; c < 64; c += 2) {
                 const float2 x = ffma2(make_float2(s[c], s[c + 1]), sc2, nm2);
@@ -530,7 +591,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             }
             const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
             const float2 at = fadd2(a01, a23);
-            l = l * alpha + (at.x + at.y);
+            l = l * alpha + (at.x + at.y) * (cached ? ivs : 1.f);
             m = m_new;
             // P_j overwrites P_{j-1} in TMEM, and a rescale touches O: both
             // need PV_{j-1} to have completed.
@@ -618,10 +679,10 @@ size_t prefill_smem_bytes(int S, int W) {
     return (1 + kKStages + kVStages) * size_t(kTile) + 1024;
 }
 
-size_t prefill_workspace_bytes(int B, int n_kv, int n_r, int n_s, int64_t cap, int S, int W, int C) {
+size_t prefill_workspace_bytes(int B, int n_kv, int n_r, int n_s, int64_t cap, int S, int W, int C, bool fp8) {
     const size_t row = size_t(kHD) * 2;
-    return align256(size_t(B) * n_r * rows_r(cap) * row) + align256(size_t(B) * n_s * rows_s(S, W) * row) +
-           align256(size_t(B) * n_kv * C * row);
+    const size_t cached = align256(size_t(B) * n_r * rows_r(cap) * row) + align256(size_t(B) * n_s * rows_s(S, W) * row);
+    return cached + align256(size_t(B) * n_kv * C * row) + (fp8 ? cached : 0);   // V copies, chunk V, FP8 key copies
 }
 
 int launch_prefill(const PrefillLaunch& a, cudaStream_t s) {
@@ -632,6 +693,10 @@ int launch_prefill(const PrefillLaunch& a, cudaStream_t s) {
     uint16_t* v16s = reinterpret_cast<uint16_t*>(ws + align256(size_t(a.B) * a.n_r * LR * row));
     uint16_t* v16c = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(v16s) +
                                                  align256(size_t(a.B) * a.n_s * LS * row));
+    uint16_t* k16r = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(v16c) +
+                                                 align256(size_t(a.B) * a.n_kv * a.C * row));
+    uint16_t* k16s = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(k16r) +
+                                                 align256(size_t(a.B) * a.n_r * LR * row));
 
     PrefillParams p;
     memset(&p, 0, sizeof p);
@@ -639,8 +704,10 @@ int launch_prefill(const PrefillLaunch& a, cudaStream_t s) {
     const CUtensorMapDataType BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, F16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     if (!make_map(&p.tm_q, a.q, uint64_t(a.B) * a.hq * a.C, BF) ||
         !make_map(&p.tm_kc, a.k_chunk, uint64_t(a.B) * a.n_kv * a.C, BF) ||
-        !make_map(&p.tm_kr, a.kr, uint64_t(a.B) * a.n_r * a.cap, BF) ||
-        !make_map(&p.tm_ks, a.ks, uint64_t(a.B) * a.n_s * SW, BF) ||
+        (!a.fp8 && !make_map(&p.tm_kr, a.kr, uint64_t(a.B) * a.n_r * a.cap, BF)) ||
+        (!a.fp8 && !make_map(&p.tm_ks, a.ks, uint64_t(a.B) * a.n_s * SW, BF)) ||
+        (a.fp8 && !make_map(&p.tm_kr16, k16r, uint64_t(a.B) * a.n_r * LR, BF)) ||
+        (a.fp8 && !make_map(&p.tm_ks16, k16s, uint64_t(a.B) * a.n_s * LS, BF)) ||
         !make_map(&p.tm_vc, v16c, uint64_t(a.B) * a.n_kv * a.C, F16) ||
         !make_map(&p.tm_vr, v16r, uint64_t(a.B) * a.n_r * LR, F16) ||
         !make_map(&p.tm_vs, v16s, uint64_t(a.B) * a.n_s * LS, F16))
@@ -656,6 +723,9 @@ int launch_prefill(const PrefillLaunch& a, cudaStream_t s) {
     p.timeout_ns = a.timeout_ns;
     memcpy(p.rank, a.rank, sizeof p.rank);
     memcpy(p.is_r, a.is_r, sizeof p.is_r);
+    p.fp8 = a.fp8;
+    memcpy(p.k_scale, a.k_scale, sizeof p.k_scale);
+    memcpy(p.v_scale, a.v_scale, sizeof p.v_scale);
 
     ConvertParams c;
     memset(&c, 0, sizeof c);
@@ -669,16 +739,29 @@ int launch_prefill(const PrefillLaunch& a, cudaStream_t s) {
     c.LR = LR; c.LS = LS;
     memcpy(c.rank, a.rank, sizeof c.rank);
     memcpy(c.is_r, a.is_r, sizeof c.is_r);
+    c.fp8 = a.fp8;
+    c.kr8 = static_cast<const uint8_t*>(a.kr);
+    c.ks8 = static_cast<const uint8_t*>(a.ks);
+    c.k16r = k16r;
+    c.k16s = k16s;
     if (int64_t(a.B) * a.n_kv > 65535) return DUO_ERR_UNSUPPORTED;
-    convert_v_kernel<<<dim3(64, unsigned(a.B * a.n_kv), 2), 256, 0, s>>>(c);
+    convert_v_kernel<<<dim3(64, unsigned(a.B * a.n_kv), a.fp8 ? 3 : 2), 256, 0, s>>>(c);
     if (cudaGetLastError() != cudaSuccess) return DUO_ERR_CUDA;
 
     const size_t smem = prefill_smem_bytes(a.S, a.W);
-    cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (e != cudaSuccess) return DUO_ERR_CUDA;
     const int64_t grid = int64_t(p.n_qt) * a.B * a.hq;
     if (grid > 0x7fffffff) return DUO_ERR_UNSUPPORTED;
-    prefill_kernel<<<unsigned(grid), kThreads, smem, s>>>(p);
+    if (a.fp8) {
+        if (cudaFuncSetAttribute(prefill_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+            cudaSuccess)
+            return DUO_ERR_CUDA;
+        prefill_kernel<true><<<unsigned(grid), kThreads, smem, s>>>(p);
+    } else {
+        if (cudaFuncSetAttribute(prefill_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+            cudaSuccess)
+            return DUO_ERR_CUDA;
+        prefill_kernel<false><<<unsigned(grid), kThreads, smem, s>>>(p);
+    }
     return cudaGetLastError() == cudaSuccess ? DUO_OK : DUO_ERR_CUDA;
 }
 

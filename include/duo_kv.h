@@ -306,9 +306,14 @@ DUO_API int duo_prefill_workspace_bytes(const duo_kv* kv, int32_t chunk, size_t*
  * and from k_chunk).  The DuoAttention guide's "Hardware-Fused Prefill":
  * dense causal attention for retrieval heads, block-sparse sink + local
  * attention for streaming heads.  Products of probabilities and values run
- * in fp16 (fp32 accumulation), so |v| must stay below 65504.  Requirements:
- * head_dim 128 (else UNSUPPORTED); chunk >= 1; prefix_len[b] must equal the
- * tokens appended so far (the ring state is derived from it). */
+ * in fp16 (fp32 accumulation), so |v| must stay below 65504.  FP8 caches:
+ * the cached prefix is read dequantised (codes times the scales), the
+ * chunk's own keys and values exactly as given; the value scales of the
+ * layer must lie in [2^-8, 2^7] (else UNSUPPORTED: probabilities are scaled
+ * by them in fp16), and the workspace also holds bf16 copies of the cached
+ * keys' codes.  Requirements: head_dim 128 (else UNSUPPORTED); chunk >= 1;
+ * prefix_len[b] must equal the tokens appended so far (the ring state is
+ * derived from it). */
 DUO_API int duo_prefill_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const uint16_t* k_chunk,
                      const uint16_t* v_chunk, const int32_t* prefix_len, int32_t chunk,
                      float scale, float* out, void* workspace, size_t workspace_bytes,

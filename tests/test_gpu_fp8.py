@@ -7,7 +7,9 @@
   GQA group size, ragged lengths that cross the 256-key tiles, any split of
   the keys over CTAs, saturating scales and extreme query magnitudes, and the
   full 128K GQA workload (sampled heads) at the launch configuration the
-  benchmark uses.
+  benchmark uses;
+* chunked prefill attends to the cached prefix dequantised and to the
+  chunk's own keys and values as given.
 """
 import numpy as np
 import pytest
@@ -170,4 +172,67 @@ def test_fp8_gqa128k_config_sampled():
     got, ref = _decode_step(cache, w, hist, lens0, ks, vs, pairs=pairs)
     assert cache.status() == 0
     assert_close(got, ref, "fp8 gqa128k sampled")
+    cache.close()
+
+
+# ------------------------------------------------------------------ prefill on an FP8 cache
+def _chunk(w, prefix, C):
+    q = torch.empty(w.batch, w.hq, C, w.d, dtype=torch.bfloat16)
+    k = torch.empty(w.batch, w.n_kv, C, w.d, dtype=torch.bfloat16)
+    v = torch.empty_like(k)
+    for b in range(w.batch):
+        P = int(prefix[b])
+        for h in range(w.hq):
+            q[b, h] = W.tokens(w, 0, b, h, W.TENSOR_Q, P, P + C)
+        for g in range(w.n_kv):
+            k[b, g] = W.tokens(w, 0, b, g, W.TENSOR_K, P, P + C)
+            v[b, g] = W.tokens(w, 0, b, g, W.TENSOR_V, P, P + C)
+    return q, k, v
+
+
+@pytest.mark.parametrize("chunks,S,Wn", [([300, 700, 129], 16, 64), ([256, 384], 64, 1024)])
+def test_fp8_prefill_matches_oracle(chunks, S, Wn):
+    """Chunked prefill on an FP8 cache: each chunk attends to the cached
+    prefix dequantised and to its own keys / values as given (they are
+    appended, hence quantised, only afterwards)."""
+    w = W.scaled(W.WORKLOADS["gqa128k"], batch=2, layers=1, t0_range=None, t0=0, sink=S, window=Wn)
+    ks, vs = _scales(w, 51)
+    dev = _dev()
+    cache = _cache(w, sum(chunks), ks, vs)
+    hist = History(w)
+    dq = DequantHistory(hist, ks, vs)
+    mask = W.retrieval_mask(w, 0)
+    prefix = np.zeros(w.batch, dtype=np.int64)
+    for C in chunks:
+        q, k, v = _chunk(w, prefix, C)
+        pre = torch.from_numpy(prefix.astype(np.int32)).to(dev)
+        out = cache.prefill(0, q.to(dev), k.to(dev), v.to(dev), pre, w.scale)
+        cache.append(0, k.to(dev), v.to(dev), pre)
+
+        def hist_of(kind):
+            def f(b, g):
+                P = int(prefix[b])
+                cached = dq.get(b, g, kind, P) if P else np.zeros((0, w.d))
+                own = hist.kv(0, b, g, kind, P + C)[P:].double().numpy()
+                return np.concatenate([cached, own])
+            return f
+        ref = O.prefill_attention(q.double().numpy(), hist_of(W.TENSOR_K), hist_of(W.TENSOR_V), prefix, mask,
+                                  w.sink, w.window, w.scale)
+        assert_close(out.cpu().double().numpy(), ref, f"fp8 prefill chunk {C} after {prefix.tolist()}")
+        prefix = prefix + C
+    assert cache.status() == 0
+    cache.close()
+
+
+def test_fp8_prefill_rejects_value_scales_out_of_range():
+    from head_wise_kv_b200 import _lib as L
+    w = W.scaled(W.WORKLOADS["gqa128k"], batch=1, layers=1, t0_range=None, t0=0, sink=16, window=64)
+    ks, vs = _scales(w, 52)
+    vs[0, 0] = 1000.0
+    cache = _cache(w, 256, ks, vs)
+    q, k, v = _chunk(w, np.zeros(1, np.int64), 128)
+    dev = _dev()
+    with pytest.raises(L.DuoError) as e:
+        cache.prefill(0, q.to(dev), k.to(dev), v.to(dev), torch.zeros(1, dtype=torch.int32, device=dev), w.scale)
+    assert e.value.code == L.DUO_ERR_UNSUPPORTED
     cache.close()
