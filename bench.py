@@ -35,6 +35,9 @@ FALLBACK_HBM_GBS = 6650.0
 # from the ncu capture summarised in profiles/decode_tc_kernel_gqa128k.md.  Must be
 # reset to None whenever the decode kernel changes.
 DECODE_TRAFFIC_BYTES = 1126346000 + 3740672
+# The same for decode_tc_kernel<4, FP8> on the FP8 cache of this workload
+# (profiles/decode_tc_kernel_fp8_gqa128k.md); None once that kernel changes.
+DECODE_FP8_TRAFFIC_BYTES = 566199040 + 3438592
 
 
 # ---------------------------------------------------------------- helpers
@@ -383,7 +386,8 @@ def run_fp8_decode(local, steps=512, warmup=16):
         "kv_bytes_per_layer_step": int(fp8_bytes),
         "roofline": {"bound": "hbm", "kernel": "decode_tc_kernel FP8 (kind::f8f6f4)", "achieved": round(achieved, 1),
                      "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": round(achieved / hbm_peak, 4), "traffic": None},
+                     "frac": round(achieved / hbm_peak, 4), "traffic": DECODE_FP8_TRAFFIC_BYTES,
+                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch"},
         "gpu_launches": 2 * steps,
     }
 
