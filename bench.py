@@ -331,19 +331,25 @@ def run_ours(args, rank, world, local):
 
 
 # ---------------------------------------------------------------- FP8 decode
-def run_fp8_decode(local, steps=512, warmup=16):
-    """The same layer-step (append of the new token + decode) on an FP8 E4M3
-    cache of the same workload (scales 1.0: the N(0,1) data sits well inside
-    E4M3's range).  Reports the decode launch against the HBM roofline at
-    one byte per cached element."""
+def run_variant_decode(local, kv_dtype="fp8", paged=False, steps=512, warmup=16):
+    """The same layer-step (append of the new token + decode) on another
+    cache of the same workload: FP8 E4M3 (scales 1.0: the N(0,1) data sits
+    well inside E4M3's range; roofline at one byte per cached element), or a
+    paged cache (256-token pages handed out in a shuffled order)."""
     from head_wise_kv_b200 import DuoKVCache
     dev = torch.device("cuda", local)
     base, gw, lens0 = rank_workload(0, 1)
     mask = W.retrieval_mask(gw, 0)
     cap = int(lens0.max()) + base.steps
     B = base.batch
+    page = 256
+    per_seq = (cap + page - 1) // page
     cache = DuoKVCache(1, B, base.hq, base.n_kv, base.d, base.sink, base.window, cap, mask[None], device=dev,
-                       kv_dtype="fp8")
+                       kv_dtype=kv_dtype, page_tokens=page if paged else 0, num_pages=B * per_seq if paged else 0)
+    if paged:
+        perm = np.random.default_rng(0).permutation(B * per_seq).astype(np.int32).reshape(B, per_seq)
+        table = torch.from_numpy(perm).to(dev)
+        cache.set_page_table(table)
     fill_rank(cache, gw, lens0, 0, dev)
     qs, ks, vs = step_inputs(gw, lens0, 0, base.steps)
     dq = [q.to(dev) for q in qs]
@@ -372,21 +378,24 @@ def run_fp8_decode(local, steps=512, warmup=16):
     assert cache.status() == 0, "device status set during the FP8 timed region"
     dec_ms = sum(ev[i][1].elapsed_time(ev[i][2]) for i in range(steps)) / steps
     step_ms = ev[0][0].elapsed_time(ev[-1][2]) / steps
-    fp8_bytes = sum(kv_bytes(lens0 + (i % base.steps) + 1, mask, base.d, base.sink, base.window, cap)
-                    for i in range(steps)) / steps / 2
+    elem = 1 if kv_dtype == "fp8" else 2
+    nbytes = sum(kv_bytes(lens0 + (i % base.steps) + 1, mask, base.d, base.sink, base.window, cap)
+                 for i in range(steps)) / steps * elem / 2
     hbm_peak, peak_kind = peaks()
-    achieved = fp8_bytes / (dec_ms * 1e-3) / 1e9
+    achieved = nbytes / (dec_ms * 1e-3) / 1e9
     cache.close()
+    what = ("an FP8 E4M3 cache (retrieval and streaming heads)" if kv_dtype == "fp8" else "a bf16 cache") + \
+        (", retrieval heads paged (256-token pages, shuffled)" if paged else "")
     return {
-        "workload": "gqa128k with an FP8 E4M3 cache (retrieval and streaming heads), append + decode per "
-                    "layer-step, 32 distinct steps cycled",
+        "workload": f"gqa128k with {what}, append + decode per layer-step, 32 distinct steps cycled",
         "steps": steps, "warmup": warmup,
         "layer_step_us": round(step_ms * 1e3, 3),
         "decode_us": round(dec_ms * 1e3, 3),
-        "kv_bytes_per_layer_step": int(fp8_bytes),
-        "roofline": {"bound": "hbm", "kernel": "decode_tc_kernel FP8 (kind::f8f6f4)", "achieved": round(achieved, 1),
-                     "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": round(achieved / hbm_peak, 4), "traffic": DECODE_FP8_TRAFFIC_BYTES,
+        "kv_bytes_per_layer_step": int(nbytes),
+        "roofline": {"bound": "hbm", "kernel": f"decode_tc_kernel {kv_dtype}{' paged' if paged else ''}",
+                     "achieved": round(achieved, 1), "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": round(achieved / hbm_peak, 4),
+                     "traffic": DECODE_FP8_TRAFFIC_BYTES if (kv_dtype == "fp8" and not paged) else None,
                      "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch"},
         "gpu_launches": 2 * steps,
     }
@@ -582,9 +591,9 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the chunked-prefill measurement")
-    ap.add_argument("--only", choices=["decode", "prefill", "fp8"], default=None,
+    ap.add_argument("--only", choices=["decode", "prefill", "fp8", "paged"], default=None,
                     help="measure one path only (profiling runs)")
-    ap.add_argument("--no-fp8", action="store_true", help="skip the FP8-cache decode measurement")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the FP8-cache and paged-cache decode measurements")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
     rank, world, local = dist_init()
@@ -594,14 +603,20 @@ def main(argv=None):
         elif args.only == "prefill":
             res = {"metric": "chunked prefill attention", "prefill": run_prefill(local)} if rank == 0 else None
         elif args.only == "fp8":
-            res = ({"metric": "FP8-cache decode", "decode_fp8": run_fp8_decode(local, args.steps, args.warmup)}
+            res = ({"metric": "FP8-cache decode",
+                    "decode_fp8": run_variant_decode(local, "fp8", False, args.steps, args.warmup)}
+                   if rank == 0 else None)
+        elif args.only == "paged":
+            res = ({"metric": "paged-cache decode",
+                    "decode_paged": run_variant_decode(local, "bf16", True, args.steps, args.warmup)}
                    if rank == 0 else None)
         else:
             res, ctx = run_ours(args, rank, world, local)
             if world == 1 and not args.no_prefill and args.only != "decode":
                 res["prefill"] = run_prefill(local)
             if world == 1 and not args.no_fp8 and args.only != "decode":
-                res["decode_fp8"] = run_fp8_decode(local)
+                res["decode_fp8"] = run_variant_decode(local, "fp8")
+                res["decode_paged"] = run_variant_decode(local, "bf16", True)
             if rank == 0 and world == 1 and not args.no_cpu_baseline:
                 res["cpu_baseline"] = cpu_baseline(ctx)
         if rank == 0 and res is not None:

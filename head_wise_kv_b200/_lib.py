@@ -35,6 +35,7 @@ DUO_STATUS_OVER_CAPACITY = 1
 DUO_STATUS_EMPTY_SEQUENCE = 2
 DUO_STATUS_WAIT_TIMEOUT = 4
 DUO_STATUS_BAD_LENGTH = 8
+DUO_STATUS_NO_PAGE = 16
 
 # C entry points declared in include/duo_kv.h (checked by the CPU tests)
 EXPORTED = (
@@ -42,7 +43,7 @@ EXPORTED = (
     "duo_kv_append", "duo_decode_workspace_bytes", "duo_decode_attn",
     "duo_prefill_workspace_bytes", "duo_prefill_attn", "duo_kv_read_status",
     "duo_kv_set_decode_ctas", "duo_strerror", "duo_decode_attn_static_ws",
-    "duo_kv_append_rows", "duo_decode_attn_rows", "duo_lse_merge", "duo_alpha_blend",
+    "duo_kv_append_rows", "duo_decode_attn_rows", "duo_lse_merge", "duo_alpha_blend", "duo_kv_set_page_table",
 )
 DUO_STATIC_WS_BYTES = 4 << 20
 
@@ -61,6 +62,8 @@ class duo_kv_desc(ctypes.Structure):
         ("kv_dtype", ctypes.c_int32),
         ("k_scale", ctypes.POINTER(ctypes.c_float)),
         ("v_scale", ctypes.POINTER(ctypes.c_float)),
+        ("page_tokens", ctypes.c_int32),
+        ("num_pages", ctypes.c_int64),
     ]
 
 
@@ -106,6 +109,7 @@ _c_pre_ws = _sig("duo_prefill_workspace_bytes", [_P, _I32, ctypes.POINTER(_SZ)])
 _c_prefill = _sig("duo_prefill_attn", [_P, _I32, _P, _P, _P, _P, _I32, ctypes.c_float, _P, _P, _SZ, _P])
 _c_status = _sig("duo_kv_read_status", [_P, ctypes.POINTER(_I32), _I32, _P])
 _c_set_ctas = _sig("duo_kv_set_decode_ctas", [_P, _I32])
+_c_set_pages = _sig("duo_kv_set_page_table", [_P, _P, _I32])
 _c_strerror = _sig("duo_strerror", [ctypes.c_int], ctypes.c_char_p)
 
 
@@ -125,7 +129,7 @@ def duo_strerror(code: int) -> str:
 
 
 def make_desc(num_layers, batch, num_q_heads, num_kv_heads, head_dim, sink, window, capacity, mask_u8,
-              kv_dtype=DUO_KV_BF16, k_scale=None, v_scale=None):
+              kv_dtype=DUO_KV_BF16, k_scale=None, v_scale=None, page_tokens=0, num_pages=0):
     """Build a duo_kv_desc; ``mask_u8`` is a host bytes-like [layers][n_kv];
     k_scale / v_scale optional float sequences [layers * n_kv] (FP8).  The
     host arrays are kept alive by the returned pair."""
@@ -139,7 +143,8 @@ def make_desc(num_layers, batch, num_q_heads, num_kv_heads, head_dim, sink, wind
         keep.append(arr)
         return ctypes.cast(arr, ctypes.POINTER(ctypes.c_float))
     d = duo_kv_desc(num_layers, batch, num_q_heads, num_kv_heads, head_dim, sink, window, capacity,
-                    ctypes.cast(buf, ctypes.POINTER(ctypes.c_uint8)), kv_dtype, floats(k_scale), floats(v_scale))
+                    ctypes.cast(buf, ctypes.POINTER(ctypes.c_uint8)), kv_dtype, floats(k_scale), floats(v_scale),
+                    page_tokens, num_pages)
     return d, keep
 
 
@@ -224,3 +229,7 @@ def duo_kv_read_status(handle, clear: bool, stream: int) -> int:
 
 def duo_kv_set_decode_ctas(handle, ctas: int) -> None:
     _check(_c_set_ctas(handle, ctas), "duo_kv_set_decode_ctas")
+
+
+def duo_kv_set_page_table(handle, d_table: int, max_pages: int) -> None:
+    _check(_c_set_pages(handle, d_table, max_pages), "duo_kv_set_page_table")

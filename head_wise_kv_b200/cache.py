@@ -34,10 +34,14 @@ class DuoKVCache:
     retrieval_mask: [num_layers][num_kv_heads] (1 = retrieval KV head).
     kv_dtype: "bf16" or "fp8" (E4M3 codes; k_scale / v_scale per
     [num_layers][num_kv_heads], default 1.0).
+    page_tokens > 0: paged retrieval caches, a pool of num_pages pages per
+    layer; the page table (int32 [batch][max_pages] on the device) is given
+    with set_page_table.
     """
 
     def __init__(self, num_layers, batch, num_q_heads, num_kv_heads, head_dim, sink, window, capacity,
-                 retrieval_mask, device="cuda", kv_dtype="bf16", k_scale=None, v_scale=None):
+                 retrieval_mask, device="cuda", kv_dtype="bf16", k_scale=None, v_scale=None, page_tokens=0,
+                 num_pages=0):
         self.device = torch.device(device)
         if self.device.type != "cuda":
             raise ValueError("DuoKVCache lives on a CUDA device")
@@ -60,7 +64,9 @@ class DuoKVCache:
         self._desc, self._mask_buf = L.make_desc(
             num_layers, batch, num_q_heads, num_kv_heads, head_dim, sink, window, capacity, mask.tobytes(),
             L.DUO_KV_FP8_E4M3 if self.fp8 else L.DUO_KV_BF16, self.k_scale.ravel().tolist(),
-            self.v_scale.ravel().tolist())
+            self.v_scale.ravel().tolist(), page_tokens, num_pages)
+        self.page_tokens, self.num_pages = page_tokens, num_pages
+        self._page_table = None
         self.total_bytes, self.cache_bytes = L.duo_kv_required_bytes(self._desc)
         with torch.cuda.device(self.device):
             self.buf = torch.empty(self.total_bytes, dtype=torch.uint8, device=self.device)
@@ -72,6 +78,16 @@ class DuoKVCache:
     def _alloc_workspace(self):
         n = L.duo_decode_workspace_bytes(self.handle)
         self._ws = torch.empty(max(n, 256), dtype=torch.uint8, device=self.device)
+
+    def set_page_table(self, table):
+        """table: int32 [batch][max_pages] on the cache's device (kept
+        referenced; its contents may change between calls)."""
+        if table.dtype != torch.int32 or table.dim() != 2 or table.shape[0] != self.B:
+            raise ValueError("page table must be int32 [batch][max_pages]")
+        if table.device != self.device or not table.is_contiguous():
+            raise ValueError("page table must be a contiguous tensor on the cache's device")
+        L.duo_kv_set_page_table(self.handle, table.data_ptr(), table.shape[1])
+        self._page_table = table
 
     def set_decode_ctas(self, ctas: int):
         L.duo_kv_set_decode_ctas(self.handle, ctas)
@@ -106,8 +122,13 @@ class DuoKVCache:
 
         def typed(t):
             return t if self.fp8 else t.view(torch.bfloat16)
-        kr = typed(region(v.k_retrieval, B * nr * cap * d * eb)).view(B, nr, cap, d)
-        vr = typed(region(v.v_retrieval, B * nr * cap * d * eb)).view(B, nr, cap, d)
+        if self.page_tokens > 0:   # the pool [num_pages][n_r][page_tokens][d]
+            shape = (self.num_pages, nr, self.page_tokens, d)
+        else:
+            shape = (B, nr, cap, d)
+        n_el = shape[0] * shape[1] * shape[2] * shape[3]
+        kr = typed(region(v.k_retrieval, n_el * eb)).view(*shape)
+        vr = typed(region(v.v_retrieval, n_el * eb)).view(*shape)
         ks = typed(region(v.k_streaming, B * ns * SW * d * eb)).view(B, ns, SW, d)
         vs = typed(region(v.v_streaming, B * ns * SW * d * eb)).view(B, ns, SW, d)
         pos = region(v.positions, B * SW * 4).view(torch.int32).view(B, SW)

@@ -32,6 +32,13 @@ int check_desc(const duo_kv_desc* d) {
     if (g != 1 && g != 2 && g != 4 && g != 8) return DUO_ERR_UNSUPPORTED;
     if (d->num_kv_heads > duo::kMaxKvHeads) return DUO_ERR_UNSUPPORTED;
     if (d->kv_dtype != DUO_KV_BF16 && d->kv_dtype != DUO_KV_FP8_E4M3) return DUO_ERR_INVALID_ARG;
+    if (d->page_tokens < 0) return DUO_ERR_INVALID_ARG;
+    if (d->page_tokens > 0) {
+        if (d->page_tokens % 256 != 0 || d->num_pages < 1) return DUO_ERR_INVALID_ARG;
+        if (d->head_dim != 128) return DUO_ERR_UNSUPPORTED;
+        // TMA coordinates are int32: pool rows of one page, pages * heads
+        if (d->num_pages * int64_t(d->num_kv_heads) >= (int64_t(1) << 31)) return DUO_ERR_UNSUPPORTED;
+    }
     if (d->kv_dtype == DUO_KV_FP8_E4M3) {
         if (d->head_dim != 128) return DUO_ERR_UNSUPPORTED;
         const size_t n = size_t(d->num_layers) * d->num_kv_heads;
@@ -68,7 +75,8 @@ size_t plan_layout(const duo_kv_desc* d, std::vector<duo::LayerLayout>* layers, 
             L.rank[g] = r ? L.n_r++ : L.n_s++;
         }
         L.r_before[d->num_kv_heads] = L.n_r;
-        const size_t kr = B * L.n_r * size_t(d->capacity) * D * E;
+        const size_t kr = d->page_tokens > 0 ? size_t(d->num_pages) * L.n_r * size_t(d->page_tokens) * D * E
+                                             : B * L.n_r * size_t(d->capacity) * D * E;
         const size_t ks = B * L.n_s * SW * D * E;
         L.off_kr = off; off = align_up(off + kr);
         L.off_vr = off; off = align_up(off + kr);
@@ -109,6 +117,8 @@ int duo_kv_alloc(const duo_kv_desc* desc, void* dev_buf, size_t buf_bytes, duo_s
     h->desc.retrieval_mask = nullptr;
     h->desc.k_scale = h->desc.v_scale = nullptr;
     h->fp8 = desc->kv_dtype == DUO_KV_FP8_E4M3;
+    h->page_tokens = desc->page_tokens;
+    h->num_pages = desc->num_pages;
     {
         const size_t n = size_t(desc->num_layers) * desc->num_kv_heads;
         h->k_scale.assign(n, 1.f);
@@ -144,9 +154,12 @@ int duo_kv_alloc(const duo_kv_desc* desc, void* dev_buf, size_t buf_bytes, duo_s
         h->maps.resize(h->layers.size());
         for (size_t l = 0; l < h->layers.size(); ++l) {
             const duo::LayerLayout& L = h->layers[l];
+            const bool paged = desc->page_tokens > 0;
             if (!duo::make_decode_maps(&h->maps[l], h->base + L.off_kr, h->base + L.off_vr, h->base + L.off_ks,
-                                       h->base + L.off_vs, desc->batch, L.n_r, L.n_s, desc->capacity, int(SW),
-                                       h->fp8 != 0)) {
+                                       h->base + L.off_vs,
+                                       paged ? desc->num_pages * L.n_r : int64_t(desc->batch) * L.n_r,
+                                       paged ? desc->page_tokens : desc->capacity, int64_t(desc->batch) * L.n_s,
+                                       int(SW), h->fp8 != 0)) {
                 delete h;
                 return DUO_ERR_CUDA;
             }
@@ -220,6 +233,13 @@ static int append_impl(duo_kv* kv, int32_t layer, const uint16_t* k_new, const u
     for (int g = 0; g < kv->desc.num_kv_heads; ++g) {
         p.k_scale[g] = kv->k_scale[size_t(layer) * kv->desc.num_kv_heads + g];
         p.v_scale[g] = kv->v_scale[size_t(layer) * kv->desc.num_kv_heads + g];
+    }
+    if (kv->page_tokens > 0) {
+        if (!kv->page_table && L.n_r > 0) return DUO_ERR_INVALID_ARG;   // no page table set
+        p.page_tokens = kv->page_tokens;
+        p.num_pages = kv->num_pages;
+        p.max_pages = kv->max_pages;
+        p.page_table = kv->page_table;
     }
     return cuda_err(duo::launch_append(p, stream));
 }
@@ -313,6 +333,14 @@ static int decode_impl(duo_kv* kv, int32_t layer, const uint16_t* q, const int32
         p.k_scale[g] = kv->k_scale[size_t(layer) * kv->desc.num_kv_heads + g];
         p.v_scale[g] = kv->v_scale[size_t(layer) * kv->desc.num_kv_heads + g];
     }
+    p.blk = 16;
+    if (kv->page_tokens > 0) {
+        if (!kv->page_table && L.n_r > 0) return DUO_ERR_INVALID_ARG;   // no page table set
+        p.page_tokens = kv->page_tokens;
+        p.num_pages = kv->num_pages;
+        p.max_pages = kv->max_pages;
+        p.page_table = kv->page_table;
+    }
     return cuda_err(duo::launch_decode(p, D, G, stream));
 }
 
@@ -362,7 +390,7 @@ static size_t prefill_ws(const duo_kv* kv, int32_t chunk) {
     }
     const duo_kv_desc& d = kv->desc;
     return duo::prefill_workspace_bytes(d.batch, d.num_kv_heads, n_r, n_s, d.capacity, d.sink, d.window, chunk,
-                                        kv->fp8 != 0);
+                                        kv->fp8 != 0 || kv->page_tokens > 0);
 }
 
 int duo_prefill_workspace_bytes(const duo_kv* kv, int32_t chunk, size_t* bytes) {
@@ -432,6 +460,13 @@ int duo_prefill_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const uint16_
         a.k_scale[g] = kv->k_scale[size_t(layer) * d.num_kv_heads + g];
         a.v_scale[g] = kv->v_scale[size_t(layer) * d.num_kv_heads + g];
     }
+    if (kv->page_tokens > 0) {
+        if (!kv->page_table && L.n_r > 0) return DUO_ERR_INVALID_ARG;   // no page table set
+        a.page_tokens = kv->page_tokens;
+        a.num_pages = kv->num_pages;
+        a.max_pages = kv->max_pages;
+        a.page_table = kv->page_table;
+    }
     return duo::launch_prefill(a, stream);
 }
 
@@ -444,6 +479,14 @@ int duo_kv_read_status(duo_kv* kv, int32_t* status, int32_t clear, duo_stream_t 
     if (e == cudaSuccess && clear && (*status & DUO_STATUS_WAIT_TIMEOUT))
         e = cudaMemsetAsync(kv->seg_count, 0, size_t(kv->desc.batch) * kv->desc.num_kv_heads * 4, stream);
     return cuda_err(e);
+}
+
+int duo_kv_set_page_table(duo_kv* kv, const int32_t* d_table, int32_t max_pages) {
+    if (!kv || kv->page_tokens <= 0 || !d_table || max_pages < 1) return DUO_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(d_table) & 3) return DUO_ERR_ALIGNMENT;
+    kv->page_table = d_table;
+    kv->max_pages = max_pages;
+    return DUO_OK;
 }
 
 int duo_kv_set_decode_ctas(duo_kv* kv, int32_t ctas) {

@@ -103,9 +103,23 @@ __global__ void __launch_bounds__(kThreads) append_kernel(const __grid_constant_
             if (part == 0) set_status(p.status, DUO_STATUS_OVER_CAPACITY);
             return;
         }
+        size_t dst;
+        if (p.page_tokens > 0) {
+            // paged: row -> (page from the table, offset in the page); a page
+            // holds [n_r][page_tokens][d] for one sequence
+            const int64_t slot = row / p.page_tokens;
+            const int page = slot < p.max_pages ? p.page_table[size_t(b) * p.max_pages + slot] : -1;
+            if (page < 0 || page >= p.num_pages) {
+                if (part == 0) set_status(p.status, DUO_STATUS_NO_PAGE);
+                return;
+            }
+            dst = ((size_t(page) * p.n_r + p.rank[g]) * size_t(p.page_tokens) + size_t(row % p.page_tokens)) * D +
+                  part * 8;
+        } else {
+            dst = ((size_t(b) * p.n_r + p.rank[g]) * size_t(p.cap) + row) * D + part * 8;
+        }
         const uint4 kv = *reinterpret_cast<const uint4*>(p.k_new + src);
         const uint4 vv = *reinterpret_cast<const uint4*>(p.v_new + src);
-        const size_t dst = ((size_t(b) * p.n_r + p.rank[g]) * size_t(p.cap) + row) * D + part * 8;
         put8(p, p.kr, dst, kv, p.k_scale[g]);
         put8(p, p.vr, dst, vv, p.v_scale[g]);
     } else if (survives) {

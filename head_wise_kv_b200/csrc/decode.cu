@@ -465,7 +465,7 @@ __global__ void __launch_bounds__(32 * G) merge_kernel(const __grid_constant__ D
     float* out = p.out + (size_t(b) * p.hq + qh) * D;
     const int64_t total = bpre[p.B];
     const SeqRows x = seq_rows(p, b);
-    const int nbr = blocks_of(x.nr), nbs = blocks_of(x.ns);
+    const int nbr = blocks_of(x.nr, p.blk), nbs = blocks_of(x.ns, p.blk);
     const int64_t seg_gb = bpre[b] + int64_t(p.r_before[g]) * nbr + int64_t(g - p.r_before[g]) * nbs;
     const int seg_nb = p.is_r[g] ? nbr : nbs;
     const int c0 = seg_nb < 1 ? 0 : cta_owner(seg_gb, total, p.num_ctas);

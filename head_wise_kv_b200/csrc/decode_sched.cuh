@@ -2,7 +2,7 @@
 //
 // Every (sequence b, KV head g) pair is a *segment* of keys: the retrieval
 // rows or the filled ring slots it reads.  All segments are laid end to end
-// in blocks of 16 tokens and a persistent grid of C CTAs takes C equal
+// in blocks of p.blk tokens and a persistent grid of C CTAs takes C equal
 // contiguous ranges of that axis; a CTA walks its range piece by piece (a
 // piece = the part of one segment inside the range).  Partial results go to
 // workspace slot (segment + CTA), unique because moving along the axis
@@ -16,9 +16,9 @@
 namespace duo {
 namespace {
 
-constexpr int kBlk = 16;   // partition granularity in tokens
-
-__device__ __forceinline__ int blocks_of(int64_t rows) { return int((rows + kBlk - 1) / kBlk); }
+// Blocks of p.blk tokens (16, or a whole tile for paged caches so that no
+// tile straddles a page).
+__device__ __forceinline__ int blocks_of(int64_t rows, int blk) { return int((rows + blk - 1) / blk); }
 
 __device__ __forceinline__ int64_t rows_r(int len, int64_t cap) {
     int64_t r = len < 0 ? 0 : len;
@@ -84,7 +84,8 @@ __device__ void build_prefix(const DecodeParams& p, int32_t* bpre) {
         int c = 0;
         if (b < p.B) {
             const SeqRows x = seq_rows(p, b);
-            c = p.n_r * seg_units(blocks_of(x.nr), p.seg_weight) + p.n_s * seg_units(blocks_of(x.ns), p.seg_weight);
+            c = p.n_r * seg_units(blocks_of(x.nr, p.blk), p.seg_weight) +
+                p.n_s * seg_units(blocks_of(x.ns, p.blk), p.seg_weight);
             int32_t* rows = bpre + p.B + 1;
             rows[b] = int32_t(x.r0);
             rows[p.B + b] = int32_t(x.nr);
@@ -140,7 +141,7 @@ __device__ __forceinline__ Piece locate(const DecodeParams& p, const int32_t* bp
     pc.b = lo;
     const int32_t* tab = bpre + p.B + 1;
     const int64_t r0 = tab[lo], rr = tab[p.B + lo], rs = tab[2 * p.B + lo];
-    const int nbr = blocks_of(rr), nbs = blocks_of(rs);
+    const int nbr = blocks_of(rr, p.blk), nbs = blocks_of(rs, p.blk);
     const int ur = seg_units(nbr, p.seg_weight), us = seg_units(nbs, p.seg_weight);
     const int64_t local = gb - bpre[lo];
     const int32_t* hb = bpre + 4 * p.B + 1;
@@ -163,8 +164,8 @@ __device__ __forceinline__ Piece locate(const DecodeParams& p, const int32_t* bp
     const int64_t seg_end = pc.seg_gb + pc.seg_nb;
     pc.end_gb = seg_end < range_end ? seg_end : range_end;
     const int64_t rows = retr ? rr : rs;
-    pc.tok0 = gb > pc.seg_gb ? (gb - pc.seg_gb) * kBlk : 0;
-    const int64_t t1 = (pc.end_gb - pc.seg_gb) * kBlk;
+    pc.tok0 = gb > pc.seg_gb ? (gb - pc.seg_gb) * p.blk : 0;
+    const int64_t t1 = (pc.end_gb - pc.seg_gb) * p.blk;
     pc.tok1 = t1 < rows ? t1 : rows;
     if (pc.tok1 < pc.tok0) pc.tok1 = pc.tok0;   // the range ends before the segment's first key
     pc.whole = (gb <= pc.seg_gb) && (pc.end_gb == seg_end);

@@ -212,6 +212,32 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const D
     return ok != 0;
 }
 
+// TMA coordinates of the tile that starts t keys into a piece: (row, head)
+// of the [heads][rows] maps; paged retrieval caches address the pool
+// [pages * n_r][page_tokens] through the tile's page (a missing page sets
+// DUO_STATUS_NO_PAGE and reads as zeros: its coordinate is outside the map).
+// A paged tile must start on a page boundary (T divides page_tokens and
+// the pieces start on tile boundaries; a row range must start on a
+// multiple of 256, else DUO_STATUS_BAD_LENGTH).
+template <int T>
+__device__ __forceinline__ void tile_coords(const DecodeParams& p, const Piece& pc, int64_t t, int page, int& y,
+                                            int& z) {
+    if (pc.retr && p.page_tokens > 0) {
+        const int64_t row = pc.row0 + t;
+        y = int(row % p.page_tokens);
+        if (y + T > p.page_tokens) set_status(p.status, DUO_STATUS_BAD_LENGTH);
+        if (page < 0 || page >= p.num_pages) {
+            set_status(p.status, DUO_STATUS_NO_PAGE);
+            z = -1;
+        } else {
+            z = page * p.n_r + pc.rank;
+        }
+    } else {
+        y = int(pc.row0 + t);
+        z = pc.b * (pc.retr ? p.n_r : p.n_s) + pc.rank;
+    }
+}
+
 // Lane 0 polls for the warp, napping between polls: for waits that span a
 // whole piece, so that the poll takes no issue slots from the warps on the
 // critical path.
@@ -289,12 +315,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     const uint32_t sQ = sV + nst * kTileBytes;            // 2 q operands (piece parity)
     const uint32_t sP = sQ + 2 * C::QB;                   // 2 P^T operands (tile parity)
     int32_t* bpre = reinterpret_cast<int32_t*>(smem + 2 * nst * kTileBytes + 2 * C::QB + 2 * C::PB);
+    // paged caches: the pool page of each of this CTA's tiles, in the
+    // producers' order (p.pg_cap entries after the sequence table)
+    int32_t* pg = bpre + (seq_table_bytes(p.B, p.n_kv) + 15) / 16 * 4;
 
     constexpr int kMaxStages = 3;
     __shared__ __align__(8) uint64_t full_k[kMaxStages], full_v[kMaxStages], empty_k[kMaxStages],
         empty_v[kMaxStages], q_full[2],
         q_empty[2], s_full[2], s_free[2], p_full[2], p_free[2], o_full[2], o_empty[2], epi_full[2], mma_fin,
-        qs_full[4];
+        qs_full[4], pg_ready;
     // FP8: 2^-a of each piece's q prescale, a ring of four (the q warp runs
     // at most three pieces ahead of the softmax, see the q warp)
     __shared__ float q_scale[4];
@@ -328,6 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         }
         mbar_init(smem_addr(&mma_fin), 1);
         for (int s = 0; s < 4; ++s) mbar_init(smem_addr(&qs_full[s]), 1);
+        mbar_init(smem_addr(&pg_ready), 1);
         abort_sh = 0;
         fence_mbar_init();
     }
@@ -365,19 +395,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             if (lane == 0) {
                 const uint64_t policy = l2_evict_first_policy();
                 uint32_t it = 0;
-                bool ok = true;
+                bool ok = p.page_tokens <= 0 || timed_wait(smem_addr(&pg_ready), 0, p, abort_flag);
                 for (int64_t gb = gb_begin; ok && gb < gb_end;) {
                     Piece pc;
                     if (!next_piece(p, bpre, gb, gb_end, pc)) break;
                     const CUtensorMap* mk = pc.retr ? &p.tm_kr : &p.tm_ks;
-                    const int z = pc.b * (pc.retr ? p.n_r : p.n_s) + pc.rank;
+                    const bool paged = pc.retr && p.page_tokens > 0;
                     for (int64_t t = pc.tok0; t < pc.tok1; t += C::T, ++it) {
                         const int st = int(it % uint32_t(nst));
                         if (!timed_wait(smem_addr(&empty_k[st]), ((it / nst) & 1) ^ 1, p, abort_flag)) {
                             ok = false;
                             break;
                         }
-                        const int y = int(pc.row0 + t);
+                        int y, z;
+                        tile_coords<C::T>(p, pc, t, paged ? (it < uint32_t(p.pg_cap) ? pg[it] : -1) : 0, y, z);
                         const uint32_t fk = smem_addr(&full_k[st]);
                         mbar_arrive_expect_tx(fk, kTileBytes);
                         if constexpr (F8) {
@@ -396,6 +427,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             }
         } else if (warp == kQWarp) {
             // ======================================================== q staging
+            if (p.page_tokens > 0) {
+                // Paged caches: look up the pool page of every retrieval tile
+                // now, before HBM is busy (a dependent global read per tile
+                // would stall the producers), in the producers' tile order.
+                uint32_t idx = 0;
+                for (int64_t gb = gb_begin; gb < gb_end;) {
+                    Piece pc;
+                    if (!next_piece(p, bpre, gb, gb_end, pc)) break;
+                    const int nt = tiles_of<C::T>(pc);
+                    if (pc.retr)
+                        for (int k = lane; k < nt; k += 32) {
+                            const int64_t slot = (pc.row0 + pc.tok0 + int64_t(k) * C::T) / p.page_tokens;
+                            const int page = slot < p.max_pages ? p.page_table[size_t(pc.b) * p.max_pages + slot] : -1;
+                            if (idx + k < uint32_t(p.pg_cap)) pg[idx + k] = page;
+                        }
+                    idx += nt;
+                }
+                if (idx > uint32_t(p.pg_cap) && lane == 0) set_status(p.status, DUO_STATUS_NO_PAGE);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_addr(&pg_ready));
+            }
             // Runs up to two pieces ahead of the S products (two q buffers).
             int pi = 0;
             for (int64_t gb = gb_begin; gb < gb_end; ++pi) {
@@ -486,19 +538,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             if (lane == 0) {
                 const uint64_t policy = l2_evict_first_policy();
                 uint32_t it = 0;
-                bool ok = true;
+                bool ok = p.page_tokens <= 0 || timed_wait(smem_addr(&pg_ready), 0, p, abort_flag);
                 for (int64_t gb = gb_begin; ok && gb < gb_end;) {
                     Piece pc;
                     if (!next_piece(p, bpre, gb, gb_end, pc)) break;
                     const CUtensorMap* mv = pc.retr ? &p.tm_vr : &p.tm_vs;
-                    const int z = pc.b * (pc.retr ? p.n_r : p.n_s) + pc.rank;
+                    const bool paged = pc.retr && p.page_tokens > 0;
                     for (int64_t t = pc.tok0; t < pc.tok1; t += C::T, ++it) {
                         const int st = int(it % uint32_t(nst));
                         if (!timed_wait(smem_addr(&empty_v[st]), ((it / nst) & 1) ^ 1, p, abort_flag)) {
                             ok = false;
                             break;
                         }
-                        const int y = int(pc.row0 + t);
+                        int y, z;
+                        tile_coords<C::T>(p, pc, t, paged ? (it < uint32_t(p.pg_cap) ? pg[it] : -1) : 0, y, z);
                         const uint32_t fv = smem_addr(&full_v[st]);
                         mbar_arrive_expect_tx(fv, kTileBytes);
                         if constexpr (F8) {
@@ -921,8 +974,23 @@ template <int G, bool F8>
 cudaError_t launch_g(const DecodeParams& p, cudaStream_t s) {
     using C = Tr<G, F8>;
     DecodeParams q = p;
-    q.seg_weight = F8 ? kSegWeightF8 : kSegWeight;
-    const size_t fixed = 2 * size_t(C::QB + C::PB) + seq_table_bytes(p.B, p.n_kv) + 1024;
+    // partition: 16-token blocks, or whole tiles for paged caches (no tile
+    // straddles a page); the segment weight is a fixed number of keys
+    q.blk = p.page_tokens > 0 ? C::T : 16;
+    q.seg_weight = (F8 ? kSegWeightF8 : kSegWeight) * 16 / q.blk;
+    q.pg_cap = 0;
+    if (p.page_tokens > 0) {
+        // tiles one CTA can see: its share of the largest possible axis, plus
+        // one partial tile per piece (at most one piece per segment, plus one)
+        const int64_t ur = (p.cap + q.blk - 1) / q.blk + q.seg_weight;
+        const int64_t us = (p.S + p.W + q.blk - 1) / q.blk + q.seg_weight;
+        const int64_t axis = int64_t(p.B) * (int64_t(p.n_r) * ur + int64_t(p.n_s) * us);
+        const int64_t cap = (axis + p.num_ctas - 1) / p.num_ctas + 2 + int64_t(p.B) * p.n_kv;
+        if (cap > (1 << 20)) return cudaErrorInvalidConfiguration;
+        q.pg_cap = int(cap);
+    }
+    const size_t fixed = 2 * size_t(C::QB + C::PB) + (seq_table_bytes(p.B, p.n_kv) + 15) / 16 * 16 +
+                         size_t(q.pg_cap) * 4 + 1024;
     q.stages = fixed + 3 * 2 * size_t(kTileBytes) <= size_t(227) * 1024 ? 3 : 2;
     const size_t smem = fixed + size_t(q.stages) * 2 * kTileBytes;
     if (smem > size_t(227) * 1024) return cudaErrorInvalidConfiguration;
@@ -962,12 +1030,12 @@ bool make_map3(CUtensorMap* m, const void* base, uint64_t rows, uint64_t heads, 
 
 }  // namespace
 
-bool make_decode_maps(DecodeMaps* m, const void* kr, const void* vr, const void* ks, const void* vs, int B, int n_r,
-                      int n_s, int64_t cap, int SW, bool fp8) {
-    return make_map3(&m->kr, kr, uint64_t(cap), uint64_t(B) * n_r, fp8) &&
-           make_map3(&m->vr, vr, uint64_t(cap), uint64_t(B) * n_r, fp8) &&
-           make_map3(&m->ks, ks, uint64_t(SW), uint64_t(B) * n_s, fp8) &&
-           make_map3(&m->vs, vs, uint64_t(SW), uint64_t(B) * n_s, fp8);
+bool make_decode_maps(DecodeMaps* m, const void* kr, const void* vr, const void* ks, const void* vs, int64_t r_heads,
+                      int64_t r_rows, int64_t s_heads, int SW, bool fp8) {
+    return make_map3(&m->kr, kr, uint64_t(r_rows), uint64_t(r_heads), fp8) &&
+           make_map3(&m->vr, vr, uint64_t(r_rows), uint64_t(r_heads), fp8) &&
+           make_map3(&m->ks, ks, uint64_t(SW), uint64_t(s_heads), fp8) &&
+           make_map3(&m->vs, vs, uint64_t(SW), uint64_t(s_heads), fp8);
 }
 
 cudaError_t launch_decode_tc(const DecodeParams& p, int group, cudaStream_t s) {

@@ -42,6 +42,10 @@ struct duo_kv {
     int num_sms = 0;
     int decode_ctas = 0;                    // 0 = default persistent wave
     int fp8 = 0;                            // caches hold E4M3 codes
+    int page_tokens = 0;                    // > 0: paged retrieval caches (pools of num_pages pages)
+    int64_t num_pages = 0;
+    const int32_t* page_table = nullptr;    // device [B][max_pages], caller-owned
+    int max_pages = 0;
     std::vector<float> k_scale, v_scale;    // [L][n_kv] (FP8)
     std::vector<duo::DecodeMaps> maps;      // per layer (head_dim 128 only)
 };
@@ -69,7 +73,13 @@ struct DecodeParams {
     int64_t cap;
     int B, n_kv, hq, n_r, n_s, S, W;
     int num_ctas;
-    int seg_weight;           // partition weight of a segment start, in 16-token blocks (0 = none)
+    int blk;                  // partition block in tokens (16; a whole tile for paged caches)
+    int seg_weight;           // partition weight of a segment start, in blocks (0 = none)
+    int page_tokens;          // > 0: paged retrieval caches
+    int64_t num_pages;
+    int max_pages;
+    const int32_t* page_table;   // [B][max_pages]
+    int pg_cap;                  // tensor-core kernel: entries of its shared page list
     int fp8;                  // caches hold E4M3 codes (tensor-core kernel only)
     int stages;               // tensor-core kernel pipeline depth (set by its launcher)
     float scale_log2;
@@ -96,6 +106,10 @@ struct AppendParams {
     int64_t cap;
     int B, n_kv, n_r, n_s, S, W, d, n_new_max;
     int fp8;                      // store E4M3 codes of value / scale
+    int page_tokens;              // > 0: paged retrieval caches
+    int64_t num_pages;
+    int max_pages;
+    const int32_t* page_table;
     int32_t rank[kMaxKvHeads];
     uint8_t is_r[kMaxKvHeads];
     float k_scale[kMaxKvHeads], v_scale[kMaxKvHeads];
@@ -117,6 +131,10 @@ struct PrefillLaunch {
     int B, hq, n_kv, C, S, W, n_r, n_s;
     int fp8;                // cached prefix holds E4M3 codes
     float k_scale[kMaxKvHeads], v_scale[kMaxKvHeads];
+    int page_tokens;        // > 0: paged retrieval caches (prefix gathered into the workspace)
+    int64_t num_pages;
+    int max_pages;
+    const int32_t* page_table;
     float scale;
     unsigned long long timeout_ns;
     int32_t rank[kMaxKvHeads];
@@ -129,14 +147,17 @@ int decode_ctas_default(int num_sms, int d, int group);
 size_t decode_workspace_bytes(int slots, int d, int group);
 cudaError_t launch_decode(const DecodeParams& p, int d, int group, cudaStream_t s);
 cudaError_t launch_decode_tc(const DecodeParams& p, int group, cudaStream_t s);   // attention only
-bool make_decode_maps(DecodeMaps* m, const void* kr, const void* vr, const void* ks, const void* vs, int B, int n_r,
-                      int n_s, int64_t cap, int SW, bool fp8);
+// Retrieval maps over [B * n_r][cap] rows, or for paged caches over the
+// pool [num_pages * n_r][page_tokens] (pass r_heads = num_pages * n_r, r_rows = page_tokens).
+bool make_decode_maps(DecodeMaps* m, const void* kr, const void* vr, const void* ks, const void* vs, int64_t r_heads,
+                      int64_t r_rows, int64_t s_heads, int SW, bool fp8);
 cudaError_t launch_lse_merge(int parts, int rows, int d, const float* part_out, const float* part_lse, float* out,
                              float* lse, cudaStream_t s);
 cudaError_t launch_blend(int64_t n, int hq, int d, const float* alpha, const float* full, const float* strm,
                          float* out, cudaStream_t s);
 size_t prefill_smem_bytes(int S, int W);
-size_t prefill_workspace_bytes(int B, int n_kv, int n_r, int n_s, int64_t cap, int S, int W, int C, bool fp8);
+size_t prefill_workspace_bytes(int B, int n_kv, int n_r, int n_s, int64_t cap, int S, int W, int C,
+                               bool key_copies);   // key copies: FP8 or paged caches
 int launch_prefill(const PrefillLaunch& a, cudaStream_t s);   // returns a DUO_* code
 
 // ----------------------------------------------------------------- device helpers

@@ -80,6 +80,7 @@ struct PrefillParams {
     float scale_log2;
     unsigned long long timeout_ns;
     int fp8;                                    // cached keys / values are E4M3 codes
+    int kcopy;                                  // cached keys read from the workspace copies (FP8 or paged)
     int32_t rank[kMaxKvHeads];
     uint8_t is_r[kMaxKvHeads];
     float k_scale[kMaxKvHeads], v_scale[kMaxKvHeads];
@@ -92,11 +93,16 @@ struct ConvertParams {
     uint16_t* v16r;         // fp16 copies: [B][n_r][LR][d], [B][n_s][LS][d], [B][n_kv][C][d]
     uint16_t* v16s;
     uint16_t* v16c;
-    const uint8_t* kr8;     // FP8 caches: key codes, and bf16 copies of them [B][n_r][LR][d], [B][n_s][LS][d]
-    const uint8_t* ks8;
-    uint16_t* k16r;
+    const void* kr;         // cached keys (bf16 or E4M3; retrieval: a contiguous cache or the page pool)
+    const void* ks;
+    uint16_t* k16r;         // bf16 copies of the cached keys [B][n_r][LR][d], [B][n_s][LS][d]
     uint16_t* k16s;
     int fp8;
+    int page_tokens;        // > 0: retrieval rows live in pages
+    int max_pages;
+    int64_t num_pages;
+    const int32_t* page_table;
+    int32_t* status;
     const int32_t* prefix;
     int64_t cap;
     int B, n_kv, n_r, n_s, S, W, C, LR, LS;
@@ -289,29 +295,28 @@ __global__ void __launch_bounds__(256) convert_v_kernel(const __grid_constant__ 
     const int b = bg / c.n_kv, g = bg % c.n_kv;
     const int P = max(c.prefix[b], 0);
     const bool keys = blockIdx.z == 2;
-    const uint16_t* src = nullptr;
-    const uint8_t* src8 = nullptr;
+    const size_t E = c.fp8 ? 1 : 2;                       // bytes per cached element
+    const size_t row_bytes = kHD * E;
+    const uint8_t* base = nullptr;                        // cached rows (contiguous) or the page pool
+    const uint16_t* chunk = nullptr;
+    bool paged = false;
     uint16_t* dst;
     int64_t n_conv, n_rows;
     if (blockIdx.z == 1) {
-        src = c.vc + size_t(bg) * c.C * kHD;
+        chunk = c.vc + size_t(bg) * c.C * kHD;
         dst = c.v16c + size_t(bg) * c.C * kHD;
         n_conv = n_rows = c.C;
     } else if (c.is_r[g]) {
         const size_t r = size_t(b) * c.n_r + c.rank[g];
-        if (c.fp8)
-            src8 = (keys ? c.kr8 : reinterpret_cast<const uint8_t*>(c.vr)) + r * size_t(c.cap) * kHD;
-        else
-            src = c.vr + r * size_t(c.cap) * kHD;
+        const uint8_t* pool = static_cast<const uint8_t*>(keys ? c.kr : static_cast<const void*>(c.vr));
+        paged = c.page_tokens > 0;
+        base = paged ? pool : pool + r * size_t(c.cap) * row_bytes;
         dst = (keys ? c.k16r : c.v16r) + r * size_t(c.LR) * kHD;
         n_conv = min(int64_t(P), c.cap);
         n_rows = (n_conv + kBN - 1) / kBN * kBN;          // tail of the last prefix tile
     } else {
         const size_t r = size_t(b) * c.n_s + c.rank[g];
-        if (c.fp8)
-            src8 = (keys ? c.ks8 : reinterpret_cast<const uint8_t*>(c.vs)) + r * size_t(c.S + c.W) * kHD;
-        else
-            src = c.vs + r * size_t(c.S + c.W) * kHD;
+        base = static_cast<const uint8_t*>(keys ? c.ks : static_cast<const void*>(c.vs)) + r * size_t(c.S + c.W) * row_bytes;
         dst = (keys ? c.k16s : c.v16s) + r * size_t(c.LS) * kHD;
         n_conv = min(P, c.S + c.W);                         // filled slots
         n_rows = c.LS;
@@ -320,18 +325,41 @@ __global__ void __launch_bounds__(256) convert_v_kernel(const __grid_constant__ 
     for (int64_t x = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; x < pieces;
          x += int64_t(gridDim.x) * blockDim.x) {
         const int64_t row = x / (kHD / 8);
+        const int col8 = int(x % (kHD / 8));              // 8-element chunk of the row
         uint4 v = make_uint4(0, 0, 0, 0);
         if (row < n_conv) {
-            if (src8) {
-                const uint2 cc = *reinterpret_cast<const uint2*>(src8 + x * 8);
-                v = keys ? e4m3x8_to_bf16(cc) : e4m3x8_to_f16(cc);
-            } else {
-                const uint4 w = *reinterpret_cast<const uint4*>(src + x * 8);
+            if (chunk) {
+                const uint4 w = *reinterpret_cast<const uint4*>(chunk + x * 8);
                 const float2 a = bf2_to_f2(w.x), bb = bf2_to_f2(w.y), cc = bf2_to_f2(w.z), dd = bf2_to_f2(w.w);
-                v.x = pack_half2(a.x, a.y);
-                v.y = pack_half2(bb.x, bb.y);
-                v.z = pack_half2(cc.x, cc.y);
-                v.w = pack_half2(dd.x, dd.y);
+                v = make_uint4(pack_half2(a.x, a.y), pack_half2(bb.x, bb.y), pack_half2(cc.x, cc.y),
+                               pack_half2(dd.x, dd.y));
+            } else {
+                const uint8_t* rowp = nullptr;
+                if (paged) {
+                    const int64_t slot = row / c.page_tokens;
+                    const int page = slot < c.max_pages ? c.page_table[size_t(b) * c.max_pages + slot] : -1;
+                    if (page >= 0 && page < c.num_pages)
+                        rowp = base + ((size_t(page) * c.n_r + c.rank[g]) * size_t(c.page_tokens) +
+                                       size_t(row % c.page_tokens)) * row_bytes;
+                    else if (col8 == 0)
+                        atomicOr(reinterpret_cast<int*>(c.status), DUO_STATUS_NO_PAGE);
+                } else {
+                    rowp = base + size_t(row) * row_bytes;
+                }
+                if (rowp && c.fp8) {
+                    const uint2 cc = *reinterpret_cast<const uint2*>(rowp + col8 * 8);
+                    v = keys ? e4m3x8_to_bf16(cc) : e4m3x8_to_f16(cc);
+                } else if (rowp) {
+                    const uint4 w = *reinterpret_cast<const uint4*>(rowp + col8 * 16);
+                    if (keys) {
+                        v = w;                                  // bf16 keys: a copy
+                    } else {
+                        const float2 a = bf2_to_f2(w.x), bb = bf2_to_f2(w.y), cc = bf2_to_f2(w.z),
+                                     dd = bf2_to_f2(w.w);
+                        v = make_uint4(pack_half2(a.x, a.y), pack_half2(bb.x, bb.y), pack_half2(cc.x, cc.y),
+                                       pack_half2(dd.x, dd.y));
+                    }
+                }
             }
         }
         *reinterpret_cast<uint4*>(dst + x * 8) = v;
@@ -419,16 +447,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 const KeyTile kt = plan.get(j);
                 const CUtensorMap* map;
                 int row;
-                // FP8 caches: cached keys come from their bf16 copies (rows LR / LS)
-                const bool copy = !is_k || p.fp8;
+                // FP8 or paged caches: cached keys come from their bf16 copies (rows LR / LS)
+                const bool copy = !is_k || p.kcopy;
                 if (kt.src == kSrcCache) {
-                    map = is_k ? (p.fp8 ? &p.tm_kr16 : &p.tm_kr) : &p.tm_vr;
+                    map = is_k ? (p.kcopy ? &p.tm_kr16 : &p.tm_kr) : &p.tm_vr;
                     row = int((int64_t(b) * p.n_r + kv_rank) * (copy ? int64_t(p.LR) : p.cap) + kt.row0);
                 } else if (kt.src == kSrcChunk) {
                     map = is_k ? &p.tm_kc : &p.tm_vc;
                     row = (b * p.n_kv + g) * p.C + kt.row0;
                 } else {
-                    map = is_k ? (p.fp8 ? &p.tm_ks16 : &p.tm_ks) : &p.tm_vs;
+                    map = is_k ? (p.kcopy ? &p.tm_ks16 : &p.tm_ks) : &p.tm_vs;
                     row = (b * p.n_s + kv_rank) * (copy ? p.LS : p.S + p.W) + (kt.src == kSrcWindow ? p.S : 0) +
                           kt.row0;
                 }
@@ -679,10 +707,11 @@ size_t prefill_smem_bytes(int S, int W) {
     return (1 + kKStages + kVStages) * size_t(kTile) + 1024;
 }
 
-size_t prefill_workspace_bytes(int B, int n_kv, int n_r, int n_s, int64_t cap, int S, int W, int C, bool fp8) {
+size_t prefill_workspace_bytes(int B, int n_kv, int n_r, int n_s, int64_t cap, int S, int W, int C,
+                               bool key_copies) {
     const size_t row = size_t(kHD) * 2;
     const size_t cached = align256(size_t(B) * n_r * rows_r(cap) * row) + align256(size_t(B) * n_s * rows_s(S, W) * row);
-    return cached + align256(size_t(B) * n_kv * C * row) + (fp8 ? cached : 0);   // V copies, chunk V, FP8 key copies
+    return cached + align256(size_t(B) * n_kv * C * row) + (key_copies ? cached : 0);   // V copies, chunk V, key copies
 }
 
 int launch_prefill(const PrefillLaunch& a, cudaStream_t s) {
@@ -701,13 +730,14 @@ int launch_prefill(const PrefillLaunch& a, cudaStream_t s) {
     PrefillParams p;
     memset(&p, 0, sizeof p);
     const int SW = a.S + a.W;
+    const bool kcopy = a.fp8 || a.page_tokens > 0;
     const CUtensorMapDataType BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, F16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     if (!make_map(&p.tm_q, a.q, uint64_t(a.B) * a.hq * a.C, BF) ||
         !make_map(&p.tm_kc, a.k_chunk, uint64_t(a.B) * a.n_kv * a.C, BF) ||
-        (!a.fp8 && !make_map(&p.tm_kr, a.kr, uint64_t(a.B) * a.n_r * a.cap, BF)) ||
-        (!a.fp8 && !make_map(&p.tm_ks, a.ks, uint64_t(a.B) * a.n_s * SW, BF)) ||
-        (a.fp8 && !make_map(&p.tm_kr16, k16r, uint64_t(a.B) * a.n_r * LR, BF)) ||
-        (a.fp8 && !make_map(&p.tm_ks16, k16s, uint64_t(a.B) * a.n_s * LS, BF)) ||
+        (!kcopy && !make_map(&p.tm_kr, a.kr, uint64_t(a.B) * a.n_r * a.cap, BF)) ||
+        (!kcopy && !make_map(&p.tm_ks, a.ks, uint64_t(a.B) * a.n_s * SW, BF)) ||
+        (kcopy && !make_map(&p.tm_kr16, k16r, uint64_t(a.B) * a.n_r * LR, BF)) ||
+        (kcopy && !make_map(&p.tm_ks16, k16s, uint64_t(a.B) * a.n_s * LS, BF)) ||
         !make_map(&p.tm_vc, v16c, uint64_t(a.B) * a.n_kv * a.C, F16) ||
         !make_map(&p.tm_vr, v16r, uint64_t(a.B) * a.n_r * LR, F16) ||
         !make_map(&p.tm_vs, v16s, uint64_t(a.B) * a.n_s * LS, F16))
@@ -724,6 +754,7 @@ int launch_prefill(const PrefillLaunch& a, cudaStream_t s) {
     memcpy(p.rank, a.rank, sizeof p.rank);
     memcpy(p.is_r, a.is_r, sizeof p.is_r);
     p.fp8 = a.fp8;
+    p.kcopy = a.fp8 || a.page_tokens > 0;
     memcpy(p.k_scale, a.k_scale, sizeof p.k_scale);
     memcpy(p.v_scale, a.v_scale, sizeof p.v_scale);
 
@@ -740,12 +771,17 @@ int launch_prefill(const PrefillLaunch& a, cudaStream_t s) {
     memcpy(c.rank, a.rank, sizeof c.rank);
     memcpy(c.is_r, a.is_r, sizeof c.is_r);
     c.fp8 = a.fp8;
-    c.kr8 = static_cast<const uint8_t*>(a.kr);
-    c.ks8 = static_cast<const uint8_t*>(a.ks);
+    c.kr = a.kr;
+    c.ks = a.ks;
     c.k16r = k16r;
     c.k16s = k16s;
+    c.page_tokens = a.page_tokens;
+    c.max_pages = a.max_pages;
+    c.num_pages = a.num_pages;
+    c.page_table = a.page_table;
+    c.status = a.status;
     if (int64_t(a.B) * a.n_kv > 65535) return DUO_ERR_UNSUPPORTED;
-    convert_v_kernel<<<dim3(64, unsigned(a.B * a.n_kv), a.fp8 ? 3 : 2), 256, 0, s>>>(c);
+    convert_v_kernel<<<dim3(64, unsigned(a.B * a.n_kv), p.kcopy ? 3 : 2), 256, 0, s>>>(c);
     if (cudaGetLastError() != cudaSuccess) return DUO_ERR_CUDA;
 
     const size_t smem = prefill_smem_bytes(a.S, a.W);

@@ -73,7 +73,10 @@ enum {
     DUO_STATUS_EMPTY_SEQUENCE = 2,  /* decode with len[b] < 1: output zeroed  */
     DUO_STATUS_WAIT_TIMEOUT = 4,    /* a pipeline wait exceeded its limit:     */
                                     /* the output of that launch is invalid    */
-    DUO_STATUS_BAD_LENGTH = 8       /* negative length or append count         */
+    DUO_STATUS_BAD_LENGTH = 8,      /* negative length or append count         */
+    DUO_STATUS_NO_PAGE = 16         /* paged cache: a retrieval row's page is  */
+                                    /* missing (-1 or >= num_pages): not       */
+                                    /* written / its tile read as zeros        */
 };
 
 /* Element type of the K/V caches. */
@@ -99,7 +102,18 @@ enum {
  * stores code = E4M3(fp32(x) / fp32(scale)) (round to nearest even,
  * saturating at 448) and reads scale * E4M3(code).  k_scale and v_scale are
  * HOST arrays [num_layers][num_kv_heads] of finite positive scales (NULL =
- * all 1.0), copied during duo_kv_alloc.  FP8 needs head_dim 128. */
+ * all 1.0), copied during duo_kv_alloc.  FP8 needs head_dim 128.
+ *
+ * page_tokens > 0 pages the retrieval caches (paged attention, "Attention
+ * Variants and Memory Efficiency", "What the Inference Runtime Can Change":
+ * fixed-size blocks, not contiguous in memory): each layer keeps a pool of
+ * num_pages pages of [n_retrieval][page_tokens][d] elements, one page = the
+ * page_tokens consecutive positions of one sequence for all of the layer's
+ * retrieval heads.  Which page holds which positions is a caller-owned
+ * device table set with duo_kv_set_page_table and shared by all layers.
+ * capacity stays the largest length a sequence may reach (positions are
+ * checked against it).  page_tokens must be a multiple of 256; paging needs
+ * head_dim 128.  0 = one contiguous [capacity] range per sequence and head. */
 typedef struct {
     int32_t num_layers;
     int32_t batch;
@@ -113,6 +127,8 @@ typedef struct {
     int32_t kv_dtype;           /* DUO_KV_BF16 (0) or DUO_KV_FP8_E4M3 (1) */
     const float* k_scale;       /* FP8 only, see above                     */
     const float* v_scale;
+    int32_t page_tokens;        /* 0 = contiguous retrieval caches        */
+    int64_t num_pages;          /* pages per layer pool (page_tokens > 0) */
 } duo_kv_desc;
 
 /* Opaque host-side handle (host memory only). */
@@ -122,7 +138,8 @@ typedef struct duo_kv duo_kv;
  * manage the cache themselves).  Layouts, in elements of the cache's
  * kv_dtype (bf16 bit patterns, or one E4M3 byte each -- the pointers then
  * address bytes):
- *   k_retrieval, v_retrieval: [B][n_retrieval][capacity][d]
+ *   k_retrieval, v_retrieval: [B][n_retrieval][capacity][d], or, paged,
+ *                             the pool [num_pages][n_retrieval][page_tokens][d]
  *   k_streaming, v_streaming: [B][n_streaming][S + W][d]
  *   positions:                [B][S + W] int32, original position of the
  *                             token in each streaming slot, -1 = empty
@@ -324,6 +341,15 @@ DUO_API int duo_prefill_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const
  * and if DUO_STATUS_WAIT_TIMEOUT was set, the decode merge counters too (a
  * launch that gave up may have left them non-zero). */
 DUO_API int duo_kv_read_status(duo_kv* kv, int32_t* status, int32_t clear, duo_stream_t stream);
+
+/* Paged caches: the device table that maps a sequence's positions to pages,
+ * int32 [batch][max_pages]: entry [b][i] is the pool page (0 .. num_pages-1,
+ * the same index in every layer's pool) holding positions
+ * i*page_tokens .. (i+1)*page_tokens - 1 of sequence b, or -1 for none.
+ * The table stays the caller's; the library reads it in later calls
+ * (stream-ordered), so the caller updates it as sequences grow.  Host only;
+ * INVALID_ARG on a contiguous cache or max_pages < 1. */
+DUO_API int duo_kv_set_page_table(duo_kv* kv, const int32_t* d_table, int32_t max_pages);
 
 /* Override the number of CTAs the decode kernel splits the keys over
  * (0 = one persistent wave, the default).  For tests of split invariance;

@@ -167,3 +167,30 @@ def test_fp8_descriptor_checks():
     d, keep = L.make_desc(2, 3, 32, 8, 128, 64, 256, 1000, np.zeros((2, 8), np.uint8).tobytes(),
                           L.DUO_KV_FP8_E4M3, [0.5] * n, [2.0] * n)
     assert L.duo_kv_required_bytes(d)[1] > 0
+
+
+def test_paged_cache_bytes_and_checks():
+    """Paged retrieval caches: each layer's retrieval part is a pool of
+    num_pages pages of n_r x page_tokens rows (streaming rings unchanged)."""
+    L = _lib()
+    layers, B, n_kv, d, S, Wn = 2, 3, 8, 128, 64, 256
+    mask = np.zeros((layers, n_kv), np.uint8)
+    mask[:, ::2] = 1                              # 4 retrieval heads per layer
+    d0, k0 = L.make_desc(layers, B, 32, n_kv, d, S, Wn, 1000, mask.tobytes(), L.DUO_KV_BF16, None, None, 256, 10)
+    _, cache = L.duo_kv_required_bytes(d0)
+    want = layers * (2 * 2 * d * (10 * 4 * 256) + B * 2 * 2 * d * 4 * (S + Wn))
+    assert cache == want
+    d8, k8 = L.make_desc(layers, B, 32, n_kv, d, S, Wn, 1000, mask.tobytes(), L.DUO_KV_FP8_E4M3, None, None, 256,
+                         10)
+    assert L.duo_kv_required_bytes(d8)[1] * 2 == want
+    for pt, npg, code in ((100, 10, L.DUO_ERR_INVALID_ARG), (256, 0, L.DUO_ERR_INVALID_ARG),
+                          (-256, 10, L.DUO_ERR_INVALID_ARG)):
+        dd, kk = L.make_desc(layers, B, 32, n_kv, d, S, Wn, 1000, mask.tobytes(), L.DUO_KV_BF16, None, None, pt,
+                             npg)
+        with pytest.raises(L.DuoError) as e:
+            L.duo_kv_required_bytes(dd)
+        assert e.value.code == code
+    dd, kk = L.make_desc(layers, B, 8, n_kv, 64, S, Wn, 1000, mask.tobytes(), L.DUO_KV_BF16, None, None, 256, 10)
+    with pytest.raises(L.DuoError) as e:
+        L.duo_kv_required_bytes(dd)
+    assert e.value.code == L.DUO_ERR_UNSUPPORTED
