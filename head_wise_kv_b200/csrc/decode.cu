@@ -164,7 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         abort_flag = 0;
         fence_mbar_init();
     }
-    build_prefix(p, bpre);
+    build_prefix<16>(p, bpre);
     __syncthreads();
     // The merge kernel may be scheduled now; it waits (griddepcontrol.wait)
     // for this grid's completion before it reads any partial.
@@ -184,7 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         uint32_t it = 0;
         bool ok = true;
         for (int64_t gb = gb_begin; gb < gb_end && ok;) {
-            const Piece pc = locate(p, bpre, gb, gb_end);
+            const Piece pc = locate<16>(p, bpre, gb, gb_end);
             const uint16_t *kp, *vp;
             seg_ptrs<D>(p, pc.b, pc.g, pc.row0, kp, vp);
             for (int64_t t = pc.tok0; t < pc.tok1; t += kTile, ++it) {
@@ -227,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     const int lo_idx = rs_first<C>(li);   // first (step * G + head) score this lane owns
 
     for (int64_t gb = gb_begin; gb < gb_end;) {
-        const Piece pc = locate(p, bpre, gb, gb_end);
+        const Piece pc = locate<16>(p, bpre, gb, gb_end);
         gb = pc.end_gb;
 
         // q of the G query heads of this KV head, this lane's dims, fp32
@@ -456,7 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 template <int D, int G>
 __global__ void __launch_bounds__(32 * G) merge_kernel(const __grid_constant__ DecodeParams p) {
     extern __shared__ int32_t bpre[];
-    build_prefix(p, bpre);
+    build_prefix<16>(p, bpre);
     __syncthreads();
     const int seg = blockIdx.x;
     const int b = seg / p.n_kv, g = seg % p.n_kv;
@@ -465,7 +465,7 @@ __global__ void __launch_bounds__(32 * G) merge_kernel(const __grid_constant__ D
     float* out = p.out + (size_t(b) * p.hq + qh) * D;
     const int64_t total = bpre[p.B];
     const SeqRows x = seq_rows(p, b);
-    const int nbr = blocks_of(x.nr, p.blk), nbs = blocks_of(x.ns, p.blk);
+    const int nbr = blocks_of<16>(x.nr), nbs = blocks_of<16>(x.ns);
     const int64_t seg_gb = bpre[b] + int64_t(p.r_before[g]) * nbr + int64_t(g - p.r_before[g]) * nbs;
     const int seg_nb = p.is_r[g] ? nbr : nbs;
     const int c0 = seg_nb < 1 ? 0 : cta_owner(seg_gb, total, p.num_ctas);

@@ -16,9 +16,12 @@
 namespace duo {
 namespace {
 
-// Blocks of p.blk tokens (16, or a whole tile for paged caches so that no
-// tile straddles a page).
-__device__ __forceinline__ int blocks_of(int64_t rows, int blk) { return int((rows + blk - 1) / blk); }
+// Blocks of BLK tokens (16, or a whole tile for paged caches so that no
+// tile straddles a page).  BLK is a compile-time constant: a division by a
+// run-time 64-bit value is an out-of-line routine, and code first reached
+// at a piece boundary while HBM is saturated costs microseconds to fetch.
+template <int BLK>
+__device__ __forceinline__ int blocks_of(int64_t rows) { return int((rows + BLK - 1) / BLK); }
 
 __device__ __forceinline__ int64_t rows_r(int len, int64_t cap) {
     int64_t r = len < 0 ? 0 : len;
@@ -74,6 +77,7 @@ __host__ __device__ constexpr size_t seq_table_bytes(int B, int n_kv) {
 __device__ __forceinline__ int seg_units(int nb, int weight) { return nb > 0 ? nb + weight : 0; }
 
 // Fill the table (shared); warp 0 does a chunked shuffle scan.  Caller syncs afterwards.
+template <int BLK>
 __device__ void build_prefix(const DecodeParams& p, int32_t* bpre) {
     if (threadIdx.x >= 32) return;
     const int lane = threadIdx.x;
@@ -84,8 +88,8 @@ __device__ void build_prefix(const DecodeParams& p, int32_t* bpre) {
         int c = 0;
         if (b < p.B) {
             const SeqRows x = seq_rows(p, b);
-            c = p.n_r * seg_units(blocks_of(x.nr, p.blk), p.seg_weight) +
-                p.n_s * seg_units(blocks_of(x.ns, p.blk), p.seg_weight);
+            c = p.n_r * seg_units(blocks_of<BLK>(x.nr), p.seg_weight) +
+                p.n_s * seg_units(blocks_of<BLK>(x.ns), p.seg_weight);
             int32_t* rows = bpre + p.B + 1;
             rows[b] = int32_t(x.r0);
             rows[p.B + b] = int32_t(x.nr);
@@ -129,6 +133,7 @@ struct Piece {
 };
 
 // Locate the piece that starts at global block gb (gb < range end).
+template <int BLK>
 __device__ __forceinline__ Piece locate(const DecodeParams& p, const int32_t* bpre, int64_t gb,
                                         int64_t range_end) {
     Piece pc;
@@ -141,7 +146,7 @@ __device__ __forceinline__ Piece locate(const DecodeParams& p, const int32_t* bp
     pc.b = lo;
     const int32_t* tab = bpre + p.B + 1;
     const int64_t r0 = tab[lo], rr = tab[p.B + lo], rs = tab[2 * p.B + lo];
-    const int nbr = blocks_of(rr, p.blk), nbs = blocks_of(rs, p.blk);
+    const int nbr = blocks_of<BLK>(rr), nbs = blocks_of<BLK>(rs);
     const int ur = seg_units(nbr, p.seg_weight), us = seg_units(nbs, p.seg_weight);
     const int64_t local = gb - bpre[lo];
     const int32_t* hb = bpre + 4 * p.B + 1;
@@ -164,8 +169,8 @@ __device__ __forceinline__ Piece locate(const DecodeParams& p, const int32_t* bp
     const int64_t seg_end = pc.seg_gb + pc.seg_nb;
     pc.end_gb = seg_end < range_end ? seg_end : range_end;
     const int64_t rows = retr ? rr : rs;
-    pc.tok0 = gb > pc.seg_gb ? (gb - pc.seg_gb) * p.blk : 0;
-    const int64_t t1 = (pc.end_gb - pc.seg_gb) * p.blk;
+    pc.tok0 = gb > pc.seg_gb ? (gb - pc.seg_gb) * BLK : 0;
+    const int64_t t1 = (pc.end_gb - pc.seg_gb) * BLK;
     pc.tok1 = t1 < rows ? t1 : rows;
     if (pc.tok1 < pc.tok0) pc.tok1 = pc.tok0;   // the range ends before the segment's first key
     pc.whole = (gb <= pc.seg_gb) && (pc.end_gb == seg_end);
@@ -175,10 +180,11 @@ __device__ __forceinline__ Piece locate(const DecodeParams& p, const int32_t* bp
 // The next piece that holds keys, starting at global block gb (advanced
 // past it); false when the range has none left.  With a segment weight a
 // range may start or end inside a weight, which gives a piece without keys.
+template <int BLK>
 __device__ __forceinline__ bool next_piece(const DecodeParams& p, const int32_t* bpre, int64_t& gb,
                                            int64_t range_end, Piece& pc) {
     while (gb < range_end) {
-        pc = locate(p, bpre, gb, range_end);
+        pc = locate<BLK>(p, bpre, gb, range_end);
         gb = pc.end_gb;
         if (pc.tok1 > pc.tok0) return true;
     }

@@ -169,7 +169,7 @@ __device__ __forceinline__ int tiles_of(const Piece& pc) { return int((pc.tok1 -
 
 // Position in the CTA's sequence of tiles (T keys each): piece `pi` (pc),
 // tile t of its nt; gb is where the search for the next piece starts.
-template <int T>
+template <int T, int BLK>
 struct TileCursor {
     Piece pc;
     int pi, t, nt;
@@ -181,14 +181,14 @@ struct TileCursor {
         pi = 0;
         t = 0;
         gb = gb_begin;
-        valid = next_piece(p, bpre, gb, gb_end, pc);
+        valid = next_piece<BLK>(p, bpre, gb, gb_end, pc);
         if (valid) nt = tiles_of<T>(pc);
     }
     __device__ void advance(const DecodeParams& p, const int32_t* bpre, int64_t gb_end) {
         if (++t < nt) return;
         t = 0;
         ++pi;
-        valid = next_piece(p, bpre, gb, gb_end, pc);
+        valid = next_piece<BLK>(p, bpre, gb, gb_end, pc);
         if (valid) nt = tiles_of<T>(pc);
     }
 };
@@ -219,12 +219,12 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const D
 // A paged tile must start on a page boundary (T divides page_tokens and
 // the pieces start on tile boundaries; a row range must start on a
 // multiple of 256, else DUO_STATUS_BAD_LENGTH).
-template <int T>
+template <int T, bool PAGED>
 __device__ __forceinline__ void tile_coords(const DecodeParams& p, const Piece& pc, int64_t t, int page, int& y,
                                             int& z) {
-    if (pc.retr && p.page_tokens > 0) {
-        const int64_t row = pc.row0 + t;
-        y = int(row % p.page_tokens);
+    if (PAGED && pc.retr) {
+        const uint32_t row = uint32_t(pc.row0 + t);   // < capacity < 2^31: 32-bit arithmetic
+        y = int(row % uint32_t(p.page_tokens));
         if (y + T > p.page_tokens) set_status(p.status, DUO_STATUS_BAD_LENGTH);
         if (page < 0 || page >= p.num_pages) {
             set_status(p.status, DUO_STATUS_NO_PAGE);
@@ -303,9 +303,10 @@ constexpr int kBarSoftmax = 1, kBarEpilogue = 2;
 
 __device__ __forceinline__ uint16_t bf16_bits(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
 
-template <int G, bool F8>
+template <int G, bool F8, bool PAGED>
 __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_constant__ DecodeParams p) {
     using C = Tr<G, F8>;
+    constexpr int BLK = PAGED ? C::T : 16;   // partition block (tokens)
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -375,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     // Launched as a programmatic dependent: everything above overlaps the
     // previous kernel in the stream; nothing it writes is read before this.
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    build_prefix(p, bpre);
+    build_prefix<BLK>(p, bpre);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -395,12 +396,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             if (lane == 0) {
                 const uint64_t policy = l2_evict_first_policy();
                 uint32_t it = 0;
-                bool ok = p.page_tokens <= 0 || timed_wait(smem_addr(&pg_ready), 0, p, abort_flag);
+                bool ok = !PAGED || timed_wait(smem_addr(&pg_ready), 0, p, abort_flag);
                 for (int64_t gb = gb_begin; ok && gb < gb_end;) {
                     Piece pc;
-                    if (!next_piece(p, bpre, gb, gb_end, pc)) break;
+                    if (!next_piece<BLK>(p, bpre, gb, gb_end, pc)) break;
                     const CUtensorMap* mk = pc.retr ? &p.tm_kr : &p.tm_ks;
-                    const bool paged = pc.retr && p.page_tokens > 0;
+                    const bool paged = PAGED && pc.retr;
                     for (int64_t t = pc.tok0; t < pc.tok1; t += C::T, ++it) {
                         const int st = int(it % uint32_t(nst));
                         if (!timed_wait(smem_addr(&empty_k[st]), ((it / nst) & 1) ^ 1, p, abort_flag)) {
@@ -408,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                             break;
                         }
                         int y, z;
-                        tile_coords<C::T>(p, pc, t, paged ? (it < uint32_t(p.pg_cap) ? pg[it] : -1) : 0, y, z);
+                        tile_coords<C::T, PAGED>(p, pc, t, paged ? (it < uint32_t(p.pg_cap) ? pg[it] : -1) : 0, y, z);
                         const uint32_t fk = smem_addr(&full_k[st]);
                         mbar_arrive_expect_tx(fk, kTileBytes);
                         if constexpr (F8) {
@@ -427,19 +428,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             }
         } else if (warp == kQWarp) {
             // ======================================================== q staging
-            if (p.page_tokens > 0) {
+            if constexpr (PAGED) {
                 // Paged caches: look up the pool page of every retrieval tile
                 // now, before HBM is busy (a dependent global read per tile
                 // would stall the producers), in the producers' tile order.
                 uint32_t idx = 0;
                 for (int64_t gb = gb_begin; gb < gb_end;) {
                     Piece pc;
-                    if (!next_piece(p, bpre, gb, gb_end, pc)) break;
+                    if (!next_piece<BLK>(p, bpre, gb, gb_end, pc)) break;
                     const int nt = tiles_of<C::T>(pc);
                     if (pc.retr)
                         for (int k = lane; k < nt; k += 32) {
-                            const int64_t slot = (pc.row0 + pc.tok0 + int64_t(k) * C::T) / p.page_tokens;
-                            const int page = slot < p.max_pages ? p.page_table[size_t(pc.b) * p.max_pages + slot] : -1;
+                            const uint32_t slot = uint32_t(pc.row0 + pc.tok0 + int64_t(k) * C::T) / uint32_t(p.page_tokens);
+                            const int page = slot < uint32_t(p.max_pages) ? p.page_table[size_t(pc.b) * p.max_pages + slot] : -1;
                             if (idx + k < uint32_t(p.pg_cap)) pg[idx + k] = page;
                         }
                     idx += nt;
@@ -452,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             int pi = 0;
             for (int64_t gb = gb_begin; gb < gb_end; ++pi) {
                 Piece pc;
-                if (!next_piece(p, bpre, gb, gb_end, pc)) break;
+                if (!next_piece<BLK>(p, bpre, gb, gb_end, pc)) break;
                 if (!warp_wait(smem_addr(&q_empty[pi & 1]), ((pi >> 1) & 1) ^ 1, p, abort_flag)) break;
                 const uint16_t* qb = p.q + (size_t(pc.b) * p.hq + size_t(pc.g) * G) * kD;
                 const uint32_t qs = sQ + (pi & 1) * C::QB;
@@ -538,12 +539,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             if (lane == 0) {
                 const uint64_t policy = l2_evict_first_policy();
                 uint32_t it = 0;
-                bool ok = p.page_tokens <= 0 || timed_wait(smem_addr(&pg_ready), 0, p, abort_flag);
+                bool ok = !PAGED || timed_wait(smem_addr(&pg_ready), 0, p, abort_flag);
                 for (int64_t gb = gb_begin; ok && gb < gb_end;) {
                     Piece pc;
-                    if (!next_piece(p, bpre, gb, gb_end, pc)) break;
+                    if (!next_piece<BLK>(p, bpre, gb, gb_end, pc)) break;
                     const CUtensorMap* mv = pc.retr ? &p.tm_vr : &p.tm_vs;
-                    const bool paged = pc.retr && p.page_tokens > 0;
+                    const bool paged = PAGED && pc.retr;
                     for (int64_t t = pc.tok0; t < pc.tok1; t += C::T, ++it) {
                         const int st = int(it % uint32_t(nst));
                         if (!timed_wait(smem_addr(&empty_v[st]), ((it / nst) & 1) ^ 1, p, abort_flag)) {
@@ -551,7 +552,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                             break;
                         }
                         int y, z;
-                        tile_coords<C::T>(p, pc, t, paged ? (it < uint32_t(p.pg_cap) ? pg[it] : -1) : 0, y, z);
+                        tile_coords<C::T, PAGED>(p, pc, t, paged ? (it < uint32_t(p.pg_cap) ? pg[it] : -1) : 0, y, z);
                         const uint32_t fv = smem_addr(&full_v[st]);
                         mbar_arrive_expect_tx(fv, kTileBytes);
                         if constexpr (F8) {
@@ -574,7 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             // with it the release of stage j) never waits on the arrival of
             // K_{j+1}.
             if (lane == 0) {
-                TileCursor<C::T> cq, cv;   // next S tile, next PV tile
+                TileCursor<C::T, BLK> cq, cv;   // next S tile, next PV tile
                 cq.start(p, bpre, gb_begin, gb_end);
                 cv.start(p, bpre, gb_begin, gb_end);
                 uint32_t jq = 0, jv = 0;
@@ -671,7 +672,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             int pi = 0;
             for (int64_t gb = gb_begin; gb < gb_end; ++pi) {
                 Piece pc;
-                if (!next_piece(p, bpre, gb, gb_end, pc)) break;
+                if (!next_piece<BLK>(p, bpre, gb, gb_end, pc)) break;
                 const bool got = warp_wait_lazy(smem_addr(&epi_full[pi & 1]), (pi >> 1) & 1, p, abort_flag) &&
                                  warp_wait_lazy(smem_addr(&o_full[pi & 1]), (pi >> 1) & 1, p, abort_flag);
                 if (barrier_any<kBarEpilogue>(!got)) break;
@@ -775,7 +776,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             int pi = 0;
             for (int64_t gb = gb_begin; ok && gb < gb_end; ++pi) {
                 Piece pc;
-                if (!next_piece(p, bpre, gb, gb_end, pc)) break;
+                if (!next_piece<BLK>(p, bpre, gb, gb_end, pc)) break;
                 const uint32_t tmem_o = tmem + lane_off + C::O0 + (pi & 1) * C::OB;
                 float sc = p.scale_log2;   // log2(e) * scale, per score
                 if constexpr (F8) {
@@ -970,16 +971,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     }
 }
 
-template <int G, bool F8>
+template <int G, bool F8, bool PAGED>
 cudaError_t launch_g(const DecodeParams& p, cudaStream_t s) {
     using C = Tr<G, F8>;
     DecodeParams q = p;
     // partition: 16-token blocks, or whole tiles for paged caches (no tile
     // straddles a page); the segment weight is a fixed number of keys
-    q.blk = p.page_tokens > 0 ? C::T : 16;
+    q.blk = PAGED ? C::T : 16;   // the kernel's partition block (kept for the host's bound below)
     q.seg_weight = (F8 ? kSegWeightF8 : kSegWeight) * 16 / q.blk;
     q.pg_cap = 0;
-    if (p.page_tokens > 0) {
+    if (PAGED) {
         // tiles one CTA can see: its share of the largest possible axis, plus
         // one partial tile per piece (at most one piece per segment, plus one)
         const int64_t ur = (p.cap + q.blk - 1) / q.blk + q.seg_weight;
@@ -995,7 +996,7 @@ cudaError_t launch_g(const DecodeParams& p, cudaStream_t s) {
     const size_t smem = fixed + size_t(q.stages) * 2 * kTileBytes;
     if (smem > size_t(227) * 1024) return cudaErrorInvalidConfiguration;
     cudaError_t e =
-        cudaFuncSetAttribute(decode_tc_kernel<G, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        cudaFuncSetAttribute(decode_tc_kernel<G, F8, PAGED>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(unsigned(p.num_ctas));
@@ -1007,7 +1008,7 @@ cudaError_t launch_g(const DecodeParams& p, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<G, F8>, q);
+    e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<G, F8, PAGED>, q);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -1038,23 +1039,21 @@ bool make_decode_maps(DecodeMaps* m, const void* kr, const void* vr, const void*
            make_map3(&m->vs, vs, uint64_t(SW), uint64_t(s_heads), fp8);
 }
 
-cudaError_t launch_decode_tc(const DecodeParams& p, int group, cudaStream_t s) {
-    if (p.fp8) {
-        switch (group) {
-            case 1: return launch_g<1, true>(p, s);
-            case 2: return launch_g<2, true>(p, s);
-            case 4: return launch_g<4, true>(p, s);
-            case 8: return launch_g<8, true>(p, s);
-        }
-    } else {
-        switch (group) {
-            case 1: return launch_g<1, false>(p, s);
-            case 2: return launch_g<2, false>(p, s);
-            case 4: return launch_g<4, false>(p, s);
-            case 8: return launch_g<8, false>(p, s);
-        }
+template <bool F8, bool PAGED>
+cudaError_t launch_group(const DecodeParams& p, int group, cudaStream_t s) {
+    switch (group) {
+        case 1: return launch_g<1, F8, PAGED>(p, s);
+        case 2: return launch_g<2, F8, PAGED>(p, s);
+        case 4: return launch_g<4, F8, PAGED>(p, s);
+        case 8: return launch_g<8, F8, PAGED>(p, s);
     }
     return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_decode_tc(const DecodeParams& p, int group, cudaStream_t s) {
+    const bool paged = p.page_tokens > 0;
+    if (p.fp8) return paged ? launch_group<true, true>(p, group, s) : launch_group<true, false>(p, group, s);
+    return paged ? launch_group<false, true>(p, group, s) : launch_group<false, false>(p, group, s);
 }
 
 }  // namespace duo
