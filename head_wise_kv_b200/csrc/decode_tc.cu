@@ -94,16 +94,21 @@ constexpr int kSegWeightF8 = DUO_DECODE_SEG_WEIGHT_FP8;
 // Shapes of the two element types.
 //   bf16: 128-key tiles; S^T one column per head (q as is); P as hi + lo
 //         bf16 terms, so O^T holds two columns per head.
-//   FP8:  256-key tiles (two 128-key halves of S^T); q and P each as a sum of
-//         four E4M3 terms (~16 significant bits), columns term * G + h; the
-//         products run as kind::f8f6f4 straight on the cached codes.
+//   FP8:  256-key tiles (two 128-key halves of S^T); q as a sum of four
+//         E4M3 terms (~16 significant bits), P rounded to fp16 (11 bits, as
+//         the prefill's P) and split into three E4M3 terms, columns
+//         term * G + h; the products run as kind::f8f6f4 straight on the
+//         cached codes.
 template <int G, bool F8>
 struct Tr {
     static constexpr int T = F8 ? 256 : 128;                       // keys per tile
     static constexpr int HALVES = T / 128;                         // 128-key blocks of S^T
     static constexpr int QT = F8 ? 4 : 1;                          // q terms
-    static constexpr int PT = F8 ? 4 : 2;                          // P terms
-    static constexpr int N = F8 ? ((4 * G + 15) / 16) * 16 : 16;   // MMA N
+    static constexpr int PT = F8 ? 3 : 2;                          // P terms
+    static constexpr int N = F8 ? ((4 * G + 15) / 16) * 16 : 16;   // MMA N (QT * G >= PT * G columns)
+    // O^T columns read back: PT * G rounded up to a power of two (the
+    // columns past PT * G hold zeros: their P^T rows are never written)
+    static constexpr int OL = PT * G <= 2 ? 2 : PT * G <= 4 ? 4 : PT * G <= 8 ? 8 : PT * G <= 16 ? 16 : 32;
     static constexpr uint32_t SB = HALVES * N < 32 ? 32 : HALVES * N;   // TMEM columns of one S buffer
     static constexpr uint32_t OB = N < 32 ? 32 : N;                     // of one O buffer
     static constexpr uint32_t S0 = 0, S1 = SB, O0 = 2 * SB;
@@ -677,8 +682,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                                  warp_wait_lazy(smem_addr(&o_full[pi & 1]), (pi >> 1) & 1, p, abort_flag);
                 if (barrier_any<kBarEpilogue>(!got)) break;
                 tc_fence_after();
-                uint32_t u[C::PT * G];
-                tmem_ldn<C::PT * G>(tmem + lane_off + C::O0 + (pi & 1) * C::OB, u);
+                uint32_t u[C::OL];
+                tmem_ldn<C::OL>(tmem + lane_off + C::O0 + (pi & 1) * C::OB, u);
                 tmem_wait_ld();
                 float L[G], M[G], o[G];
                 const float vs = F8 ? p.v_scale[pc.g] : 1.f;   // FP8: O^T is in value-code units
@@ -851,23 +856,28 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                     // P^T buffer sb is free once PV_{j-2} has completed
                     if (!warp_wait(smem_addr(&p_free[sb]), ((j >> 1) & 1) ^ 1, p, abort_flag)) continue;
                     if constexpr (F8) {
-                        // key `row` (+128) of P^T as four E4M3 terms, rows term * G + h
+                        // keys `row` and `row` + 128 of P^T: P' rounded to fp16, then
+                        // three E4M3 terms peeled off in fp16 (each residual is exact
+                        // in fp16; three 4-bit terms cover its 11 bits); rows term * G + h
                         const uint32_t pb = sP + sb * C::PB + (row & 15);
 #pragma unroll
                         for (int h = 0; h < G; ++h) {
-                            // P' = 2^7 exp2(s - m); 0 off-piece
-                            float r0 = fast_exp2(s[0][h] - m[h] + C::POFF), r1 = fast_exp2(s[1][h] - m[h] + C::POFF);
+                            const float r0 = fast_exp2(s[0][h] - m[h] + C::POFF);   // 0 off-piece
+                            const float r1 = fast_exp2(s[1][h] - m[h] + C::POFF);
                             l[h] += r0 + r1;
+                            uint32_t p16;
+                            asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(p16) : "f"(r1), "f"(r0));
 #pragma unroll
-                            for (int term = 0; term < 4; ++term) {
-                                const uint16_t c2 = e4m3x2(r1, r0);
+                            for (int term = 0; term < 3; ++term) {
+                                uint16_t c2;
+                                asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(c2) : "r"(p16));
                                 const uint32_t off = small_off(term * G + h, row >> 4);
                                 st_shared_u8(pb + off, c2 & 0xffu);
                                 st_shared_u8(pb + C::PHALF + off, uint32_t(c2) >> 8);
-                                if (term < 3) {
-                                    const float2 v = e4m3x2_value(c2);
-                                    r0 -= v.x;
-                                    r1 -= v.y;
+                                if (term < 2) {
+                                    uint32_t dq;
+                                    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(dq) : "h"(c2));
+                                    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(p16) : "r"(p16), "r"(dq));
                                 }
                             }
                         }
@@ -905,15 +915,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                         // rescale O^T (rows = dims) once PV_{j-1} has landed
                         if (!warp_wait(smem_addr(&p_free[(j - 1) & 1]), ((j - 1) >> 1) & 1, p, abort_flag)) continue;
                         tc_fence_after();
-                        uint32_t u[C::PT * G];
-                        tmem_ldn<C::PT * G>(tmem_o, u);
+                        uint32_t u[C::OL];
+                        tmem_ldn<C::OL>(tmem_o, u);
                         tmem_wait_ld();
 #pragma unroll
                         for (int term = 0; term < C::PT; ++term)
 #pragma unroll
                             for (int h = 0; h < G; ++h)
                                 u[term * G + h] = __float_as_uint(__uint_as_float(u[term * G + h]) * alpha[h]);
-                        tmem_stn<C::PT * G>(tmem_o, u);
+                        tmem_stn<C::OL>(tmem_o, u);
                         tmem_wait_st();
                     }
                     tc_fence_before();
