@@ -37,7 +37,7 @@ FALLBACK_HBM_GBS = 6650.0
 DECODE_TRAFFIC_BYTES = 1126346000 + 3740672
 # The same for decode_tc_kernel<4, FP8> on the FP8 cache of this workload
 # (profiles/decode_tc_kernel_fp8_gqa128k.md); None once that kernel changes.
-DECODE_FP8_TRAFFIC_BYTES = None
+DECODE_FP8_TRAFFIC_BYTES = 566144768 + 5809408
 
 
 # ---------------------------------------------------------------- helpers

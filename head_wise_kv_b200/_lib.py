@@ -36,6 +36,7 @@ DUO_STATUS_EMPTY_SEQUENCE = 2
 DUO_STATUS_WAIT_TIMEOUT = 4
 DUO_STATUS_BAD_LENGTH = 8
 DUO_STATUS_NO_PAGE = 16
+DUO_STATUS_SHARED_PAGE = 32
 
 # C entry points declared in include/duo_kv.h (checked by the CPU tests)
 EXPORTED = (
@@ -44,6 +45,7 @@ EXPORTED = (
     "duo_prefill_workspace_bytes", "duo_prefill_attn", "duo_kv_read_status",
     "duo_kv_set_decode_ctas", "duo_strerror", "duo_decode_attn_static_ws",
     "duo_kv_append_rows", "duo_decode_attn_rows", "duo_lse_merge", "duo_alpha_blend", "duo_kv_set_page_table",
+    "duo_kv_fork",
 )
 DUO_STATIC_WS_BYTES = 4 << 20
 
@@ -110,6 +112,7 @@ _c_prefill = _sig("duo_prefill_attn", [_P, _I32, _P, _P, _P, _P, _I32, ctypes.c_
 _c_status = _sig("duo_kv_read_status", [_P, ctypes.POINTER(_I32), _I32, _P])
 _c_set_ctas = _sig("duo_kv_set_decode_ctas", [_P, _I32])
 _c_set_pages = _sig("duo_kv_set_page_table", [_P, _P, _I32])
+_c_fork = _sig("duo_kv_fork", [_P, _I32, _I32, _I32, _P])
 _c_strerror = _sig("duo_strerror", [ctypes.c_int], ctypes.c_char_p)
 
 
@@ -233,3 +236,7 @@ def duo_kv_set_decode_ctas(handle, ctas: int) -> None:
 
 def duo_kv_set_page_table(handle, d_table: int, max_pages: int) -> None:
     _check(_c_set_pages(handle, d_table, max_pages), "duo_kv_set_page_table")
+
+
+def duo_kv_fork(handle, src: int, dst: int, length: int, stream: int) -> None:
+    _check(_c_fork(handle, src, dst, length, stream), "duo_kv_fork")

@@ -89,6 +89,12 @@ class DuoKVCache:
         L.duo_kv_set_page_table(self.handle, table.data_ptr(), table.shape[1])
         self._page_table = table
 
+    def fork(self, src: int, dst: int, length: int):
+        """Sequence dst continues from the first ``length`` tokens of
+        sequence src (every layer).  Paged caches share the pages that the
+        page table maps to the same pool page for both; see duo_kv_fork."""
+        L.duo_kv_fork(self.handle, src, dst, length, _stream(self.device))
+
     def set_decode_ctas(self, ctas: int):
         L.duo_kv_set_decode_ctas(self.handle, ctas)
         self._alloc_workspace()

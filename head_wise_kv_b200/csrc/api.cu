@@ -489,6 +489,43 @@ int duo_kv_set_page_table(duo_kv* kv, const int32_t* d_table, int32_t max_pages)
     return DUO_OK;
 }
 
+int duo_kv_fork(duo_kv* kv, int32_t src, int32_t dst, int32_t len, duo_stream_t stream) {
+    if (!kv || src < 0 || dst < 0 || src >= kv->desc.batch || dst >= kv->desc.batch || src == dst)
+        return DUO_ERR_INVALID_ARG;
+    if (len < 0 || len > kv->desc.capacity) return DUO_ERR_INVALID_ARG;
+    const bool paged = kv->page_tokens > 0;
+    const int units = paged ? (len + kv->page_tokens - 1) / kv->page_tokens : 1;
+    if (paged && len > 0 && (!kv->page_table || units > kv->max_pages)) return DUO_ERR_INVALID_ARG;
+    const int64_t E = kv->fp8 ? 1 : 2;
+    for (int l = 0; l < kv->desc.num_layers; ++l) {
+        const duo::LayerLayout& L = kv->layers[l];
+        duo::ForkParams p{};
+        p.kr = reinterpret_cast<uint8_t*>(kv->base + L.off_kr);
+        p.vr = reinterpret_cast<uint8_t*>(kv->base + L.off_vr);
+        p.ks = reinterpret_cast<uint8_t*>(kv->base + L.off_ks);
+        p.vs = reinterpret_cast<uint8_t*>(kv->base + L.off_vs);
+        p.pos = reinterpret_cast<int32_t*>(kv->base + L.off_pos);
+        p.status = kv->status;
+        p.page_table = kv->page_table;
+        p.cap = kv->desc.capacity;
+        p.row_bytes = int64_t(kv->desc.head_dim) * E;
+        p.num_pages = kv->num_pages;
+        p.src = src;
+        p.dst = dst;
+        p.len = len;
+        p.n_r = L.n_r;
+        p.n_s = L.n_s;
+        p.S = kv->desc.sink;
+        p.W = kv->desc.window;
+        p.page_tokens = kv->page_tokens;
+        p.max_pages = kv->max_pages;
+        p.n_units = len > 0 ? units : 0;
+        const int rc = cuda_err(duo::launch_fork(p, static_cast<cudaStream_t>(stream)));
+        if (rc) return rc;
+    }
+    return DUO_OK;
+}
+
 int duo_kv_set_decode_ctas(duo_kv* kv, int32_t ctas) {
     if (!kv || ctas < 0 || ctas > (1 << 20)) return DUO_ERR_INVALID_ARG;
     kv->decode_ctas = ctas;

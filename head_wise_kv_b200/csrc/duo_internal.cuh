@@ -115,6 +115,24 @@ struct AppendParams {
     float k_scale[kMaxKvHeads], v_scale[kMaxKvHeads];
 };
 
+// Prefix sharing (fork.cu): one layer, sequence src -> dst, first len tokens.
+struct ForkParams {
+    uint8_t* kr;
+    uint8_t* vr;
+    uint8_t* ks;
+    uint8_t* vs;
+    int32_t* pos;
+    int32_t* status;
+    const int32_t* page_table;    // paged caches
+    int64_t cap;                  // contiguous: rows per (sequence, retrieval head)
+    int64_t row_bytes;            // d x bytes per element
+    int64_t num_pages;
+    int src, dst, len;
+    int n_r, n_s, S, W;
+    int page_tokens, max_pages;
+    int n_units;                  // retrieval jobs per head: pages of the prefix, or 1
+};
+
 struct PrefillLaunch {
     const void* q;
     const void* k_chunk;
@@ -143,6 +161,7 @@ struct PrefillLaunch {
 
 // Host-side launchers (defined in the kernel translation units).
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
+cudaError_t launch_fork(const ForkParams& p, cudaStream_t s);
 int decode_ctas_default(int num_sms, int d, int group);
 size_t decode_workspace_bytes(int slots, int d, int group);
 cudaError_t launch_decode(const DecodeParams& p, int d, int group, cudaStream_t s);

@@ -74,9 +74,13 @@ enum {
     DUO_STATUS_WAIT_TIMEOUT = 4,    /* a pipeline wait exceeded its limit:     */
                                     /* the output of that launch is invalid    */
     DUO_STATUS_BAD_LENGTH = 8,      /* negative length or append count         */
-    DUO_STATUS_NO_PAGE = 16         /* paged cache: a retrieval row's page is  */
+    DUO_STATUS_NO_PAGE = 16,        /* paged cache: a retrieval row's page is  */
                                     /* missing (-1 or >= num_pages): not       */
                                     /* written / its tile read as zeros        */
+    DUO_STATUS_SHARED_PAGE = 32     /* duo_kv_fork: the prefix's partly filled */
+                                    /* last page is the same pool page for     */
+                                    /* both sequences (both would append into  */
+                                    /* it): not copied                         */
 };
 
 /* Element type of the K/V caches. */
@@ -350,6 +354,27 @@ DUO_API int duo_kv_read_status(duo_kv* kv, int32_t* status, int32_t clear, duo_s
  * (stream-ordered), so the caller updates it as sequences grow.  Host only;
  * INVALID_ARG on a contiguous cache or max_pages < 1. */
 DUO_API int duo_kv_set_page_table(duo_kv* kv, const int32_t* d_table, int32_t max_pages);
+
+/* Prefix sharing: make sequence dst continue from the first len tokens of
+ * sequence src, in every layer (paged attention's block sharing, "Attention
+ * Variants and Memory Efficiency", "What the Inference Runtime Can Change":
+ * prefix sharing keeps one copy of the blocks of a common prefix).
+ *   src, dst: sequence indices (different, < batch);
+ *   len:      host int, tokens src holds (0 <= len <= capacity); afterwards
+ *             dst holds the same len tokens and appends from position len.
+ * Streaming heads (sinks, ring and position table) are copied.  Retrieval
+ * heads of a contiguous cache copy rows [0, len).  Paged caches: the caller
+ * first sets dst's page-table entries for the prefix's pages; an entry equal
+ * to src's shares that pool page (nothing is copied), any other page
+ * receives a copy of src's rows.  The page holding the last, partly filled
+ * block of the prefix (len not a multiple of page_tokens) must differ
+ * between the two (DUO_STATUS_SHARED_PAGE otherwise); shared pages must not
+ * be written through either sequence afterwards (they hold positions < len,
+ * which appends never revisit).  Sets DUO_STATUS_NO_PAGE for a missing page
+ * and DUO_STATUS_BAD_LENGTH when src's newest ring slot does not hold
+ * position len - 1 (src holds a different number of tokens).  One launch per
+ * layer on `stream`, ordered like appends. */
+DUO_API int duo_kv_fork(duo_kv* kv, int32_t src, int32_t dst, int32_t len, duo_stream_t stream);
 
 /* Override the number of CTAs the decode kernel splits the keys over
  * (0 = one persistent wave, the default).  For tests of split invariance;
