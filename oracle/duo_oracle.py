@@ -48,6 +48,16 @@ The pages fix neither the 8-bit format nor the scaling; readings taken:
     prefill: the cached prefix dequantized, the chunk's own keys and values
     as given, because they are attended before they are appended).
 
+INT4 KV cache (the same passage: 4 bits per element, a 4x footprint
+reduction).  The pages give no integer format or scaling either; readings:
+  * a code is a signed 4-bit integer c in [-8, 7] (two's complement nibble);
+  * the same caller scales as FP8, one per (layer, KV head) for keys and one
+    for values (exactly 4x, as the pages state: no per-group metadata);
+  * c = round-half-to-even of fp32(x) / fp32(scale), clamped to [-8, 7]; the
+    stored value stands for scale * c;
+  * two codes per byte, element 2i in the low nibble of byte i and element
+    2i + 1 in the high nibble.
+
 Parity pins for every function live in ``tests/test_oracle_pins.py``.
 """
 from __future__ import annotations
@@ -61,6 +71,7 @@ __all__ = [
     "StreamingCache", "ring_positions", "keep_set", "key_mask", "kv_head_of",
     "attend", "decode_attention", "prefill_attention", "brute_force_attention", "blended_decode",
     "E4M3_MAX", "e4m3_decode", "e4m3_encode", "quantize_kv", "dequantize_kv",
+    "INT4_MIN", "INT4_MAX", "int4_encode", "int4_pack", "int4_unpack", "quantize_kv_int4", "dequantize_kv_int4",
 ]
 
 
@@ -348,3 +359,44 @@ def quantize_kv(x, scale: float) -> np.ndarray:
 def dequantize_kv(codes, scale: float) -> np.ndarray:
     """Values the cache codes stand for: scale * E4M3(code), float64 (exact)."""
     return float(np.float32(scale)) * e4m3_decode(codes)
+
+
+# ---------------------------------------------------------------- INT4 KV cache
+INT4_MIN, INT4_MAX = -8, 7
+
+
+def int4_encode(x) -> np.ndarray:
+    """Signed 4-bit code of each value of x: the nearest integer (ties to the
+    even one), clamped to [-8, 7]; NaN gives 0.  x as float64 (pass fp32
+    quotients for fp32 inputs)."""
+    x = np.asarray(x, dtype=np.float64)
+    r = np.rint(np.where(np.isnan(x), 0.0, x))          # round half to even
+    return np.clip(r, INT4_MIN, INT4_MAX).astype(np.int8)
+
+
+def int4_pack(codes) -> np.ndarray:
+    """Pack codes [..., d] (d even) two per byte: element 2i in the low
+    nibble of byte i, element 2i + 1 in the high nibble (two's complement)."""
+    c = np.asarray(codes, dtype=np.int64)
+    lo = c[..., 0::2] & 0xF
+    hi = c[..., 1::2] & 0xF
+    return (lo | (hi << 4)).astype(np.uint8)
+
+
+def int4_unpack(packed) -> np.ndarray:
+    """Codes [..., 2n] of packed bytes [..., n], sign-extended from 4 bits."""
+    b = np.asarray(packed, dtype=np.int64) & 0xFF
+    nib = np.stack([b & 0xF, b >> 4], axis=-1).reshape(*b.shape[:-1], 2 * b.shape[-1])
+    return np.where(nib >= 8, nib - 16, nib).astype(np.int8)
+
+
+def quantize_kv_int4(x, scale: float) -> np.ndarray:
+    """Packed INT4 cache bytes [..., d/2] of K or V values x [..., d]: the
+    code of fp32(x) / fp32(scale), the quotient rounded once in fp32."""
+    q = np.asarray(x, dtype=np.float32) / np.float32(scale)
+    return int4_pack(int4_encode(q.astype(np.float64)))
+
+
+def dequantize_kv_int4(packed, scale: float) -> np.ndarray:
+    """Values packed INT4 cache bytes stand for: scale * code, float64 (exact)."""
+    return float(np.float32(scale)) * int4_unpack(packed).astype(np.float64)

@@ -507,3 +507,69 @@ def test_planted_e4m3_ties_away_is_caught(monkeypatch):
     monkeypatch.setattr(O, "e4m3_encode", away)
     with pytest.raises(AssertionError):
         test_e4m3_ties_saturation_nan_and_round_trip()
+
+
+# ------------------------------------------------------------------ INT4 KV codes
+def test_int4_encode_closed_forms():
+    # nearest integer, ties to the even one, clamped to [-8, 7]
+    x = [0.0, 0.49, 0.5, 1.5, 2.5, -0.5, -1.5, -2.5, 3.51, 6.5, 7.4, 7.5, 100.0, -7.5, -8.4, -8.5, -100.0, np.nan]
+    assert list(O.int4_encode(x)) == [0, 0, 0, 2, 2, 0, -2, -2, 4, 6, 7, 7, 7, -8, -8, -8, -8, 0]
+    # every code is reached exactly by its own value
+    assert list(O.int4_encode(np.arange(-8, 8))) == list(range(-8, 8))
+
+
+def test_int4_encode_matches_library_rounding():
+    """torch.round rounds half to even (a library routine); clamp is a clamp."""
+    rng = np.random.default_rng(21)
+    x = np.concatenate([rng.uniform(-10, 10, 20000), np.arange(-10.5, 10.5, 0.5)]).astype(np.float32)
+    lib = torch.from_numpy(x).round().clamp(-8, 7).to(torch.int8).numpy()
+    assert np.array_equal(O.int4_encode(x.astype(np.float64)), lib)
+
+
+def test_int4_pack_layout_and_round_trip():
+    # element 2i in the low nibble, 2i+1 in the high nibble, two's complement
+    assert list(O.int4_pack([1, -1, -8, 7, 0, 3])) == [0xF1, 0x78, 0x30]
+    assert list(O.int4_unpack([0xF1, 0x78, 0x30])) == [1, -1, -8, 7, 0, 3]
+    every = np.array([[a, b] for a in range(-8, 8) for b in range(-8, 8)])      # all 256 bytes
+    packed = O.int4_pack(every)[:, 0]
+    assert sorted(packed.tolist()) == list(range(256))
+    assert np.array_equal(O.int4_unpack(packed[:, None]), every)
+
+
+def test_quantize_kv_int4_is_one_fp32_division_then_rounding():
+    x = torch.randn(4096, dtype=torch.float32).to(torch.bfloat16).float().numpy().reshape(32, 128)
+    for s in (1.0, 0.37, 0.3, 1 / 64):
+        q32 = (torch.from_numpy(x) / torch.tensor(s, dtype=torch.float32)).round().clamp(-8, 7).to(torch.int64)
+        codes = q32.numpy()
+        want = ((codes[:, 0::2] & 0xF) | ((codes[:, 1::2] & 0xF) << 4)).astype(np.uint8)
+        assert np.array_equal(O.quantize_kv_int4(x, s), want)
+        back = O.dequantize_kv_int4(O.quantize_kv_int4(x, s), s)
+        inside = (x / s >= -8.5) & (x / s <= 7.5)
+        # within the grid the error is at most half a step (plus the fp32 division's rounding)
+        assert np.all(np.abs(back[inside] - x[inside]) <= 0.5 * np.float32(s) * (1 + 1e-6) + 1e-12)
+    # a value whose fp32 quotient is an exact tie while the fp64 quotient is
+    # above it: 1.75 / fp32(0.7) is 2.5 in fp32 (code 2), 2.50000004 in fp64 (3)
+    s = np.float32(0.7)
+    v = np.float32(1.75)
+    assert np.float32(v / s) == np.float32(2.5) and float(v) / float(s) > 2.5
+    assert O.int4_unpack(O.quantize_kv_int4(np.array([v, v]), float(s)))[0] == 2
+
+
+def test_planted_int4_ties_away_is_caught(monkeypatch):
+    def wrong(x):
+        x = np.asarray(x, dtype=np.float64)
+        x = np.where(np.isnan(x), 0.0, x)
+        r = np.sign(x) * np.floor(np.abs(x) + 0.5)                       # half away from zero
+        return np.clip(r, -8, 7).astype(np.int8)
+    monkeypatch.setattr(O, "int4_encode", wrong)
+    with pytest.raises(AssertionError):
+        test_int4_encode_closed_forms()
+
+
+def test_planted_int4_nibble_swap_is_caught(monkeypatch):
+    def wrong(codes):
+        c = np.asarray(codes, dtype=np.int64)
+        return ((c[..., 1::2] & 0xF) | ((c[..., 0::2] & 0xF) << 4)).astype(np.uint8)
+    monkeypatch.setattr(O, "int4_pack", wrong)
+    with pytest.raises(AssertionError):
+        test_int4_pack_layout_and_round_trip()
