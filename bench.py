@@ -395,8 +395,10 @@ def run_ours(args, rank, world, local):
 def run_variant_decode(local, kv_dtype="fp8", paged=False, steps=512, warmup=16):
     """The same layer-step (append of the new token + decode) on another
     cache of the same workload: FP8 E4M3 (scales 1.0: the N(0,1) data sits
-    well inside E4M3's range; roofline at one byte per cached element), or a
-    paged cache (256-token pages handed out in a shuffled order)."""
+    well inside E4M3's range; roofline at one byte per cached element), INT4
+    (scales 0.5: about the largest |value| / 7 of the data; roofline at half a
+    byte per element), or a paged cache (256-token pages handed out in a
+    shuffled order)."""
     from head_wise_kv_b200 import DuoKVCache
     dev = torch.device("cuda", local)
     base, gw, lens0 = rank_workload(0, 1)
@@ -405,8 +407,10 @@ def run_variant_decode(local, kv_dtype="fp8", paged=False, steps=512, warmup=16)
     B = base.batch
     page = 256
     per_seq = (cap + page - 1) // page
+    sc = np.full((1, base.n_kv), 0.5, np.float32) if kv_dtype == "int4" else None
     cache = DuoKVCache(1, B, base.hq, base.n_kv, base.d, base.sink, base.window, cap, mask[None], device=dev,
-                       kv_dtype=kv_dtype, page_tokens=page if paged else 0, num_pages=B * per_seq if paged else 0)
+                       kv_dtype=kv_dtype, k_scale=sc, v_scale=sc, page_tokens=page if paged else 0,
+                       num_pages=B * per_seq if paged else 0)
     if paged:
         perm = np.random.default_rng(0).permutation(B * per_seq).astype(np.int32).reshape(B, per_seq)
         table = torch.from_numpy(perm).to(dev)
@@ -425,7 +429,7 @@ def run_variant_decode(local, kv_dtype="fp8", paged=False, steps=512, warmup=16)
         cache.append(0, dk[s], dv[s], lb[s])
         cache.decode(0, dq[s], la[s], base.scale, out=out)
     torch.cuda.synchronize()
-    assert cache.status() == 0, "device status set during the FP8 warm-up"
+    assert cache.status() == 0, "device status set during the warm-up"
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for i in range(steps):                   # layer-steps, events only at the ends
@@ -445,13 +449,14 @@ def run_variant_decode(local, kv_dtype="fp8", paged=False, steps=512, warmup=16)
     torch.cuda.synchronize()
     assert cache.status() == 0, "device status set during the timed region"
     dec_ms = sum(ev[i][0].elapsed_time(ev[i][1]) for i in range(steps)) / steps
-    elem = 1 if kv_dtype == "fp8" else 2
+    elem = {"fp8": 1, "int4": 0.5, "bf16": 2}[kv_dtype]
     nbytes = sum(kv_bytes(lens0 + (i % base.steps) + 1, mask, base.d, base.sink, base.window, cap)
                  for i in range(steps)) / steps * elem / 2
     hbm_peak, peak_kind = peaks()
     achieved = nbytes / (dec_ms * 1e-3) / 1e9
     cache.close()
-    what = ("an FP8 E4M3 cache (retrieval and streaming heads)" if kv_dtype == "fp8" else "a bf16 cache") + \
+    what = {"fp8": "an FP8 E4M3 cache (retrieval and streaming heads)",
+            "int4": "an INT4 cache (retrieval and streaming heads, scales 0.5)", "bf16": "a bf16 cache"}[kv_dtype] + \
         (", retrieval heads paged (256-token pages, shuffled)" if paged else "")
     return {
         "workload": f"gqa128k with {what}, append + decode per layer-step, 32 distinct steps cycled",
@@ -658,9 +663,10 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the chunked-prefill measurement")
-    ap.add_argument("--only", choices=["decode", "prefill", "fp8", "paged"], default=None,
+    ap.add_argument("--only", choices=["decode", "prefill", "fp8", "int4", "paged"], default=None,
                     help="measure one path only (profiling runs)")
-    ap.add_argument("--no-fp8", action="store_true", help="skip the FP8-cache and paged-cache decode measurements")
+    ap.add_argument("--no-fp8", action="store_true",
+                    help="skip the FP8-, INT4- and paged-cache decode measurements")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
     rank, world, local = dist_init()
@@ -673,6 +679,10 @@ def main(argv=None):
             res = ({"metric": "FP8-cache decode",
                     "decode_fp8": run_variant_decode(local, "fp8", False, args.steps, args.warmup)}
                    if rank == 0 else None)
+        elif args.only == "int4":
+            res = ({"metric": "INT4-cache decode",
+                    "decode_int4": run_variant_decode(local, "int4", False, args.steps, args.warmup)}
+                   if rank == 0 else None)
         elif args.only == "paged":
             res = ({"metric": "paged-cache decode",
                     "decode_paged": run_variant_decode(local, "bf16", True, args.steps, args.warmup)}
@@ -683,6 +693,7 @@ def main(argv=None):
                 res["prefill"] = run_prefill(local)
             if world == 1 and not args.no_fp8 and args.only != "decode":
                 res["decode_fp8"] = run_variant_decode(local, "fp8")
+                res["decode_int4"] = run_variant_decode(local, "int4")
                 res["decode_paged"] = run_variant_decode(local, "bf16", True)
             if rank == 0 and world == 1 and not args.no_cpu_baseline:
                 res["cpu_baseline"] = cpu_baseline(ctx)

@@ -30,6 +30,7 @@ DUO_ERR_ALIGNMENT = -6
 
 DUO_KV_BF16 = 0
 DUO_KV_FP8_E4M3 = 1
+DUO_KV_INT4 = 2
 
 DUO_STATUS_OVER_CAPACITY = 1
 DUO_STATUS_EMPTY_SEQUENCE = 2

@@ -32,8 +32,8 @@ class DuoKVCache:
     """Mixed-head KV cache for ``num_layers`` layers and ``batch`` sequences.
 
     retrieval_mask: [num_layers][num_kv_heads] (1 = retrieval KV head).
-    kv_dtype: "bf16" or "fp8" (E4M3 codes; k_scale / v_scale per
-    [num_layers][num_kv_heads], default 1.0).
+    kv_dtype: "bf16", "fp8" (E4M3 codes) or "int4" (signed 4-bit codes, two
+    per byte); k_scale / v_scale per [num_layers][num_kv_heads], default 1.0.
     page_tokens > 0: paged retrieval caches, a pool of num_pages pages per
     layer; the page table (int32 [batch][max_pages] on the device) is given
     with set_page_table.
@@ -51,10 +51,11 @@ class DuoKVCache:
         self.mask = mask.copy()
         self.L, self.B, self.hq, self.n_kv, self.d = num_layers, batch, num_q_heads, num_kv_heads, head_dim
         self.S, self.W, self.cap = sink, window, capacity
-        if kv_dtype not in ("bf16", "fp8"):
-            raise ValueError("kv_dtype must be 'bf16' or 'fp8'")
+        if kv_dtype not in ("bf16", "fp8", "int4"):
+            raise ValueError("kv_dtype must be 'bf16', 'fp8' or 'int4'")
         self.kv_dtype = kv_dtype
         self.fp8 = kv_dtype == "fp8"
+        self.int4 = kv_dtype == "int4"
 
         def scales(x):
             if x is None:
@@ -63,7 +64,8 @@ class DuoKVCache:
         self.k_scale, self.v_scale = scales(k_scale), scales(v_scale)
         self._desc, self._mask_buf = L.make_desc(
             num_layers, batch, num_q_heads, num_kv_heads, head_dim, sink, window, capacity, mask.tobytes(),
-            L.DUO_KV_FP8_E4M3 if self.fp8 else L.DUO_KV_BF16, self.k_scale.ravel().tolist(),
+            {"bf16": L.DUO_KV_BF16, "fp8": L.DUO_KV_FP8_E4M3, "int4": L.DUO_KV_INT4}[kv_dtype],
+            self.k_scale.ravel().tolist(),
             self.v_scale.ravel().tolist(), page_tokens, num_pages)
         self.page_tokens, self.num_pages = page_tokens, num_pages
         self._page_table = None
@@ -115,7 +117,8 @@ class DuoKVCache:
 
     def layer_views(self, layer: int) -> dict:
         """Torch views of one layer's cache regions (see duo_kv_layer_view):
-        bf16 tensors, or uint8 E4M3 codes for an FP8 cache."""
+        bf16 tensors, uint8 E4M3 codes for an FP8 cache, or uint8 bytes of
+        two INT4 codes each (last dimension d / 2) for an INT4 cache."""
         v = L.duo_kv_layer_view_get(self.handle, layer)
         base = self.buf.data_ptr()
         B, d, SW, cap = self.B, self.d, self.S + self.W, self.cap
@@ -124,19 +127,21 @@ class DuoKVCache:
             off = ptr - base
             return self.buf[off:off + nbytes]
         nr, ns = v.n_retrieval, v.n_streaming
-        eb = 1 if self.fp8 else 2
+        quant = self.fp8 or self.int4
+        eb = 1 if quant else 2
+        dl = d // 2 if self.int4 else d          # last dimension of a row in its element type
 
         def typed(t):
-            return t if self.fp8 else t.view(torch.bfloat16)
+            return t if quant else t.view(torch.bfloat16)
         if self.page_tokens > 0:   # the pool [num_pages][n_r][page_tokens][d]
-            shape = (self.num_pages, nr, self.page_tokens, d)
+            shape = (self.num_pages, nr, self.page_tokens, dl)
         else:
-            shape = (B, nr, cap, d)
+            shape = (B, nr, cap, dl)
         n_el = shape[0] * shape[1] * shape[2] * shape[3]
         kr = typed(region(v.k_retrieval, n_el * eb)).view(*shape)
         vr = typed(region(v.v_retrieval, n_el * eb)).view(*shape)
-        ks = typed(region(v.k_streaming, B * ns * SW * d * eb)).view(B, ns, SW, d)
-        vs = typed(region(v.v_streaming, B * ns * SW * d * eb)).view(B, ns, SW, d)
+        ks = typed(region(v.k_streaming, B * ns * SW * dl * eb)).view(B, ns, SW, dl)
+        vs = typed(region(v.v_streaming, B * ns * SW * dl * eb)).view(B, ns, SW, dl)
         pos = region(v.positions, B * SW * 4).view(torch.int32).view(B, SW)
         rank = [v.head_rank[g] for g in range(self.n_kv)]
         is_r = [bool(v.is_retrieval[g]) for g in range(self.n_kv)]

@@ -31,7 +31,8 @@ int check_desc(const duo_kv_desc* d) {
     const int g = d->num_q_heads / d->num_kv_heads;
     if (g != 1 && g != 2 && g != 4 && g != 8) return DUO_ERR_UNSUPPORTED;
     if (d->num_kv_heads > duo::kMaxKvHeads) return DUO_ERR_UNSUPPORTED;
-    if (d->kv_dtype != DUO_KV_BF16 && d->kv_dtype != DUO_KV_FP8_E4M3) return DUO_ERR_INVALID_ARG;
+    if (d->kv_dtype != DUO_KV_BF16 && d->kv_dtype != DUO_KV_FP8_E4M3 && d->kv_dtype != DUO_KV_INT4)
+        return DUO_ERR_INVALID_ARG;
     if (d->page_tokens < 0) return DUO_ERR_INVALID_ARG;
     if (d->page_tokens > 0) {
         if (d->page_tokens % 256 != 0 || d->num_pages < 1) return DUO_ERR_INVALID_ARG;
@@ -39,7 +40,7 @@ int check_desc(const duo_kv_desc* d) {
         // TMA coordinates are int32: pool rows of one page, pages * heads
         if (d->num_pages * int64_t(d->num_kv_heads) >= (int64_t(1) << 31)) return DUO_ERR_UNSUPPORTED;
     }
-    if (d->kv_dtype == DUO_KV_FP8_E4M3) {
+    if (d->kv_dtype != DUO_KV_BF16) {
         if (d->head_dim != 128) return DUO_ERR_UNSUPPORTED;
         const size_t n = size_t(d->num_layers) * d->num_kv_heads;
         for (const float* s : {d->k_scale, d->v_scale})
@@ -62,7 +63,8 @@ size_t plan_layout(const duo_kv_desc* d, std::vector<duo::LayerLayout>* layers, 
     size_t off = header_bytes(d);
     size_t cache = 0;
     const size_t D = size_t(d->head_dim), B = size_t(d->batch), SW = size_t(d->sink) + d->window;
-    const size_t E = d->kv_dtype == DUO_KV_FP8_E4M3 ? 1 : 2;   // bytes per cached element
+    // bytes per cached row: bf16, one E4M3 code per element, or two INT4 codes per byte
+    const size_t RB = d->kv_dtype == DUO_KV_INT4 ? D / 2 : (d->kv_dtype == DUO_KV_FP8_E4M3 ? D : 2 * D);
     for (int l = 0; l < d->num_layers; ++l) {
         duo::LayerLayout L;
         memset(L.rank, 0, sizeof L.rank);
@@ -75,9 +77,9 @@ size_t plan_layout(const duo_kv_desc* d, std::vector<duo::LayerLayout>* layers, 
             L.rank[g] = r ? L.n_r++ : L.n_s++;
         }
         L.r_before[d->num_kv_heads] = L.n_r;
-        const size_t kr = d->page_tokens > 0 ? size_t(d->num_pages) * L.n_r * size_t(d->page_tokens) * D * E
-                                             : B * L.n_r * size_t(d->capacity) * D * E;
-        const size_t ks = B * L.n_s * SW * D * E;
+        const size_t kr = d->page_tokens > 0 ? size_t(d->num_pages) * L.n_r * size_t(d->page_tokens) * RB
+                                             : B * L.n_r * size_t(d->capacity) * RB;
+        const size_t ks = B * L.n_s * SW * RB;
         L.off_kr = off; off = align_up(off + kr);
         L.off_vr = off; off = align_up(off + kr);
         L.off_ks = off; off = align_up(off + ks);
@@ -116,7 +118,8 @@ int duo_kv_alloc(const duo_kv_desc* desc, void* dev_buf, size_t buf_bytes, duo_s
     h->desc = *desc;
     h->desc.retrieval_mask = nullptr;
     h->desc.k_scale = h->desc.v_scale = nullptr;
-    h->fp8 = desc->kv_dtype == DUO_KV_FP8_E4M3;
+    h->fp8 = desc->kv_dtype != DUO_KV_BF16;   // quantised: E4M3 or INT4 codes
+    h->int4 = desc->kv_dtype == DUO_KV_INT4;
     h->page_tokens = desc->page_tokens;
     h->num_pages = desc->num_pages;
     {
@@ -159,7 +162,7 @@ int duo_kv_alloc(const duo_kv_desc* desc, void* dev_buf, size_t buf_bytes, duo_s
                                        h->base + L.off_vs,
                                        paged ? desc->num_pages * L.n_r : int64_t(desc->batch) * L.n_r,
                                        paged ? desc->page_tokens : desc->capacity, int64_t(desc->batch) * L.n_s,
-                                       int(SW), h->fp8 != 0)) {
+                                       int(SW), h->fp8 != 0, h->int4 != 0)) {
                 delete h;
                 return DUO_ERR_CUDA;
             }
@@ -230,6 +233,7 @@ static int append_impl(duo_kv* kv, int32_t layer, const uint16_t* k_new, const u
     memcpy(p.rank, L.rank, sizeof p.rank);
     memcpy(p.is_r, L.is_r, sizeof p.is_r);
     p.fp8 = kv->fp8;
+    p.int4 = kv->int4;
     for (int g = 0; g < kv->desc.num_kv_heads; ++g) {
         p.k_scale[g] = kv->k_scale[size_t(layer) * kv->desc.num_kv_heads + g];
         p.v_scale[g] = kv->v_scale[size_t(layer) * kv->desc.num_kv_heads + g];
@@ -329,6 +333,7 @@ static int decode_impl(duo_kv* kv, int32_t layer, const uint16_t* q, const int32
     memcpy(p.r_before, L.r_before, sizeof p.r_before);
     memcpy(p.is_r, L.is_r, sizeof p.is_r);
     p.fp8 = kv->fp8;
+    p.int4 = kv->int4;
     for (int g = 0; g < kv->desc.num_kv_heads; ++g) {
         p.k_scale[g] = kv->k_scale[size_t(layer) * kv->desc.num_kv_heads + g];
         p.v_scale[g] = kv->v_scale[size_t(layer) * kv->desc.num_kv_heads + g];
@@ -456,6 +461,7 @@ int duo_prefill_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const uint16_
     memcpy(a.rank, L.rank, sizeof a.rank);
     memcpy(a.is_r, L.is_r, sizeof a.is_r);
     a.fp8 = kv->fp8;
+    a.int4 = kv->int4;
     for (int g = 0; g < d.num_kv_heads; ++g) {
         a.k_scale[g] = kv->k_scale[size_t(layer) * d.num_kv_heads + g];
         a.v_scale[g] = kv->v_scale[size_t(layer) * d.num_kv_heads + g];
@@ -496,7 +502,6 @@ int duo_kv_fork(duo_kv* kv, int32_t src, int32_t dst, int32_t len, duo_stream_t 
     const bool paged = kv->page_tokens > 0;
     const int units = paged ? (len + kv->page_tokens - 1) / kv->page_tokens : 1;
     if (paged && len > 0 && (!kv->page_table || units > kv->max_pages)) return DUO_ERR_INVALID_ARG;
-    const int64_t E = kv->fp8 ? 1 : 2;
     for (int l = 0; l < kv->desc.num_layers; ++l) {
         const duo::LayerLayout& L = kv->layers[l];
         duo::ForkParams p{};
@@ -508,7 +513,7 @@ int duo_kv_fork(duo_kv* kv, int32_t src, int32_t dst, int32_t len, duo_stream_t 
         p.status = kv->status;
         p.page_table = kv->page_table;
         p.cap = kv->desc.capacity;
-        p.row_bytes = int64_t(kv->desc.head_dim) * E;
+        p.row_bytes = kv->int4 ? kv->desc.head_dim / 2 : int64_t(kv->desc.head_dim) * (kv->fp8 ? 1 : 2);
         p.num_pages = kv->num_pages;
         p.src = src;
         p.dst = dst;

@@ -42,10 +42,28 @@ __device__ __forceinline__ uint2 e4m3_codes(uint4 x, float scale) {
     return make_uint2(uint32_t(c[0]) | (uint32_t(c[1]) << 16), uint32_t(c[2]) | (uint32_t(c[3]) << 16));
 }
 
+// Eight bf16 values -> their eight INT4 codes, packed two per byte (element
+// 2i in the low nibble of byte i): IEEE fp32 division, round half to even
+// (cvt.rni), clamp to [-8, 7].
+__device__ __forceinline__ uint32_t int4_codes(uint4 x, float scale) {
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    uint32_t out = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int lo = __float2int_rn(__fdiv_rn(__uint_as_float(w[i] << 16), scale));
+        const int hi = __float2int_rn(__fdiv_rn(__uint_as_float(w[i] & 0xffff0000u), scale));
+        const uint32_t cl = uint32_t(min(max(lo, -8), 7)) & 0xFu, ch = uint32_t(min(max(hi, -8), 7)) & 0xFu;
+        out |= (cl | (ch << 4)) << (8 * i);
+    }
+    return out;
+}
+
 // Store 8 elements (16 bytes of bf16) at element offset `dst` of a cache:
-// as given, or as E4M3 codes (8 bytes).
+// as given, as E4M3 codes (8 bytes) or as INT4 codes (4 bytes).
 __device__ __forceinline__ void put8(const AppendParams& p, uint16_t* base, size_t dst, uint4 v, float scale) {
-    if (p.fp8)
+    if (p.int4)
+        *reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(base) + dst / 2) = int4_codes(v, scale);
+    else if (p.fp8)
         *reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(base) + dst) = e4m3_codes(v, scale);
     else
         *reinterpret_cast<uint4*>(base + dst) = v;

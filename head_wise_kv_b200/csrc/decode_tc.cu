@@ -75,6 +75,13 @@ constexpr int kQWarp = 7;
 constexpr int kEpiWarp0 = 8;               // epilogue warps 8-11
 constexpr uint32_t kSlab = 128 * 128;         // 128 rows x 64 bf16: one dim-half of a bf16 tile
 constexpr uint32_t kTileBytes = 32768;        // one K or V tile: 128 bf16 rows or 256 FP8 rows
+// INT4 caches: the producers bring 256-row tiles of packed codes (64 bytes a
+// row) into a staging ring; eight converter warps (12-15 for K, 16-19 for V)
+// expand them to E4M3 in the FP8 tile layout, and the rest of the kernel is
+// the FP8 one.
+constexpr int kConvWarp0 = 12;
+constexpr int kThreadsI4 = 640;
+constexpr uint32_t kTile4Bytes = 16384;       // one K or V tile of 256 INT4 rows
 constexpr float kNegBig = -1.0e30f;
 constexpr float kRescaleThreshold = 8.0f;     // log2 units: probabilities stay <= 2^8
 // Partition weight of a segment start in 16-token blocks: starting a piece
@@ -130,6 +137,33 @@ struct Tr {
     static constexpr uint32_t IPV = idesc_f16(kD, N, !F8, true, false);     // A = V^T (MN-major), B = P^T
     static_assert(QT * G <= N && PT * G <= N, "terms must fit the MMA N");
 };
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+// Eight INT4 codes (two's complement nibbles, element i in bits 4i..4i+3)
+// -> their eight values as E4M3 bytes (exact: every integer in [-8, 7] is an
+// E4M3 value).  Each output byte is assembled from three byte permutes,
+// using the permute's rule that a selector with bit 3 set yields the sign of
+// the chosen byte replicated (0x00 here, as every table byte is positive):
+//   1. selector = the nibble, table E4M3(0..7): the code of c >= 0, else 0;
+//   2. selector = the nibble with bit 3 flipped, table E4M3(|k - 8|), k = 0..7:
+//      the magnitude code of c = k - 8 < 0, else 0;
+//   3. the nibble's sign bit moved to bit 7 of its byte.
+__device__ __forceinline__ uint2 int4x8_to_e4m3(uint32_t w) {
+    constexpr uint32_t kPos0 = 0x44403800u, kPos1 = 0x4E4C4A48u;   // E4M3 of 0, 1, ..., 7
+    constexpr uint32_t kNeg0 = 0x4A4C4E50u, kNeg1 = 0x38404448u;   // E4M3 of 8, 7, ..., 1
+    const uint32_t wx = w ^ 0x88888888u;
+    const uint32_t s_odd = w & 0x80808080u;             // bit 8k+7: sign of element 2k+1
+    const uint32_t s_even = (w << 4) & 0x80808080u;     // bit 8k+7: sign of element 2k
+    uint2 r;
+    r.x = prmt(kPos0, kPos1, w) | prmt(kNeg0, kNeg1, wx) | prmt(s_even, s_odd, 0x5140u);
+    r.y = prmt(kPos0, kPos1, w >> 16) | prmt(kNeg0, kNeg1, wx >> 16) | prmt(s_even, s_odd, 0x7362u);
+    return r;
+}
 
 // Two values -> two E4M3 codes (round to nearest even, saturating); the
 // first operand lands in the upper byte.
@@ -308,19 +342,26 @@ constexpr int kBarSoftmax = 1, kBarEpilogue = 2;
 
 __device__ __forceinline__ uint16_t bf16_bits(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
 
-template <int G, bool F8, bool PAGED>
-__global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_constant__ DecodeParams p) {
+template <int G, bool F8, bool PAGED, bool I4>
+__global__ void __launch_bounds__(I4 ? kThreadsI4 : kThreads, 1)
+    decode_tc_kernel(const __grid_constant__ DecodeParams p) {
     using C = Tr<G, F8>;
+    static_assert(!I4 || F8, "INT4 caches run the FP8 arithmetic");
+    constexpr int NT = I4 ? kThreadsI4 : kThreads;
     constexpr int BLK = PAGED ? C::T : 16;   // partition block (tokens)
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int nst = p.stages;
+    const int ns4 = I4 ? p.stages4 : 0;
     const uint32_t sK = smem_addr(smem);                  // nst K tiles
     const uint32_t sV = sK + nst * kTileBytes;            // nst V tiles
-    const uint32_t sQ = sV + nst * kTileBytes;            // 2 q operands (piece parity)
+    const uint32_t s4K = sV + nst * kTileBytes;           // INT4: ns4 staged K tiles of codes
+    const uint32_t s4V = s4K + ns4 * kTile4Bytes;         //       ns4 staged V tiles
+    const uint32_t sQ = s4V + ns4 * kTile4Bytes;          // 2 q operands (piece parity)
     const uint32_t sP = sQ + 2 * C::QB;                   // 2 P^T operands (tile parity)
-    int32_t* bpre = reinterpret_cast<int32_t*>(smem + 2 * nst * kTileBytes + 2 * C::QB + 2 * C::PB);
+    int32_t* bpre = reinterpret_cast<int32_t*>(smem + 2 * nst * kTileBytes + 2 * ns4 * kTile4Bytes + 2 * C::QB +
+                                               2 * C::PB);
     // paged caches: the pool page of each of this CTA's tiles, in the
     // producers' order (p.pg_cap entries after the sequence table)
     int32_t* pg = bpre + (seq_table_bytes(p.B, p.n_kv) + 15) / 16 * 4;
@@ -329,7 +370,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     __shared__ __align__(8) uint64_t full_k[kMaxStages], full_v[kMaxStages], empty_k[kMaxStages],
         empty_v[kMaxStages], q_full[2],
         q_empty[2], s_full[2], s_free[2], p_full[2], p_free[2], o_full[2], o_empty[2], epi_full[2], mma_fin,
-        qs_full[4], pg_ready;
+        qs_full[4], pg_ready, full4_k[kMaxStages], full4_v[kMaxStages], empty4_k[kMaxStages],
+        empty4_v[kMaxStages];
     // FP8: 2^-a of each piece's q prescale, a ring of four (the q warp runs
     // at most three pieces ahead of the softmax, see the q warp)
     __shared__ float q_scale[4];
@@ -345,10 +387,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < nst; ++s) {
-            mbar_init(smem_addr(&full_k[s]), 1);
-            mbar_init(smem_addr(&full_v[s]), 1);
+            // INT4: an E4M3 tile is full once its four converter warps have arrived
+            mbar_init(smem_addr(&full_k[s]), I4 ? 4 : 1);
+            mbar_init(smem_addr(&full_v[s]), I4 ? 4 : 1);
             mbar_init(smem_addr(&empty_k[s]), 1);
             mbar_init(smem_addr(&empty_v[s]), 1);
+        }
+        for (int s = 0; s < ns4; ++s) {
+            mbar_init(smem_addr(&full4_k[s]), 1);
+            mbar_init(smem_addr(&full4_v[s]), 1);
+            mbar_init(smem_addr(&empty4_k[s]), 4);
+            mbar_init(smem_addr(&empty4_v[s]), 4);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(smem_addr(&q_full[s]), 1);
@@ -368,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         fence_mbar_init();
     }
     // q and P^T rows past the heads in use stay zero (their S / O columns are never read)
-    for (uint32_t o = threadIdx.x * 16; o < 2 * (C::QB + C::PB); o += kThreads * 16)
+    for (uint32_t o = threadIdx.x * 16; o < 2 * (C::QB + C::PB); o += NT * 16)
         st_shared_v4(sQ + o, make_uint4(0, 0, 0, 0));
     fence_proxy_async_smem();
     if (warp == 1) tmem_alloc(smem_addr(&tmem_base_sh), C::COLS);
@@ -408,27 +457,35 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                     const CUtensorMap* mk = pc.retr ? &p.tm_kr : &p.tm_ks;
                     const bool paged = PAGED && pc.retr;
                     for (int64_t t = pc.tok0; t < pc.tok1; t += C::T, ++it) {
-                        const int st = int(it % uint32_t(nst));
-                        if (!timed_wait(smem_addr(&empty_k[st]), ((it / nst) & 1) ^ 1, p, abort_flag)) {
+                        // INT4: the staging ring, filled with codes for the converters
+                        const int nr = I4 ? ns4 : nst;
+                        const int st = int(it % uint32_t(nr));
+                        uint64_t* empty = I4 ? &empty4_k[st] : &empty_k[st];
+                        if (!timed_wait(smem_addr(empty), ((it / nr) & 1) ^ 1, p, abort_flag)) {
                             ok = false;
                             break;
                         }
                         int y, z;
                         tile_coords<C::T, PAGED>(p, pc, t, paged ? (it < uint32_t(p.pg_cap) ? pg[it] : -1) : 0, y, z);
-                        const uint32_t fk = smem_addr(&full_k[st]);
-                        mbar_arrive_expect_tx(fk, kTileBytes);
-                        if constexpr (F8) {
+                        const uint32_t fk = smem_addr(I4 ? &full4_k[st] : &full_k[st]);
+                        if constexpr (I4) {
+                            mbar_arrive_expect_tx(fk, kTile4Bytes);
+                            tma_load_3d(s4K + st * kTile4Bytes, mk, 0, y, z, fk, policy);   // 256 rows x 64 bytes
+                        } else if constexpr (F8) {
+                            mbar_arrive_expect_tx(fk, kTileBytes);
                             tma_load_3d(sK + st * kTileBytes, mk, 0, y, z, fk, policy);   // 256 rows x 128 codes
                         } else {
+                            mbar_arrive_expect_tx(fk, kTileBytes);
                             tma_load_3d(sK + st * kTileBytes, mk, 0, y, z, fk, policy);
                             tma_load_3d(sK + st * kTileBytes + kSlab, mk, 64, y, z, fk, policy);
                         }
                     }
                 }
                 // do not leave while copies may still land in this CTA's shared memory
-                for (uint32_t k = 0; k < uint32_t(nst) && k < it; ++k) {
+                const int nr = I4 ? ns4 : nst;
+                for (uint32_t k = 0; k < uint32_t(nr) && k < it; ++k) {
                     const uint32_t last = it - 1 - k;
-                    mbar_wait(smem_addr(&full_k[last % nst]), (last / nst) & 1, p.timeout_ns);
+                    mbar_wait(smem_addr(I4 ? &full4_k[last % nr] : &full_k[last % nr]), (last / nr) & 1, p.timeout_ns);
                 }
             }
         } else if (warp == kQWarp) {
@@ -551,26 +608,33 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                     const CUtensorMap* mv = pc.retr ? &p.tm_vr : &p.tm_vs;
                     const bool paged = PAGED && pc.retr;
                     for (int64_t t = pc.tok0; t < pc.tok1; t += C::T, ++it) {
-                        const int st = int(it % uint32_t(nst));
-                        if (!timed_wait(smem_addr(&empty_v[st]), ((it / nst) & 1) ^ 1, p, abort_flag)) {
+                        const int nr = I4 ? ns4 : nst;
+                        const int st = int(it % uint32_t(nr));
+                        uint64_t* empty = I4 ? &empty4_v[st] : &empty_v[st];
+                        if (!timed_wait(smem_addr(empty), ((it / nr) & 1) ^ 1, p, abort_flag)) {
                             ok = false;
                             break;
                         }
                         int y, z;
                         tile_coords<C::T, PAGED>(p, pc, t, paged ? (it < uint32_t(p.pg_cap) ? pg[it] : -1) : 0, y, z);
-                        const uint32_t fv = smem_addr(&full_v[st]);
-                        mbar_arrive_expect_tx(fv, kTileBytes);
-                        if constexpr (F8) {
+                        const uint32_t fv = smem_addr(I4 ? &full4_v[st] : &full_v[st]);
+                        if constexpr (I4) {
+                            mbar_arrive_expect_tx(fv, kTile4Bytes);
+                            tma_load_3d(s4V + st * kTile4Bytes, mv, 0, y, z, fv, policy);
+                        } else if constexpr (F8) {
+                            mbar_arrive_expect_tx(fv, kTileBytes);
                             tma_load_3d(sV + st * kTileBytes, mv, 0, y, z, fv, policy);
                         } else {
+                            mbar_arrive_expect_tx(fv, kTileBytes);
                             tma_load_3d(sV + st * kTileBytes, mv, 0, y, z, fv, policy);
                             tma_load_3d(sV + st * kTileBytes + kSlab, mv, 64, y, z, fv, policy);
                         }
                     }
                 }
-                for (uint32_t k = 0; k < uint32_t(nst) && k < it; ++k) {
+                const int nr = I4 ? ns4 : nst;
+                for (uint32_t k = 0; k < uint32_t(nr) && k < it; ++k) {
                     const uint32_t last = it - 1 - k;
-                    mbar_wait(smem_addr(&full_v[last % nst]), (last / nst) & 1, p.timeout_ns);
+                    mbar_wait(smem_addr(I4 ? &full4_v[last % nr] : &full_v[last % nr]), (last / nr) & 1, p.timeout_ns);
                 }
             }
         } else if (warp == 1) {
@@ -666,6 +730,55 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                 // every MMA issued by this thread has completed before TMEM is freed
                 umma_commit(smem_addr(&mma_fin));
                 mbar_wait(smem_addr(&mma_fin), 0, p.timeout_ns);
+            }
+        } else if (I4 && warp >= kConvWarp0) {
+            // ======================================================== INT4 -> E4M3
+            // Warps 12-15 expand the K tiles, 16-19 the V tiles, in the
+            // producers' order.  Thread u of 128 takes the 16-byte pieces u,
+            // u + 128, ... of a staged tile (row r = piece / 4, bytes 16 j ..
+            // 16 j + 15 = dims 32 j .. 32 j + 31) and writes their 32 codes as
+            // the 16-byte chunks 2 j and 2 j + 1 of row r in the layout the FP8
+            // tensor map produces (128-byte rows, chunk c of row r stored at
+            // position c xor (r mod 8)).
+            if constexpr (I4) {
+                const bool is_k = warp < kConvWarp0 + 4;
+                const int ct = (warp - kConvWarp0) % 4 * 32 + lane;
+                const uint32_t src0 = is_k ? s4K : s4V, dst0 = is_k ? sK : sV;
+                uint64_t* full4 = is_k ? full4_k : full4_v;
+                uint64_t* empty4 = is_k ? empty4_k : empty4_v;
+                uint64_t* full8 = is_k ? full_k : full_v;
+                uint64_t* empty8 = is_k ? empty_k : empty_v;
+                uint32_t it = 0;
+                bool ok = true;
+                for (int64_t gb = gb_begin; ok && gb < gb_end;) {
+                    Piece pc;
+                    if (!next_piece<BLK>(p, bpre, gb, gb_end, pc)) break;
+                    for (int64_t t = pc.tok0; t < pc.tok1; t += C::T, ++it) {
+                        const int s4 = int(it % uint32_t(ns4)), st = int(it % uint32_t(nst));
+                        if (!warp_wait(smem_addr(&full4[s4]), (it / ns4) & 1, p, abort_flag) ||
+                            !warp_wait(smem_addr(&empty8[st]), ((it / nst) & 1) ^ 1, p, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint32_t src = src0 + s4 * kTile4Bytes, dst = dst0 + st * kTileBytes;
+#pragma unroll 2
+                        for (int u = ct; u < int(kTile4Bytes / 16); u += 128) {
+                            const int r = u >> 2, j = u & 3;
+                            const uint4 w = ld_shared_v4(src + u * 16);
+                            const uint2 a = int4x8_to_e4m3(w.x), b = int4x8_to_e4m3(w.y);
+                            const uint2 c = int4x8_to_e4m3(w.z), d = int4x8_to_e4m3(w.w);
+                            const uint32_t row = dst + r * 128, sw = r & 7;
+                            st_shared_v4(row + (((2 * j) ^ sw) << 4), make_uint4(a.x, a.y, b.x, b.y));
+                            st_shared_v4(row + (((2 * j + 1) ^ sw) << 4), make_uint4(c.x, c.y, d.x, d.y));
+                        }
+                        fence_proxy_async_smem();   // the tensor cores read the codes through the async proxy
+                        __syncwarp();
+                        if (lane == 0) {
+                            mbar_arrive(smem_addr(&full8[st]));
+                            mbar_arrive(smem_addr(&empty4[s4]));
+                        }
+                    }
+                }
             }
         } else if (warp >= kEpiWarp0) {
             // ======================================================== epilogue
@@ -981,7 +1094,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     }
 }
 
-template <int G, bool F8, bool PAGED>
+template <int G, bool F8, bool PAGED, bool I4>
 cudaError_t launch_g(const DecodeParams& p, cudaStream_t s) {
     using C = Tr<G, F8>;
     DecodeParams q = p;
@@ -1002,15 +1115,17 @@ cudaError_t launch_g(const DecodeParams& p, cudaStream_t s) {
     }
     const size_t fixed = 2 * size_t(C::QB + C::PB) + (seq_table_bytes(p.B, p.n_kv) + 15) / 16 * 16 +
                          size_t(q.pg_cap) * 4 + 1024;
-    q.stages = fixed + 3 * 2 * size_t(kTileBytes) <= size_t(227) * 1024 ? 3 : 2;
-    const size_t smem = fixed + size_t(q.stages) * 2 * kTileBytes;
+    // INT4: two E4M3 stages fed by a two-deep ring of staged codes
+    q.stages = I4 ? 2 : (fixed + 3 * 2 * size_t(kTileBytes) <= size_t(227) * 1024 ? 3 : 2);
+    q.stages4 = I4 ? 2 : 0;
+    const size_t smem = fixed + size_t(q.stages) * 2 * kTileBytes + size_t(q.stages4) * 2 * kTile4Bytes;
     if (smem > size_t(227) * 1024) return cudaErrorInvalidConfiguration;
-    cudaError_t e =
-        cudaFuncSetAttribute(decode_tc_kernel<G, F8, PAGED>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<G, F8, PAGED, I4>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(unsigned(p.num_ctas));
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(I4 ? kThreadsI4 : kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
@@ -1018,52 +1133,56 @@ cudaError_t launch_g(const DecodeParams& p, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<G, F8, PAGED>, q);
+    e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<G, F8, PAGED, I4>, q);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
 // 3-D map over [heads][rows][128 dims] with 128-byte swizzle: bf16 in boxes
-// of 64 dims x 128 rows (two per tile), FP8 codes in boxes of 128 x 256 rows.
-bool make_map3(CUtensorMap* m, const void* base, uint64_t rows, uint64_t heads, bool fp8) {
+// of 64 dims x 128 rows (two per tile), FP8 codes in boxes of 128 x 256 rows;
+// INT4 codes (64 bytes a row) in unswizzled boxes of 64 bytes x 256 rows.
+bool make_map3(CUtensorMap* m, const void* base, uint64_t rows, uint64_t heads, bool fp8, bool int4) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
-    const uint64_t eb = fp8 ? 1 : 2;
+    const uint64_t rb = int4 ? kD / 2 : (fp8 ? kD : 2 * kD);   // bytes per row
+    const uint64_t inner = int4 ? rb : uint64_t(kD);           // elements per row in the map's type
     rows = rows < 1 ? 1 : rows;
-    cuuint64_t dims[3] = {uint64_t(kD), rows, heads < 1 ? 1 : heads};
-    cuuint64_t strides[2] = {uint64_t(kD) * eb, rows * uint64_t(kD) * eb};
-    cuuint32_t box[3] = {fp8 ? 128u : 64u, fp8 ? 256u : 128u, 1};
+    cuuint64_t dims[3] = {inner, rows, heads < 1 ? 1 : heads};
+    cuuint64_t strides[2] = {rb, rows * rb};
+    cuuint32_t box[3] = {int4 ? uint32_t(rb) : (fp8 ? 128u : 64u), fp8 ? 256u : 128u, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     return enc(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base),
-               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               int4 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
 
 bool make_decode_maps(DecodeMaps* m, const void* kr, const void* vr, const void* ks, const void* vs, int64_t r_heads,
-                      int64_t r_rows, int64_t s_heads, int SW, bool fp8) {
-    return make_map3(&m->kr, kr, uint64_t(r_rows), uint64_t(r_heads), fp8) &&
-           make_map3(&m->vr, vr, uint64_t(r_rows), uint64_t(r_heads), fp8) &&
-           make_map3(&m->ks, ks, uint64_t(SW), uint64_t(s_heads), fp8) &&
-           make_map3(&m->vs, vs, uint64_t(SW), uint64_t(s_heads), fp8);
+                      int64_t r_rows, int64_t s_heads, int SW, bool fp8, bool int4) {
+    return make_map3(&m->kr, kr, uint64_t(r_rows), uint64_t(r_heads), fp8, int4) &&
+           make_map3(&m->vr, vr, uint64_t(r_rows), uint64_t(r_heads), fp8, int4) &&
+           make_map3(&m->ks, ks, uint64_t(SW), uint64_t(s_heads), fp8, int4) &&
+           make_map3(&m->vs, vs, uint64_t(SW), uint64_t(s_heads), fp8, int4);
 }
 
-template <bool F8, bool PAGED>
+template <bool F8, bool PAGED, bool I4>
 cudaError_t launch_group(const DecodeParams& p, int group, cudaStream_t s) {
     switch (group) {
-        case 1: return launch_g<1, F8, PAGED>(p, s);
-        case 2: return launch_g<2, F8, PAGED>(p, s);
-        case 4: return launch_g<4, F8, PAGED>(p, s);
-        case 8: return launch_g<8, F8, PAGED>(p, s);
+        case 1: return launch_g<1, F8, PAGED, I4>(p, s);
+        case 2: return launch_g<2, F8, PAGED, I4>(p, s);
+        case 4: return launch_g<4, F8, PAGED, I4>(p, s);
+        case 8: return launch_g<8, F8, PAGED, I4>(p, s);
     }
     return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_decode_tc(const DecodeParams& p, int group, cudaStream_t s) {
     const bool paged = p.page_tokens > 0;
-    if (p.fp8) return paged ? launch_group<true, true>(p, group, s) : launch_group<true, false>(p, group, s);
-    return paged ? launch_group<false, true>(p, group, s) : launch_group<false, false>(p, group, s);
+    if (p.int4) return paged ? launch_group<true, true, true>(p, group, s) : launch_group<true, false, true>(p, group, s);
+    if (p.fp8) return paged ? launch_group<true, true, false>(p, group, s) : launch_group<true, false, false>(p, group, s);
+    return paged ? launch_group<false, true, false>(p, group, s) : launch_group<false, false, false>(p, group, s);
 }
 
 }  // namespace duo

@@ -41,7 +41,8 @@ struct duo_kv {
     int device = 0;
     int num_sms = 0;
     int decode_ctas = 0;                    // 0 = default persistent wave
-    int fp8 = 0;                            // caches hold E4M3 codes
+    int fp8 = 0;                            // caches hold quantised codes (E4M3, or INT4 when int4)
+    int int4 = 0;                           // caches hold packed INT4 codes
     int page_tokens = 0;                    // > 0: paged retrieval caches (pools of num_pages pages)
     int64_t num_pages = 0;
     const int32_t* page_table = nullptr;    // device [B][max_pages], caller-owned
@@ -81,7 +82,9 @@ struct DecodeParams {
     const int32_t* page_table;   // [B][max_pages]
     int pg_cap;                  // tensor-core kernel: entries of its shared page list
     int fp8;                  // caches hold E4M3 codes (tensor-core kernel only)
+    int int4;                 // caches hold packed INT4 codes (with fp8 = 1: the same arithmetic)
     int stages;               // tensor-core kernel pipeline depth (set by its launcher)
+    int stages4;              // INT4: depth of the staged-code ring (set by the launcher)
     float scale_log2;
     unsigned long long timeout_ns;
     int32_t rank[kMaxKvHeads];
@@ -106,6 +109,7 @@ struct AppendParams {
     int64_t cap;
     int B, n_kv, n_r, n_s, S, W, d, n_new_max;
     int fp8;                      // store E4M3 codes of value / scale
+    int int4;                     // store packed INT4 codes of value / scale
     int page_tokens;              // > 0: paged retrieval caches
     int64_t num_pages;
     int max_pages;
@@ -147,7 +151,8 @@ struct PrefillLaunch {
     void* workspace;        // fp16 value copies (and bf16 key copies of an FP8 prefix), prefill_workspace_bytes(...) bytes
     int64_t cap;
     int B, hq, n_kv, C, S, W, n_r, n_s;
-    int fp8;                // cached prefix holds E4M3 codes
+    int fp8;                // cached prefix holds E4M3 codes (or INT4 codes when int4)
+    int int4;
     float k_scale[kMaxKvHeads], v_scale[kMaxKvHeads];
     int page_tokens;        // > 0: paged retrieval caches (prefix gathered into the workspace)
     int64_t num_pages;
@@ -169,7 +174,7 @@ cudaError_t launch_decode_tc(const DecodeParams& p, int group, cudaStream_t s); 
 // Retrieval maps over [B * n_r][cap] rows, or for paged caches over the
 // pool [num_pages * n_r][page_tokens] (pass r_heads = num_pages * n_r, r_rows = page_tokens).
 bool make_decode_maps(DecodeMaps* m, const void* kr, const void* vr, const void* ks, const void* vs, int64_t r_heads,
-                      int64_t r_rows, int64_t s_heads, int SW, bool fp8);
+                      int64_t r_rows, int64_t s_heads, int SW, bool fp8, bool int4);
 cudaError_t launch_lse_merge(int parts, int rows, int d, const float* part_out, const float* part_lse, float* out,
                              float* lse, cudaStream_t s);
 cudaError_t launch_blend(int64_t n, int hq, int d, const float* alpha, const float* full, const float* strm,

@@ -98,6 +98,7 @@ struct ConvertParams {
     uint16_t* k16r;         // bf16 copies of the cached keys [B][n_r][LR][d], [B][n_s][LS][d]
     uint16_t* k16s;
     int fp8;
+    int int4;               // cached codes are packed INT4 (two per byte)
     int page_tokens;        // > 0: retrieval rows live in pages
     int max_pages;
     int64_t num_pages;
@@ -282,10 +283,33 @@ __device__ __forceinline__ uint4 e4m3x8_to_bf16(uint2 c) {
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// Eight INT4 codes (element 2i in the low nibble of byte i) -> their
+// integer values as fp16 or bf16 (exact: |c| <= 8).
+__device__ __forceinline__ int int4_at(uint32_t w, int i) {
+    return int(w << (28 - 4 * i)) >> 28;                  // sign-extend nibble i
+}
+
+__device__ __forceinline__ uint4 int4x8_to_f16(uint32_t w) {
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[i] = pack_half2(float(int4_at(w, 2 * i)), float(int4_at(w, 2 * i + 1)));
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__device__ __forceinline__ uint4 int4x8_to_bf16(uint32_t w) {
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 b = __floats2bfloat162_rn(float(int4_at(w, 2 * i)), float(int4_at(w, 2 * i + 1)));
+        o[i] = *reinterpret_cast<const uint32_t*>(&b);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 // One thread per 8 values (16 bytes of output).  blockIdx.y = b * n_kv + g;
 // blockIdx.z = 0: the head's cached value rows, 1: its chunk's value rows,
-// 2 (FP8 caches only): its cached key rows.  Values become fp16; cached
-// FP8 codes become their (unscaled) values, fp16 for V and bf16 for K -- the
+// 2 (quantised caches only): its cached key rows.  Values become fp16; cached
+// FP8 or INT4 codes become their (unscaled) values, fp16 for V and bf16 for K -- the
 // scales are applied in the attention kernel.  Rows that hold no key (past
 // the prefix or the filled ring slots) up to the end of the last tile the
 // attention reads are written as zeros, so masked columns always meet
@@ -295,8 +319,8 @@ __global__ void __launch_bounds__(256) convert_v_kernel(const __grid_constant__ 
     const int b = bg / c.n_kv, g = bg % c.n_kv;
     const int P = max(c.prefix[b], 0);
     const bool keys = blockIdx.z == 2;
-    const size_t E = c.fp8 ? 1 : 2;                       // bytes per cached element
-    const size_t row_bytes = kHD * E;
+    // bytes per cached row: bf16, E4M3 codes, or INT4 codes two per byte
+    const size_t row_bytes = c.int4 ? kHD / 2 : (c.fp8 ? kHD : 2 * kHD);
     const uint8_t* base = nullptr;                        // cached rows (contiguous) or the page pool
     const uint16_t* chunk = nullptr;
     bool paged = false;
@@ -346,7 +370,10 @@ __global__ void __launch_bounds__(256) convert_v_kernel(const __grid_constant__ 
                 } else {
                     rowp = base + size_t(row) * row_bytes;
                 }
-                if (rowp && c.fp8) {
+                if (rowp && c.int4) {
+                    const uint32_t cc = *reinterpret_cast<const uint32_t*>(rowp + col8 * 4);
+                    v = keys ? int4x8_to_bf16(cc) : int4x8_to_f16(cc);
+                } else if (rowp && c.fp8) {
                     const uint2 cc = *reinterpret_cast<const uint2*>(rowp + col8 * 8);
                     v = keys ? e4m3x8_to_bf16(cc) : e4m3x8_to_f16(cc);
                 } else if (rowp) {
@@ -771,6 +798,7 @@ int launch_prefill(const PrefillLaunch& a, cudaStream_t s) {
     memcpy(c.rank, a.rank, sizeof c.rank);
     memcpy(c.is_r, a.is_r, sizeof c.is_r);
     c.fp8 = a.fp8;
+    c.int4 = a.int4;
     c.kr = a.kr;
     c.ks = a.ks;
     c.k16r = k16r;

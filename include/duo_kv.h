@@ -86,7 +86,8 @@ enum {
 /* Element type of the K/V caches. */
 enum {
     DUO_KV_BF16 = 0,        /* bf16, as given                                  */
-    DUO_KV_FP8_E4M3 = 1     /* FP8 E4M3 codes with per-(layer, KV head) scales  */
+    DUO_KV_FP8_E4M3 = 1,    /* FP8 E4M3 codes with per-(layer, KV head) scales  */
+    DUO_KV_INT4 = 2         /* INT4 codes, two per byte, same scales            */
 };
 
 /* Cache shape.  retrieval_mask is a HOST array [num_layers][num_kv_heads],
@@ -108,6 +109,12 @@ enum {
  * HOST arrays [num_layers][num_kv_heads] of finite positive scales (NULL =
  * all 1.0), copied during duo_kv_alloc.  FP8 needs head_dim 128.
  *
+ * kv_dtype = DUO_KV_INT4 stores each element in 4 bits (the same passage: a
+ * 4x cut): code c = round-half-to-even(fp32(x) / fp32(scale)) clamped to
+ * [-8, 7], two's complement, two codes per byte (element 2i in the low
+ * nibble of byte i, 2i + 1 in the high nibble); the cache reads scale * c.
+ * Same scale arrays and head_dim 128 requirement as FP8.
+ *
  * page_tokens > 0 pages the retrieval caches (paged attention, "Attention
  * Variants and Memory Efficiency", "What the Inference Runtime Can Change":
  * fixed-size blocks, not contiguous in memory): each layer keeps a pool of
@@ -128,8 +135,8 @@ typedef struct {
     int32_t window;
     int64_t capacity;
     const uint8_t* retrieval_mask;
-    int32_t kv_dtype;           /* DUO_KV_BF16 (0) or DUO_KV_FP8_E4M3 (1) */
-    const float* k_scale;       /* FP8 only, see above                     */
+    int32_t kv_dtype;           /* DUO_KV_BF16 (0), DUO_KV_FP8_E4M3 (1) or DUO_KV_INT4 (2) */
+    const float* k_scale;       /* FP8 / INT4 only, see above              */
     const float* v_scale;
     int32_t page_tokens;        /* 0 = contiguous retrieval caches        */
     int64_t num_pages;          /* pages per layer pool (page_tokens > 0) */

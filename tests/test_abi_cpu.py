@@ -169,6 +169,40 @@ def test_fp8_descriptor_checks():
     assert L.duo_kv_required_bytes(d)[1] > 0
 
 
+@pytest.mark.parametrize("cfg", ["mha32k", "gqa128k", "mtok"])
+def test_int4_cache_bytes_follow_memory_equation_at_half_a_byte(cfg):
+    """INT4 caches: the memory equation with 4 bits per element (the guide's
+    4x cut), i.e. a quarter of the bf16 bytes."""
+    L = _lib()
+    w = W.WORKLOADS[cfg]
+    masks = W.retrieval_masks(w)
+    cap = W.capacity(w)
+    d, keep = L.make_desc(w.layers, w.batch, w.hq, w.n_kv, w.d, w.sink, w.window, cap, masks.tobytes(),
+                          L.DUO_KV_INT4)
+    _, cache = L.duo_kv_required_bytes(d)
+    want = w.batch * O.duo_cache_bytes(w.layers, w.n_kv, w.d, cap, w.sink, w.window, masks.sum(1).tolist(),
+                                       elem_bytes=0.5)
+    assert cache == want
+    d16, keep16 = L.make_desc(w.layers, w.batch, w.hq, w.n_kv, w.d, w.sink, w.window, cap, masks.tobytes())
+    assert 4 * cache == L.duo_kv_required_bytes(d16)[1]
+
+
+def test_int4_descriptor_checks():
+    L = _lib()
+    n = 2 * 8
+    d, keep = _desc(L, d=64, hq=8)
+    d.kv_dtype = L.DUO_KV_INT4
+    with pytest.raises(L.DuoError) as e:
+        L.duo_kv_required_bytes(d)
+    assert e.value.code == L.DUO_ERR_UNSUPPORTED
+    mask = np.zeros((2, 8), np.uint8)
+    d, keep = L.make_desc(2, 3, 32, 8, 128, 64, 256, 1000, mask.tobytes(), L.DUO_KV_INT4, None,
+                          [1.0] * (n - 1) + [0.0])
+    with pytest.raises(L.DuoError) as e:
+        L.duo_kv_required_bytes(d)
+    assert e.value.code == L.DUO_ERR_INVALID_ARG
+
+
 def test_paged_cache_bytes_and_checks():
     """Paged retrieval caches: each layer's retrieval part is a pool of
     num_pages pages of n_r x page_tokens rows (streaming rings unchanged)."""
