@@ -146,22 +146,23 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 
 // Eight INT4 codes (two's complement nibbles, element i in bits 4i..4i+3)
 // -> their eight values as E4M3 bytes (exact: every integer in [-8, 7] is an
-// E4M3 value).  Each output byte is assembled from three byte permutes,
-// using the permute's rule that a selector with bit 3 set yields the sign of
-// the chosen byte replicated (0x00 here, as every table byte is positive):
-//   1. selector = the nibble, table E4M3(0..7): the code of c >= 0, else 0;
-//   2. selector = the nibble with bit 3 flipped, table E4M3(|k - 8|), k = 0..7:
-//      the magnitude code of c = k - 8 < 0, else 0;
-//   3. the nibble's sign bit moved to bit 7 of its byte.
+// E4M3 value), four per byte permute.  A permute selector with bit 3 set
+// yields the sign of the chosen byte replicated, so with the nibble itself
+// as the selector:
+//   table E4M3(0..7) (signs 0):            the code of c >= 0, else 0x00;
+//   nibble xor 8, table E4M3(-8..-1):      the code of c < 0, else 0xFF;
+//   bytes whose bit 7 is the sign of each element, replicated: 0xFF for c < 0;
+// and code = first | (second & third).  The right shift by 16 runs as a
+// multiply-high and the left shift as a multiply, off the integer pipe.
 __device__ __forceinline__ uint2 int4x8_to_e4m3(uint32_t w) {
     constexpr uint32_t kPos0 = 0x44403800u, kPos1 = 0x4E4C4A48u;   // E4M3 of 0, 1, ..., 7
-    constexpr uint32_t kNeg0 = 0x4A4C4E50u, kNeg1 = 0x38404448u;   // E4M3 of 8, 7, ..., 1
-    const uint32_t wx = w ^ 0x88888888u;
-    const uint32_t s_odd = w & 0x80808080u;             // bit 8k+7: sign of element 2k+1
-    const uint32_t s_even = (w << 4) & 0x80808080u;     // bit 8k+7: sign of element 2k
+    constexpr uint32_t kNeg0 = 0xCACCCED0u, kNeg1 = 0xB8C0C4C8u;   // E4M3 of -8, -7, ..., -1
+    const uint32_t hi = __umulhi(w, 0x10000u);                      // w >> 16: elements 4..7
+    const uint32_t w4 = w * 16u;                                    // bit 8k+7: sign of element 2k
+    const uint32_t wx = w ^ 0x88888888u, hx = hi ^ 0x8888u;
     uint2 r;
-    r.x = prmt(kPos0, kPos1, w) | prmt(kNeg0, kNeg1, wx) | prmt(s_even, s_odd, 0x5140u);
-    r.y = prmt(kPos0, kPos1, w >> 16) | prmt(kNeg0, kNeg1, wx >> 16) | prmt(s_even, s_odd, 0x7362u);
+    r.x = prmt(kPos0, kPos1, w) | (prmt(kNeg0, kNeg1, wx) & prmt(w4, w, 0xD9C8u));
+    r.y = prmt(kPos0, kPos1, hi) | (prmt(kNeg0, kNeg1, hx) & prmt(w4, w, 0xFBEAu));
     return r;
 }
 
@@ -761,6 +762,8 @@ __global__ void __launch_bounds__(I4 ? kThreadsI4 : kThreads, 1)
                             break;
                         }
                         const uint32_t src = src0 + s4 * kTile4Bytes, dst = dst0 + st * kTileBytes;
+                        // every code is consumed (stored) before the staging slot is
+                        // handed back to the producer
 #pragma unroll 2
                         for (int u = ct; u < int(kTile4Bytes / 16); u += 128) {
                             const int r = u >> 2, j = u & 3;
