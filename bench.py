@@ -38,6 +38,8 @@ DECODE_TRAFFIC_BYTES = 1126346000 + 3740672
 # The same for decode_tc_kernel<4, FP8> on the FP8 cache of this workload
 # (profiles/decode_tc_kernel_fp8_gqa128k.md); None once that kernel changes.
 DECODE_FP8_TRAFFIC_BYTES = 566144768 + 5809408
+# The same for the INT4 instantiation (profiles/decode_tc_kernel_int4_gqa128k.md).
+DECODE_INT4_TRAFFIC_BYTES = 283192320 + 3347456
 
 
 # ---------------------------------------------------------------- helpers
@@ -467,7 +469,8 @@ def run_variant_decode(local, kv_dtype="fp8", paged=False, steps=512, warmup=16)
         "roofline": {"bound": "hbm", "kernel": f"decode_tc_kernel {kv_dtype}{' paged' if paged else ''}",
                      "achieved": round(achieved, 1), "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4),
-                     "traffic": DECODE_FP8_TRAFFIC_BYTES if (kv_dtype == "fp8" and not paged) else None,
+                     "traffic": None if paged else {"fp8": DECODE_FP8_TRAFFIC_BYTES,
+                                                     "int4": DECODE_INT4_TRAFFIC_BYTES}.get(kv_dtype),
                      "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch"},
         "gpu_launches": 2 * steps,
     }
