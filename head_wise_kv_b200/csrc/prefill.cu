@@ -236,6 +236,9 @@ __device__ __forceinline__ bool timed_wait(uint32_t bar, uint32_t parity, const 
 // Lane 0 waits on the mbarrier for the warp (fewer shared-memory polls).
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const PrefillParams& p,
                                           volatile int* abort_flag) {
+    // fast path: the phase has completed already (each lane probes it; a
+    // phase, once completed, stays so until this warp consumes it)
+    if (__all_sync(0xffffffffu, mbar_test_wait(bar, parity))) return true;
     int ok = 1;
     if ((threadIdx.x & 31) == 0) ok = timed_wait(bar, parity, p, abort_flag) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
