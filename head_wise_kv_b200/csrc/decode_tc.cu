@@ -243,13 +243,22 @@ __device__ __forceinline__ bool timed_wait(uint32_t bar, uint32_t parity, const 
 }
 
 // Lane 0 waits for the warp.
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const DecodeParams& p,
-                                          volatile int* abort_flag) {
+// Lane 0 waits (bounded), the warp takes its verdict.
+__device__ __forceinline__ bool warp_wait_lead(uint32_t bar, uint32_t parity, const DecodeParams& p,
+                                               volatile int* abort_flag) {
     int ok = 1;
     if ((threadIdx.x & 31) == 0) ok = timed_wait(bar, parity, p, abort_flag) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
     __syncwarp();
     return ok != 0;
+}
+
+// The same with a fast path for a phase that has completed already (each
+// lane probes it): for waits that usually find their data there.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const DecodeParams& p,
+                                          volatile int* abort_flag) {
+    if (__all_sync(0xffffffffu, mbar_test_wait(bar, parity))) return true;
+    return warp_wait_lead(bar, parity, p, abort_flag);
 }
 
 // TMA coordinates of the tile that starts t keys into a piece: (row, head)
@@ -756,8 +765,8 @@ __global__ void __launch_bounds__(I4 ? kThreadsI4 : kThreads, 1)
                     if (!next_piece<BLK>(p, bpre, gb, gb_end, pc)) break;
                     for (int64_t t = pc.tok0; t < pc.tok1; t += C::T, ++it) {
                         const int s4 = int(it % uint32_t(ns4)), st = int(it % uint32_t(nst));
-                        if (!warp_wait(smem_addr(&full4[s4]), (it / ns4) & 1, p, abort_flag) ||
-                            !warp_wait(smem_addr(&empty8[st]), ((it / nst) & 1) ^ 1, p, abort_flag)) {
+                        if (!warp_wait_lead(smem_addr(&full4[s4]), (it / ns4) & 1, p, abort_flag) ||
+                            !warp_wait_lead(smem_addr(&empty8[st]), ((it / nst) & 1) ^ 1, p, abort_flag)) {
                             ok = false;
                             break;
                         }
