@@ -557,7 +557,7 @@ def run_prefill(local, reps=3):
                      "peak": sustained, "peak_kind": f"{kind} sustained bf16", "unit": "TFLOP/s",
                      "frac": round(tflops / sustained, 4), "frac_of_burst": round(tflops / burst, 4),
                      "traffic": None},
-        "gpu_launches": 2 * n_chunks * reps,
+        "gpu_launches": 4 * n_chunks * reps,   # per chunk: V conversion, attention, split merge, append
     }
 
 

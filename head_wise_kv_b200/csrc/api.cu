@@ -394,7 +394,7 @@ static size_t prefill_ws(const duo_kv* kv, int32_t chunk) {
         n_s = std::max(n_s, L.n_s);
     }
     const duo_kv_desc& d = kv->desc;
-    return duo::prefill_workspace_bytes(d.batch, d.num_kv_heads, n_r, n_s, d.capacity, d.sink, d.window, chunk,
+    return duo::prefill_workspace_bytes(d.batch, d.num_q_heads, d.num_kv_heads, n_r, n_s, d.capacity, d.sink, d.window, chunk,
                                         kv->fp8 != 0 || kv->page_tokens > 0);
 }
 

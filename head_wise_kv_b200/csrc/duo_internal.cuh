@@ -180,7 +180,7 @@ cudaError_t launch_lse_merge(int parts, int rows, int d, const float* part_out, 
 cudaError_t launch_blend(int64_t n, int hq, int d, const float* alpha, const float* full, const float* strm,
                          float* out, cudaStream_t s);
 size_t prefill_smem_bytes(int S, int W);
-size_t prefill_workspace_bytes(int B, int n_kv, int n_r, int n_s, int64_t cap, int S, int W, int C,
+size_t prefill_workspace_bytes(int B, int hq, int n_kv, int n_r, int n_s, int64_t cap, int S, int W, int C,
                                bool key_copies);   // key copies: FP8 or paged caches
 int launch_prefill(const PrefillLaunch& a, cudaStream_t s);   // returns a DUO_* code
 

@@ -62,6 +62,11 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO = 256, kTmemP = 384;
 constexpr float kNegBig = -1.0e30f;
 constexpr float kRescaleThreshold = 8.0f;    // log2 units
+// A retrieval query tile with at least this many key tiles is shared by two
+// CTAs (the first and the second half of its keys), so that the last wave of
+// a launch is made of shorter pieces; their partial outputs are combined by
+// log-sum-exp in merge_parts_kernel.
+constexpr int kSplitMin = 128;
 
 // Instruction descriptors: S = Q K^T in bf16 (both K-major), O += P V in fp16
 // (P from TMEM, V MN-major); M = 128, N = 128.
@@ -74,6 +79,8 @@ struct PrefillParams {
     CUtensorMap tm_vc, tm_vr, tm_vs;            // fp16 copies of the values (workspace)
     const int32_t* prefix;
     float* out;
+    float* part_o;          // [2][B][hq][C][d] normalised partial outputs of split query tiles
+    float* part_lse;        // [2][B][hq][C] their log2-sum-exp (scaled scores)
     int32_t* status;
     int64_t cap;
     int B, hq, n_kv, G, C, n_qt, S, W, n_r, n_s, LR, LS;
@@ -136,7 +143,8 @@ struct Plan {
     int n_w;           // window tiles (streaming)
     int nw_rows;       // filled window slots
     int c0_lo, c0_hi, c1_lo, c1_hi;   // chunk tile ranges (inclusive; empty if lo > hi)
-    int n;
+    int n;             // tiles this CTA visits
+    int jb;            // index of its first tile in the row's order (split query tiles)
 
     __device__ void init(bool is_retrieval, int P_, int i0_, int C_, int S_, int W_) {
         retr = is_retrieval;
@@ -165,10 +173,22 @@ struct Plan {
             }
         }
         n = n_a + n_w + (c0_hi - c0_lo + 1) + (c1_hi >= c1_lo ? c1_hi - c1_lo + 1 : 0);
+        jb = 0;
     }
+
+    // Keep only the first (part 0) or second (part 1) half of the tiles.
+    __device__ void take_half(int part) {
+        const int h = n / 2;
+        jb = part ? h : 0;
+        n = part ? n - h : h;
+    }
+
+    // Tile j of this CTA holds cached keys (they come first).
+    __device__ bool cached(int j) const { return j + jb < n_a + n_w; }
 
     __device__ KeyTile get(int j) const {
         KeyTile t;
+        j += jb;
         if (j < n_a) {
             t.src = retr ? kSrcCache : kSrcSink;
             t.row0 = j * kBN;
@@ -418,7 +438,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
 
     // ---------------------------------------------------------------- work item
     const int per_qt = p.B * p.hq;
-    const int qt = p.n_qt - 1 - int(blockIdx.x) / per_qt;   // heaviest query tiles first
+    const int qt = p.n_qt - 1 - int(blockIdx.x) / (2 * per_qt);   // heaviest query tiles first
+    const int part = (int(blockIdx.x) / per_qt) & 1;                // share of a split query tile
     const int rem = int(blockIdx.x) % per_qt;
     const int h = rem % p.hq, b = rem / p.hq;
     const int g = h / p.G;
@@ -427,6 +448,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     const bool retr = p.is_r[g] != 0;
     Plan plan;
     plan.init(retr, P < 0 ? 0 : P, i0, p.C, p.S, p.W);
+    const bool split = retr && plan.n >= kSplitMin;
+    if (part == 1 && !split) return;   // the whole CTA leaves before any set-up
+    if (split) plan.take_half(part);
 
     if (threadIdx.x == 0) {
         mbar_init(smem_addr(&bar_q), 1);
@@ -627,7 +651,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             if (softmax_barrier_any(!got || *abort_flag)) { ok = false; break; }
             mx = fmaxf(red_max[st][0][r], red_max[st][1][r]);
 
-            const bool cached = F8 && j < plan.n_a + plan.n_w;   // tiles of the cache come first
+            const bool cached = F8 && plan.cached(j);   // tiles of the cache come first
             const float fs = cached ? p.scale_log2 * ksc : p.scale_log2;   // score factor of this tile
             const float mt = mx * fs;                    // factor > 0 keeps the order
             const bool grow = mt > m + kRescaleThreshold;
@@ -683,7 +707,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 tc_fence_after();
                 const float lt = red_l[0][r] + red_l[1][r];
                 const float inv = lt > 0.f ? 1.f / lt : 0.f;
-                float* dst = p.out + ((size_t(b) * p.hq + h) * p.C + i) * kHD + cb;
+                // a split query tile leaves its normalised half and the row's
+                // log2-sum-exp for merge_parts_kernel
+                const size_t row = (size_t(split ? part * p.B + b : b) * p.hq + h) * p.C + i;
+                float* dst = (split ? p.part_o : p.out) + row * kHD + cb;
+                if (split && hf == 0 && i < p.C) p.part_lse[row] = lt > 0.f ? m + __log2f(lt) : -CUDART_INF_F;
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     uint32_t u[32];
@@ -707,6 +735,44 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+}
+
+// ------------------------------------------------------------------ split merge
+struct MergeParams {
+    const float* part_o;
+    const float* part_lse;
+    float* out;
+    const int32_t* prefix;
+    int B, hq, G, C, S, W;
+    uint8_t is_r[kMaxKvHeads];
+};
+
+// One warp per query row of a split query tile: out = sum_p w_p o_p / sum_p w_p
+// with w_p = 2^(lse_p - max lse), the log-sum-exp combination of two
+// attentions over disjoint key sets.  Rows of unsplit tiles were written by
+// the attention kernel and are left alone (the same split rule decides).
+__global__ void __launch_bounds__(256) merge_parts_kernel(const __grid_constant__ MergeParams a) {
+    const int64_t row = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;   // (b, h, i)
+    const int lane = threadIdx.x & 31;
+    if (row >= int64_t(a.B) * a.hq * a.C) return;
+    const int i = int(row % a.C);
+    const int h = int((row / a.C) % a.hq), b = int(row / (int64_t(a.C) * a.hq));
+    const bool retr = a.is_r[h / a.G] != 0;
+    if (!retr) return;
+    const int P = a.prefix[b];
+    Plan plan;
+    plan.init(true, P < 0 ? 0 : P, i / kBM * kBM, a.C, a.S, a.W);
+    if (plan.n < kSplitMin || P < 0) return;
+    const size_t r0 = size_t(row), r1 = size_t(a.B) * a.hq * a.C + r0;
+    const float l0 = a.part_lse[r0], l1 = a.part_lse[r1];
+    const float mx = fmaxf(l0, l1);
+    const float w0 = exp2f(l0 - mx), w1 = exp2f(l1 - mx);
+    const float inv = 1.f / (w0 + w1);
+    const float4 o0 = reinterpret_cast<const float4*>(a.part_o + r0 * kHD)[lane];
+    const float4 o1 = reinterpret_cast<const float4*>(a.part_o + r1 * kHD)[lane];
+    reinterpret_cast<float4*>(a.out + r0 * kHD)[lane] =
+        make_float4((w0 * o0.x + w1 * o1.x) * inv, (w0 * o0.y + w1 * o1.y) * inv, (w0 * o0.z + w1 * o1.z) * inv,
+                    (w0 * o0.w + w1 * o1.w) * inv);
 }
 
 // ------------------------------------------------------------------ host side
@@ -737,11 +803,13 @@ size_t prefill_smem_bytes(int S, int W) {
     return (1 + kKStages + kVStages) * size_t(kTile) + 1024;
 }
 
-size_t prefill_workspace_bytes(int B, int n_kv, int n_r, int n_s, int64_t cap, int S, int W, int C,
+size_t prefill_workspace_bytes(int B, int hq, int n_kv, int n_r, int n_s, int64_t cap, int S, int W, int C,
                                bool key_copies) {
     const size_t row = size_t(kHD) * 2;
     const size_t cached = align256(size_t(B) * n_r * rows_r(cap) * row) + align256(size_t(B) * n_s * rows_s(S, W) * row);
-    return cached + align256(size_t(B) * n_kv * C * row) + (key_copies ? cached : 0);   // V copies, chunk V, key copies
+    const size_t parts = align256(2 * size_t(B) * hq * C * kHD * 4) + align256(2 * size_t(B) * hq * C * 4);
+    // V copies, chunk V, key copies, split partials
+    return cached + align256(size_t(B) * n_kv * C * row) + (key_copies ? cached : 0) + parts;
 }
 
 int launch_prefill(const PrefillLaunch& a, cudaStream_t s) {
@@ -756,6 +824,12 @@ int launch_prefill(const PrefillLaunch& a, cudaStream_t s) {
                                                  align256(size_t(a.B) * a.n_kv * a.C * row));
     uint16_t* k16s = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(k16r) +
                                                  align256(size_t(a.B) * a.n_r * LR * row));
+    // split partials after the key copies (whose space exists only with key copies)
+    const bool kc = a.fp8 || a.page_tokens > 0;
+    char* parts = kc ? reinterpret_cast<char*>(k16s) + align256(size_t(a.B) * a.n_s * LS * row)
+                     : reinterpret_cast<char*>(k16r);
+    float* part_o = reinterpret_cast<float*>(parts);
+    float* part_lse = reinterpret_cast<float*>(parts + align256(2 * size_t(a.B) * a.hq * a.C * kHD * 4));
 
     PrefillParams p;
     memset(&p, 0, sizeof p);
@@ -774,6 +848,8 @@ int launch_prefill(const PrefillLaunch& a, cudaStream_t s) {
         return DUO_ERR_CUDA;
     p.prefix = a.prefix;
     p.out = a.out;
+    p.part_o = part_o;
+    p.part_lse = part_lse;
     p.status = a.status;
     p.cap = a.cap;
     p.B = a.B; p.hq = a.hq; p.n_kv = a.n_kv; p.G = a.hq / a.n_kv; p.C = a.C;
@@ -816,7 +892,7 @@ int launch_prefill(const PrefillLaunch& a, cudaStream_t s) {
     if (cudaGetLastError() != cudaSuccess) return DUO_ERR_CUDA;
 
     const size_t smem = prefill_smem_bytes(a.S, a.W);
-    const int64_t grid = int64_t(p.n_qt) * a.B * a.hq;
+    const int64_t grid = 2 * int64_t(p.n_qt) * a.B * a.hq;   // two shares per query tile (unsplit: one leaves)
     if (grid > 0x7fffffff) return DUO_ERR_UNSUPPORTED;
     if (a.fp8) {
         if (cudaFuncSetAttribute(prefill_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
@@ -829,6 +905,17 @@ int launch_prefill(const PrefillLaunch& a, cudaStream_t s) {
             return DUO_ERR_CUDA;
         prefill_kernel<false><<<unsigned(grid), kThreads, smem, s>>>(p);
     }
+    if (cudaGetLastError() != cudaSuccess) return DUO_ERR_CUDA;
+    MergeParams mp;
+    memset(&mp, 0, sizeof mp);
+    mp.part_o = part_o;
+    mp.part_lse = part_lse;
+    mp.out = a.out;
+    mp.prefix = a.prefix;
+    mp.B = a.B; mp.hq = a.hq; mp.G = a.hq / a.n_kv; mp.C = a.C; mp.S = a.S; mp.W = a.W;
+    memcpy(mp.is_r, a.is_r, sizeof mp.is_r);
+    const int64_t warps = int64_t(a.B) * a.hq * a.C;
+    merge_parts_kernel<<<unsigned((warps + 7) / 8), 256, 0, s>>>(mp);
     return cudaGetLastError() == cudaSuccess ? DUO_OK : DUO_ERR_CUDA;
 }
 

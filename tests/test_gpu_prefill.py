@@ -171,3 +171,47 @@ def test_prefill64k_first_and_last_chunks_sampled():
     rows = sorted(set(rng.choice(w.chunk, 48, replace=False).tolist()) | {0, 1, 127, 128, 1022, 1023, 1024,
                                                                           4095})
     _run_chunks(w, [w.chunk] * (w.prompt // w.chunk), rows=rows, check=[0, 7, 15])
+
+
+@pytest.mark.parametrize("kv_dtype", ["bf16", "fp8"])
+def test_long_prefix_split_query_tiles(kv_dtype):
+    """A 17,000-token prefix makes every retrieval query tile long enough to be
+    shared by two CTAs (their halves merged by log-sum-exp); two sequences
+    with different prefixes, a ragged chunk of 333 rows (a partial last query
+    tile), retrieval and streaming heads."""
+    from head_wise_kv_b200 import DuoKVCache
+    w = _small(batch=2)
+    dev = _dev()
+    first = np.array([17000, 16390])
+    C = 333
+    ks = vs = None
+    if kv_dtype == "fp8":
+        rng = np.random.default_rng(9)
+        ks = rng.uniform(0.5, 2.0, (w.layers, w.n_kv)).astype(np.float32)
+        vs = rng.uniform(0.5, 2.0, (w.layers, w.n_kv)).astype(np.float32)
+    cache = DuoKVCache(w.layers, w.batch, w.hq, w.n_kv, w.d, w.sink, w.window, int(first.max()) + C,
+                       W.retrieval_masks(w), device=dev, kv_dtype=kv_dtype, k_scale=ks, v_scale=vs)
+    hist = History(w)
+    mask = W.retrieval_mask(w, 0)
+    k, v = _chunk_kv(w, 0, np.zeros(2, np.int64), int(first.max()))
+    cache.append(0, k.to(dev), v.to(dev), torch.zeros(2, dtype=torch.int32, device=dev),
+                 torch.from_numpy(first.astype(np.int32)).to(dev))
+    q = _chunk_q(w, 0, first, C)
+    k, v = _chunk_kv(w, 0, first, C)
+    out = cache.prefill(0, q.to(dev), k.to(dev), v.to(dev), torch.from_numpy(first.astype(np.int32)).to(dev),
+                        w.scale)
+
+    def hist_of(kind):
+        def f(b, g):
+            P = int(first[b])
+            x = hist.kv(0, b, g, kind, P + C).float().numpy()
+            if kv_dtype == "fp8":
+                s = float((ks if kind == W.TENSOR_K else vs)[0, g])
+                x = np.concatenate([O.dequantize_kv(O.quantize_kv(x[:P], s), s), x[P:]])
+            return x
+        return f
+    ref = O.prefill_attention(q.double().numpy(), hist_of(W.TENSOR_K), hist_of(W.TENSOR_V), first, mask,
+                              w.sink, w.window, w.scale)
+    assert_close(out.cpu().double().numpy(), ref, f"{kv_dtype} long prefix, split query tiles")
+    assert cache.status() == 0
+    cache.close()
