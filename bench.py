@@ -34,12 +34,12 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM read + write bytes per launch of decode_tc_kernel<4> on this workload,
 # from the ncu capture summarised in profiles/decode_tc_kernel_gqa128k.md.  Must be
 # reset to None whenever the decode kernel changes.
-DECODE_TRAFFIC_BYTES = 1126346000 + 3740672
+DECODE_TRAFFIC_BYTES = 1126401536 + 3869184
 # The same for decode_tc_kernel<4, FP8> on the FP8 cache of this workload
 # (profiles/decode_tc_kernel_fp8_gqa128k.md); None once that kernel changes.
-DECODE_FP8_TRAFFIC_BYTES = 566144768 + 5809408
+DECODE_FP8_TRAFFIC_BYTES = 566236416 + 2974976
 # The same for the INT4 instantiation (profiles/decode_tc_kernel_int4_gqa128k.md).
-DECODE_INT4_TRAFFIC_BYTES = 283192320 + 3347456
+DECODE_INT4_TRAFFIC_BYTES = 283220992 + 3125248
 
 
 # ---------------------------------------------------------------- helpers
