@@ -281,6 +281,21 @@ __device__ __forceinline__ bool softmax_barrier_any(bool flag) {
     return out != 0;
 }
 
+// The same over the two softmax warps that share a TMEM lane quarter (the two
+// halves of the same 32 query rows): named barrier 4 + quarter, 64 threads.
+__device__ __forceinline__ bool pair_barrier_any(int quarter, bool flag) {
+    uint32_t out;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\t"
+        "setp.ne.u32 pi, %1, 0;\n\t"
+        "bar.red.or.pred po, %2, 64, pi;\n\t"
+        "selp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(out)
+        : "r"(uint32_t(flag)), "r"(4 + quarter)
+        : "memory");
+    return out != 0;
+}
+
 // ------------------------------------------------------------------ V -> fp16 (and FP8 codes -> 16 bits)
 // Eight E4M3 codes -> their values as fp16 (exact: every E4M3 value is an
 // fp16 value), or as bf16 (also exact).
@@ -646,9 +661,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 for (int c = 8; c < 64; c += 2) t8[(c >> 1) & 7] = fmax3(t8[(c >> 1) & 7], s[c], s[c + 1]);
                 mx = fmax3(fmax3(t8[0], t8[1], t8[2]), fmax3(t8[3], t8[4], t8[5]), fmaxf(t8[6], t8[7]));
             }
-            // exchange the half-row maxima; the barrier also agrees on aborting
+            // exchange the half-row maxima with the warp that holds the other
+            // half of these rows; the barrier also agrees on aborting
             red_max[st][hf][r] = mx;
-            if (softmax_barrier_any(!got || *abort_flag)) { ok = false; break; }
+            if (pair_barrier_any(wq, !got || *abort_flag)) { ok = false; break; }
             mx = fmaxf(red_max[st][0][r], red_max[st][1][r]);
 
             const bool cached = F8 && plan.cached(j);   // tiles of the cache come first
@@ -699,6 +715,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_addr(&p_full));
         }
+        // the pairs may have left at different tiles: agree before the epilogue
+        ok = !softmax_barrier_any(!ok);
         // epilogue: O / (l of both halves)
         if (ok) {
             const bool got = warp_wait(smem_addr(&o_done), (plan.n - 1) & 1, p, abort_flag);
