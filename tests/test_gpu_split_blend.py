@@ -8,6 +8,7 @@ through the C ABI, against the fp64 oracle.
 * Gated forward: on a cache whose heads all keep full history, the streaming
   attention is two row ranges (sinks, recent window) merged, then blended
   with full attention per query head.
+Both on bf16, FP8 and INT4 caches (the oracle reads the dequantised history).
 """
 import numpy as np
 import pytest
@@ -24,9 +25,15 @@ def _dev():
     return torch.device("cuda", 0)
 
 
-def _cache(w, cap, mask):
+SCALES = {"bf16": None, "fp8": 0.25, "int4": 0.5}   # one K and V scale for every head
+
+
+def _cache(w, cap, mask, kv_dtype="bf16"):
     from head_wise_kv_b200 import DuoKVCache
-    return DuoKVCache(1, w.batch, w.hq, w.n_kv, w.d, w.sink, w.window, cap, mask[None], device=_dev())
+    sc = SCALES[kv_dtype]
+    sc = None if sc is None else np.full((1, w.n_kv), sc, np.float32)
+    return DuoKVCache(1, w.batch, w.hq, w.n_kv, w.d, w.sink, w.window, cap, mask[None], device=_dev(),
+                      kv_dtype=kv_dtype, k_scale=sc, v_scale=sc)
 
 
 def _history(w, T):
@@ -49,26 +56,35 @@ def _fill_rows(cache, w, lens, lo, hi, dev):
     cache.append_rows(0, k.to(dev), v.to(dev), i32([0] * w.batch), i32(lo), i32(hi), n_new=i32(lens))
 
 
-def _oracle_full(w, q, lens, mask):
+def _oracle_full(w, q, lens, mask, kv_dtype="bf16"):
     hist = History(w)
+    sc = SCALES[kv_dtype]
+
+    def read(x):
+        if kv_dtype == "fp8":
+            return O.dequantize_kv(O.quantize_kv(x, sc), sc)
+        if kv_dtype == "int4":
+            return O.dequantize_kv_int4(O.quantize_kv_int4(x, sc), sc)
+        return x
 
     def kh(b, g):
-        return hist.kv(0, b, g, W.TENSOR_K, int(lens[b])).float().numpy()
+        return read(hist.kv(0, b, g, W.TENSOR_K, int(lens[b])).float().numpy())
 
     def vh(b, g):
-        return hist.kv(0, b, g, W.TENSOR_V, int(lens[b])).float().numpy()
+        return read(hist.kv(0, b, g, W.TENSOR_V, int(lens[b])).float().numpy())
     return kh, vh
 
 
+@pytest.mark.parametrize("kv_dtype", ["bf16", "fp8", "int4"])
 @pytest.mark.parametrize("R,cap", [(2, 1600), (3, 1100), (4, 1024)])
-def test_sequence_split_decode_merges_to_full_result(R, cap):
+def test_sequence_split_decode_merges_to_full_result(R, cap, kv_dtype):
     from head_wise_kv_b200 import seqsplit
     from head_wise_kv_b200.cache import lse_merge
     w = W.scaled(W.WORKLOADS["gqa128k"], batch=2, t0_range=None, t0=0, sink=16, window=64)
     dev = _dev()
     mask = W.retrieval_mask(w, 0)
     lens = np.array([2900, 1301])            # after this step's append
-    caches = [_cache(w, cap, mask) for _ in range(R)]
+    caches = [_cache(w, cap, mask, kv_dtype) for _ in range(R)]
     for r, c in enumerate(caches):
         lo, hi = seqsplit.slice_bounds(cap, r)
         _fill_rows(c, w, lens, [lo] * w.batch, [hi] * w.batch, dev)
@@ -82,23 +98,24 @@ def test_sequence_split_decode_merges_to_full_result(R, cap):
         outs.append(o)
         lses.append(l)
     out, lse = lse_merge(torch.stack(outs), torch.stack(lses))
-    kh, vh = _oracle_full(w, q, lens, mask)
+    kh, vh = _oracle_full(w, q, lens, mask, kv_dtype)
     ref, ref_lse = O.decode_attention(q.double().numpy(), kh, vh, lens, mask, w.sink, w.window, w.scale)
-    assert_close(out.cpu().double().numpy(), ref, f"split over {R}")
+    assert_close(out.cpu().double().numpy(), ref, f"{kv_dtype} split over {R}")
     assert np.abs(lse.cpu().double().numpy() - ref_lse).max() < 1e-3
     for c in caches:
         assert c.status() == 0
         c.close()
 
 
+@pytest.mark.parametrize("kv_dtype", ["bf16", "fp8", "int4"])
 @pytest.mark.parametrize("lens", [[700, 90], [79, 12], [5, 300]])
-def test_gated_forward_matches_oracle(lens):
+def test_gated_forward_matches_oracle(lens, kv_dtype):
     from head_wise_kv_b200.cache import alpha_blend, lse_merge
     w = W.scaled(W.WORKLOADS["gqa128k"], batch=2, hq=8, n_kv=4, t0_range=None, t0=0, sink=16, window=64)
     dev = _dev()
     lens = np.array(lens)
     full_mask = np.ones(w.n_kv, np.uint8)         # identification keeps every head's full history
-    cache = _cache(w, int(lens.max()), full_mask)
+    cache = _cache(w, int(lens.max()), full_mask, kv_dtype)
     _fill_rows(cache, w, lens, [0] * w.batch, [1 << 30] * w.batch, dev)
     q = W.decode_q(w, 0, lens).to(dev)
     L = torch.from_numpy(lens.astype(np.int32)).to(dev)
@@ -111,10 +128,10 @@ def test_gated_forward_matches_oracle(lens):
     strm, _ = lse_merge(torch.stack([o_s, o_w]), torch.stack([l_s, l_w]))
     alpha = torch.from_numpy(np.random.default_rng(3).uniform(0, 1, w.hq).astype(np.float32)).to(dev)
     out = alpha_blend(alpha, full, strm)
-    kh, vh = _oracle_full(w, q.cpu(), lens, full_mask)
+    kh, vh = _oracle_full(w, q.cpu(), lens, full_mask, kv_dtype)
     ref = O.blended_decode(q.cpu().double().numpy(), kh, vh, lens, w.n_kv, alpha.cpu().double().numpy(), S, Wn,
                            w.scale)
-    assert_close(out.cpu().double().numpy(), ref, "gated forward")
+    assert_close(out.cpu().double().numpy(), ref, f"{kv_dtype} gated forward")
     cache.close()
 
 
