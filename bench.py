@@ -37,9 +37,9 @@ FALLBACK_HBM_GBS = 6650.0
 DECODE_TRAFFIC_BYTES = 1126401536 + 3869184
 # The same for decode_tc_kernel<4, FP8> on the FP8 cache of this workload
 # (profiles/decode_tc_kernel_fp8_gqa128k.md); None once that kernel changes.
-DECODE_FP8_TRAFFIC_BYTES = None
+DECODE_FP8_TRAFFIC_BYTES = 562110464 + 3260160
 # The same for the INT4 instantiation (profiles/decode_tc_kernel_int4_gqa128k.md).
-DECODE_INT4_TRAFFIC_BYTES = None
+DECODE_INT4_TRAFFIC_BYTES = 281120256 + 3440640
 
 
 # ---------------------------------------------------------------- helpers
