@@ -46,7 +46,7 @@ EXPORTED = (
     "duo_prefill_workspace_bytes", "duo_prefill_attn", "duo_kv_read_status",
     "duo_kv_set_decode_ctas", "duo_strerror", "duo_decode_attn_static_ws",
     "duo_kv_append_rows", "duo_decode_attn_rows", "duo_lse_merge", "duo_alpha_blend", "duo_kv_set_page_table",
-    "duo_kv_fork",
+    "duo_kv_fork", "duo_kv_check_wait_timeout",
 )
 DUO_STATIC_WS_BYTES = 4 << 20
 
@@ -114,6 +114,7 @@ _c_status = _sig("duo_kv_read_status", [_P, ctypes.POINTER(_I32), _I32, _P])
 _c_set_ctas = _sig("duo_kv_set_decode_ctas", [_P, _I32])
 _c_set_pages = _sig("duo_kv_set_page_table", [_P, _P, _I32])
 _c_fork = _sig("duo_kv_fork", [_P, _I32, _I32, _I32, _P])
+_c_waitcheck = _sig("duo_kv_check_wait_timeout", [_P, ctypes.c_uint64, _P])
 _c_strerror = _sig("duo_strerror", [ctypes.c_int], ctypes.c_char_p)
 
 
@@ -241,3 +242,7 @@ def duo_kv_set_page_table(handle, d_table: int, max_pages: int) -> None:
 
 def duo_kv_fork(handle, src: int, dst: int, length: int, stream: int) -> None:
     _check(_c_fork(handle, src, dst, length, stream), "duo_kv_fork")
+
+
+def duo_kv_check_wait_timeout(handle, limit_ns: int, stream: int) -> None:
+    _check(_c_waitcheck(handle, limit_ns, stream), "duo_kv_check_wait_timeout")

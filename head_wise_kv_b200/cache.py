@@ -97,6 +97,10 @@ class DuoKVCache:
         page table maps to the same pool page for both; see duo_kv_fork."""
         L.duo_kv_fork(self.handle, src, dst, length, _stream(self.device))
 
+    def check_wait_timeout(self, limit_ns: int):
+        """Make one bounded device wait run out (see duo_kv_check_wait_timeout)."""
+        L.duo_kv_check_wait_timeout(self.handle, limit_ns, _stream(self.device))
+
     def set_decode_ctas(self, ctas: int):
         L.duo_kv_set_decode_ctas(self.handle, ctas)
         self._alloc_workspace()

@@ -487,6 +487,11 @@ int duo_kv_read_status(duo_kv* kv, int32_t* status, int32_t clear, duo_stream_t 
     return cuda_err(e);
 }
 
+int duo_kv_check_wait_timeout(duo_kv* kv, uint64_t limit_ns, duo_stream_t stream) {
+    if (!kv || limit_ns == 0 || limit_ns > kWaitLimitNs) return DUO_ERR_INVALID_ARG;
+    return cuda_err(duo::launch_wait_check(kv->status, limit_ns, static_cast<cudaStream_t>(stream)));
+}
+
 int duo_kv_set_page_table(duo_kv* kv, const int32_t* d_table, int32_t max_pages) {
     if (!kv || kv->page_tokens <= 0 || !d_table || max_pages < 1) return DUO_ERR_INVALID_ARG;
     if (reinterpret_cast<uintptr_t>(d_table) & 3) return DUO_ERR_ALIGNMENT;

@@ -167,6 +167,7 @@ struct PrefillLaunch {
 // Host-side launchers (defined in the kernel translation units).
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 cudaError_t launch_fork(const ForkParams& p, cudaStream_t s);
+cudaError_t launch_wait_check(int32_t* status, unsigned long long limit_ns, cudaStream_t s);
 int decode_ctas_default(int num_sms, int d, int group);
 size_t decode_workspace_bytes(int slots, int d, int group);
 cudaError_t launch_decode(const DecodeParams& p, int d, int group, cudaStream_t s);

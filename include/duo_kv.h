@@ -353,6 +353,15 @@ DUO_API int duo_prefill_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const
  * launch that gave up may have left them non-zero). */
 DUO_API int duo_kv_read_status(duo_kv* kv, int32_t* status, int32_t clear, duo_stream_t stream);
 
+/* Diagnostic of the bounded waits: launches one warp that waits on an
+ * mbarrier nothing completes, with the bounded-wait routine every pipeline
+ * wait of the attention kernels uses, limited to limit_ns (0 < limit_ns <= 1 s,
+ * the kernels' own limit), after which it sets DUO_STATUS_WAIT_TIMEOUT in the
+ * handle's status word exactly as a timed-out kernel does.  No fault, trap or
+ * unbounded wait is involved; the stream and context stay usable.  For tests
+ * of the timeout reporting (duo_kv_read_status). */
+DUO_API int duo_kv_check_wait_timeout(duo_kv* kv, uint64_t limit_ns, duo_stream_t stream);
+
 /* Paged caches: the device table that maps a sequence's positions to pages,
  * int32 [batch][max_pages]: entry [b][i] is the pool page (0 .. num_pages-1,
  * the same index in every layer's pool) holding positions

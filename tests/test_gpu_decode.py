@@ -142,3 +142,39 @@ def test_gqa128k_config_sampled():
     retrieval): two decode steps, every sequence and query head compared."""
     w = W.scaled(W.WORKLOADS["gqa128k"], steps=2)
     _run_steps(w, 2)
+
+
+def test_timed_out_wait_is_reported_and_the_context_stays_usable():
+    """A device wait that nothing completes gives up after its bound and sets
+    DUO_STATUS_WAIT_TIMEOUT (the same routine and status path as every
+    pipeline wait); reading the status with clear resets it, and decode then
+    runs and matches the oracle."""
+    import time
+    from head_wise_kv_b200 import _lib as L
+    w = W.scaled(W.WORKLOADS["gqa128k"], batch=2, layers=1, t0_range=None, t0=0, sink=16, window=64)
+    from head_wise_kv_b200 import DuoKVCache
+    dev = torch.device("cuda", 0)
+    cache = DuoKVCache(w.layers, w.batch, w.hq, w.n_kv, w.d, w.sink, w.window, 700, W.retrieval_masks(w),
+                       device=dev)
+    lens0 = np.array([600, 333])
+    hist = History(w)
+    fill(cache, hist, 0, lens0, dev)
+    torch.cuda.synchronize()
+    assert cache.status() == 0
+    t0 = time.perf_counter()
+    cache.check_wait_timeout(2_000_000)           # 2 ms
+    st = cache.status(clear=True)
+    elapsed = time.perf_counter() - t0
+    assert st & L.DUO_STATUS_WAIT_TIMEOUT
+    assert 0.002 <= elapsed < 5.0
+    assert cache.status() == 0
+    q, k, v = new_token_inputs(w, 0, lens0)
+    cache.append(0, k.to(dev), v.to(dev), torch.from_numpy(lens0.astype(np.int32)).to(dev))
+    lens = lens0 + 1
+    out = cache.decode(0, q.to(dev), torch.from_numpy(lens.astype(np.int32)).to(dev), w.scale)
+    ref, _ = oracle_decode(hist, 0, q, lens, W.retrieval_mask(w, 0))
+    assert_close(out.cpu().double().numpy(), ref, "decode after a reported timeout")
+    assert cache.status() == 0
+    with pytest.raises(L.DuoError):
+        cache.check_wait_timeout(0)
+    cache.close()
