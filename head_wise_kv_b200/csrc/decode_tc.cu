@@ -46,6 +46,9 @@
 //              kernel is launched.
 //   warp 7 also writes the output of segments without keys and sets the
 //              length status bits.
+//   INT4 caches add warps 12-19 (640 threads): the producers bring the packed
+//              codes into a staging ring and these warps expand them to E4M3
+//              tiles (12-15 K, 16-19 V) for the FP8 arithmetic.
 //
 // Every mbarrier wait is bounded; on a timeout the CTA sets
 // DUO_STATUS_WAIT_TIMEOUT, stops, waits (bounded) for its copies and MMAs in
