@@ -316,7 +316,10 @@ DUO_API int duo_decode_attn_static_ws(duo_kv* kv, int32_t layer, const uint16_t*
 
 /* Workspace bytes duo_prefill_attn needs for chunks of up to `chunk` rows
  * (host only): fp16 copies of the values one call reads -- the retrieval
- * heads' cached rows, the streaming rings and the chunk. */
+ * heads' cached rows, the streaming rings and the chunk --, bf16 copies of
+ * the cached keys for FP8, INT4 or paged caches, and the partial outputs of
+ * query tiles whose keys are shared by two CTAs (2 x B x Hq x chunk x d
+ * fp32 plus their log-sum-exps). */
 DUO_API int duo_prefill_workspace_bytes(const duo_kv* kv, int32_t chunk, size_t* bytes);
 
 /* Chunked-prefill attention for one layer (before the chunk is appended).
