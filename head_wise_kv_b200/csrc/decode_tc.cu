@@ -90,9 +90,11 @@ constexpr float kRescaleThreshold = 8.0f;     // log2 units: probabilities stay 
 // Partition weight of a segment start in 16-token blocks: starting a piece
 // (its first tile's latency, the hand-over of the last one) costs about as
 // much time as streaming this many blocks.  Measured on the 128K GQA
-// workload: 0 -> 193 us, 8 -> 188, 16 -> 183, 24..48 -> 181.5-183, 64 -> 183.
+// workload: 0 -> 193 us, 8 -> 188, 16 -> 183, 24..48 -> 181.5-183, 64 -> 183;
+// with the current kernel on one box, 24 -> 182.3-183.6, 32 -> 183.8-184.6,
+// 40 -> 184.1-184.3 (layer-step).
 #ifndef DUO_DECODE_SEG_WEIGHT
-#define DUO_DECODE_SEG_WEIGHT 32
+#define DUO_DECODE_SEG_WEIGHT 24
 #endif
 constexpr int kSegWeight = DUO_DECODE_SEG_WEIGHT;
 // FP8 streams twice the keys per byte, so a piece start costs more blocks.
