@@ -34,7 +34,7 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM read + write bytes per launch of decode_tc_kernel<4> on this workload,
 # from the ncu capture summarised in profiles/decode_tc_kernel_gqa128k.md.  Must be
 # reset to None whenever the decode kernel changes.
-DECODE_TRAFFIC_BYTES = None
+DECODE_TRAFFIC_BYTES = 1124017664 + 6327552
 # The same for decode_tc_kernel<4, FP8> on the FP8 cache of this workload
 # (profiles/decode_tc_kernel_fp8_gqa128k.md); None once that kernel changes.
 DECODE_FP8_TRAFFIC_BYTES = 562110464 + 3260160
