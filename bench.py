@@ -150,6 +150,13 @@ def rank_workload(rank: int, world: int):
 # ---------------------------------------------------------------- our arm
 def fill_rank(cache, gw, lens0, first_b, dev, slab=16384):
     """Bulk-append the seeded history of this rank's sequences."""
+    fill_targets([(cache, None)], gw, lens0, first_b, dev, slab)
+
+
+def fill_targets(targets, gw, lens0, first_b, dev, slab=16384):
+    """Bulk-append the seeded history into every (cache, rows) target; rows =
+    None appends whole sequences, rows = (lo, hi) (int32 [B] on the device)
+    keeps retrieval positions [lo, hi) (a slice of a sequence-split cache)."""
     B = len(lens0)
     top = int(lens0.max())
     for p0 in range(0, top, slab):
@@ -163,8 +170,14 @@ def fill_rank(cache, gw, lens0, first_b, dev, slab=16384):
                 if c:
                     k[b, g, :c] = W.tokens(gw, 0, first_b + b, g, W.TENSOR_K, p0, p0 + c)
                     v[b, g, :c] = W.tokens(gw, 0, first_b + b, g, W.TENSOR_V, p0, p0 + c)
-        cache.append(0, k.to(dev), v.to(dev), torch.from_numpy(np.minimum(lens0, p0).astype(np.int32)).to(dev),
-                     torch.from_numpy(cnt).to(dev))
+        kd, vd = k.to(dev), v.to(dev)
+        lb = torch.from_numpy(np.minimum(lens0, p0).astype(np.int32)).to(dev)
+        cd = torch.from_numpy(cnt).to(dev)
+        for cache, rows in targets:
+            if rows is None:
+                cache.append(0, kd, vd, lb, cd)
+            else:
+                cache.append_rows(0, kd, vd, lb, rows[0], rows[1], cd)
 
 
 def step_inputs(gw, lens0, first_b, steps):
@@ -476,6 +489,186 @@ def run_variant_decode(local, kv_dtype="fp8", paged=False, steps=512, warmup=16)
     }
 
 
+def _step_tensors(gw, base, lens0, dev):
+    qs, ks, vs = step_inputs(gw, lens0, 0, base.steps)
+    dq = [q.to(dev) for q in qs]
+    dk = [k.to(dev) for k in ks]
+    dv = [v.to(dev) for v in vs]
+    lb = [torch.from_numpy((lens0 + s).astype(np.int32)).to(dev) for s in range(base.steps)]
+    la = [torch.from_numpy((lens0 + s + 1).astype(np.int32)).to(dev) for s in range(base.steps)]
+    return dq, dk, dv, lb, la
+
+
+def run_seqsplit(local, R=2, steps=256, warmup=16):
+    """Sequence-split decode (f4): every sequence's retrieval positions cut
+    into R contiguous slices, as R GPUs would hold them.  Here the R slices
+    are R independent caches on one GPU, run one after another (none waits on
+    another).  Per layer-step: each slice appends the new token
+    (append_rows), decodes its rows (decode_rows; the last slice also the
+    streaming heads), and lse_merge combines the R partial (out, lse) -- the
+    exchange between GPUs (an all-gather of 16.5 KB per sequence and layer)
+    is the one step not run here."""
+    from head_wise_kv_b200 import DuoKVCache, seqsplit
+    from head_wise_kv_b200.cache import lse_merge
+    dev = torch.device("cuda", local)
+    base, gw, lens0 = rank_workload(0, 1)
+    mask = W.retrieval_mask(gw, 0)
+    B = base.batch
+    total = int(lens0.max()) + base.steps
+    cap = (total + R - 1) // R
+    caches = [DuoKVCache(1, B, base.hq, base.n_kv, base.d, base.sink, base.window, cap, mask[None], device=dev)
+              for _ in range(R)]
+    bounds = []
+    for r in range(R):
+        lo, hi = seqsplit.slice_bounds(cap, r)
+        bounds.append((torch.full((B,), lo, dtype=torch.int32, device=dev),
+                       torch.full((B,), hi, dtype=torch.int32, device=dev)))
+    fill_targets(list(zip(caches, bounds)), gw, lens0, 0, dev)
+    dq, dk, dv, lb, la = _step_tensors(gw, base, lens0, dev)
+    rows = [[seqsplit.local_rows(la[s], cap, r) for s in range(base.steps)] for r in range(R)]
+    zero = torch.zeros(B, dtype=torch.int32, device=dev)
+    po = torch.empty(R, B, base.hq, base.d, dtype=torch.float32, device=dev)
+    pl = torch.empty(R, B, base.hq, dtype=torch.float32, device=dev)
+    out = torch.empty(B, base.hq, base.d, dtype=torch.float32, device=dev)
+    lse = torch.empty(B, base.hq, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i, ev=None):
+        s = i % base.steps
+        for r, c in enumerate(caches):
+            c.append_rows(0, dk[s], dv[s], lb[s], bounds[r][0], bounds[r][1])
+        for r, c in enumerate(caches):
+            if ev is not None:
+                ev[r][0].record(stream)
+            c.decode_rows(0, dq[s], rows[r][s], base.scale, s_len=la[s] if r == R - 1 else zero, out=po[r],
+                          lse=pl[r])
+            if ev is not None:
+                ev[r][1].record(stream)
+        lse_merge(po, pl, out=out, lse=lse)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    assert all(c.status() == 0 for c in caches), "device status set during the warm-up"
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    step_ms = e0.elapsed_time(e1) / steps
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(R)]
+           for _ in range(steps)]
+    for i in range(steps):
+        step(i, evs[i])
+    torch.cuda.synchronize()
+    assert all(c.status() == 0 for c in caches), "device status set during the timed region"
+    slice_ms = [sum(evs[i][r][0].elapsed_time(evs[i][r][1]) for i in range(steps)) / steps for r in range(R)]
+    nbytes = sum(kv_bytes(lens0 + (i % base.steps) + 1, mask, base.d, base.sink, base.window, total)
+                 for i in range(steps)) / steps
+    hbm_peak, peak_kind = peaks()
+    achieved = nbytes / (sum(slice_ms) * 1e-3) / 1e9
+    for c in caches:
+        c.close()
+    return {
+        "workload": f"gqa128k, every sequence's retrieval positions split into {R} slices of {cap} rows "
+                    f"(R caches on one GPU, run one after another), append_rows + decode_rows per slice + "
+                    f"lse_merge per layer-step, 32 distinct steps cycled",
+        "steps": steps, "warmup": warmup,
+        "layer_step_us": round(step_ms * 1e3, 3),
+        "slice_decode_us": [round(x * 1e3, 3) for x in slice_ms],
+        "kv_bytes_per_layer_step": int(nbytes),
+        "roofline": {"bound": "hbm", "kernel": "decode_tc_kernel over row ranges (all slices)",
+                     "achieved": round(achieved, 1), "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": round(achieved / hbm_peak, 4), "traffic": None},
+        "gpu_launches": (2 * R + 1) * steps,
+    }
+
+
+def run_gated(local, steps=256, warmup=16):
+    """Gated (alpha-blended) decode (f3) on the gqa128k shape with every KV
+    head keeping its whole history (the setting of the identification pass):
+    per layer-step the append, full attention for every head, streaming
+    attention as two row ranges (the sinks and the recent window) merged by
+    log-sum-exp, and out = alpha_h full + (1 - alpha_h) streaming per query
+    head (alpha seeded uniform in [0, 1))."""
+    from head_wise_kv_b200 import DuoKVCache
+    from head_wise_kv_b200.cache import alpha_blend, lse_merge
+    dev = torch.device("cuda", local)
+    base, gw, lens0 = rank_workload(0, 1)
+    B, S, Wn = base.batch, base.sink, base.window
+    full_mask = np.ones(base.n_kv, np.uint8)
+    cap = int(lens0.max()) + base.steps
+    cache = DuoKVCache(1, B, base.hq, base.n_kv, base.d, S, Wn, cap, full_mask[None], device=dev)
+    fill_rank(cache, gw, lens0, 0, dev)
+    dq, dk, dv, lb, la = _step_tensors(gw, base, lens0, dev)
+    sink_end = [torch.clamp(x, max=S) for x in la]
+    win_begin = [torch.clamp(x - Wn, min=S) for x in la]
+    alpha = torch.from_numpy(np.random.default_rng(3).uniform(0, 1, base.hq).astype(np.float32)).to(dev)
+    full = torch.empty(B, base.hq, base.d, dtype=torch.float32, device=dev)
+    po = torch.empty(2, B, base.hq, base.d, dtype=torch.float32, device=dev)
+    pl = torch.empty(2, B, base.hq, dtype=torch.float32, device=dev)
+    strm = torch.empty(B, base.hq, base.d, dtype=torch.float32, device=dev)
+    slse = torch.empty(B, base.hq, dtype=torch.float32, device=dev)
+    out = torch.empty_like(full)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i, ev=None):
+        s = i % base.steps
+        cache.append(0, dk[s], dv[s], lb[s])
+        if ev is not None:
+            ev[0].record(stream)
+        cache.decode(0, dq[s], la[s], base.scale, out=full)
+        if ev is not None:
+            ev[1].record(stream)
+        cache.decode_rows(0, dq[s], sink_end[s], base.scale, out=po[0], lse=pl[0])
+        cache.decode_rows(0, dq[s], la[s], base.scale, r_begin=win_begin[s], out=po[1], lse=pl[1])
+        lse_merge(po, pl, out=strm, lse=slse)
+        alpha_blend(alpha, full, strm, out=out)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    assert cache.status() == 0, "device status set during the warm-up"
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    step_ms = e0.elapsed_time(e1) / steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        step(i, evs[i])
+    torch.cuda.synchronize()
+    assert cache.status() == 0, "device status set during the timed region"
+    full_ms = sum(evs[i][0].elapsed_time(evs[i][1]) for i in range(steps)) / steps
+    n_kv, row = base.n_kv, 4 * base.d
+    fb = sb = 0
+    for i in range(steps):
+        for T in lens0 + (i % base.steps) + 1:
+            T = int(T)
+            fb += n_kv * row * T
+            sb += n_kv * row * (min(T, S) + max(0, T - max(T - Wn, S)))
+    fb, sb = fb / steps, sb / steps
+    hbm_peak, peak_kind = peaks()
+    achieved = fb / (full_ms * 1e-3) / 1e9
+    cache.close()
+    return {
+        "workload": "gqa128k shape, all 8 KV heads keep their whole history; append + full decode + streaming "
+                    "decode (sink rows and window rows, lse-merged) + per-head alpha blend per layer-step, "
+                    "32 distinct steps cycled",
+        "steps": steps, "warmup": warmup,
+        "layer_step_us": round(step_ms * 1e3, 3),
+        "full_decode_us": round(full_ms * 1e3, 3),
+        "kv_bytes_per_layer_step": {"full": int(fb), "streaming": int(sb)},
+        "roofline": {"bound": "hbm", "kernel": "decode_tc_kernel (full attention of every head)",
+                     "achieved": round(achieved, 1), "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": round(achieved / hbm_peak, 4), "traffic": None},
+        "gpu_launches": 6 * steps,
+    }
+
+
 # ---------------------------------------------------------------- chunked prefill
 def prefill_pairs(prompt, chunk, n_r_q, n_s_q, S, Wn):
     """Mask-valid (query, key) pairs of a chunked prefill: retrieval query heads
@@ -666,10 +859,11 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the chunked-prefill measurement")
-    ap.add_argument("--only", choices=["decode", "prefill", "fp8", "int4", "paged"], default=None,
+    ap.add_argument("--only", choices=["decode", "prefill", "fp8", "int4", "paged", "seqsplit", "gated"],
+                    default=None,
                     help="measure one path only (profiling runs)")
     ap.add_argument("--no-fp8", action="store_true",
-                    help="skip the FP8-, INT4- and paged-cache decode measurements")
+                    help="skip the FP8-, INT4-, paged-cache, sequence-split and gated decode measurements")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
     rank, world, local = dist_init()
@@ -686,6 +880,14 @@ def main(argv=None):
             res = ({"metric": "INT4-cache decode",
                     "decode_int4": run_variant_decode(local, "int4", False, args.steps, args.warmup)}
                    if rank == 0 else None)
+        elif args.only == "seqsplit":
+            res = ({"metric": "sequence-split decode",
+                    "decode_seqsplit": run_seqsplit(local, 2, min(args.steps, 256), args.warmup)}
+                   if rank == 0 else None)
+        elif args.only == "gated":
+            res = ({"metric": "gated (alpha-blended) decode",
+                    "decode_gated": run_gated(local, min(args.steps, 256), args.warmup)}
+                   if rank == 0 else None)
         elif args.only == "paged":
             res = ({"metric": "paged-cache decode",
                     "decode_paged": run_variant_decode(local, "bf16", True, args.steps, args.warmup)}
@@ -698,6 +900,8 @@ def main(argv=None):
                 res["decode_fp8"] = run_variant_decode(local, "fp8")
                 res["decode_int4"] = run_variant_decode(local, "int4")
                 res["decode_paged"] = run_variant_decode(local, "bf16", True)
+                res["decode_seqsplit"] = run_seqsplit(local)
+                res["decode_gated"] = run_gated(local)
             if rank == 0 and world == 1 and not args.no_cpu_baseline:
                 res["cpu_baseline"] = cpu_baseline(ctx)
         if rank == 0 and res is not None:
