@@ -229,3 +229,33 @@ def test_paged_cache_bytes_and_checks():
     with pytest.raises(L.DuoError) as e:
         L.duo_kv_required_bytes(dd)
     assert e.value.code == L.DUO_ERR_UNSUPPORTED
+
+
+def test_merge_blend_and_row_calls_check_arguments_before_cuda():
+    """Argument errors come back as codes before any launch; empty work is a
+    no-op that succeeds (fake, never dereferenced addresses stand in for
+    device pointers)."""
+    L = _lib()
+    P = 0x100000          # 256-byte aligned stand-in address
+    bad = [
+        (L.duo_lse_merge, (0, 4, 64, P, P, P, P, None), L.DUO_ERR_INVALID_ARG),      # no parts
+        (L.duo_lse_merge, (2, -1, 64, P, P, P, P, None), L.DUO_ERR_INVALID_ARG),     # negative rows
+        (L.duo_lse_merge, (2, 4, 0, P, P, P, P, None), L.DUO_ERR_INVALID_ARG),       # d = 0
+        (L.duo_lse_merge, (2, 4, 64, None, P, P, P, None), L.DUO_ERR_INVALID_ARG),   # no partial outputs
+        (L.duo_lse_merge, (2, 4, 64, P, P, None, P, None), L.DUO_ERR_INVALID_ARG),   # no output
+        (L.duo_lse_merge, (2, 4, 64, P + 2, P, P, P, None), L.DUO_ERR_ALIGNMENT),    # fp32 misaligned
+        (L.duo_alpha_blend, (-1, 8, 64, P, P, P, P, None), L.DUO_ERR_INVALID_ARG),
+        (L.duo_alpha_blend, (2, 0, 64, P, P, P, P, None), L.DUO_ERR_INVALID_ARG),
+        (L.duo_alpha_blend, (2, 8, 64, None, P, P, P, None), L.DUO_ERR_INVALID_ARG),
+        (L.duo_alpha_blend, (2, 8, 64, P, P, P + 1, P, None), L.DUO_ERR_ALIGNMENT),
+        (L.duo_decode_attn_rows, (None, 0, P, None, P, None, 0.1, P, P, P, 1 << 20, None), L.DUO_ERR_INVALID_ARG),
+        (L.duo_kv_append_rows, (None, 0, P, P, P, None, 1, P, P, None), L.DUO_ERR_INVALID_ARG),
+        (L.duo_kv_set_page_table, (None, P, 4), L.DUO_ERR_INVALID_ARG),
+        (L.duo_kv_check_wait_timeout, (None, 1000, None), L.DUO_ERR_INVALID_ARG),
+    ]
+    for fn, args, code in bad:
+        with pytest.raises(L.DuoError) as e:
+            fn(*args)
+        assert e.value.code == code, (fn.__name__, args)
+    L.duo_lse_merge(3, 0, 64, P, P, P, P, None)          # no rows: nothing to launch
+    L.duo_alpha_blend(0, 8, 64, P, P, P, P, None)        # no sequences: nothing to launch
