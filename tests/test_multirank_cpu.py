@@ -88,3 +88,21 @@ def test_sequence_split_partials_gather_to_every_rank(tmp_path):
     full, _ = O.attend(q, k, v, 0.3)
     wts = np.exp(lses - np.logaddexp(lses[0], lses[1]))
     np.testing.assert_allclose(wts @ outs, full, rtol=1e-5, atol=1e-6)
+
+
+def test_slices_partition_every_sequence_exactly():
+    """R slices of `cap` rows: each sequence's first L positions are covered
+    once, slice r holding [r cap, r cap + rows_r) with 0 <= rows_r <= cap."""
+    import torch
+    from head_wise_kv_b200 import seqsplit
+    rng = np.random.default_rng(5)
+    for R, cap in [(2, 160), (3, 1100), (4, 1)]:
+        L = torch.tensor(rng.integers(0, R * cap + 1, size=7), dtype=torch.int32)
+        held = [seqsplit.local_rows(L, cap, r) for r in range(R)]
+        assert torch.equal(sum(h.to(torch.int64) for h in held), L.to(torch.int64))
+        for r, h in enumerate(held):
+            lo, hi = seqsplit.slice_bounds(cap, r)
+            assert (lo, hi) == (r * cap, (r + 1) * cap)
+            assert bool(((h >= 0) & (h <= cap)).all())
+            # a slice holds rows only once every earlier slice is full
+            assert bool(((h == 0) | (L >= lo)).all())
