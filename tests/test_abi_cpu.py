@@ -259,3 +259,51 @@ def test_merge_blend_and_row_calls_check_arguments_before_cuda():
         assert e.value.code == code, (fn.__name__, args)
     L.duo_lse_merge(3, 0, 64, P, P, P, P, None)          # no rows: nothing to launch
     L.duo_alpha_blend(0, 8, 64, P, P, P, P, None)        # no sequences: nothing to launch
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "duo_kv.h"
+
+int main(void) {
+    /* 2 layers, batch 3, 32 query / 8 KV heads, d = 128, S = 64, W = 256,
+       capacity 1000, even KV heads retrieval, bf16 */
+    uint8_t mask[2 * 8];
+    for (int i = 0; i < 16; ++i) mask[i] = (i % 2) == 0;
+    duo_kv_desc d;
+    memset(&d, 0, sizeof d);
+    d.num_layers = 2; d.batch = 3; d.num_q_heads = 32; d.num_kv_heads = 8; d.head_dim = 128;
+    d.sink = 64; d.window = 256; d.capacity = 1000; d.retrieval_mask = mask; d.kv_dtype = DUO_KV_BF16;
+    size_t total = 0, cache = 0;
+    int rc = duo_kv_required_bytes(&d, &total, &cache);
+    d.head_dim = 96;
+    int bad = duo_kv_required_bytes(&d, &total, NULL);
+    duo_kv* h = NULL;
+    int nul = duo_kv_alloc(NULL, NULL, 0, NULL, &h);
+    printf("%d %zu %zu %d %d %s\n", rc, total, cache, bad, nul, duo_strerror(bad));
+    return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """include/duo_kv.h compiles as C99 and a C program linked to
+    libduo_kv.so sizes a cache exactly as the Python binding does."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc") or shutil.which("cc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    L = _lib()
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(L.LIB_PATH)
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-L", libdir, "-lduo_kv", f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    d, keep = _desc(L)
+    total, cache = L.duo_kv_required_bytes(d)
+    assert [int(x) for x in out[:5]] == [0, total, cache, L.DUO_ERR_UNSUPPORTED, L.DUO_ERR_INVALID_ARG]
+    assert " ".join(out[5:]) == L.duo_strerror(L.DUO_ERR_UNSUPPORTED)
