@@ -11,7 +11,7 @@
 // guide: dense attention for retrieval heads, a block-sparse sliding-window
 // kernel for streaming heads).
 //
-// Two launches per call:
+// Three launches per call:
 //  1. convert_v_kernel writes an fp16 copy of every V row the attention can
 //     read (cached prefix, ring slots, the chunk) into the caller's workspace,
 //     zeroing tile tails.  P is multiplied in fp16 rather than bf16 (rounding
@@ -31,6 +31,10 @@
 //                   64-key half each): masked scores, running max with lazy
 //                   rescaling (O rescaled only when the max grows by more
 //                   than 2^8), P_j as packed fp16 written to TMEM, O / l.
+//
+//  3. merge_parts_kernel combines the two halves of every query tile that
+//     was split over two CTAs (long retrieval prefixes) by log-sum-exp; rows
+//     of unsplit tiles were written directly and are left alone.
 //
 // Every mbarrier wait is bounded; on a timeout the CTA sets
 // DUO_STATUS_WAIT_TIMEOUT, stops, waits (bounded) for its own copies and
