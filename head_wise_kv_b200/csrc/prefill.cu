@@ -18,6 +18,8 @@
 //     P to bf16 alone costs ~1.5e-3 relative error in the output, fp16
 //     ~2e-4), and one tcgen05 MMA needs both operands in the same type; this
 //     way each V row is converted once per call instead of once per CTA.
+//     For FP8 / INT4 or paged caches it also writes bf16 copies of the cached
+//     keys (codes as exact values; pages gathered into one range per head).
 //  2. prefill_kernel, one CTA per (sequence, query head, 128-row query tile),
 //     11 warps:
 //       warp 0      TMA: Q once, then K tiles (bf16, 128 keys x 128 dims as
