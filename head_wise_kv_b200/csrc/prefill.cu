@@ -11,10 +11,12 @@
 // guide: dense attention for retrieval heads, a block-sparse sliding-window
 // kernel for streaming heads).
 //
-// Three launches per call:
+// Four launches per call:
 //  1. convert_v_kernel writes an fp16 copy of every V row the attention can
 //     read (cached prefix, ring slots, the chunk) into the caller's workspace,
-//     zeroing tile tails.  P is multiplied in fp16 rather than bf16 (rounding
+//     zeroing tile tails; a second, usually empty launch of it rescales the
+//     values of any head whose largest |v| reaches 2^15 by a power of two
+//     2^-E (undone in the epilogue), so no finite bf16 value overflows fp16.  P is multiplied in fp16 rather than bf16 (rounding
 //     P to bf16 alone costs ~1.5e-3 relative error in the output, fp16
 //     ~2e-4), and one tcgen05 MMA needs both operands in the same type; this
 //     way each V row is converted once per call instead of once per CTA.
@@ -73,6 +75,12 @@ constexpr float kRescaleThreshold = 8.0f;    // log2 units
 // a launch is made of shorter pieces; their partial outputs are combined by
 // log-sum-exp in merge_parts_kernel.
 constexpr int kSplitMin = 128;
+// CTAs per (head, source) of the value conversion pass.
+constexpr int kConvCtas = 64;
+// fp16 copies of the values keep |v| * 2^-E below 2^15, E >= 0 a power-of-two
+// exponent per (sequence, KV head): far from fp16's 65504 limit, and the
+// unnormalised P V sums (P <= 2^8 with lazy rescaling) stay far inside fp32.
+constexpr int kV16MaxLog2 = 15;
 
 // Instruction descriptors: S = Q K^T in bf16 (both K-major), O += P V in fp16
 // (P from TMEM, V MN-major); M = 128, N = 128.
@@ -88,6 +96,7 @@ struct PrefillParams {
     float* part_o;          // [2][B][hq][C][d] normalised partial outputs of split query tiles
     float* part_lse;        // [2][B][hq][C] their log2-sum-exp (scaled scores)
     int32_t* status;
+    const int32_t* vexp;    // [B * n_kv] value exponent E of each head's fp16 copies (out *= 2^E)
     int64_t cap;
     int B, hq, n_kv, G, C, n_qt, S, W, n_r, n_s, LR, LS;
     float scale_log2;
@@ -118,6 +127,8 @@ struct ConvertParams {
     const int32_t* page_table;
     int32_t* status;
     const int32_t* prefix;
+    float* vmax;            // [B * n_kv][2][kConvCtas] largest |v| each first-pass CTA converted
+    int32_t* vexp;          // [B * n_kv] E: the fp16 copies hold v * 2^-E (read by the attention epilogue)
     int64_t cap;
     int B, n_kv, n_r, n_s, S, W, C, LR, LS;
     int32_t rank[kMaxKvHeads];
@@ -358,11 +369,39 @@ __device__ __forceinline__ uint4 int4x8_to_bf16(uint32_t w) {
 // the prefix or the filled ring slots) up to the end of the last tile the
 // attention reads are written as zeros, so masked columns always meet
 // finite values.
+//
+// Range of the values.  bf16 reaches 3.4e38, fp16 only 65504, so each head's
+// copies hold v * 2^-E with E >= 0 the smallest exponent that keeps every
+// |v| * 2^-E below 2^kV16MaxLog2 (a power-of-two scale: exact, apart from
+// values that fall into fp16's subnormal range, 2^-24 and below, far under
+// the head's largest value); the attention epilogue multiplies by 2^E.  The
+// first pass (REDO = false) converts with E = 0 and records the largest |v|
+// of every CTA; the second pass (REDO = true, values only) computes E per
+// head, writes it for the attention kernel, and leaves at once when E = 0
+// (every value already fits) or converts the head's values again with 2^-E.
+template <bool REDO>
 __global__ void __launch_bounds__(256) convert_v_kernel(const __grid_constant__ ConvertParams c) {
     const int bg = blockIdx.y;
     const int b = bg / c.n_kv, g = bg % c.n_kv;
     const int P = max(c.prefix[b], 0);
     const bool keys = blockIdx.z == 2;
+    __shared__ uint32_t red[8];
+    float vmul = 1.f;
+    if (REDO) {
+        uint32_t mx = 0;   // |v| >= 0, so the float bits order as unsigned integers
+        for (int t = threadIdx.x; t < 2 * kConvCtas; t += blockDim.x)
+            mx = max(mx, __float_as_uint(c.vmax[size_t(bg) * 2 * kConvCtas + t]));
+        mx = __reduce_max_sync(0xffffffffu, mx);
+        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+        __syncthreads();
+        mx = 0;
+        for (int w = 0; w < int(blockDim.x >> 5); ++w) mx = max(mx, red[w]);
+        const int e = int((mx >> 23) & 0xffu) - 127;        // floor(log2 max |v|)
+        const int E = max(0, e - (kV16MaxLog2 - 1));       // <= 114: 2^-E and 2^E are normal floats
+        if (blockIdx.x == 0 && blockIdx.z == 0 && threadIdx.x == 0) c.vexp[bg] = E;
+        if (E == 0) return;
+        vmul = __uint_as_float(uint32_t(127 - E) << 23);
+    }
     // bytes per cached row: bf16, E4M3 codes, or INT4 codes two per byte
     const size_t row_bytes = c.int4 ? kHD / 2 : (c.fp8 ? kHD : 2 * kHD);
     const uint8_t* base = nullptr;                        // cached rows (contiguous) or the page pool
@@ -389,6 +428,25 @@ __global__ void __launch_bounds__(256) convert_v_kernel(const __grid_constant__ 
         n_conv = min(P, c.S + c.W);                         // filled slots
         n_rows = c.LS;
     }
+    // eight bf16 values -> fp16 of v * vmul, with the largest |v| seen
+    auto to_f16 = [vmul](const uint4 w, float& amax) {
+        const float2 a = bf2_to_f2(w.x), bb = bf2_to_f2(w.y), cc = bf2_to_f2(w.z), dd = bf2_to_f2(w.w);
+        if (!REDO)
+            amax = fmaxf(amax, fmaxf(fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(bb.x), fabsf(bb.y))),
+                                     fmaxf(fmaxf(fabsf(cc.x), fabsf(cc.y)), fmaxf(fabsf(dd.x), fabsf(dd.y)))));
+        return make_uint4(pack_half2(a.x * vmul, a.y * vmul), pack_half2(bb.x * vmul, bb.y * vmul),
+                          pack_half2(cc.x * vmul, cc.y * vmul), pack_half2(dd.x * vmul, dd.y * vmul));
+    };
+    auto scaled_f16 = [vmul](uint4 v) {    // fp16 values (codes) * vmul; only reached when REDO
+        uint32_t* x = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&x[i]));
+            x[i] = pack_half2(f.x * vmul, f.y * vmul);
+        }
+        return v;
+    };
+    float amax = 0.f;
     const int64_t pieces = n_rows * (kHD / 8);
     for (int64_t x = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; x < pieces;
          x += int64_t(gridDim.x) * blockDim.x) {
@@ -397,10 +455,7 @@ __global__ void __launch_bounds__(256) convert_v_kernel(const __grid_constant__ 
         uint4 v = make_uint4(0, 0, 0, 0);
         if (row < n_conv) {
             if (chunk) {
-                const uint4 w = *reinterpret_cast<const uint4*>(chunk + x * 8);
-                const float2 a = bf2_to_f2(w.x), bb = bf2_to_f2(w.y), cc = bf2_to_f2(w.z), dd = bf2_to_f2(w.w);
-                v = make_uint4(pack_half2(a.x, a.y), pack_half2(bb.x, bb.y), pack_half2(cc.x, cc.y),
-                               pack_half2(dd.x, dd.y));
+                v = to_f16(*reinterpret_cast<const uint4*>(chunk + x * 8), amax);
             } else {
                 const uint8_t* rowp = nullptr;
                 if (paged) {
@@ -409,31 +464,36 @@ __global__ void __launch_bounds__(256) convert_v_kernel(const __grid_constant__ 
                     if (page >= 0 && page < c.num_pages)
                         rowp = base + ((size_t(page) * c.n_r + c.rank[g]) * size_t(c.page_tokens) +
                                        size_t(row % c.page_tokens)) * row_bytes;
-                    else if (col8 == 0)
+                    else if (col8 == 0 && !REDO)
                         atomicOr(reinterpret_cast<int*>(c.status), DUO_STATUS_NO_PAGE);
                 } else {
                     rowp = base + size_t(row) * row_bytes;
                 }
+                // codes are at most 448 (E4M3) or 8 (INT4) in magnitude: no range to record
                 if (rowp && c.int4) {
                     const uint32_t cc = *reinterpret_cast<const uint32_t*>(rowp + col8 * 4);
                     v = keys ? int4x8_to_bf16(cc) : int4x8_to_f16(cc);
+                    if (REDO) v = scaled_f16(v);
                 } else if (rowp && c.fp8) {
                     const uint2 cc = *reinterpret_cast<const uint2*>(rowp + col8 * 8);
                     v = keys ? e4m3x8_to_bf16(cc) : e4m3x8_to_f16(cc);
+                    if (REDO) v = scaled_f16(v);
                 } else if (rowp) {
                     const uint4 w = *reinterpret_cast<const uint4*>(rowp + col8 * 16);
-                    if (keys) {
-                        v = w;                                  // bf16 keys: a copy
-                    } else {
-                        const float2 a = bf2_to_f2(w.x), bb = bf2_to_f2(w.y), cc = bf2_to_f2(w.z),
-                                     dd = bf2_to_f2(w.w);
-                        v = make_uint4(pack_half2(a.x, a.y), pack_half2(bb.x, bb.y), pack_half2(cc.x, cc.y),
-                                       pack_half2(dd.x, dd.y));
-                    }
+                    v = keys ? w : to_f16(w, amax);             // bf16 keys: a copy
                 }
             }
         }
         *reinterpret_cast<uint4*>(dst + x * 8) = v;
+    }
+    if (!REDO && !keys) {
+        uint32_t mx = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
+        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            for (int w = 1; w < int(blockDim.x >> 5); ++w) mx = max(mx, red[w]);
+            c.vmax[(size_t(bg) * 2 + blockIdx.z) * kConvCtas + blockIdx.x] = __uint_as_float(mx);
+        }
     }
 }
 
@@ -730,7 +790,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             if (!softmax_barrier_any(!got)) {
                 tc_fence_after();
                 const float lt = red_l[0][r] + red_l[1][r];
-                const float inv = lt > 0.f ? 1.f / lt : 0.f;
+                // the fp16 value copies hold v * 2^-E (E = 0 unless some |v| >= 2^15)
+                const float vpow = __uint_as_float(uint32_t(127 + p.vexp[b * p.n_kv + g]) << 23);
+                const float inv = lt > 0.f ? vpow / lt : 0.f;
                 // a split query tile leaves its normalised half and the row's
                 // log2-sum-exp for merge_parts_kernel
                 const size_t row = (size_t(split ? part * p.B + b : b) * p.hq + h) * p.C + i;
@@ -832,8 +894,9 @@ size_t prefill_workspace_bytes(int B, int hq, int n_kv, int n_r, int n_s, int64_
     const size_t row = size_t(kHD) * 2;
     const size_t cached = align256(size_t(B) * n_r * rows_r(cap) * row) + align256(size_t(B) * n_s * rows_s(S, W) * row);
     const size_t parts = align256(2 * size_t(B) * hq * C * kHD * 4) + align256(2 * size_t(B) * hq * C * 4);
-    // V copies, chunk V, key copies, split partials
-    return cached + align256(size_t(B) * n_kv * C * row) + (key_copies ? cached : 0) + parts;
+    const size_t range = align256(size_t(B) * n_kv * 2 * kConvCtas * 4) + align256(size_t(B) * n_kv * 4);
+    // V copies, chunk V, key copies, split partials, value ranges
+    return cached + align256(size_t(B) * n_kv * C * row) + (key_copies ? cached : 0) + parts + range;
 }
 
 int launch_prefill(const PrefillLaunch& a, cudaStream_t s) {
@@ -854,6 +917,9 @@ int launch_prefill(const PrefillLaunch& a, cudaStream_t s) {
                      : reinterpret_cast<char*>(k16r);
     float* part_o = reinterpret_cast<float*>(parts);
     float* part_lse = reinterpret_cast<float*>(parts + align256(2 * size_t(a.B) * a.hq * a.C * kHD * 4));
+    char* range = reinterpret_cast<char*>(part_lse) + align256(2 * size_t(a.B) * a.hq * a.C * 4);
+    float* vmax = reinterpret_cast<float*>(range);
+    int32_t* vexp = reinterpret_cast<int32_t*>(range + align256(size_t(a.B) * a.n_kv * 2 * kConvCtas * 4));
 
     PrefillParams p;
     memset(&p, 0, sizeof p);
@@ -875,6 +941,7 @@ int launch_prefill(const PrefillLaunch& a, cudaStream_t s) {
     p.part_o = part_o;
     p.part_lse = part_lse;
     p.status = a.status;
+    p.vexp = vexp;
     p.cap = a.cap;
     p.B = a.B; p.hq = a.hq; p.n_kv = a.n_kv; p.G = a.hq / a.n_kv; p.C = a.C;
     p.n_qt = (a.C + kBM - 1) / kBM;
@@ -911,8 +978,13 @@ int launch_prefill(const PrefillLaunch& a, cudaStream_t s) {
     c.num_pages = a.num_pages;
     c.page_table = a.page_table;
     c.status = a.status;
+    c.vmax = vmax;
+    c.vexp = vexp;
     if (int64_t(a.B) * a.n_kv > 65535) return DUO_ERR_UNSUPPORTED;
-    convert_v_kernel<<<dim3(64, unsigned(a.B * a.n_kv), p.kcopy ? 3 : 2), 256, 0, s>>>(c);
+    convert_v_kernel<false><<<dim3(kConvCtas, unsigned(a.B * a.n_kv), p.kcopy ? 3 : 2), 256, 0, s>>>(c);
+    if (cudaGetLastError() != cudaSuccess) return DUO_ERR_CUDA;
+    // value exponents; a head's values are converted again only when some |v| >= 2^15
+    convert_v_kernel<true><<<dim3(kConvCtas, unsigned(a.B * a.n_kv), 2), 256, 0, s>>>(c);
     if (cudaGetLastError() != cudaSuccess) return DUO_ERR_CUDA;
 
     const size_t smem = prefill_smem_bytes(a.S, a.W);

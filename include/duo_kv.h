@@ -231,7 +231,13 @@ DUO_API int duo_kv_append_rows(duo_kv* kv, int32_t layer, const uint16_t* k_new,
 /* Workspace bytes duo_decode_attn needs (host only). */
 DUO_API int duo_decode_workspace_bytes(const duo_kv* kv, size_t* bytes);
 
-/* Decode attention for one layer, every sequence and query head at once.
+/* Decode attention for one layer, every sequence and query head at once
+ * (the DuoAttention guide, section 2, "Retrieval Heads vs. Streaming
+ * Heads": full attention for retrieval heads, attention over the sinks and
+ * the recent window for streaming heads; window rule from "Attention
+ * Variants and Memory Efficiency", "Sliding-Window and Mixed Attention":
+ * keys max(0, t - W + 1) .. t; query head h reads KV head h / G, as in
+ * "Multi-Query and Grouped-Query Attention").
  *   q:    [B][Hq][d] bf16, the query of each sequence's newest token;
  *   len:  device int32 [B], tokens held after this step's append (>= 1);
  *         the query sits at position t = len[b] - 1;
@@ -319,7 +325,8 @@ DUO_API int duo_decode_attn_static_ws(duo_kv* kv, int32_t layer, const uint16_t*
  * heads' cached rows, the streaming rings and the chunk --, bf16 copies of
  * the cached keys for FP8, INT4 or paged caches, and the partial outputs of
  * query tiles whose keys are shared by two CTAs (2 x B x Hq x chunk x d
- * fp32 plus their log-sum-exps). */
+ * fp32 plus their log-sum-exps), and each (sequence, KV head)'s value
+ * range (a few hundred bytes). */
 DUO_API int duo_prefill_workspace_bytes(const duo_kv* kv, int32_t chunk, size_t* bytes);
 
 /* Chunked-prefill attention for one layer (before the chunk is appended).
@@ -337,7 +344,11 @@ DUO_API int duo_prefill_workspace_bytes(const duo_kv* kv, int32_t chunk, size_t*
  * and from k_chunk).  The DuoAttention guide's "Hardware-Fused Prefill":
  * dense causal attention for retrieval heads, block-sparse sink + local
  * attention for streaming heads.  Products of probabilities and values run
- * in fp16 (fp32 accumulation), so |v| must stay below 65504.  FP8 caches:
+ * in fp16 (fp32 accumulation) on copies of the values scaled per
+ * (sequence, KV head) by a power of two 2^-E, E >= 0 the smallest exponent
+ * that keeps the head's |v| * 2^-E below 2^15, and the output is multiplied
+ * back by 2^E: any finite bf16 value is accepted (E = 0, no scaling, for
+ * heads whose values all lie below 2^15).  FP8 caches:
  * the cached prefix is read dequantised (codes times the scales), the
  * chunk's own keys and values exactly as given; the value scales of the
  * layer must lie in [2^-8, 2^7] (else UNSUPPORTED: probabilities are scaled
