@@ -42,15 +42,26 @@ def gather_partials(out: torch.Tensor, lse: torch.Tensor, group=None):
     return torch.stack(outs), torch.stack(lses)
 
 
-def split_decode_step(cache, layer: int, q, lengths, scale: float, capacity_per_rank: int, rank: int,
-                      world: int, group=None):
-    """One decode of one layer for a sequence split over `world` ranks.
-    lengths: int32 [B] total tokens held (after the step's append).  Returns
-    the merged (out, lse) on every rank."""
+def rank_rows(lengths: torch.Tensor, capacity_per_rank: int, rank: int, world: int):
+    """What `rank` reads for sequences of the given total lengths (int32
+    [B]): its retrieval rows (local_rows) and the streaming ring slots.  Every
+    rank holds complete rings, but only the last one reads them, so that each
+    streaming key enters the merged result once."""
     rows = local_rows(lengths, capacity_per_rank, rank)
     s_len = lengths if rank == world - 1 else torch.zeros_like(lengths)
+    return rows, s_len
+
+
+def split_decode_step(cache, layer: int, q, lengths, scale: float, capacity_per_rank: int, rank: int,
+                      world: int, group=None, gather=None):
+    """One decode of one layer for a sequence split over `world` ranks.
+    lengths: int32 [B] total tokens held (after the step's append).  Returns
+    the merged (out, lse) on every rank.  gather(out, lse, group) collects
+    every rank's partials as ([R][...], [R][...]); the default is
+    gather_partials over torch.distributed."""
+    rows, s_len = rank_rows(lengths, capacity_per_rank, rank, world)
     out, lse = cache.decode_rows(layer, q, rows, scale, s_len=s_len)
     if world == 1:
         return out, lse
-    parts_out, parts_lse = gather_partials(out, lse, group)
+    parts_out, parts_lse = (gather or gather_partials)(out, lse, group)
     return lse_merge(parts_out, parts_lse)

@@ -152,3 +152,72 @@ def test_lse_merge_ignores_empty_parts():
         np.testing.assert_allclose(out[row].cpu().numpy(), wts[0] * oo[0, row] + wts[1] * oo[2, row], rtol=1e-5,
                                    atol=1e-6)
     assert torch.all(out[4] == 0) and lse[4].item() == float("-inf")
+
+
+class _ThreadAllGather:
+    """All-gather among R host threads of one process: a stand-in for the
+    NCCL all-gather of gather_partials when the R ranks' caches share one
+    GPU.  Kernels never wait on one another: the threads meet on the host
+    after each has enqueued its own decode."""
+
+    def __init__(self, world):
+        import threading
+        self.world = world
+        self.slots = [None] * world
+        self.barrier = threading.Barrier(world, timeout=120)
+
+    def __call__(self, out, lse, rank):
+        self.slots[rank] = (out, lse)
+        self.barrier.wait()
+        parts = (torch.stack([s[0] for s in self.slots]), torch.stack([s[1] for s in self.slots]))
+        self.barrier.wait()
+        return parts
+
+
+@pytest.mark.parametrize("R,cap", [(2, 1600), (3, 1100), (4, 1024)])
+def test_split_decode_step_on_every_rank(R, cap):
+    """seqsplit.split_decode_step as R ranks call it (one host thread per
+    rank, each with its own cache holding its slice): the rank-dependent row
+    ranges (only the last rank reads the streaming rings), the exchange and
+    the merge give every rank the oracle's result."""
+    import threading
+    from head_wise_kv_b200 import seqsplit
+    w = W.scaled(W.WORKLOADS["gqa128k"], batch=3, t0_range=None, t0=0, sink=16, window=64)
+    dev = _dev()
+    mask = W.retrieval_mask(w, 0)
+    lens = np.array([2900, 1301, 40])        # the last sequence: fewer tokens than the ring holds
+    lens = np.minimum(lens, R * cap)
+    caches = [_cache(w, cap, mask) for _ in range(R)]
+    for r, c in enumerate(caches):
+        lo, hi = seqsplit.slice_bounds(cap, r)
+        _fill_rows(c, w, lens, [lo] * w.batch, [hi] * w.batch, dev)
+    q = W.decode_q(w, 0, lens).to(dev)
+    L = torch.from_numpy(lens.astype(np.int32)).to(dev)
+    torch.cuda.synchronize()
+    gather = _ThreadAllGather(R)
+    results, errors_ = [None] * R, []
+
+    def rank_main(r):
+        try:
+            torch.cuda.set_device(dev)
+            results[r] = seqsplit.split_decode_step(caches[r], 0, q, L, w.scale, cap, r, R, group=r,
+                                                    gather=gather)
+        except Exception as e:                 # reported below
+            errors_.append(e)
+            gather.barrier.abort()
+    threads = [threading.Thread(target=rank_main, args=(r,)) for r in range(R)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert not errors_, errors_
+    torch.cuda.synchronize()
+    kh, vh = _oracle_full(w, q.cpu(), lens, mask)
+    ref, ref_lse = O.decode_attention(q.cpu().double().numpy(), kh, vh, lens, mask, w.sink, w.window, w.scale)
+    for r, (out, lse) in enumerate(results):
+        assert_close(out.cpu().double().numpy(), ref, f"rank {r} of {R}")
+        assert np.abs(lse.cpu().double().numpy() - ref_lse).max() < 1e-3
+        assert torch.equal(out, results[0][0]) and torch.equal(lse, results[0][1])
+    for c in caches:
+        assert c.status() == 0
+        c.close()
