@@ -1,7 +1,9 @@
 """duo_decode_attn_static_ws: decode for callers that cannot allocate device
 memory (their host program owns it all, or they must not call cudaMalloc in
-the serving loop).  It must give the same result as duo_decode_attn with a
-caller workspace, call after call, using only the library's built-in scratch.
+the serving loop).  It runs the same kernel as duo_decode_attn with the same
+split of the keys, only on the library's built-in scratch, so its output and
+log-sum-exp must equal duo_decode_attn's bit for bit, call after call; one
+call is also compared with the fp64 oracle at the parity bar.
 
 Collected last on purpose: if it fails, a run that stops at the first
 failure has already run every other test.
@@ -11,7 +13,7 @@ import pytest
 import torch
 
 import duo_workloads as W
-from _harness import MAX_ABS, REL_L2, History, errors, fill, new_token_inputs
+from _harness import History, assert_close, fill, new_token_inputs, oracle_decode
 
 pytestmark = pytest.mark.gpu
 
@@ -31,6 +33,7 @@ def test_static_scratch_decode_matches_workspace_decode():
     w = W.scaled(W.WORKLOADS["gqa128k"], batch=4, t0_range=(2000, 40000), steps=2)
     lens0 = W.context_lengths(w)
     cache, dev = _setup(w, lens0)
+    hist = History(w)
     assert L.duo_decode_workspace_bytes(cache.handle) <= L.DUO_STATIC_WS_BYTES
     stream = torch.cuda.current_stream(dev).cuda_stream
     for s in range(2):   # two calls in a row, the second after another append
@@ -48,10 +51,12 @@ def test_static_scratch_decode_matches_workspace_decode():
         L.duo_decode_attn_static_ws(cache.handle, 0, qd.data_ptr(), lens.data_ptr(), w.scale, got.data_ptr(),
                                     got_lse.data_ptr(), stream)
         torch.cuda.synchronize()
-        m, r = errors(got.cpu().numpy(), ref.cpu().numpy())
-        assert np.isfinite(got.cpu().numpy()).all()
-        assert m <= MAX_ABS and r <= REL_L2, f"call {s}: max-abs {m:.3e}, rel-L2 {r:.3e}"
-        assert np.abs(got_lse.cpu().numpy() - ref_lse.cpu().numpy()).max() < 1e-3
+        assert torch.equal(got, ref), f"call {s}: output differs from the workspace decode"
+        assert torch.equal(got_lse, ref_lse), f"call {s}: lse differs from the workspace decode"
+        if s == 1:
+            o_ref, o_lse = oracle_decode(hist, 0, q, lens_b + 1, W.retrieval_mask(w, 0))
+            assert_close(got.cpu().double().numpy(), o_ref, f"call {s} against the oracle")
+            assert np.abs(got_lse.cpu().double().numpy() - o_lse).max() < 1e-3
     assert cache.status() == 0
     cache.close()
 
