@@ -80,3 +80,25 @@ def test_gated_streaming_rows_cover_the_keep_set(S, Wn):
         if T:
             assert sink_rows | win_rows == _key_set(T - 1, False, S, Wn)
         assert len(sink_rows | win_rows) == min(T, S + Wn)
+
+
+def test_decode_kv_bytes_of_the_million_token_step():
+    """One decode step of the 32-layer million-token workload: per layer 2
+    retrieval heads over T + 1 = 1,048,577 keys and 6 streaming heads over
+    S + W = 1,088 slots, 512 bytes per key (K and V, d = 128, bf16): 34.47 GB
+    per step, 1.077 GB per layer."""
+    w = W.WORKLOADS["mtok"]
+    T = w.t0 + 1
+    per_layer = 2 * 512 * T + 6 * 512 * 1088
+    total = sum(bench.kv_bytes([T], W.retrieval_mask(w, l), w.d, w.sink, w.window, T) for l in range(w.layers))
+    assert total == 32 * per_layer == 34_466_725_888
+    assert round(per_layer / 1e9, 3) == 1.077
+
+
+def test_decode_kv_bytes_of_the_mha32k_step():
+    """MHA-32K, first decode step: 8 retrieval heads over 32,769 keys and 24
+    streaming heads over 320 slots, 512 bytes per key: ~138.1 MB."""
+    w = W.WORKLOADS["mha32k"]
+    lens = W.context_lengths(w) + 1
+    got = bench.kv_bytes(lens, W.retrieval_mask(w, 0), w.d, w.sink, w.window, 10 ** 9)
+    assert got == 8 * 512 * 32769 + 24 * 512 * 320 == 138_153_984
