@@ -34,12 +34,21 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM read + write bytes per launch of decode_tc_kernel<4> on this workload,
 # from the ncu capture summarised in profiles/decode_tc_kernel_gqa128k.md.  Must be
 # reset to None whenever the decode kernel changes.
-DECODE_TRAFFIC_BYTES = 1124017664 + 6327552
+DECODE_TRAFFIC_BYTES = 1123973888 + 2843648
 # The same for decode_tc_kernel<4, FP8> on the FP8 cache of this workload
 # (profiles/decode_tc_kernel_fp8_gqa128k.md); None once that kernel changes.
-DECODE_FP8_TRAFFIC_BYTES = 562110464 + 3260160
+DECODE_FP8_TRAFFIC_BYTES = 562082816 + 2980608
 # The same for the INT4 instantiation (profiles/decode_tc_kernel_int4_gqa128k.md).
-DECODE_INT4_TRAFFIC_BYTES = 281120256 + 3440640
+DECODE_INT4_TRAFFIC_BYTES = None
+# Paged cache, the two slice launches of the sequence split, and the gated
+# forward's full-attention launch (profiles/decode_tc_kernel_variants_gqa128k.md).
+DECODE_PAGED_TRAFFIC_BYTES = 1120186112 + 3314944
+DECODE_SEQSPLIT_TRAFFIC_BYTES = 838107904 + 3008768 + 291869440 + 1110784
+DECODE_GATED_TRAFFIC_BYTES = 2231675904 + 2985984
+# decode_tc_kernel<1> on one copy of the MHA-32K cache, and decode_tc_kernel<4>
+# on one layer of the million-token cache (profiles/decode_tc_kernel_mha32k_mtok.md).
+MHA32K_DECODE_TRAFFIC_BYTES = 139629056 + 3043072
+MTOK_DECODE_TRAFFIC_BYTES = 1085130496 + 3013632
 
 
 # ---------------------------------------------------------------- helpers
@@ -266,6 +275,7 @@ def run_ours(args, rank, world, local):
     torch.cuda.synchronize()
     dec_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(KR)]
     app_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(KR)]
+    each_ms = [ev[i][0].elapsed_time(ev[i][2]) for i in range(KR)]
 
     # algorithmic bytes of the decode launch, averaged over the steps timed
     bytes_steps = [kv_bytes(lens0 + (i % steps) + 1, mask, base.d, base.sink, base.window, cap) for i in range(KR)]
@@ -381,8 +391,12 @@ def run_ours(args, rank, world, local):
             "parallelism": f"replicas/dp{world} (independent sequences per GPU)",
         },
         "hbm_gbs_step": round(step_gbs * world, 1),
+        "value_stats": {"timing": "value: mean over the timed region (events at its two ends); "
+                                  "layer_step_us_each: each layer-step timed alone in a second pass",
+                        "layer_step_us_each": _stats_us(each_ms)},
         "append_us": round(1e3 * sum(app_ms) / KR, 3),
         "decode_us": round(1e3 * dec_avg_ms, 3),
+        "decode_us_median": round(1e3 * statistics.median(dec_ms), 3),
         "roofline": {
             "bound": "hbm",
             "kernel": "decode_tc_kernel (split-K tcgen05 attention with the log-sum-exp merge in-kernel)",
@@ -482,8 +496,8 @@ def run_variant_decode(local, kv_dtype="fp8", paged=False, steps=512, warmup=16)
         "roofline": {"bound": "hbm", "kernel": f"decode_tc_kernel {kv_dtype}{' paged' if paged else ''}",
                      "achieved": round(achieved, 1), "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4),
-                     "traffic": None if paged else {"fp8": DECODE_FP8_TRAFFIC_BYTES,
-                                                     "int4": DECODE_INT4_TRAFFIC_BYTES}.get(kv_dtype),
+                     "traffic": DECODE_PAGED_TRAFFIC_BYTES if paged and kv_dtype == "bf16" else
+                     None if paged else {"fp8": DECODE_FP8_TRAFFIC_BYTES, "int4": DECODE_INT4_TRAFFIC_BYTES}.get(kv_dtype),
                      "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch"},
         "gpu_launches": 2 * steps,
     }
@@ -580,7 +594,9 @@ def run_seqsplit(local, R=2, steps=256, warmup=16):
         "kv_bytes_per_layer_step": int(nbytes),
         "roofline": {"bound": "hbm", "kernel": "decode_tc_kernel over row ranges (all slices)",
                      "achieved": round(achieved, 1), "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": round(achieved / hbm_peak, 4), "traffic": None},
+                     "frac": round(achieved / hbm_peak, 4),
+                     "traffic": DECODE_SEQSPLIT_TRAFFIC_BYTES if R == 2 else None,
+                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, both slice launches"},
         "gpu_launches": (2 * R + 1) * steps,
     }
 
@@ -664,8 +680,229 @@ def run_gated(local, steps=256, warmup=16):
         "kv_bytes_per_layer_step": {"full": int(fb), "streaming": int(sb)},
         "roofline": {"bound": "hbm", "kernel": "decode_tc_kernel (full attention of every head)",
                      "achieved": round(achieved, 1), "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": round(achieved / hbm_peak, 4), "traffic": None},
+                     "frac": round(achieved / hbm_peak, 4), "traffic": DECODE_GATED_TRAFFIC_BYTES,
+                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch"},
         "gpu_launches": 6 * steps,
+    }
+
+
+# ---------------------------------------------------------------- the other decode workloads
+def _l2_flush_buffer(dev):
+    """A buffer twice the device's L2: writing it evicts whatever a step left
+    in L2."""
+    l2 = int(getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 0) or (126 << 20))
+    return torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+
+
+def _stats_us(ms):
+    return {"median": round(statistics.median(ms) * 1e3, 3), "mean": round(sum(ms) / len(ms) * 1e3, 3)}
+
+
+def run_tiny(local, steps=512, warmup=16):
+    """Tiny workload (1 layer, MHA 4 heads, d=64, B=1, T0=512, 16 decode
+    steps cycled, heads {0,2} retrieval, S=16, W=64): the latency floor of a
+    layer-step.  L2 is flushed before every step (a write of twice its size),
+    and each step is timed on its own with CUDA events; median reported."""
+    from head_wise_kv_b200 import DuoKVCache
+    dev = torch.device("cuda", local)
+    w = W.WORKLOADS["tiny"]
+    mask = W.retrieval_mask(w, 0)
+    lens0 = W.context_lengths(w)
+    cap = int(lens0.max()) + w.steps
+    cache = DuoKVCache(1, w.batch, w.hq, w.n_kv, w.d, w.sink, w.window, cap, mask[None], device=dev)
+    fill_rank(cache, w, lens0, 0, dev)
+    dq, dk, dv, lb, la = _step_tensors(w, w, lens0, dev)
+    out = torch.empty(w.batch, w.hq, w.d, dtype=torch.float32, device=dev)
+    flush = _l2_flush_buffer(dev)
+    stream = torch.cuda.current_stream(dev)
+    n = warmup + steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for i in range(n):
+        s = i % w.steps
+        flush.zero_()
+        ev[i][0].record(stream)
+        cache.append(0, dk[s], dv[s], lb[s])
+        cache.decode(0, dq[s], la[s], w.scale, out=out)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    assert cache.status() == 0, "device status set during the tiny benchmark"
+    ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(warmup, n)]
+    nbytes = sum(kv_bytes(lens0 + (i % w.steps) + 1, mask, w.d, w.sink, w.window, cap) for i in range(steps)) / steps
+    med = statistics.median(ms)
+    hbm_peak, peak_kind = peaks()
+    achieved = nbytes / (med * 1e-3) / 1e9
+    cache.close()
+    return {
+        "workload": "tiny: 1 layer, MHA 4 heads, d=64, B=1, T0=512, 16 decode steps cycled, heads {0,2} "
+                    "retrieval, S=16, W=64, K and q RoPE'd",
+        "steps": steps, "warmup": warmup,
+        "layer_step_us": _stats_us(ms),
+        "kv_bytes_per_layer_step": int(nbytes),
+        "l2": "flushed before every step (write of 2x L2); each step timed alone with CUDA events",
+        "roofline": {"bound": "latency", "kernel": "append_kernel + decode_kernel + merge_kernel (d=64)",
+                     "achieved": round(achieved, 1), "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": round(achieved / hbm_peak, 6), "traffic": None,
+                     "note": "0.3 MB per step: three launches' latency, not bandwidth, sets the time"},
+        "gpu_launches": 3 * steps,
+    }
+
+
+def run_mha32k(local, steps=1024, warmup=32, copies=4):
+    """MHA-32K workload (Llama-2-7B attention: 32 = 32 heads, d=128, B=1,
+    T0=32768, 64 decode steps with append/evict, 8 retrieval heads, S=64,
+    W=256, key rows 0..3 x4).  One step reads ~138 MB, about L2's size, so
+    `copies` caches with the same history are used in rotation (step i on
+    copy i mod copies): between two uses of a copy the other copies stream
+    ~3x L2, so every step reads its keys from HBM."""
+    from head_wise_kv_b200 import DuoKVCache
+    dev = torch.device("cuda", local)
+    w = W.WORKLOADS["mha32k"]
+    mask = W.retrieval_mask(w, 0)
+    lens0 = W.context_lengths(w)
+    cap = int(lens0.max()) + w.steps
+    caches = [DuoKVCache(1, w.batch, w.hq, w.n_kv, w.d, w.sink, w.window, cap, mask[None], device=dev)
+              for _ in range(copies)]
+    fill_targets([(c, None) for c in caches], w, lens0, 0, dev)
+    dq, dk, dv, lb, la = _step_tensors(w, w, lens0, dev)
+    out = torch.empty(w.batch, w.hq, w.d, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def which(i):
+        return caches[i % copies], (i // copies) % w.steps
+
+    for i in range(warmup):
+        c, s = which(i)
+        c.append(0, dk[s], dv[s], lb[s])
+        c.decode(0, dq[s], la[s], w.scale, out=out)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):                   # events only at the ends
+        c, s = which(i)
+        c.append(0, dk[s], dv[s], lb[s])
+        c.decode(0, dq[s], la[s], w.scale, out=out)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    step_ms = e0.elapsed_time(e1) / steps
+    ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(steps)]
+    for i in range(steps):                   # per-step and per-launch times
+        c, s = which(i)
+        ev[i][0].record(stream)
+        c.append(0, dk[s], dv[s], lb[s])
+        ev[i][1].record(stream)
+        c.decode(0, dq[s], la[s], w.scale, out=out)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    assert all(c.status() == 0 for c in caches), "device status set during the MHA-32K benchmark"
+    step_each = [ev[i][0].elapsed_time(ev[i][2]) for i in range(steps)]
+    dec_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(steps)]
+    nbytes = sum(kv_bytes(lens0 + ((i // copies) % w.steps) + 1, mask, w.d, w.sink, w.window, cap)
+                 for i in range(steps)) / steps
+    hbm_peak, peak_kind = peaks()
+    dec_avg = sum(dec_ms) / steps
+    achieved = nbytes / (dec_avg * 1e-3) / 1e9
+    for c in caches:
+        c.close()
+    return {
+        "workload": "mha32k: Llama-2-7B attention, MHA 32 heads, d=128, B=1, T0=32768, 8 retrieval heads, "
+                    "S=64, W=256, key rows 0-3 x4, append + decode per layer-step, 64 distinct steps cycled",
+        "steps": steps, "warmup": warmup,
+        "layer_step_us": round(step_ms * 1e3, 3),
+        "layer_step_us_each": _stats_us(step_each),
+        "decode_us": _stats_us(dec_ms),
+        "kv_bytes_per_layer_step": int(nbytes),
+        "hbm_gbs_step": round(nbytes / (step_ms * 1e-3) / 1e9, 1),
+        "l2": f"{copies} cache copies in rotation ({copies} x {nbytes / 1e6:.0f} MB > 3x L2): every step "
+              f"reads its keys from HBM",
+        "roofline": {"bound": "hbm", "kernel": "decode_tc_kernel (G=1)", "achieved": round(achieved, 1),
+                     "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
+                     "traffic": MHA32K_DECODE_TRAFFIC_BYTES,
+                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch"},
+        "gpu_launches": 2 * steps,
+    }
+
+
+def run_mtok(local, steps=10, warmup=3, slab=65536, layers=None):
+    """Million-token workload: 32 layers of GQA 32q/8kv, d=128, B=1,
+    T=1,048,576, 2 of 8 KV heads retrieval per layer, S=64, W=1024.  The
+    caches are filled by bulk appends of N(0,1) bf16 keys and values drawn
+    on the device (a seeded torch generator; 34 GB of history, which host
+    draws would take minutes to produce; the timing does not depend on the
+    values).  One step = append + decode in each of the 32 layers in turn;
+    the steps re-append position T (the same bytes)."""
+    from head_wise_kv_b200 import DuoKVCache
+    dev = torch.device("cuda", local)
+    w = W.WORKLOADS["mtok"]
+    if layers is not None:        # profiling: the first `layers` layers (the same launch per layer)
+        w = W.scaled(w, layers=layers)
+    masks = W.retrieval_masks(w)
+    T0 = w.t0
+    cache = DuoKVCache(w.layers, 1, w.hq, w.n_kv, w.d, w.sink, w.window, T0 + 1, masks, device=dev)
+    gen = torch.Generator(device=dev).manual_seed(W.WORKLOADS["mtok"].seed)
+    for layer in range(w.layers):
+        for p0 in range(0, T0, slab):
+            n = min(slab, T0 - p0)
+            k = torch.randn(1, w.n_kv, n, w.d, generator=gen, device=dev).to(torch.bfloat16)
+            v = torch.randn(1, w.n_kv, n, w.d, generator=gen, device=dev).to(torch.bfloat16)
+            cache.append(layer, k, v, torch.tensor([p0], dtype=torch.int32, device=dev))
+            del k, v
+    torch.cuda.synchronize()
+    assert cache.status() == 0, "device status set while filling the million-token cache"
+    qs = [torch.randn(1, w.hq, w.d, generator=gen, device=dev).to(torch.bfloat16) for _ in range(w.layers)]
+    ks = [torch.randn(1, w.n_kv, 1, w.d, generator=gen, device=dev).to(torch.bfloat16) for _ in range(w.layers)]
+    vs = [torch.randn(1, w.n_kv, 1, w.d, generator=gen, device=dev).to(torch.bfloat16) for _ in range(w.layers)]
+    lb = torch.tensor([T0], dtype=torch.int32, device=dev)
+    la = torch.tensor([T0 + 1], dtype=torch.int32, device=dev)
+    out = torch.empty(1, w.hq, w.d, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        for layer in range(w.layers):
+            cache.append(layer, ks[layer], vs[layer], lb)
+            if ev is not None:
+                ev[layer][0].record(stream)
+            cache.decode(layer, qs[layer], la, w.scale, out=out)
+            if ev is not None:
+                ev[layer][1].record(stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    step_ms = e0.elapsed_time(e1) / steps
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(w.layers)]
+           for _ in range(steps)]
+    for i in range(steps):
+        step(evs[i])
+    torch.cuda.synchronize()
+    assert cache.status() == 0, "device status set during the million-token benchmark"
+    dec_ms = [evs[i][l][0].elapsed_time(evs[i][l][1]) for i in range(steps) for l in range(w.layers)]
+    layer_bytes = [kv_bytes([T0 + 1], masks[l], w.d, w.sink, w.window, T0 + 1) for l in range(w.layers)]
+    step_bytes = sum(layer_bytes)
+    dec_avg = sum(dec_ms) / len(dec_ms)
+    hbm_peak, peak_kind = peaks()
+    achieved = (step_bytes / w.layers) / (dec_avg * 1e-3) / 1e9
+    cache.close()
+    return {
+        "workload": f"mtok: {w.layers} layers GQA 32q/8kv, d=128, B=1, T=1048576, 2/8 KV heads retrieval per "
+                    f"layer, S=64, W=1024; one step = append + decode in each layer in turn",
+        "steps": steps, "warmup": warmup,
+        "ms_per_step": round(step_ms, 4),
+        "layer_step_us": round(step_ms * 1e3 / w.layers, 3),
+        "decode_us": _stats_us(dec_ms),
+        "kv_bytes_per_step": int(step_bytes),
+        "hbm_gbs_step": round(step_bytes / (step_ms * 1e-3) / 1e9, 1),
+        "l2": "not flushed: each layer reads ~1.08 GB (> L2)",
+        "roofline": {"bound": "hbm", "kernel": "decode_tc_kernel (G=4), one launch per layer",
+                     "achieved": round(achieved, 1), "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": round(achieved / hbm_peak, 4), "traffic": MTOK_DECODE_TRAFFIC_BYTES,
+                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch (one layer)"},
+        "gpu_launches": 2 * w.layers * steps,
     }
 
 
@@ -792,40 +1029,104 @@ def cpu_baseline(ctx):
                       f"heads, first decode step), mean of {reps} repetitions, {secs:.2f} s each"}
 
 
+def cpu_baseline_prefill(sample_rows=256, chunks=(15, 7)):
+    """The fp64 oracle's chunked prefill on a bounded sample of the 64K
+    prompt: the first `sample_rows` query rows of the given chunks, every
+    query head, timed; its useful FLOP rate scales it to the whole prompt."""
+    from oracle import duo_oracle as O
+    w = W.WORKLOADS["prefill64k"]
+    mask = W.retrieval_mask(w, 0)
+    G = w.hq // w.n_kv
+    C = w.chunk
+    top = (max(chunks) + 1) * C
+    K = {g: W.tokens(w, 0, 0, g, W.TENSOR_K, 0, top).float().numpy() for g in range(w.n_kv)}
+    V = {g: W.tokens(w, 0, 0, g, W.TENSOR_V, 0, top).float().numpy() for g in range(w.n_kv)}
+    rows = np.arange(sample_rows)
+    secs, pairs = 0.0, 0
+    for c in chunks:
+        P = c * C
+        q = torch.stack([W.tokens(w, 0, 0, h, W.TENSOR_Q, P, P + C) for h in range(w.hq)])[None]
+        q = q.double().numpy()
+        t0 = time.perf_counter()
+        O.prefill_attention(q, lambda _b, g: K[g], lambda _b, g: V[g], np.array([P]), mask, w.sink, w.window,
+                            w.scale, rows=rows)
+        secs += time.perf_counter() - t0
+        t = P + rows
+        n_r_q = int(mask.sum()) * G
+        pairs += n_r_q * int((t + 1).sum()) + (w.hq - n_r_q) * int(np.minimum(t + 1, w.sink + w.window).sum())
+    rate = 4 * w.d * pairs / secs                  # useful FLOP/s
+    n_r_q = int(mask.sum()) * G
+    total = 4 * w.d * prefill_pairs(w.prompt, C, n_r_q, w.hq - n_r_q, w.sink, w.window)
+    return {"value": round(total / rate * 1e3, 1), "unit": "ms per 64K-token prompt (attention)",
+            "useful_tflops": round(rate / 1e12, 4), "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+            "sample": f"numpy fp64 oracle prefill of query rows 0..{sample_rows - 1} of chunks "
+                      f"{list(chunks)} (P = {[c * C for c in chunks]}), all 32 query heads, {secs:.2f} s; "
+                      f"scaled to the whole prompt by useful FLOPs"}
+
+
+def cpu_baseline_mtok(min_seconds=10.0, max_layers=4):
+    """The fp64 oracle's decode of whole layers of the million-token step
+    (layers 0, 1, ... until about `min_seconds` of CPU time): seconds per
+    layer measured, per 32-layer step = 32 x that."""
+    from oracle import duo_oracle as O
+    w = W.WORKLOADS["mtok"]
+    T = w.t0 + 1
+    secs, layers = 0.0, 0
+    while layers < max_layers and (layers == 0 or secs < min_seconds):
+        mask = W.retrieval_mask(w, layers)
+        keep = O.keep_set(T - 1, w.sink, w.window)
+        hk, hv = {}, {}
+        for g in range(w.n_kv):
+            if mask[g]:
+                hk[g] = W.tokens(w, layers, 0, g, W.TENSOR_K, 0, T).float().numpy()
+                hv[g] = W.tokens(w, layers, 0, g, W.TENSOR_V, 0, T).float().numpy()
+            else:   # a streaming head's history is read only at its kept positions
+                hk[g] = np.zeros((T, w.d), np.float32)
+                hv[g] = np.zeros((T, w.d), np.float32)
+                for a, e in [(0, w.sink), (T - w.window, T)]:
+                    hk[g][a:e] = W.tokens(w, layers, 0, g, W.TENSOR_K, a, e).float().numpy()
+                    hv[g][a:e] = W.tokens(w, layers, 0, g, W.TENSOR_V, a, e).float().numpy()
+        assert len(keep) == w.sink + w.window
+        q = torch.stack([W.tokens(w, layers, 0, h, W.TENSOR_Q, T - 1, T)[0] for h in range(w.hq)])[None]
+        q = q.double().numpy()
+        t0 = time.perf_counter()
+        O.decode_attention(q, lambda _b, g: hk[g], lambda _b, g: hv[g], [T], mask, w.sink, w.window, w.scale)
+        secs += time.perf_counter() - t0
+        layers += 1
+        del hk, hv
+    per_layer = secs / layers
+    return {"value": round(per_layer * 1e6, 1), "unit": "us/layer-step",
+            "ms_per_step": round(per_layer * 1e3 * w.layers, 1), "cores": len(os.sched_getaffinity(0)),
+            "kind": "oracle",
+            "sample": f"numpy fp64 oracle decode of {layers} whole layer(s) of the million-token step (all 32 "
+                      f"query heads), {secs:.2f} s; ms_per_step = 32 x the per-layer mean"}
+
+
 def run_reference(args, rank, world):
-    """The oracle as the reference arm: each step times the oracle's decode of
-    the 4 query heads of one retrieval KV head over a 4,096-token prefix of
-    one sequence's cache (cycling sequences and heads) plus one streaming KV
-    head, scaled to a full layer-step by KV bytes."""
+    """The oracle as the reference arm: every step is one full layer-step of
+    the GQA-128K workload (all 8 sequences, all 32 query heads), the same
+    decode steps the GPU arm cycles through, timed on the host cores."""
     if rank != 0:
         return None
     from oracle import duo_oracle as O
     base, gw, lens0 = rank_workload(0, 1)
     mask = W.retrieval_mask(gw, 0)
-    r_heads = [g for g in range(gw.n_kv) if mask[g]]
-    s_heads = [g for g in range(gw.n_kv) if not mask[g]]
-    Tw = 4096
-    samples = []
-    for i in range(min(8, base.batch)):
-        b, g, gs = i % base.batch, r_heads[i % len(r_heads)], s_heads[i % len(s_heads)]
-        T = int(lens0[b]) + 1
-        K = W.tokens(gw, 0, b, g, W.TENSOR_K, 0, Tw).float().numpy()
-        V = W.tokens(gw, 0, b, g, W.TENSOR_V, 0, Tw).float().numpy()
-        keep = O.keep_set(T - 1, gw.sink, gw.window)
-        Ks = W.tokens(gw, 0, b, gs, W.TENSOR_K, 0, T).float().numpy()[keep]
-        Vs = W.tokens(gw, 0, b, gs, W.TENSOR_V, 0, T).float().numpy()[keep]
-        q = torch.stack([W.tokens(gw, 0, b, h, W.TENSOR_Q, T - 1, T)[0] for h in range(gw.hq)]).double().numpy()
-        samples.append((K, V, Ks, Vs, q, g, gs))
-    G = gw.hq // gw.n_kv
-    sample_bytes = 4 * gw.d * (Tw + len(samples[0][2]))
-    total = kv_bytes(lens0 + 1, mask, gw.d, gw.sink, gw.window, 1 << 40)
+    n_steps = base.steps
+    hk, hv, qs = [], [], []
+    for b in range(base.batch):
+        Tmax = int(lens0[b]) + n_steps
+        hk.append({g: W.tokens(gw, 0, b, g, W.TENSOR_K, 0, Tmax).float().numpy() for g in range(gw.n_kv)})
+        hv.append({g: W.tokens(gw, 0, b, g, W.TENSOR_V, 0, Tmax).float().numpy() for g in range(gw.n_kv)})
+        p = int(lens0[b])
+        qs.append(torch.stack([W.tokens(gw, 0, b, h, W.TENSOR_Q, p, p + n_steps) for h in range(gw.hq)], 1))
 
     def one(i):
-        K, V, Ks, Vs, q, g, gs = samples[i % len(samples)]
-        for h in range(g * G, (g + 1) * G):
-            O.attend(q[h], K, V, gw.scale)
-        for h in range(gs * G, (gs + 1) * G):
-            O.attend(q[h], Ks, Vs, gw.scale)
+        s = i % n_steps
+        for b in range(base.batch):
+            T = int(lens0[b]) + s + 1
+            q = qs[b][s][None].double().numpy()
+            O.decode_attention(q, lambda _b, g: hk[b][g], lambda _b, g: hv[b][g], [T], mask, gw.sink,
+                               gw.window, gw.scale)
 
     for i in range(args.warmup):
         one(i)
@@ -833,16 +1134,18 @@ def run_reference(args, rank, world):
     for i in range(args.steps):
         one(i)
     secs = (time.perf_counter() - t0) / args.steps
-    val = secs * 1e6 * total / sample_bytes
+    val = secs * 1e6
     cores = len(os.sched_getaffinity(0))
-    sample = (f"per step: fp64 oracle decode of one retrieval KV head (4 query heads) over a {Tw}-token "
-              f"prefix plus one streaming KV head, scaled to the full layer-step by KV bytes")
+    sample = (f"per step: the fp64 oracle's decode of one full layer-step (all {base.batch} sequences, all "
+              f"{gw.hq} query heads, history as float32 arrays in host memory), decode steps cycled as on the GPU")
     return {
         "impl": "reference", "metric": METRIC, "value": round(val, 1), "unit": "us/layer-step",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(val / 1e3, 4),
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": "gqa128k (oracle on a bounded sample per step)", "global_batch": base.batch,
+        "config": {"workload": "gqa128k: GQA 32q/8kv d=128, B=8 ragged T~U[16384,131072], 4/8 KV heads "
+                               "retrieval, S=64 W=256, one full layer-step per step (fp64 oracle)",
+                   "global_batch": base.batch, "seq_len": [int(x) for x in lens0],
                    "parallelism": "rank 0 only"},
         "cpu_baseline": {"value": round(val, 1), "unit": "us/layer-step", "cores": cores, "kind": "oracle",
                          "sample": sample},
@@ -854,17 +1157,27 @@ def run_reference(args, rank, world):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2048)
-    ap.add_argument("--warmup", type=int, default=64)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default 2048; 20 for --impl reference, whose steps take ~1.5 s)")
+    ap.add_argument("--warmup", type=int, default=None, help="warm-up steps (default 64; 3 for --impl reference)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the chunked-prefill measurement")
-    ap.add_argument("--only", choices=["decode", "prefill", "fp8", "int4", "paged", "seqsplit", "gated"],
+    ap.add_argument("--only", choices=["decode", "prefill", "fp8", "int4", "paged", "seqsplit", "gated", "tiny",
+                                       "mha32k", "mtok"],
                     default=None,
                     help="measure one path only (profiling runs)")
     ap.add_argument("--no-fp8", action="store_true",
                     help="skip the FP8-, INT4-, paged-cache, sequence-split and gated decode measurements")
+    ap.add_argument("--mtok-layers", type=int, default=None,
+                    help="with --only mtok: run only the first N layers (profiling a smaller case)")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the tiny, MHA-32K and million-token decode measurements")
     args = ap.parse_args(argv)
+    if args.steps is None:
+        args.steps = 20 if args.impl == "reference" else 2048
+    if args.warmup is None:
+        args.warmup = 3 if args.impl == "reference" else 64
     args.warmup = max(args.warmup, 3)
     rank, world, local = dist_init()
     try:
@@ -888,6 +1201,15 @@ def main(argv=None):
             res = ({"metric": "gated (alpha-blended) decode",
                     "decode_gated": run_gated(local, min(args.steps, 256), args.warmup)}
                    if rank == 0 else None)
+        elif args.only == "tiny":
+            res = {"metric": "tiny decode", "decode_tiny": run_tiny(local)} if rank == 0 else None
+        elif args.only == "mha32k":
+            res = ({"metric": "MHA-32K decode", "decode_mha32k": run_mha32k(local, min(args.steps, 1024))}
+                   if rank == 0 else None)
+        elif args.only == "mtok":
+            res = ({"metric": "million-token decode",
+                    "decode_mtok": run_mtok(local, min(args.steps, 10), layers=args.mtok_layers)}
+                   if rank == 0 else None)
         elif args.only == "paged":
             res = ({"metric": "paged-cache decode",
                     "decode_paged": run_variant_decode(local, "bf16", True, args.steps, args.warmup)}
@@ -902,8 +1224,16 @@ def main(argv=None):
                 res["decode_paged"] = run_variant_decode(local, "bf16", True)
                 res["decode_seqsplit"] = run_seqsplit(local)
                 res["decode_gated"] = run_gated(local)
+            if world == 1 and not args.no_workloads and args.only != "decode":
+                res["decode_tiny"] = run_tiny(local)
+                res["decode_mha32k"] = run_mha32k(local)
+                res["decode_mtok"] = run_mtok(local)
             if rank == 0 and world == 1 and not args.no_cpu_baseline:
                 res["cpu_baseline"] = cpu_baseline(ctx)
+                if "prefill" in res:
+                    res["prefill"]["cpu_baseline"] = cpu_baseline_prefill()
+                if "decode_mtok" in res:
+                    res["decode_mtok"]["cpu_baseline"] = cpu_baseline_mtok()
         if rank == 0 and res is not None:
             print(json.dumps(res), flush=True)
     finally:
