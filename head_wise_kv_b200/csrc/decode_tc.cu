@@ -47,10 +47,8 @@
 //   warp 7 also writes the output of segments without keys and sets the
 //              length status bits.
 //   INT4 caches add warps 12-19 (640 threads): the producers bring the packed
-//              codes into a staging ring and these warps expand them to 8-bit
-//              integer tiles (12-15 K, 16-19 V); both products then run as
-//              exact integer MMAs (kind::i8), and the epilogue warps add up
-//              each tile's integer O^T in fp32 (see Tr).
+//              codes into a staging ring and these warps expand them to E4M3
+//              tiles (12-15 K, 16-19 V) for the FP8 arithmetic.
 //
 // Every mbarrier wait is bounded; on a timeout the CTA sets
 // DUO_STATUS_WAIT_TIMEOUT, stops, waits (bounded) for its copies and MMAs in
@@ -82,8 +80,8 @@ constexpr uint32_t kSlab = 128 * 128;         // 128 rows x 64 bf16: one dim-hal
 constexpr uint32_t kTileBytes = 32768;        // one K or V tile: 128 bf16 rows or 256 FP8 rows
 // INT4 caches: the producers bring 256-row tiles of packed codes (64 bytes a
 // row) into a staging ring; eight converter warps (12-15 for K, 16-19 for V)
-// expand them to one byte per element in the 8-bit tile layout (keys as u8
-// c + 8, values as s8 c), for integer MMAs.
+// expand them to E4M3 in the FP8 tile layout, and the rest of the kernel is
+// the FP8 one.
 constexpr int kConvWarp0 = 12;
 constexpr int kThreadsI4 = 640;
 constexpr uint32_t kTile4Bytes = 16384;       // one K or V tile of 256 INT4 rows
@@ -115,20 +113,13 @@ constexpr int kSegWeightF8 = DUO_DECODE_SEG_WEIGHT_FP8;
 //         the prefill's P) and split into three E4M3 terms, columns
 //         term * G + h; the products run as kind::f8f6f4 straight on the
 //         cached codes.
-//   INT4: 256-key tiles of 8-bit integers on kind::i8 (exact integer
-//         products): keys as u = c + 8 (u8), values as c (s8), q as three
-//         s8 terms (~21 bits), P as a 24-bit fixed-point integer in three u8
-//         terms; S^T and each tile's O^T in s32, O accumulated in fp32 by the
-//         epilogue warps (an integer accumulator cannot be rescaled).
-template <int G, bool F8, bool I4 = false>
+template <int G, bool F8>
 struct Tr {
     static constexpr int T = F8 ? 256 : 128;                       // keys per tile
     static constexpr int HALVES = T / 128;                         // 128-key blocks of S^T
-    static constexpr int QT = I4 ? 3 : F8 ? 4 : 1;                 // q terms
+    static constexpr int QT = F8 ? 4 : 1;                          // q terms
     static constexpr int PT = F8 ? 3 : 2;                          // P terms
-    static constexpr int N = I4 ? ((3 * G + 15) / 16) * 16 : F8 ? ((4 * G + 15) / 16) * 16 : 16;   // MMA N
-    // S^T columns read back per 128-key block: QT * G rounded up to a power of two
-    static constexpr int SL = QT * G <= 1 ? 1 : QT * G <= 2 ? 2 : QT * G <= 4 ? 4 : QT * G <= 8 ? 8 : QT * G <= 16 ? 16 : 32;
+    static constexpr int N = F8 ? ((4 * G + 15) / 16) * 16 : 16;   // MMA N (QT * G >= PT * G columns)
     // O^T columns read back: PT * G rounded up to a power of two (the
     // columns past PT * G hold zeros: their P^T rows are never written)
     static constexpr int OL = PT * G <= 2 ? 2 : PT * G <= 4 ? 4 : PT * G <= 8 ? 8 : PT * G <= 16 ? 16 : 32;
@@ -148,15 +139,39 @@ struct Tr {
     // no such floor: threshold 2^8, no offset, no headroom.
     static constexpr float THRESH = F8 ? 1.75f : kRescaleThreshold;   // log2 units
     static constexpr float HEAD = F8 ? 2.0f : 0.0f;
-    // log2 of the P offset: FP8 enters P' = 2^7 P, INT4 the integer rn(2^22 P) <= 2^23.75
-    static constexpr float POFF = I4 ? 22.0f : F8 ? 7.0f : 0.0f;
-    static constexpr uint32_t IQK = I4 ? idesc_i8(128, N, false, true, false, false)    // A = K (u8), B = q (s8)
-                                       : idesc_f16(128, N, !F8, false, false);          // A = K (K-major), B = q
-    static constexpr uint32_t IPV = I4 ? idesc_i8(kD, N, true, false, true, false)      // A = V^T (s8, MN-major), B = P^T (u8)
-                                       : idesc_f16(kD, N, !F8, true, false);            // A = V^T (MN-major), B = P^T
-    static_assert(QT * G <= N && PT * G <= N && SL <= N, "terms must fit the MMA N");
+    static constexpr float POFF = F8 ? 7.0f : 0.0f;                    // log2 of the P offset
+    static constexpr uint32_t IQK = idesc_f16(128, N, !F8, false, false);   // A = K (K-major), B = q
+    static constexpr uint32_t IPV = idesc_f16(kD, N, !F8, true, false);     // A = V^T (MN-major), B = P^T
+    static_assert(QT * G <= N && PT * G <= N, "terms must fit the MMA N");
 };
 
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+// Eight INT4 codes (two's complement nibbles, element i in bits 4i..4i+3)
+// -> their eight values as E4M3 bytes (exact: every integer in [-8, 7] is an
+// E4M3 value), four per byte permute.  A permute selector with bit 3 set
+// yields the sign of the chosen byte replicated, so with the nibble itself
+// as the selector:
+//   table E4M3(0..7) (signs 0):            the code of c >= 0, else 0x00;
+//   nibble xor 8, table E4M3(-8..-1):      the code of c < 0, else 0xFF;
+//   bytes whose bit 7 is the sign of each element, replicated: 0xFF for c < 0;
+// and code = first | (second & third).  The right shift by 16 runs as a
+// multiply-high and the left shift as a multiply, off the integer pipe.
+__device__ __forceinline__ uint2 int4x8_to_e4m3(uint32_t w) {
+    constexpr uint32_t kPos0 = 0x44403800u, kPos1 = 0x4E4C4A48u;   // E4M3 of 0, 1, ..., 7
+    constexpr uint32_t kNeg0 = 0xCACCCED0u, kNeg1 = 0xB8C0C4C8u;   // E4M3 of -8, -7, ..., -1
+    const uint32_t hi = __umulhi(w, 0x10000u);                      // w >> 16: elements 4..7
+    const uint32_t w4 = w * 16u;                                    // bit 8k+7: sign of element 2k
+    const uint32_t wx = w ^ 0x88888888u, hx = hi ^ 0x8888u;
+    uint2 r;
+    r.x = prmt(kPos0, kPos1, w) | (prmt(kNeg0, kNeg1, wx) & prmt(w4, w, 0xD9C8u));
+    r.y = prmt(kPos0, kPos1, hi) | (prmt(kNeg0, kNeg1, hx) & prmt(w4, w, 0xFBEAu));
+    return r;
+}
 
 // Two values -> two E4M3 codes (round to nearest even, saturating); the
 // first operand lands in the upper byte.
@@ -184,40 +199,6 @@ __device__ __forceinline__ void umma_f8(uint32_t tmem_d, uint64_t adesc, uint64_
         ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
-
-// D (TMEM, s32) (+)= A (smem, u8 / s8) * B (smem, u8 / s8): exact integer products.
-__device__ __forceinline__ void umma_i8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                        uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// Sixteen bytes of packed INT4 codes (32 elements, element 2i in the low
-// nibble of byte i) -> 32 bytes, even elements first: `ev` holds elements
-// 0, 2, ..., 30 and `od` elements 1, 3, ..., 31.  Keys become offset-binary
-// u8 (c + 8 = nibble xor 8), values two's-complement s8 (c = (u + 0x78) xor
-// 0x80 per byte: u + 0x78 never carries out of its byte).
-__device__ __forceinline__ void int4x32_to_u8(const uint4 w, uint4& ev, uint4& od) {
-    ev = make_uint4((w.x & 0x0F0F0F0Fu) ^ 0x08080808u, (w.y & 0x0F0F0F0Fu) ^ 0x08080808u,
-                    (w.z & 0x0F0F0F0Fu) ^ 0x08080808u, (w.w & 0x0F0F0F0Fu) ^ 0x08080808u);
-    od = make_uint4(((w.x >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u, ((w.y >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u,
-                    ((w.z >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u, ((w.w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u);
-}
-__device__ __forceinline__ uint4 u8_to_s8(const uint4 u) {
-    return make_uint4((u.x + 0x78787878u) ^ 0x80808080u, (u.y + 0x78787878u) ^ 0x80808080u,
-                      (u.z + 0x78787878u) ^ 0x80808080u, (u.w + 0x78787878u) ^ 0x80808080u);
-}
-
-// INT4 tiles keep each 32-element block as its even elements (16-byte chunk
-// 2j) then its odd elements (chunk 2j + 1): byte column P of a 128-byte row
-// holds dimension dim_of_col(P).  q is staged in the same order; the
-// epilogue thread of TMEM lane P (row P of O^T) writes output dimension
-// dim_of_col(P).
-__device__ __forceinline__ int dim_of_col(int P) { return ((P >> 5) << 5) + ((P & 15) << 1) + ((P >> 4) & 1); }
 
 __device__ __forceinline__ void st_shared_u8(uint32_t addr, uint32_t v) {
     asm volatile("st.shared.b8 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
@@ -316,7 +297,6 @@ __device__ __forceinline__ void tile_coords(const DecodeParams& p, const Piece& 
 // Lane 0 polls for the warp, napping between polls: for waits that span a
 // whole piece, so that the poll takes no issue slots from the warps on the
 // critical path.
-template <unsigned kNapNs = 256>
 __device__ __forceinline__ bool warp_wait_lazy(uint32_t bar, uint32_t parity, const DecodeParams& p,
                                                volatile int* abort_flag) {
     int ok = 1;
@@ -333,7 +313,7 @@ __device__ __forceinline__ bool warp_wait_lazy(uint32_t bar, uint32_t parity, co
                 ok = 0;
                 break;
             }
-            __nanosleep(kNapNs);
+            __nanosleep(256);
         }
     }
     ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -382,8 +362,8 @@ __device__ __forceinline__ uint16_t bf16_bits(float x) { return __bfloat16_as_us
 template <int G, bool F8, bool PAGED, bool I4>
 __global__ void __launch_bounds__(I4 ? kThreadsI4 : kThreads, 1)
     decode_tc_kernel(const __grid_constant__ DecodeParams p) {
-    using C = Tr<G, F8, I4>;
-    static_assert(!I4 || F8, "INT4 caches take the 256-key tiles of the 8-bit types");
+    using C = Tr<G, F8>;
+    static_assert(!I4 || F8, "INT4 caches run the FP8 arithmetic");
     constexpr int NT = I4 ? kThreadsI4 : kThreads;
     constexpr int BLK = PAGED ? C::T : 16;   // partition block (tokens)
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -412,12 +392,6 @@ __global__ void __launch_bounds__(I4 ? kThreadsI4 : kThreads, 1)
     // FP8: 2^-a of each piece's q prescale, a ring of four (the q warp runs
     // at most three pieces ahead of the softmax, see the q warp)
     __shared__ float q_scale[4];
-    // INT4: each piece's offset correction per head (8 sum_d q'_d, see the q
-    // warp), in the same ring; each tile's rescale factor of the running O
-    // per head, a ring of four tiles (a_full), from the softmax to the epilogue
-    __shared__ float q_corr[4][G];
-    __shared__ float alpha_r[4][G];
-    __shared__ __align__(8) uint64_t a_full[4], lm_empty[2];
     __shared__ uint32_t tmem_base_sh;
     __shared__ float red_max[2][4][G];
     __shared__ float red_l[2][4][G];   // [piece parity][softmax warp][head] row sums
@@ -455,8 +429,6 @@ __global__ void __launch_bounds__(I4 ? kThreadsI4 : kThreads, 1)
         }
         mbar_init(smem_addr(&mma_fin), 1);
         for (int s = 0; s < 4; ++s) mbar_init(smem_addr(&qs_full[s]), 1);
-        for (int s = 0; s < 4; ++s) mbar_init(smem_addr(&a_full[s]), 1);
-        for (int s = 0; s < 2; ++s) mbar_init(smem_addr(&lm_empty[s]), 4);
         mbar_init(smem_addr(&pg_ready), 1);
         abort_sh = 0;
         fence_mbar_init();
@@ -564,93 +536,7 @@ __global__ void __launch_bounds__(I4 ? kThreadsI4 : kThreads, 1)
                 if (!warp_wait(smem_addr(&q_empty[pi & 1]), ((pi >> 1) & 1) ^ 1, p, abort_flag)) break;
                 const uint16_t* qb = p.q + (size_t(pc.b) * p.hq + size_t(pc.g) * G) * kD;
                 const uint32_t qs = sQ + (pi & 1) * C::QB;
-                if constexpr (I4) {
-                    // q' = q * 2^a (exact) with max |q'| in [32, 64), then three
-                    // s8 terms: q' = t0 + t1 / 2^7 + t2 / 2^14 + r, |r| <= 2^-15,
-                    // each t = rn(what the previous terms left, times 2^7), so
-                    // |t| <= 64.  Item (head h, 32-dim block k) per lane; its
-                    // even dims go to chunk 2k of row term * G + h, odd dims to
-                    // chunk 2k + 1 (the order of the INT4 tiles' columns).  The
-                    // keys enter as u = c + 8: the sum of the products exceeds
-                    // q'.c by 8 sum_d q'_d, removed in the softmax.
-                    constexpr int kItems = (G * 4 + 31) / 32;
-                    uint4 raw[kItems][4];
-                    float amax = 0.f;
-#pragma unroll
-                    for (int k = 0; k < kItems; ++k) {
-                        const int c = lane + 32 * k;
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) raw[k][i] = make_uint4(0, 0, 0, 0);
-                        if (c < G * 4) {
-                            const uint16_t* src = qb + (c >> 2) * kD + (c & 3) * 32;
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) raw[k][i] = *reinterpret_cast<const uint4*>(src + 8 * i);
-                        }
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const uint32_t w[4] = {raw[k][i].x, raw[k][i].y, raw[k][i].z, raw[k][i].w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e)
-                                amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w[e] << 16)),
-                                                         fabsf(__uint_as_float(w[e] & 0xffff0000u))));
-                        }
-                    }
-                    uint32_t abits;
-                    asm volatile("redux.sync.max.u32 %0, %1, 0xffffffff;" : "=r"(abits) : "r"(__float_as_uint(amax)));
-                    const int e = abits ? int((abits >> 23) & 0xff) - 127 : 0;
-                    const int a = 5 - e < -100 ? -100 : (5 - e > 100 ? 100 : 5 - e);
-                    const float up = __uint_as_float(uint32_t(a + 127) << 23);   // 2^a
-                    int qsum[3] = {0, 0, 0};   // this lane's sum of each term over its item (one item per lane)
-#pragma unroll
-                    for (int k = 0; k < kItems; ++k) {
-                        const int c = lane + 32 * k;
-                        if (c >= G * 4) continue;
-                        float y[32];
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const uint32_t w[4] = {raw[k][i].x, raw[k][i].y, raw[k][i].z, raw[k][i].w};
-#pragma unroll
-                            for (int e2 = 0; e2 < 4; ++e2) {
-                                y[8 * i + 2 * e2] = __uint_as_float(w[e2] << 16) * up;
-                                y[8 * i + 2 * e2 + 1] = __uint_as_float(w[e2] & 0xffff0000u) * up;
-                            }
-                        }
-#pragma unroll
-                        for (int term = 0; term < 3; ++term) {
-                            uint32_t ev[4], od[4];
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) {
-                                const int te = __float2int_rn(y[2 * i]), to = __float2int_rn(y[2 * i + 1]);
-                                qsum[term] += te + to;
-                                if (term < 2) {
-                                    y[2 * i] = (y[2 * i] - float(te)) * 128.f;
-                                    y[2 * i + 1] = (y[2 * i + 1] - float(to)) * 128.f;
-                                }
-                                const uint32_t be = uint32_t(te) & 0xffu, bo = uint32_t(to) & 0xffu;
-                                if ((i & 3) == 0) {
-                                    ev[i >> 2] = be;
-                                    od[i >> 2] = bo;
-                                } else {
-                                    ev[i >> 2] |= be << (8 * (i & 3));
-                                    od[i >> 2] |= bo << (8 * (i & 3));
-                                }
-                            }
-                            const int row = term * G + (c >> 2), blk = c & 3;
-                            st_shared_v4(qs + small_off(row, 2 * blk), make_uint4(ev[0], ev[1], ev[2], ev[3]));
-                            st_shared_v4(qs + small_off(row, 2 * blk + 1), make_uint4(od[0], od[1], od[2], od[3]));
-                        }
-                    }
-                    // per head: the four lanes of its blocks hold the partial sums
-#pragma unroll
-                    for (int term = 0; term < 3; ++term) {
-                        qsum[term] += __shfl_xor_sync(0xffffffffu, qsum[term], 1);
-                        qsum[term] += __shfl_xor_sync(0xffffffffu, qsum[term], 2);
-                    }
-                    if ((lane & 3) == 0 && lane < G * 4)
-                        q_corr[pi & 3][lane >> 2] =
-                            8.f * (float(qsum[0]) + float(qsum[1]) * 0.0078125f + float(qsum[2]) * 0.00006103515625f);
-                    if (lane == 0) q_scale[pi & 3] = __uint_as_float(uint32_t(127 - a) << 23) * p.k_scale[pc.g];
-                } else if constexpr (F8) {
+                if constexpr (F8) {
                     // q' = q * 2^a (exact) with max |q'| in [128, 256), then four
                     // E4M3 terms, each the code of what the previous ones left:
                     // q' = t0 + t1 + t2 + t3 + r, |r| ~ 2^-16 |q'|.  Row
@@ -791,15 +677,7 @@ __global__ void __launch_bounds__(I4 ? kThreadsI4 : kThreads, 1)
                             tc_fence_after();
                             const uint32_t sk = sK + st * kTileBytes, sq = sQ + (cq.pi & 1) * C::QB;
                             const uint32_t ts = tmem + ((jq & 1) ? C::S1 : C::S0);
-                            if constexpr (I4) {
-                                // as FP8, on 8-bit integers (keys u8, q terms s8)
-#pragma unroll
-                                for (int hf = 0; hf < 2; ++hf)
-#pragma unroll
-                                    for (int k = 0; k < 4; ++k)
-                                        umma_i8(ts + hf * C::N, smem_desc(sk + hf * 16384 + k * 32, 16, 1024),
-                                                smem_desc(sq + k * 32, 16, 1024), C::IQK, k > 0 ? 1u : 0u);
-                            } else if constexpr (F8) {
+                            if constexpr (F8) {
                                 // two 128-key halves; K = d = 128 codes = one swizzled row, 4 x K32
 #pragma unroll
                                 for (int hf = 0; hf < 2; ++hf)
@@ -826,25 +704,13 @@ __global__ void __launch_bounds__(I4 ? kThreadsI4 : kThreads, 1)
                     }
                     if (jv < jq) {
                         const int st = int(jv % uint32_t(nst));
-                        // O^T buffers: by piece parity (accumulated over the piece's
-                        // tiles), or for INT4 by tile parity (one tile's integer sums,
-                        // taken over by the epilogue warps)
-                        const uint32_t ob = I4 ? (jv & 1) : (cv.pi & 1);
-                        const uint32_t oph = I4 ? ((jv >> 1) & 1) : ((cv.pi >> 1) & 1);
                         if (mbar_test_wait(smem_addr(&p_full[jv & 1]), (jv >> 1) & 1) &&
                             mbar_test_wait(smem_addr(&full_v[st]), (jv / nst) & 1) &&
-                            ((!I4 && cv.t > 0) || mbar_test_wait(smem_addr(&o_empty[ob]), oph ^ 1))) {
+                            (cv.t > 0 || mbar_test_wait(smem_addr(&o_empty[cv.pi & 1]), ((cv.pi >> 1) & 1) ^ 1))) {
                             tc_fence_after();
                             const uint32_t sv = sV + st * kTileBytes, sp = sP + (jv & 1) * C::PB;
-                            const uint32_t to = tmem + C::O0 + ob * C::OB;
-                            if constexpr (I4) {
-                                // V^T (s8, MN-major) times P^T (u8): 8 x K32 keys, a fresh sum per tile
-#pragma unroll
-                                for (int k = 0; k < 8; ++k)
-                                    umma_i8(to, smem_desc(sv + k * 4096, 16, 1024),
-                                            smem_desc(sp + (k >> 2) * C::PHALF + (k & 3) * 32, 16, 1024), C::IPV,
-                                            k > 0 ? 1u : 0u);
-                            } else if constexpr (F8) {
+                            const uint32_t to = tmem + C::O0 + (cv.pi & 1) * C::OB;
+                            if constexpr (F8) {
                                 // V^T MN-major: d = 128 codes is one 128-byte atom; 8 x K32 keys
 #pragma unroll
                                 for (int k = 0; k < 8; ++k)
@@ -860,7 +726,7 @@ __global__ void __launch_bounds__(I4 ? kThreadsI4 : kThreads, 1)
                             }
                             umma_commit(smem_addr(&empty_v[st]));
                             umma_commit(smem_addr(&p_free[jv & 1]));
-                            if (I4 || cv.t == cv.nt - 1) umma_commit(smem_addr(&o_full[ob]));
+                            if (cv.t == cv.nt - 1) umma_commit(smem_addr(&o_full[cv.pi & 1]));
                             ++jv;
                             cv.advance(p, bpre, gb_end);
                             progressed = true;
@@ -883,15 +749,14 @@ __global__ void __launch_bounds__(I4 ? kThreadsI4 : kThreads, 1)
                 mbar_wait(smem_addr(&mma_fin), 0, p.timeout_ns);
             }
         } else if (I4 && warp >= kConvWarp0) {
-            // ======================================================== INT4 -> 8-bit integers
+            // ======================================================== INT4 -> E4M3
             // Warps 12-15 expand the K tiles, 16-19 the V tiles, in the
             // producers' order.  Thread u of 128 takes the 16-byte pieces u,
             // u + 128, ... of a staged tile (row r = piece / 4, bytes 16 j ..
             // 16 j + 15 = dims 32 j .. 32 j + 31) and writes their 32 codes as
-            // the 16-byte chunks 2 j (even dims) and 2 j + 1 (odd dims) of row
-            // r, in the 128-byte-swizzled layout the tensor cores read (chunk c
-            // of row r stored at position c xor (r mod 8)): keys as u8 c + 8,
-            // values as s8 c.
+            // the 16-byte chunks 2 j and 2 j + 1 of row r in the layout the FP8
+            // tensor map produces (128-byte rows, chunk c of row r stored at
+            // position c xor (r mod 8)).
             if constexpr (I4) {
                 const bool is_k = warp < kConvWarp0 + 4;
                 const int ct = (warp - kConvWarp0) % 4 * 32 + lane;
@@ -919,15 +784,11 @@ __global__ void __launch_bounds__(I4 ? kThreadsI4 : kThreads, 1)
                         for (int u = ct; u < int(kTile4Bytes / 16); u += 128) {
                             const int r = u >> 2, j = u & 3;
                             const uint4 w = ld_shared_v4(src + u * 16);
-                            uint4 ev, od;
-                            int4x32_to_u8(w, ev, od);
-                            if (!is_k) {
-                                ev = u8_to_s8(ev);
-                                od = u8_to_s8(od);
-                            }
+                            const uint2 a = int4x8_to_e4m3(w.x), b = int4x8_to_e4m3(w.y);
+                            const uint2 c = int4x8_to_e4m3(w.z), d = int4x8_to_e4m3(w.w);
                             const uint32_t row = dst + r * 128, sw = r & 7;
-                            st_shared_v4(row + (((2 * j) ^ sw) << 4), ev);
-                            st_shared_v4(row + (((2 * j + 1) ^ sw) << 4), od);
+                            st_shared_v4(row + (((2 * j) ^ sw) << 4), make_uint4(a.x, a.y, b.x, b.y));
+                            st_shared_v4(row + (((2 * j + 1) ^ sw) << 4), make_uint4(c.x, c.y, d.x, d.y));
                         }
                         fence_proxy_async_smem();   // the tensor cores read the codes through the async proxy
                         __syncwarp();
@@ -944,88 +805,40 @@ __global__ void __launch_bounds__(I4 ? kThreadsI4 : kThreads, 1)
             // once the MMA thread's o_full commit for it has landed.
             const int sub = warp & 3;
             const int d = sub * 32 + lane;
-            const int dout = I4 ? dim_of_col(d) : d;   // output dimension of TMEM lane d
             const uint32_t lane_off = uint32_t(sub * 32) << 16;
             int pi = 0;
-            uint32_t jt = 0;   // INT4: tiles taken over so far (the MMA thread's PV order)
             for (int64_t gb = gb_begin; gb < gb_end; ++pi) {
                 Piece pc;
                 if (!next_piece<BLK>(p, bpre, gb, gb_end, pc)) break;
+                const bool got = warp_wait_lazy(smem_addr(&epi_full[pi & 1]), (pi >> 1) & 1, p, abort_flag) &&
+                                 warp_wait_lazy(smem_addr(&o_full[pi & 1]), (pi >> 1) & 1, p, abort_flag);
+                if (barrier_any<kBarEpilogue>(!got)) break;
+                tc_fence_after();
+                uint32_t u[C::OL];
+                tmem_ldn<C::OL>(tmem + lane_off + C::O0 + (pi & 1) * C::OB, u);
+                tmem_wait_ld();
                 float L[G], M[G], o[G];
-                const float vs = F8 ? p.v_scale[pc.g] : 1.f;   // FP8 / INT4: O^T is in value-code units
-                if constexpr (I4) {
-                    // O = sum over tiles of the tile's integer sums, rescaled
-                    // whenever the softmax moved its running max (alpha per tile)
-                    float acc[G];
+                const float vs = F8 ? p.v_scale[pc.g] : 1.f;   // FP8: O^T is in value-code units
 #pragma unroll
-                    for (int h = 0; h < G; ++h) acc[h] = 0.f;
-                    const int nt = tiles_of<C::T>(pc);
-                    bool got = true;
-                    for (int t = 0; t < nt; ++t, ++jt) {
-                        got = warp_wait_lazy<64>(smem_addr(&o_full[jt & 1]), (jt >> 1) & 1, p, abort_flag) &&
-                              warp_wait_lazy<64>(smem_addr(&a_full[jt & 3]), (jt >> 2) & 1, p, abort_flag);
-                        if (barrier_any<kBarEpilogue>(!got)) {
-                            got = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        uint32_t u[C::OL];
-                        tmem_ldn<C::OL>(tmem + lane_off + C::O0 + (jt & 1) * C::OB, u);
-                        tmem_wait_ld();
-                        float al[G];
+                for (int h = 0; h < G; ++h) {
+                    float x = 0.f;
 #pragma unroll
-                        for (int h = 0; h < G; ++h) al[h] = alpha_r[jt & 3][h];
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(smem_addr(&o_empty[jt & 1]));
-                        // P = 2^16 t0 + 2^8 t1 + t2: each term's sum is exact in s32
-#pragma unroll
-                        for (int h = 0; h < G; ++h) {
-                            const float x = fmaf(float(int(u[h])), 65536.f,
-                                                 fmaf(float(int(u[G + h])), 256.f, float(int(u[2 * G + h]))));
-                            acc[h] = fmaf(acc[h], al[h], x);
-                        }
-                    }
-                    if (!got) break;
-                    const bool gl = warp_wait_lazy(smem_addr(&epi_full[pi & 1]), (pi >> 1) & 1, p, abort_flag);
-                    if (barrier_any<kBarEpilogue>(!gl)) break;
-#pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        o[h] = acc[h] * vs;
-                        L[h] = red_l[pi & 1][0][h] + red_l[pi & 1][1][h] + red_l[pi & 1][2][h] + red_l[pi & 1][3][h];
-                        M[h] = epi_m[pi & 1][h] - C::POFF;
-                    }
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(smem_addr(&lm_empty[pi & 1]));
-                } else {
-                    const bool got = warp_wait_lazy(smem_addr(&epi_full[pi & 1]), (pi >> 1) & 1, p, abort_flag) &&
-                                     warp_wait_lazy(smem_addr(&o_full[pi & 1]), (pi >> 1) & 1, p, abort_flag);
-                    if (barrier_any<kBarEpilogue>(!got)) break;
-                    tc_fence_after();
-                    uint32_t u[C::OL];
-                    tmem_ldn<C::OL>(tmem + lane_off + C::O0 + (pi & 1) * C::OB, u);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        float x = 0.f;
-#pragma unroll
-                        for (int term = 0; term < C::PT; ++term) x += __uint_as_float(u[term * G + h]);
-                        o[h] = x * vs;
-                    }
-#pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        L[h] = red_l[pi & 1][0][h] + red_l[pi & 1][1][h] + red_l[pi & 1][2][h] + red_l[pi & 1][3][h];
-                        M[h] = epi_m[pi & 1][h] - C::POFF;   // sums are of P' = 2^POFF P
-                    }
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(smem_addr(&o_empty[pi & 1]));
+                    for (int term = 0; term < C::PT; ++term) x += __uint_as_float(u[term * G + h]);
+                    o[h] = x * vs;
                 }
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    L[h] = red_l[pi & 1][0][h] + red_l[pi & 1][1][h] + red_l[pi & 1][2][h] + red_l[pi & 1][3][h];
+                    M[h] = epi_m[pi & 1][h] - C::POFF;   // sums are of P' = 2^POFF P
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_addr(&o_empty[pi & 1]));
                 if (pc.whole) {
 #pragma unroll
                     for (int h = 0; h < G; ++h) {
                         const int qh = pc.g * G + h;
-                        p.out[(size_t(pc.b) * p.hq + qh) * kD + dout] = L[h] > 0.f ? o[h] / L[h] : 0.f;
+                        p.out[(size_t(pc.b) * p.hq + qh) * kD + d] = L[h] > 0.f ? o[h] / L[h] : 0.f;
                         if (d == 0 && p.lse != nullptr)
                             p.lse[size_t(pc.b) * p.hq + qh] =
                                 L[h] > 0.f ? (M[h] + __log2f(L[h])) * 0.69314718055994530942f : -CUDART_INF_F;
@@ -1063,26 +876,69 @@ __global__ void __launch_bounds__(I4 ? kThreadsI4 : kThreads, 1)
                     Ls[h] = 0.f;
                     acc[h] = 0.f;
                 }
-                for (int c = ow.c0; c <= ow.c1; ++c) {
-                    if (total < n && cta_start(c + 1, total, n) == cta_start(c, total, n)) continue;
-                    const size_t slot = size_t(pc.seg) + c;
+                if constexpr (I4) {
+                    // INT4: 640 threads leave 96 registers each, too few for the
+                    // batches below; two passes, one slot at a time
+                    for (int c = ow.c0; c <= ow.c1; ++c) {
+                        if (total < n && cta_start(c + 1, total, n) == cta_start(c, total, n)) continue;
+                        const size_t slot = size_t(pc.seg) + c;
 #pragma unroll
-                    for (int h = 0; h < G; ++h) Mx[h] = fmaxf(Mx[h], __ldcg(&p.ws_ml[(slot * G + h) * 2]));
-                }
-                for (int c = ow.c0; c <= ow.c1; ++c) {
-                    if (total < n && cta_start(c + 1, total, n) == cta_start(c, total, n)) continue;
-                    const size_t slot = size_t(pc.seg) + c;
+                        for (int h = 0; h < G; ++h) Mx[h] = fmaxf(Mx[h], __ldcg(&p.ws_ml[(slot * G + h) * 2]));
+                    }
+                    for (int c = ow.c0; c <= ow.c1; ++c) {
+                        if (total < n && cta_start(c + 1, total, n) == cta_start(c, total, n)) continue;
+                        const size_t slot = size_t(pc.seg) + c;
 #pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        const float f = fast_exp2(__ldcg(&p.ws_ml[(slot * G + h) * 2]) - Mx[h]);
-                        Ls[h] += __ldcg(&p.ws_ml[(slot * G + h) * 2 + 1]) * f;
-                        acc[h] += __ldcg(&p.ws_o[(slot * G + h) * kD + d]) * f;
+                        for (int h = 0; h < G; ++h) {
+                            const float f = fast_exp2(__ldcg(&p.ws_ml[(slot * G + h) * 2]) - Mx[h]);
+                            Ls[h] += __ldcg(&p.ws_ml[(slot * G + h) * 2 + 1]) * f;
+                            acc[h] += __ldcg(&p.ws_o[(slot * G + h) * kD + d]) * f;
+                        }
+                    }
+                } else {
+                    // One pass over the owners' partials, kB slots at a time: all loads
+                    // of a batch are issued before any is used (a segment of one long
+                    // sequence spans tens of CTAs, and a round trip to L2 per slot in
+                    // turn would cost tens of microseconds), with the log-sum-exp
+                    // carried from batch to batch.
+                    constexpr int kB = G <= 2 ? 16 : (G == 4 ? 8 : 4);
+                    for (int cb = ow.c0; cb <= ow.c1; cb += kB) {
+                        float mv[kB][G], lv[kB][G], ov[kB][G];
+#pragma unroll
+                        for (int k = 0; k < kB; ++k) {
+                            const int c = cb + k;
+                            const bool use = c <= ow.c1 &&
+                                             !(total < n && cta_start(c + 1, total, n) == cta_start(c, total, n));
+                            const size_t slot = size_t(pc.seg) + (use ? c : ow.c0);
+#pragma unroll
+                            for (int h = 0; h < G; ++h) {
+                                mv[k][h] = use ? __ldcg(&p.ws_ml[(slot * G + h) * 2]) : kNegBig;
+                                lv[k][h] = use ? __ldcg(&p.ws_ml[(slot * G + h) * 2 + 1]) : 0.f;
+                                ov[k][h] = use ? __ldcg(&p.ws_o[(slot * G + h) * kD + d]) : 0.f;
+                            }
+                        }
+#pragma unroll
+                        for (int h = 0; h < G; ++h) {
+                            float bm = Mx[h];
+#pragma unroll
+                            for (int k = 0; k < kB; ++k) bm = fmaxf(bm, mv[k][h]);
+                            const float r = fast_exp2(Mx[h] - bm);   // 1 when the max is kept
+                            Ls[h] *= r;
+                            acc[h] *= r;
+                            Mx[h] = bm;
+#pragma unroll
+                            for (int k = 0; k < kB; ++k) {
+                                const float f = fast_exp2(mv[k][h] - bm);   // 0 for unused entries
+                                Ls[h] += lv[k][h] * f;
+                                acc[h] += ov[k][h] * f;
+                            }
+                        }
                     }
                 }
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
                     const int qh = pc.g * G + h;
-                    p.out[(size_t(pc.b) * p.hq + qh) * kD + dout] = Ls[h] > 0.f ? acc[h] / Ls[h] : 0.f;
+                    p.out[(size_t(pc.b) * p.hq + qh) * kD + d] = Ls[h] > 0.f ? acc[h] / Ls[h] : 0.f;
                     if (d == 0 && p.lse != nullptr)
                         p.lse[size_t(pc.b) * p.hq + qh] =
                             Ls[h] > 0.f ? (Mx[h] + __log2f(Ls[h])) * 0.69314718055994530942f : -CUDART_INF_F;
@@ -1103,18 +959,9 @@ __global__ void __launch_bounds__(I4 ? kThreadsI4 : kThreads, 1)
                 if (!next_piece<BLK>(p, bpre, gb, gb_end, pc)) break;
                 const uint32_t tmem_o = tmem + lane_off + C::O0 + (pi & 1) * C::OB;
                 float sc = p.scale_log2;   // log2(e) * scale, per score
-                float qc[G];               // INT4: offset correction of the score sums
-#pragma unroll
-                for (int h = 0; h < G; ++h) qc[h] = 0.f;
                 if constexpr (F8) {
                     // (on failure the first tile's barrier below agrees on leaving)
-                    if (warp_wait(smem_addr(&qs_full[pi & 3]), (pi >> 2) & 1, p, abort_flag)) {
-                        sc *= q_scale[pi & 3];
-                        if constexpr (I4) {
-#pragma unroll
-                            for (int h = 0; h < G; ++h) qc[h] = q_corr[pi & 3][h];
-                        }
-                    }
+                    if (warp_wait(smem_addr(&qs_full[pi & 3]), (pi >> 2) & 1, p, abort_flag)) sc *= q_scale[pi & 3];
                 }
                 float m[G], l[G];
 #pragma unroll
@@ -1131,10 +978,10 @@ __global__ void __launch_bounds__(I4 ? kThreadsI4 : kThreads, 1)
                     float s[C::HALVES][G];
                     if (got) {
                         tc_fence_after();
-                        uint32_t u[C::HALVES][C::SL];
+                        uint32_t u[C::HALVES][C::QT * G];
 #pragma unroll
                         for (int hf = 0; hf < C::HALVES; ++hf)
-                            tmem_ldn<C::SL>(tmem + lane_off + (sb ? C::S1 : C::S0) + hf * C::N, u[hf]);
+                            tmem_ldn<C::QT * G>(tmem + lane_off + (sb ? C::S1 : C::S0) + hf * C::N, u[hf]);
                         tmem_wait_ld();
                         tc_fence_before();
                         __syncwarp();
@@ -1143,18 +990,10 @@ __global__ void __launch_bounds__(I4 ? kThreadsI4 : kThreads, 1)
                         for (int hf = 0; hf < C::HALVES; ++hf)
 #pragma unroll
                             for (int h = 0; h < G; ++h) {
-                                if constexpr (I4) {
-                                    // sum_k 2^-7k S_k over the q terms, less 8 sum_d q'_d
-                                    s[hf][h] = fmaf(float(int(u[hf][h])), 1.f,
-                                                    fmaf(float(int(u[hf][G + h])), 0.0078125f,
-                                                         fmaf(float(int(u[hf][2 * G + h])), 0.00006103515625f,
-                                                              -qc[h])));
-                                } else {
-                                    float x = __uint_as_float(u[hf][h]);
+                                float x = __uint_as_float(u[hf][h]);
 #pragma unroll
-                                    for (int term = 1; term < C::QT; ++term) x += __uint_as_float(u[hf][term * G + h]);
-                                    s[hf][h] = x;
-                                }
+                                for (int term = 1; term < C::QT; ++term) x += __uint_as_float(u[hf][term * G + h]);
+                                s[hf][h] = x;
                             }
                     }
                     const int64_t left = rows_total - int64_t(t) * C::T;
@@ -1191,33 +1030,7 @@ __global__ void __launch_bounds__(I4 ? kThreadsI4 : kThreads, 1)
                     }
                     // P^T buffer sb is free once PV_{j-2} has completed
                     if (!warp_wait(smem_addr(&p_free[sb]), ((j >> 1) & 1) ^ 1, p, abort_flag)) continue;
-                    if constexpr (I4) {
-                        // The epilogue warps read alpha of tile j after PV_j; entry
-                        // j mod 4 was last read for tile j - 4, before the epilogue
-                        // released the O^T buffer that PV_{j-2} (completed: p_free
-                        // above) needed.
-                        if (sw == 0 && lane == 0) {
-#pragma unroll
-                            for (int h = 0; h < G; ++h) alpha_r[j & 3][h] = alpha[h];
-                            mbar_arrive(smem_addr(&a_full[j & 3]));
-                        }
-                        // keys `row` and `row` + 128 of P^T: P'' = rn(2^22 P) <= 2^23.75
-                        // as three u8 terms (bits 16-23, 8-15, 0-7), rows term * G + h
-                        const uint32_t pb = sP + sb * C::PB + (row & 15);
-#pragma unroll
-                        for (int h = 0; h < G; ++h) {
-                            const float r0 = fast_exp2(s[0][h] - m[h] + C::POFF);   // 0 off-piece
-                            const float r1 = fast_exp2(s[1][h] - m[h] + C::POFF);
-                            l[h] += r0 + r1;
-                            const uint32_t i0 = __float2uint_rn(r0), i1 = __float2uint_rn(r1);
-#pragma unroll
-                            for (int term = 0; term < 3; ++term) {
-                                const uint32_t off = small_off(term * G + h, row >> 4);
-                                st_shared_u8(pb + off, i0 >> (16 - 8 * term));
-                                st_shared_u8(pb + C::PHALF + off, i1 >> (16 - 8 * term));
-                            }
-                        }
-                    } else if constexpr (F8) {
+                    if constexpr (F8) {
                         // keys `row` and `row` + 128 of P^T: P' rounded to fp16, then
                         // three E4M3 terms peeled off in fp16 (each residual is exact
                         // in fp16; three 4-bit terms cover its 11 bits); rows term * G + h
@@ -1273,7 +1086,7 @@ __global__ void __launch_bounds__(I4 ? kThreadsI4 : kThreads, 1)
                         }
                     }
                     fence_proxy_async_smem();
-                    if (!I4 && t > 0 && grow_any) {
+                    if (t > 0 && grow_any) {
                         // rescale O^T (rows = dims) once PV_{j-1} has landed
                         if (!warp_wait(smem_addr(&p_free[(j - 1) & 1]), ((j - 1) >> 1) & 1, p, abort_flag)) continue;
                         tc_fence_after();
@@ -1295,12 +1108,8 @@ __global__ void __launch_bounds__(I4 ? kThreadsI4 : kThreads, 1)
                 if (!ok) break;
 
                 // ---- hand the piece to the epilogue warps (per-warp row sums and
-                // the max) and go on with the next piece at once; the entries of
-                // piece pi - 2 have been read once the epilogue released them
-                // (with its O^T buffer, or for INT4 on their own barrier)
-                if (!warp_wait(smem_addr(I4 ? &lm_empty[pi & 1] : &o_empty[pi & 1]), ((pi >> 1) & 1) ^ 1, p,
-                               abort_flag))
-                    continue;
+                // the max) and go on with the next piece at once
+                if (!warp_wait(smem_addr(&o_empty[pi & 1]), ((pi >> 1) & 1) ^ 1, p, abort_flag)) continue;
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
                     float x = l[h];
@@ -1349,7 +1158,7 @@ __global__ void __launch_bounds__(I4 ? kThreadsI4 : kThreads, 1)
 
 template <int G, bool F8, bool PAGED, bool I4>
 cudaError_t launch_g(const DecodeParams& p, cudaStream_t s) {
-    using C = Tr<G, F8, I4>;
+    using C = Tr<G, F8>;
     DecodeParams q = p;
     // partition: 16-token blocks, or whole tiles for paged caches (no tile
     // straddles a page); the segment weight is a fixed number of keys
