@@ -232,8 +232,7 @@ def run_ours(args, rank, world, local):
 
     def one(i):
         s = i % steps
-        cache.append(0, dk[s], dv[s], lb[s])
-        cache.decode(0, dq[s], la[s], scale, out=out)
+        cache.step(0, dq[s], dk[s], dv[s], lb[s], la[s], scale, out=out)   # append + decode
 
     for i in range(args.warmup):
         one(i)
@@ -332,8 +331,7 @@ def run_ours(args, rank, world, local):
         if i >= 2:
             stream.wait_event(ev_out[k])               # step i-2's output has been copied out
         q_, k_, v_, lb_, la_ = views[k]
-        cache.append(0, k_, v_, lb_)
-        cache.decode(0, q_, la_, scale, out=outs2[k])
+        cache.step(0, q_, k_, v_, lb_, la_, scale, out=outs2[k])
         ev_comp[k].record(stream)
 
     def d2h(i):
@@ -383,7 +381,7 @@ def run_ours(args, rank, world, local):
         "data": "synthetic",
         "config": {
             "workload": "gqa128k: GQA 32q/8kv d=128, B=8/GPU ragged T~U[16384,131072], 4/8 KV heads "
-                        "retrieval, S=64 W=256, append+decode per layer-step, 32 distinct steps cycled",
+                        "retrieval, S=64 W=256, append+decode per layer-step (duo_decode_step), 32 distinct steps cycled",
             "global_batch": B * world,
             "seq_len": [int(x) for x in lens0],
             "kv_bytes_per_layer_step": int(avg_bytes),
@@ -455,16 +453,14 @@ def run_variant_decode(local, kv_dtype="fp8", paged=False, steps=512, warmup=16)
     stream = torch.cuda.current_stream(dev)
     for i in range(warmup):
         s = i % base.steps
-        cache.append(0, dk[s], dv[s], lb[s])
-        cache.decode(0, dq[s], la[s], base.scale, out=out)
+        cache.step(0, dq[s], dk[s], dv[s], lb[s], la[s], base.scale, out=out)
     torch.cuda.synchronize()
     assert cache.status() == 0, "device status set during the warm-up"
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for i in range(steps):                   # layer-steps, events only at the ends
         s = i % base.steps
-        cache.append(0, dk[s], dv[s], lb[s])
-        cache.decode(0, dq[s], la[s], base.scale, out=out)
+        cache.step(0, dq[s], dk[s], dv[s], lb[s], la[s], base.scale, out=out)
     e1.record(stream)
     torch.cuda.synchronize()
     step_ms = e0.elapsed_time(e1) / steps
@@ -721,8 +717,7 @@ def run_tiny(local, steps=512, warmup=16):
         s = i % w.steps
         flush.zero_()
         ev[i][0].record(stream)
-        cache.append(0, dk[s], dv[s], lb[s])
-        cache.decode(0, dq[s], la[s], w.scale, out=out)
+        cache.step(0, dq[s], dk[s], dv[s], lb[s], la[s], w.scale, out=out)
         ev[i][1].record(stream)
     torch.cuda.synchronize()
     assert cache.status() == 0, "device status set during the tiny benchmark"
@@ -772,15 +767,13 @@ def run_mha32k(local, steps=1024, warmup=32, copies=4):
 
     for i in range(warmup):
         c, s = which(i)
-        c.append(0, dk[s], dv[s], lb[s])
-        c.decode(0, dq[s], la[s], w.scale, out=out)
+        c.step(0, dq[s], dk[s], dv[s], lb[s], la[s], w.scale, out=out)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for i in range(steps):                   # events only at the ends
         c, s = which(i)
-        c.append(0, dk[s], dv[s], lb[s])
-        c.decode(0, dq[s], la[s], w.scale, out=out)
+        c.step(0, dq[s], dk[s], dv[s], lb[s], la[s], w.scale, out=out)
     e1.record(stream)
     torch.cuda.synchronize()
     step_ms = e0.elapsed_time(e1) / steps
@@ -858,12 +851,13 @@ def run_mtok(local, steps=10, warmup=3, slab=65536, layers=None):
 
     def step(ev=None):
         for layer in range(w.layers):
-            cache.append(layer, ks[layer], vs[layer], lb)
-            if ev is not None:
-                ev[layer][0].record(stream)
+            if ev is None:
+                cache.step(layer, qs[layer], ks[layer], vs[layer], lb, la, w.scale, out=out)
+                continue
+            cache.append(layer, ks[layer], vs[layer], lb)      # per-launch times: the two calls apart
+            ev[layer][0].record(stream)
             cache.decode(layer, qs[layer], la, w.scale, out=out)
-            if ev is not None:
-                ev[layer][1].record(stream)
+            ev[layer][1].record(stream)
 
     for _ in range(warmup):
         step()

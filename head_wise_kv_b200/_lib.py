@@ -46,7 +46,7 @@ EXPORTED = (
     "duo_prefill_workspace_bytes", "duo_prefill_attn", "duo_kv_read_status",
     "duo_kv_set_decode_ctas", "duo_strerror", "duo_decode_attn_static_ws",
     "duo_kv_append_rows", "duo_decode_attn_rows", "duo_lse_merge", "duo_alpha_blend", "duo_kv_set_page_table",
-    "duo_kv_fork", "duo_kv_check_wait_timeout",
+    "duo_kv_fork", "duo_kv_check_wait_timeout", "duo_decode_step",
 )
 DUO_STATIC_WS_BYTES = 4 << 20
 
@@ -115,6 +115,7 @@ _c_set_ctas = _sig("duo_kv_set_decode_ctas", [_P, _I32])
 _c_set_pages = _sig("duo_kv_set_page_table", [_P, _P, _I32])
 _c_fork = _sig("duo_kv_fork", [_P, _I32, _I32, _I32, _P])
 _c_waitcheck = _sig("duo_kv_check_wait_timeout", [_P, ctypes.c_uint64, _P])
+_c_step = _sig("duo_decode_step", [_P, _I32, _P, _P, _P, _P, _P, ctypes.c_float, _P, _P, _P, _SZ, _P])
 _c_strerror = _sig("duo_strerror", [ctypes.c_int], ctypes.c_char_p)
 
 
@@ -246,3 +247,9 @@ def duo_kv_fork(handle, src: int, dst: int, length: int, stream: int) -> None:
 
 def duo_kv_check_wait_timeout(handle, limit_ns: int, stream: int) -> None:
     _check(_c_waitcheck(handle, limit_ns, stream), "duo_kv_check_wait_timeout")
+
+
+def duo_decode_step(handle, layer, k_new, v_new, len_before, q, length, scale, out, lse, workspace,
+                    workspace_bytes, stream) -> None:
+    _check(_c_step(handle, layer, k_new, v_new, len_before, q, length, scale, out, lse, workspace, workspace_bytes,
+                   stream), "duo_decode_step")

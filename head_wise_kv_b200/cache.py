@@ -210,6 +210,28 @@ class DuoKVCache:
                           self._ws.numel(), _stream(self.device))
         return (out, lse) if lse is not None else out
 
+    def step(self, layer: int, q, k_new, v_new, len_before, lengths, scale: float, out=None, lse=None,
+             want_lse=False):
+        """One decode step: append the new token (k_new, v_new: bf16 [B][n_kv][1][d]
+        at positions len_before) and decode q (bf16 [B][Hq][d]) over lengths
+        (int32 [B], = len_before + 1); see duo_decode_step.  Returns fp32 out
+        [B][Hq][d] (and lse [B][Hq] if asked)."""
+        shp = (self.B, self.n_kv, 1, self.d)
+        kp = _need(k_new, "k_new", torch.bfloat16, shp, self.device)
+        vp = _need(v_new, "v_new", torch.bfloat16, shp, self.device)
+        bp = _need(len_before, "len_before", torch.int32, (self.B,), self.device)
+        qp = _need(q, "q", torch.bfloat16, (self.B, self.hq, self.d), self.device)
+        lp = _need(lengths, "lengths", torch.int32, (self.B,), self.device)
+        if out is None:
+            out = torch.empty(self.B, self.hq, self.d, dtype=torch.float32, device=self.device)
+        op = _need(out, "out", torch.float32, (self.B, self.hq, self.d), self.device)
+        if want_lse and lse is None:
+            lse = torch.empty(self.B, self.hq, dtype=torch.float32, device=self.device)
+        sp = _need(lse, "lse", torch.float32, (self.B, self.hq), self.device) if lse is not None else None
+        L.duo_decode_step(self.handle, layer, kp, vp, bp, qp, lp, float(scale), op, sp, self._ws.data_ptr(),
+                          self._ws.numel(), _stream(self.device))
+        return (out, lse) if lse is not None else out
+
     def prefill(self, layer: int, q, k_chunk, v_chunk, prefix_len, scale: float, out=None):
         """q: bf16 [B][Hq][C][d]; k_chunk, v_chunk: bf16 [B][n_kv][C][d];
         prefix_len: int32 [B].  Returns fp32 out [B][Hq][C][d]."""

@@ -275,9 +275,10 @@ int duo_decode_workspace_bytes(const duo_kv* kv, size_t* bytes) {
     return DUO_OK;
 }
 
-static int decode_impl(duo_kv* kv, int32_t layer, const uint16_t* q, const int32_t* len, const int32_t* r_begin,
-                       const int32_t* r_end, const int32_t* s_len, float scale, float* out, float* lse,
-                       void* workspace, size_t workspace_bytes, duo_stream_t stream) {
+// Checks a decode's arguments and fills its launch parameters.
+static int decode_setup(duo_kv* kv, int32_t layer, const uint16_t* q, const int32_t* len, const int32_t* r_begin,
+                        const int32_t* r_end, const int32_t* s_len, float scale, float* out, float* lse,
+                        void* workspace, size_t workspace_bytes, duo::DecodeParams& p) {
     if (!kv || layer < 0 || layer >= kv->desc.num_layers || !q || (!len && !r_end) || !out)
         return DUO_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(r_begin) & 3) || (reinterpret_cast<uintptr_t>(r_end) & 3) ||
@@ -294,7 +295,6 @@ static int decode_impl(duo_kv* kv, int32_t layer, const uint16_t* q, const int32
     if (!workspace || workspace_bytes < need) return DUO_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return DUO_ERR_ALIGNMENT;
     const duo::LayerLayout& L = kv->layers[layer];
-    duo::DecodeParams p;
     memset(&p, 0, sizeof p);
     if (!kv->maps.empty()) {
         p.tm_kr = kv->maps[layer].kr;
@@ -346,7 +346,33 @@ static int decode_impl(duo_kv* kv, int32_t layer, const uint16_t* q, const int32
         p.max_pages = kv->max_pages;
         p.page_table = kv->page_table;
     }
-    return cuda_err(duo::launch_decode(p, D, G, stream));
+    return DUO_OK;
+}
+
+static int decode_impl(duo_kv* kv, int32_t layer, const uint16_t* q, const int32_t* len, const int32_t* r_begin,
+                       const int32_t* r_end, const int32_t* s_len, float scale, float* out, float* lse,
+                       void* workspace, size_t workspace_bytes, duo_stream_t stream) {
+    duo::DecodeParams p;
+    const int rc = decode_setup(kv, layer, q, len, r_begin, r_end, s_len, scale, out, lse, workspace,
+                                workspace_bytes, p);
+    if (rc) return rc;
+    const int G = kv->desc.num_q_heads / kv->desc.num_kv_heads;
+    return cuda_err(duo::launch_decode(p, kv->desc.head_dim, G, stream));
+}
+
+int duo_decode_step(duo_kv* kv, int32_t layer, const uint16_t* k_new, const uint16_t* v_new,
+                    const int32_t* len_before, const uint16_t* q, const int32_t* len, float scale, float* out,
+                    float* lse, void* workspace, size_t workspace_bytes, duo_stream_t stream) {
+    if (!len || !len_before || (reinterpret_cast<uintptr_t>(len_before) & 3)) return DUO_ERR_INVALID_ARG;
+    duo::DecodeParams p;
+    int rc = decode_setup(kv, layer, q, len, nullptr, nullptr, nullptr, scale, out, lse, workspace, workspace_bytes,
+                          p);
+    if (rc) return rc;
+    rc = append_impl(kv, layer, k_new, v_new, len_before, nullptr, 1, nullptr, nullptr, stream);
+    if (rc) return rc;
+    if (kv->desc.head_dim == 128) p.len_before = len_before;   // read ahead of the append
+    const int G = kv->desc.num_q_heads / kv->desc.num_kv_heads;
+    return cuda_err(duo::launch_decode(p, kv->desc.head_dim, G, stream));
 }
 
 int duo_decode_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const int32_t* len, float scale,

@@ -71,8 +71,12 @@ __device__ __forceinline__ void put8(const AppendParams& p, uint16_t* base, size
 
 template <int D>
 __global__ void __launch_bounds__(kThreads) append_kernel(const __grid_constant__ AppendParams p) {
-    // A decode launched next as a programmatic dependent may start its
-    // set-up now; it waits (griddepcontrol.wait) for this grid's writes.
+    // Launched as a programmatic dependent: the launch overlaps the tail of
+    // the previous kernel, and nothing is read or written before it has
+    // completed.  Only then may a decode launched next start (it waits for
+    // this grid's writes, or in a decode step reads ahead of them: whatever
+    // preceded this append is complete by then).
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;");
     constexpr int TPR = D / 8;   // threads per row, 16 bytes each
     const int64_t rows_total = int64_t(p.B) * p.n_kv * p.n_new_max;
@@ -158,13 +162,24 @@ cudaError_t launch_append(const AppendParams& p, cudaStream_t s) {
     const int64_t threads = (rows + reset_items) * tpr;
     const int64_t blocks = (threads + kThreads - 1) / kThreads;
     if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(blocks));
+    cfg.blockDim = dim3(kThreads);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e;
     if (p.d == 128) {
-        append_kernel<128><<<unsigned(blocks), kThreads, 0, s>>>(p);
+        e = cudaLaunchKernelEx(&cfg, append_kernel<128>, p);
     } else if (p.d == 64) {
-        append_kernel<64><<<unsigned(blocks), kThreads, 0, s>>>(p);
+        e = cudaLaunchKernelEx(&cfg, append_kernel<64>, p);
     } else {
         return cudaErrorInvalidValue;
     }
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -398,6 +398,7 @@ __global__ void __launch_bounds__(I4 ? kThreadsI4 : kThreads, 1)
     __shared__ float epi_m[2][G];      // [piece parity][head] running max
     __shared__ bool epi_last;          // this CTA is the last owner of the piece's segment
     __shared__ int abort_sh;
+    __shared__ bool early_sh;          // step mode: read ahead of the append
     volatile int* abort_flag = &abort_sh;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -446,11 +447,28 @@ __global__ void __launch_bounds__(I4 ? kThreadsI4 : kThreads, 1)
     }
     // Launched as a programmatic dependent: everything above overlaps the
     // previous kernel in the stream; nothing it writes is read before this.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // Step mode (duo_decode_step): the previous kernel is the step's append
+    // of one token per sequence, launched once every input of the step was
+    // in place.  Until it completes only the newest row of each sequence can
+    // be stale (the last row of a retrieval segment, one slot of a streaming
+    // ring): the lengths, q and every other tile are read at once, and a
+    // producer waits for the append before the first tile that may hold such
+    // a row.  Any sequence whose length does not grow by exactly one turns
+    // this off for the launch.
+    const bool step_mode = p.len_before != nullptr;
+    if (!step_mode) asm volatile("griddepcontrol.wait;" ::: "memory");
     build_prefix<BLK>(p, bpre);
+    if (step_mode && warp == 2) {
+        bool one = true;
+        for (int b = lane; b < p.B; b += 32) one = one && p.len_before[b] >= 0 && p.len[b] == p.len_before[b] + 1;
+        one = __all_sync(0xffffffffu, one);
+        if (lane == 0) early_sh = one;
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    const bool early = step_mode && early_sh;
+    if (step_mode && !early) asm volatile("griddepcontrol.wait;" ::: "memory");
     // A following kernel launched as a programmatic dependent may be
     // scheduled now; it waits (griddepcontrol.wait) for this grid's writes.
     asm volatile("griddepcontrol.launch_dependents;");
@@ -467,13 +485,21 @@ __global__ void __launch_bounds__(I4 ? kThreadsI4 : kThreads, 1)
             if (lane == 0) {
                 const uint64_t policy = l2_evict_first_policy();
                 uint32_t it = 0;
+                bool ahead = early;   // reading ahead of the step's append
                 bool ok = !PAGED || timed_wait(smem_addr(&pg_ready), 0, p, abort_flag);
                 for (int64_t gb = gb_begin; ok && gb < gb_end;) {
                     Piece pc;
                     if (!next_piece<BLK>(p, bpre, gb, gb_end, pc)) break;
                     const CUtensorMap* mk = pc.retr ? &p.tm_kr : &p.tm_ks;
                     const bool paged = PAGED && pc.retr;
+                    // first tile that may hold the appended row: a retrieval
+                    // segment's last tile, any tile of a streaming ring
+                    const int64_t t_new = pc.retr ? bpre[2 * p.B + 1 + pc.b] - 1 : 0;
                     for (int64_t t = pc.tok0; t < pc.tok1; t += C::T, ++it) {
+                        if (ahead && t + C::T > t_new) {
+                            asm volatile("griddepcontrol.wait;" ::: "memory");
+                            ahead = false;
+                        }
                         // INT4: the staging ring, filled with codes for the converters
                         const int nr = I4 ? ns4 : nst;
                         const int st = int(it % uint32_t(nr));
@@ -618,13 +644,19 @@ __global__ void __launch_bounds__(I4 ? kThreadsI4 : kThreads, 1)
             if (lane == 0) {
                 const uint64_t policy = l2_evict_first_policy();
                 uint32_t it = 0;
+                bool ahead = early;
                 bool ok = !PAGED || timed_wait(smem_addr(&pg_ready), 0, p, abort_flag);
                 for (int64_t gb = gb_begin; ok && gb < gb_end;) {
                     Piece pc;
                     if (!next_piece<BLK>(p, bpre, gb, gb_end, pc)) break;
                     const CUtensorMap* mv = pc.retr ? &p.tm_vr : &p.tm_vs;
                     const bool paged = PAGED && pc.retr;
+                    const int64_t t_new = pc.retr ? bpre[2 * p.B + 1 + pc.b] - 1 : 0;
                     for (int64_t t = pc.tok0; t < pc.tok1; t += C::T, ++it) {
+                        if (ahead && t + C::T > t_new) {
+                            asm volatile("griddepcontrol.wait;" ::: "memory");
+                            ahead = false;
+                        }
                         const int nr = I4 ? ns4 : nst;
                         const int st = int(it % uint32_t(nr));
                         uint64_t* empty = I4 ? &empty4_v[st] : &empty_v[st];
@@ -1148,6 +1180,8 @@ __global__ void __launch_bounds__(I4 ? kThreadsI4 : kThreads, 1)
         }
     }
 
+    // step mode: the grid ends after the append it read ahead of
+    if (early && threadIdx.x == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {

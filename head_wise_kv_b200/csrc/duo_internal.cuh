@@ -91,6 +91,9 @@ struct DecodeParams {
     int32_t r_before[kMaxKvHeads + 1];
     uint8_t is_r[kMaxKvHeads];
     float k_scale[kMaxKvHeads], v_scale[kMaxKvHeads];   // FP8: this layer's scales
+    // tensor-core kernel, step mode (duo_decode_step): lengths before the
+    // append that precedes this launch in the stream (null otherwise)
+    const int32_t* len_before;
 };
 
 struct AppendParams {

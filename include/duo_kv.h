@@ -258,6 +258,25 @@ DUO_API int duo_decode_attn(duo_kv* kv, int32_t layer, const uint16_t* q, const 
                     float scale, float* out, float* lse, void* workspace, size_t workspace_bytes,
                     duo_stream_t stream);
 
+/* One decode step of one layer: append each sequence's new token, then
+ * decode attention over the cache that includes it.  The result (cache
+ * contents, out, lse, status) is that of
+ *   duo_kv_append(kv, layer, k_new, v_new, len_before, NULL, 1, stream);
+ *   duo_decode_attn(kv, layer, q, len, scale, out, lse, workspace, ...);
+ * with the same arguments, which this call checks before launching
+ * anything.  k_new, v_new: [B][n_kv][1][d] bf16; len_before, len: device
+ * int32 [B].  The two kernels overlap (head_dim 128): the attention kernel
+ * streams every key tile the append does not write while the append runs,
+ * and waits for it only before the last tile of each retrieval head and
+ * the streaming rings (the tiles that may hold the new token).  This relies
+ * on len[b] = len_before[b] + 1 for every sequence, which the kernel
+ * checks; if any sequence differs it waits for the append before reading
+ * anything, as duo_decode_attn does.  Every input must be in place when the
+ * call is made (produced by work already in the stream). */
+DUO_API int duo_decode_step(duo_kv* kv, int32_t layer, const uint16_t* k_new, const uint16_t* v_new,
+                            const int32_t* len_before, const uint16_t* q, const int32_t* len, float scale,
+                            float* out, float* lse, void* workspace, size_t workspace_bytes, duo_stream_t stream);
+
 /* Decode attention over chosen rows.  Like duo_decode_attn, except that
  * the keys come from explicit row ranges instead of the sequence length:
  *   retrieval heads: cache rows [r_begin[b], r_end[b]) (r_begin may be NULL
