@@ -34,21 +34,21 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM read + write bytes per launch of decode_tc_kernel<4> on this workload,
 # from the ncu capture summarised in profiles/decode_tc_kernel_gqa128k.md.  Must be
 # reset to None whenever the decode kernel changes.
-DECODE_TRAFFIC_BYTES = 1123986944 + 3088384
+DECODE_TRAFFIC_BYTES = 1123966208 + 3172096
 # The same for decode_tc_kernel<4, FP8> on the FP8 cache of this workload
 # (profiles/decode_tc_kernel_fp8_gqa128k.md); None once that kernel changes.
-DECODE_FP8_TRAFFIC_BYTES = 562085120 + 3248640
+DECODE_FP8_TRAFFIC_BYTES = 562046464 + 5267968
 # The same for the INT4 instantiation (profiles/decode_tc_kernel_int4_gqa128k.md).
-DECODE_INT4_TRAFFIC_BYTES = 281105408 + 3333888
+DECODE_INT4_TRAFFIC_BYTES = 281096192 + 3445248
 # Paged cache, the two slice launches of the sequence split, and the gated
 # forward's full-attention launch (profiles/decode_tc_kernel_variants_gqa128k.md).
-DECODE_PAGED_TRAFFIC_BYTES = 1120197888 + 3514624
-DECODE_SEQSPLIT_TRAFFIC_BYTES = 838102272 + 3296768 + 291869440 + 427264
-DECODE_GATED_TRAFFIC_BYTES = 2231663616 + 3192064
+DECODE_PAGED_TRAFFIC_BYTES = 1120185344 + 2994432
+DECODE_SEQSPLIT_TRAFFIC_BYTES = 838149120 + 3019264 + 291843840 + 142336
+DECODE_GATED_TRAFFIC_BYTES = 2231668992 + 3008256
 # decode_tc_kernel<1> on one copy of the MHA-32K cache, and decode_tc_kernel<4>
 # on one layer of the million-token cache (profiles/decode_tc_kernel_mha32k_mtok.md).
-MHA32K_DECODE_TRAFFIC_BYTES = 139597056 + 3098112
-MTOK_DECODE_TRAFFIC_BYTES = 1085115648 + 3074816
+MHA32K_DECODE_TRAFFIC_BYTES = 139653376 + 3044352
+MTOK_DECODE_TRAFFIC_BYTES = 1085167360 + 3202048
 
 
 # ---------------------------------------------------------------- helpers
