@@ -363,7 +363,8 @@ static int decode_impl(duo_kv* kv, int32_t layer, const uint16_t* q, const int32
 int duo_decode_step(duo_kv* kv, int32_t layer, const uint16_t* k_new, const uint16_t* v_new,
                     const int32_t* len_before, const uint16_t* q, const int32_t* len, float scale, float* out,
                     float* lse, void* workspace, size_t workspace_bytes, duo_stream_t stream) {
-    if (!len || !len_before || (reinterpret_cast<uintptr_t>(len_before) & 3)) return DUO_ERR_INVALID_ARG;
+    if (!len || !len_before) return DUO_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(len_before) & 3) return DUO_ERR_ALIGNMENT;
     duo::DecodeParams p;
     int rc = decode_setup(kv, layer, q, len, nullptr, nullptr, nullptr, scale, out, lse, workspace, workspace_bytes,
                           p);

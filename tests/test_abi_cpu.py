@@ -113,10 +113,17 @@ def test_null_handle_calls_fail_cleanly():
     for fn, args in [(L.duo_kv_append, (None, 0, 16, 16, 16, None, 1, None)),
                      (L.duo_decode_attn, (None, 0, 16, 16, 0.1, 16, None, 16, 1 << 20, None)),
                      (L.duo_prefill_attn, (None, 0, 16, 16, 16, 16, 8, 0.1, 16, None, 0, None)),
-                     (L.duo_kv_fork, (None, 0, 1, 10, None))]:
+                     (L.duo_kv_fork, (None, 0, 1, 10, None)),
+                     # step: null handle, then a null len_before / len (checked before any launch)
+                     (L.duo_decode_step, (None, 0, 16, 16, 16, 16, 16, 0.1, 16, None, 16, 1 << 20, None)),
+                     (L.duo_decode_step, (None, 0, 16, 16, None, 16, 16, 0.1, 16, None, 16, 1 << 20, None)),
+                     (L.duo_decode_step, (None, 0, 16, 16, 16, 16, None, 0.1, 16, None, 16, 1 << 20, None))]:
         with pytest.raises(L.DuoError) as e:
             fn(*args)
         assert e.value.code == L.DUO_ERR_INVALID_ARG
+    with pytest.raises(L.DuoError) as e:   # len_before not 4-byte aligned
+        L.duo_decode_step(None, 0, 16, 16, 18, 16, 16, 0.1, 16, None, 16, 1 << 20, None)
+    assert e.value.code == L.DUO_ERR_ALIGNMENT
     assert L._c_free(None) == 0
 
 
