@@ -210,7 +210,8 @@ DUO_API int duo_kv_layer_view_get(const duo_kv* kv, int32_t layer, duo_kv_layer_
  * (append_token) and the sliding-window ring of "Attention Variants and
  * Memory Efficiency"; the result equals appending the tokens one at a time.
  * FP8 caches store each value's code (see duo_kv_desc) instead of its bits.
- * Decode order per layer: append the new token, then duo_decode_attn.
+ * Decode order per layer: append the new token, then duo_decode_attn (or
+ * both in one call: duo_decode_step).
  * Prefill order per layer: duo_prefill_attn on the chunk, then append it. */
 DUO_API int duo_kv_append(duo_kv* kv, int32_t layer, const uint16_t* k_new, const uint16_t* v_new,
                   const int32_t* len_before, const int32_t* n_new, int32_t n_new_max,
