@@ -249,8 +249,7 @@ __device__ __forceinline__ bool timed_wait(uint32_t bar, uint32_t parity, const 
     return false;
 }
 
-// Lane 0 waits for the warp.
-// Lane 0 waits (bounded), the warp takes its verdict.
+// Lane 0 waits (bounded) for the warp; the warp takes its result.
 __device__ __forceinline__ bool warp_wait_lead(uint32_t bar, uint32_t parity, const DecodeParams& p,
                                                volatile int* abort_flag) {
     int ok = 1;
