@@ -192,7 +192,12 @@ DUO_API int duo_kv_alloc(const duo_kv_desc* desc, void* dev_buf, size_t buf_byte
 /* Release the host handle.  dev_buf stays the caller's.  NULL is a no-op. */
 DUO_API int duo_kv_free(duo_kv* kv);
 
-/* Fill *out with the device views of `layer`.  Host only. */
+/* Fill *out with the device views of `layer`.  Host only.  This is also the
+ * way to read the position table (the original position of every ring
+ * slot, kept after eviction): out->positions is its device address, which
+ * the caller copies or reads with its own stream, so the library needs no
+ * separate call that copies it (and stays free of allocation and
+ * synchronisation). */
 DUO_API int duo_kv_layer_view_get(const duo_kv* kv, int32_t layer, duo_kv_layer_view* out);
 
 /* Append tokens to one layer's cache (append + evict).
