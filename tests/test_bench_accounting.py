@@ -102,3 +102,34 @@ def test_decode_kv_bytes_of_the_mha32k_step():
     lens = W.context_lengths(w) + 1
     got = bench.kv_bytes(lens, W.retrieval_mask(w, 0), w.d, w.sink, w.window, 10 ** 9)
     assert got == 8 * 512 * 32769 + 24 * 512 * 320 == 138_153_984
+
+
+def test_traffic_constants_match_their_workloads():
+    """Each recorded DRAM traffic per launch (ncu, one launch of the leg's
+    own workload) lies between the leg's algorithmic KV bytes and 5 % above
+    them: reads cannot be fewer than the keys and values the launch must
+    stream, and the excess is the partial outputs and tile tails.  A constant
+    left over from another workload, cache type or kernel falls outside."""
+    base = W.WORKLOADS["gqa128k"]
+    lens = W.context_lengths(base) + 1                       # the captured (first timed) step
+    mask = W.retrieval_mask(base, 0)
+    bf16 = bench.kv_bytes(lens, mask, base.d, base.sink, base.window, cap=10 ** 9)
+    full = bench.kv_bytes(lens, np.ones_like(mask), base.d, base.sink, base.window, cap=10 ** 9)
+    mha = W.WORKLOADS["mha32k"]
+    mha_b = bench.kv_bytes(W.context_lengths(mha) + 1, W.retrieval_mask(mha, 0), mha.d, mha.sink, mha.window,
+                           cap=10 ** 9)
+    mt = W.WORKLOADS["mtok"]
+    mt_b = bench.kv_bytes([mt.t0 + 1], W.retrieval_masks(mt)[0], mt.d, mt.sink, mt.window, cap=10 ** 9)
+    cases = {
+        "bf16": (bench.DECODE_TRAFFIC_BYTES, bf16),
+        "fp8": (bench.DECODE_FP8_TRAFFIC_BYTES, bf16 // 2),
+        "int4": (bench.DECODE_INT4_TRAFFIC_BYTES, bf16 // 4),
+        "paged": (bench.DECODE_PAGED_TRAFFIC_BYTES, bf16),
+        "seqsplit (both slices)": (bench.DECODE_SEQSPLIT_TRAFFIC_BYTES, bf16),
+        "gated (all heads full)": (bench.DECODE_GATED_TRAFFIC_BYTES, full),
+        "mha32k": (bench.MHA32K_DECODE_TRAFFIC_BYTES, mha_b),
+        "mtok (one layer)": (bench.MTOK_DECODE_TRAFFIC_BYTES, mt_b),
+    }
+    for name, (traffic, alg) in cases.items():
+        assert traffic is not None, name
+        assert alg <= traffic <= 1.05 * alg, f"{name}: traffic {traffic} against algorithmic {alg}"
